@@ -1,0 +1,158 @@
+"""Seeded synthetic inputs for the compressor workloads.
+
+This module only draws random numbers and rounds them to the storage dtype; it holds
+none of the compressor's arithmetic.  Both the fp64 oracle (via the tests and the
+bench) and the CUDA path consume the buffers it produces, so parity never depends on
+the generator.
+
+Distributions (N(mu, var) notation, second argument = variance):
+
+* streams C^a, C^b, Z^a, Z^b (or C, Z for HCA): N(0, 1), drawn in fp32, then rounded to
+  bf16 (round-to-nearest-even) where the workload stores bf16;
+* optional per-row logit offsets U(-lo, lo): one offset per (stream, token row), drawn
+  independently for Z^a and Z^b, added to all c channels of that row in fp32 before the
+  bf16 rounding (the long-context workload, lo = 4, stresses the softmax range);
+* position biases B^a, B^b (m x c) and B (m' x c): N(0, 0.1), fp32;
+* hidden states H: N(0, 1) -> bf16; projections W (d x c): N(0, 1/d) -> bf16.
+
+Draw order for a given seed (numpy ``default_rng(seed)``): the streams in the order
+listed in the returned dict, then the offsets, then the biases.  Large workloads can be
+generated directly on the GPU with a seeded ``torch.Generator`` (same distributions,
+different bit stream); that path is used by the full-size parity tests and the bench.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "round_to_bf16",
+    "stream_inputs",
+    "fused_inputs",
+    "stream_inputs_torch",
+    "fused_inputs_torch",
+    "WORKLOADS",
+]
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding them."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    nan = np.isnan(x)
+    out = r.astype(np.uint32).view(np.float32).copy()
+    out[nan] = np.nan
+    return out
+
+
+def _normal(rng, shape, var=1.0):
+    return (rng.standard_normal(shape, dtype=np.float32) * np.float32(np.sqrt(var))).astype(np.float32)
+
+
+def stream_inputs(mode: str, batch: int, n: int, c: int, m: int, dtype: str = "f32",
+                  seed: int = 0, z_row_offset: float = 0.0, bias_var: float = 0.1):
+    """Host (numpy fp32) inputs for the streaming compressor.
+
+    mode "csa": keys Ca, Cb, Za, Zb ([batch, n, c]) and Ba, Bb ([m, c]).
+    mode "hca": keys C, Z ([batch, n, c]) and B ([m, c]).
+    dtype "bf16" rounds the streams to bf16 values (still stored as fp32 here).
+    """
+    rng = np.random.default_rng(seed)
+    names = ("Ca", "Cb", "Za", "Zb") if mode == "csa" else ("C", "Z")
+    out = {}
+    for k in names:
+        out[k] = _normal(rng, (batch, n, c))
+    if z_row_offset:
+        for k in names:
+            if k.startswith("Z"):
+                off = rng.uniform(-z_row_offset, z_row_offset, size=(batch, n, 1)).astype(np.float32)
+                out[k] = (out[k] + off).astype(np.float32)
+    if dtype == "bf16":
+        for k in names:
+            out[k] = round_to_bf16(out[k])
+    elif dtype != "f32":
+        raise ValueError(dtype)
+    bias_names = ("Ba", "Bb") if mode == "csa" else ("B",)
+    for k in bias_names:
+        out[k] = _normal(rng, (m, c), bias_var)
+    return out
+
+
+def fused_inputs(mode: str, batch: int, n: int, d: int, c: int, m: int, seed: int = 0,
+                 bias_var: float = 0.1):
+    """Host inputs for the fused projection path: H [batch*n, d] and the W's [d, c]
+    rounded to bf16 (stored as fp32), biases fp32."""
+    rng = np.random.default_rng(seed)
+    out = {"H": round_to_bf16(_normal(rng, (batch * n, d)))}
+    wn = ("W_kva", "W_kvb", "W_za", "W_zb") if mode == "csa" else ("W_kv", "W_z")
+    for k in wn:
+        out[k] = round_to_bf16(_normal(rng, (d, c), 1.0 / d))
+    for k in (("Ba", "Bb") if mode == "csa" else ("B",)):
+        out[k] = _normal(rng, (m, c), bias_var)
+    return out
+
+
+def stream_inputs_torch(mode: str, batch: int, n: int, c: int, m: int, dtype: str,
+                        seed: int = 0, z_row_offset: float = 0.0, bias_var: float = 0.1,
+                        device="cuda"):
+    """Same distributions as :func:`stream_inputs`, generated on ``device`` with a
+    seeded torch.Generator (for workloads too large to draw on the host quickly)."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    names = ("Ca", "Cb", "Za", "Zb") if mode == "csa" else ("C", "Z")
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = {}
+    for k in names:
+        x = torch.randn((batch, n, c), generator=g, device=device, dtype=torch.float32)
+        if z_row_offset and k.startswith("Z"):
+            off = torch.rand((batch, n, 1), generator=g, device=device, dtype=torch.float32)
+            x += off * (2 * z_row_offset) - z_row_offset
+        out[k] = x.to(tdt)
+        del x
+    for k in (("Ba", "Bb") if mode == "csa" else ("B",)):
+        out[k] = torch.randn((m, c), generator=g, device=device, dtype=torch.float32) * float(np.sqrt(bias_var))
+    return out
+
+
+def fused_inputs_torch(mode: str, batch: int, n: int, d: int, c: int, m: int, seed: int = 0,
+                       bias_var: float = 0.1, device="cuda"):
+    """Same distributions as :func:`fused_inputs`, generated on ``device``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = {}
+    H = torch.empty((batch * n, d), device=device, dtype=torch.bfloat16)
+    rows = max(1, (1 << 28) // d)          # draw in slabs to bound fp32 temporaries
+    for r0 in range(0, batch * n, rows):
+        r1 = min(batch * n, r0 + rows)
+        H[r0:r1] = torch.randn((r1 - r0, d), generator=g, device=device, dtype=torch.float32)
+    out["H"] = H
+    wn = ("W_kva", "W_kvb", "W_za", "W_zb") if mode == "csa" else ("W_kv", "W_z")
+    for k in wn:
+        out[k] = (torch.randn((d, c), generator=g, device=device, dtype=torch.float32)
+                  * float(1.0 / np.sqrt(d))).to(torch.bfloat16)
+    for k in (("Ba", "Bb") if mode == "csa" else ("B",)):
+        out[k] = torch.randn((m, c), generator=g, device=device, dtype=torch.float32) * float(np.sqrt(bias_var))
+    return out
+
+
+# The five workloads, named by what they are.
+WORKLOADS = {
+    "csa_f32_n1024": dict(kind="stream", mode="csa", batch=1, n=1024, c=512, m=4,
+                          in_dtype="f32", out_dtype="f32"),
+    "hca_bf16_n65536": dict(kind="stream", mode="hca", batch=1, n=65536, c=512, m=128,
+                            in_dtype="bf16", out_dtype="bf16"),
+    "csa_fused_n32768_d7168": dict(kind="fused", mode="csa", batch=1, n=32768, d=7168, c=512,
+                                   m=4, out_dtype="bf16"),
+    "hca_fused_4x131072_d4096": dict(kind="fused", mode="hca", batch=4, n=131072, d=4096,
+                                     c=512, m=128, out_dtype="bf16"),
+    "csa_long_n1048576": dict(kind="stream", mode="csa", batch=1, n=1 << 20, c=512, m=4,
+                              in_dtype="bf16", out_dtype="bf16", z_row_offset=4.0),
+    "hca_long_n1048576": dict(kind="stream", mode="hca", batch=1, n=1 << 20, c=512, m=128,
+                              in_dtype="bf16", out_dtype="bf16", z_row_offset=4.0),
+}
