@@ -1,0 +1,381 @@
+"""Throughput of the B200 token-level KV compressor (one JSON line on rank 0).
+
+Default workload: the long-context streams, batch 1, n = 2^20 tokens, c = 512, bf16
+C^a, C^b, Z^a, Z^b ~ N(0, 1) with per-row logit offsets U(-4, 4); one step runs the CSA
+compressor (m = 4, overlap) and the HCA compressor (m' = 128, C := C^a, Z := Z^a) over
+the same streams, i.e. both softmax-pool kernels of the hot path.  Inputs (4.3 GB) are
+far larger than L2 (126 MB), so no flush is needed between steps.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch under torchrun: every rank runs the same per-GPU workload on its own
+seeded inputs (weak scaling, no data-path collective); times are max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference implementation this
+project has) on a bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "input tokens/s and compressed entries/s at c=512; HBM GB/s % of peak"
+N_TOK = 1 << 20
+C = 512
+M_CSA = 4
+M_HCA = 128
+Z_OFF = 4.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(batch=1, n=N_TOK, c=C):
+    """Compulsory bytes per launch: every stream element the window definition reads,
+    the biases, and the output (bf16 in, bf16 out)."""
+    ne = n // M_CSA
+    csa = (2 * batch * ne * M_CSA * c * 2            # Z^a, C^a: a-ranges of all entries
+           + 2 * batch * max(ne - 1, 0) * M_CSA * c * 2  # Z^b, C^b: b-ranges of entries 1..
+           + 2 * M_CSA * c * 4                          # B^a, B^b
+           + batch * ne * c * 2)                        # output
+    nh = n // M_HCA
+    hca = (2 * batch * nh * M_HCA * c * 2 + M_HCA * c * 4 + batch * nh * c * 2)
+    return csa, hca
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        self.gpu = gpu_id  # nvidia-smi -i accepts the UUID (it ignores CUDA_VISIBLE_DEVICES)
+        self.t0 = self.t1 = None
+
+    def mark(self, start: bool):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.6)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        import datetime
+
+        rows = []
+        for r in out.strip().splitlines():
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if self.t0 is not None and not (self.t0 <= ts <= self.t1 + 0.05):
+                continue  # keep only samples taken inside the timed region
+            rows.append(f)
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[6 + k].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ oracle
+
+def oracle_inputs(tokens: int, seed=0):
+    """Host copy of the first `tokens` tokens of the workload (seeded, bf16 values)."""
+    from kv_token_compressor_b200 import synth
+
+    d = synth.stream_inputs("csa", 1, tokens, C, M_CSA, "bf16", seed=seed, z_row_offset=Z_OFF)
+    rng = np.random.default_rng(seed + 1)
+    d["Bh"] = (rng.standard_normal((M_HCA, C), dtype=np.float32) * np.float32(np.sqrt(0.1)))
+    return d
+
+
+def oracle_time(d):
+    """Seconds the fp64 oracle (as it stands) takes for CSA m=4 overlap then HCA m'=128
+    on the same streams."""
+    from oracle import compressor as O
+
+    t0 = time.perf_counter()
+    O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], M_CSA, True)
+    O.hca_compress(d["Ca"], d["Za"], d["Bh"], M_HCA)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(budget_s=12.0):
+    probe = 4096
+    rate = probe / oracle_time(oracle_inputs(probe))
+    tokens = int(max(probe, min(1 << 18, rate * budget_s)) // M_HCA * M_HCA)
+    dt = oracle_time(oracle_inputs(tokens))
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {tokens} of the {N_TOK} tokens (CSA m=4 + HCA m'=128, fp64 numpy, "
+                      f"single-threaded elementwise), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    probe = 2048
+    probe_rate = probe / oracle_time(oracle_inputs(probe))
+    per_step = 120.0 / max(steps + warm, 1)  # seconds: the whole run within a few minutes
+    tokens = int(max(M_HCA, min(1 << 16, probe_rate * per_step)) // M_HCA * M_HCA)
+    d = oracle_inputs(tokens)
+    for _ in range(warm):
+        oracle_time(d)
+    times = [oracle_time(d) for _ in range(steps)]
+    t = sum(times)
+    value = steps * tokens / t
+    ne = tokens // M_CSA + tokens // M_HCA
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "entries_per_s": steps * ne / t, "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+        "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "long-context streams n=2^20 c=512 bf16: CSA m=4 overlap + HCA m'=128",
+                   "sample_tokens_per_step": tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {tokens} tokens per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ ours
+
+def run_ours(args):
+    import torch
+
+    from kv_token_compressor_b200 import kvc, synth
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    t = synth.stream_inputs_torch("csa", 1, N_TOK, C, M_CSA, "bf16", seed=rank,
+                                  z_row_offset=Z_OFF, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    Bh = torch.randn((M_HCA, C), generator=g, device=dev) * float(np.sqrt(0.1))
+    out_c = torch.empty((1, N_TOK // M_CSA, C), device=dev, dtype=torch.bfloat16)
+    out_h = torch.empty((1, N_TOK // M_HCA, C), device=dev, dtype=torch.bfloat16)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=M_CSA,
+                         out=out_c, out_dtype=torch.bfloat16, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kvc.hca_compress(t["Ca"], t["Za"], Bh, m=M_HCA, out=out_h, out_dtype=torch.bfloat16,
+                         stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if kvc.device_status(stream) != kvc.KVC_OK:
+        raise SystemExit("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", ""))
+    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0"))
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.mark(True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark(False)
+    barrier(world)
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    csa_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    hca_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    csa_ms = max_over_ranks(csa_ms, world)
+    hca_ms = max_over_ranks(hca_ms, world)
+
+    # e2e through the public API with host buffers: H2D of the step's inputs from pinned
+    # memory, both compressors, D2H of both outputs, all inside the timed region.
+    host = {k: t[k].cpu().pin_memory() for k in ("Ca", "Cb", "Za", "Zb", "Ba", "Bb")}
+    host["Bh"] = Bh.cpu().pin_memory()
+    h_out_c = torch.empty(out_c.shape, dtype=out_c.dtype).pin_memory()
+    h_out_h = torch.empty(out_h.shape, dtype=out_h.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = h_out_c.numel() * 2 + h_out_h.numel() * 2
+
+    def e2e_step():
+        dv = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        kvc.csa_compress(dv["Ca"], dv["Cb"], dv["Za"], dv["Zb"], dv["Ba"], dv["Bb"], m=M_CSA,
+                         out=out_c, out_dtype=torch.bfloat16, stream=stream)
+        kvc.hca_compress(dv["Ca"], dv["Za"], dv["Bh"], m=M_HCA, out=out_h,
+                         out_dtype=torch.bfloat16, stream=stream)
+        h_out_c.copy_(out_c, non_blocking=True)
+        h_out_h.copy_(out_h, non_blocking=True)
+        del dv
+
+    del t
+    torch.cuda.empty_cache()
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+
+    peak, peak_kind = peaks()
+    csa_bytes, hca_bytes = algorithmic_bytes()
+    csa_gbs = csa_bytes / (csa_ms * 1e-3) / 1e9
+    hca_gbs = hca_bytes / (hca_ms * 1e-3) / 1e9
+    ms_step = elapsed_ms / args.steps
+    tokens_per_s = world * N_TOK / (ms_step * 1e-3)
+    entries = N_TOK // M_CSA + N_TOK // M_HCA
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            traffic = json.load(f).get("csa_compress_bf16_n1048576")
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s",
+            "entries_per_s": world * entries / (ms_step * 1e-3),
+            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "long-context streams: batch 1, n=2^20, c=512, bf16 in/out; "
+                                   "CSA m=4 overlap + HCA m'=128 on the same streams",
+                       "batch": 1, "n": N_TOK, "c": C, "m": M_CSA, "m_hca": M_HCA,
+                       "l2": "inputs 4.3 GB > 126 MB L2, no flush",
+                       "parallelism": f"weak: {world} independent replicas"},
+            "roofline": {"bound": "hbm", "kernel": "csa_compress (csa_small_m_kernel<bf16,bf16,4>)",
+                         "achieved": csa_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": csa_gbs / peak, "peak_kind": peak_kind, "traffic": traffic,
+                         "algorithmic_bytes": csa_bytes},
+            "kernels": {
+                "csa_compress": {"ms": csa_ms, "GB/s": csa_gbs, "frac": csa_gbs / peak,
+                                 "tokens_per_s": N_TOK / (csa_ms * 1e-3),
+                                 "entries_per_s": (N_TOK // M_CSA) / (csa_ms * 1e-3)},
+                "hca_compress": {"ms": hca_ms, "GB/s": hca_gbs, "frac": hca_gbs / peak,
+                                 "tokens_per_s": N_TOK / (hca_ms * 1e-3),
+                                 "entries_per_s": (N_TOK // M_HCA) / (hca_ms * 1e-3)},
+            },
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+            "e2e": {"value": world * N_TOK / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,143 @@
+/*
+ * kvc.h — C ABI of the B200 (sm_100a) token-level KV compressor.
+ *
+ * The compressor turns every m consecutive tokens of a sequence into one compressed
+ * KV entry by a per-channel softmax-weighted pool.  Sources (web pages):
+ *   [SC]  "序列压缩注意力" (sequence-compressed attention):
+ *         eq. attn-seqcomp-csa-proj     C^a = H W^{KV_a}, C^b = H W^{KV_b}, Z^a = H W^{Z_a}, Z^b = H W^{Z_b}
+ *         eq. attn-seqcomp-csa-softmax  [S^a; S^b] = Softmax_row([Z^a_{mi..m(i+1)-1} + B^a; Z^b_{m(i-1)..mi-1} + B^b])
+ *         eq. attn-seqcomp-csa-pool     C^Comp_i = sum_j S^a_j (.) C^a_j + sum_j S^b_j (.) C^b_j
+ *         table attn-seqcomp-overlap    a-range(i) = [mi, m(i+1)-1], b-range(i) = [m(i-1), mi-1]
+ *         eq. attn-seqcomp-overlap-bound  Z^b_{-m:-1} = -inf, C^b_{-m:-1} = 0 (entry 0)
+ *         eq. attn-seqcomp-hca          S = Softmax_row(Z + B), C^Comp_i = sum_{j in segment i} S_j (.) C_j, m' = 128
+ *   [CSA] "Ch 04 · CSA" (DeepSeek-V4 book), §3 Token-Level Compressor (same equations, 12-token example).
+ *   [HCA] "Ch 05 · HCA" (DeepSeek-V4 book), §2 compression formulas.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  All tensors are dense, row-major, channel fastest:
+ *   streams  [batch, n, c]   (sequence b, token t, channel ch at ((b*n)+t)*c+ch)
+ *   biases   [m, c] fp32     (row k = in-block position k)
+ *   H        [batch*n, d]    bf16 (sequence b = rows b*n .. b*n+n-1)
+ *   W        [d, c]          bf16 (as in C = H W)
+ *   out      [batch, N_e, c] with N_e = floor(n/m) = kvc_num_entries(n, m).
+ * Entries.  Sequence b's entry i reads only tokens of sequence b.  The trailing n mod m
+ *   tokens of a sequence form no complete block and are not compressed.
+ * Ownership.  Every tensor pointer is a DEVICE pointer on the current CUDA device,
+ *   owned by the caller.  The library never allocates, frees or retains them.
+ * Asynchrony.  Work is enqueued on `stream` (NULL = the legacy default stream) and the
+ *   call returns after the enqueue; no implicit synchronisation, no host<->device copy.
+ * Arithmetic.  Inputs are widened to fp32; logits, softmax and the weighted sum are
+ *   fp32 (the fused path accumulates H W in fp32 on the tensor cores and never rounds
+ *   the streams); bf16 outputs are rounded to nearest even.
+ * Errors.  Arguments are validated on the host before any launch; on error nothing is
+ *   enqueued and the status says why:
+ *     KVC_ERR_NULL         a required pointer is NULL
+ *     KVC_ERR_SHAPE        negative size, c not a multiple of 8, m < 1, overlap not 0/1,
+ *                          size overflow, fused d % 64 != 0 or c % 128 != 0
+ *     KVC_ERR_DTYPE        unknown dtype or unsupported dtype combination
+ *     KVC_ERR_ALIGN        a stream, H, W or out pointer is not 16-byte aligned, or a
+ *                          bias pointer is not 4-byte aligned
+ *     KVC_ERR_UNSUPPORTED  valid but outside what the kernels implement (e.g. window too long)
+ *     KVC_ERR_CUDA         the launch (or a CUDA query it needs) failed
+ *     KVC_ERR_TIMEOUT      reported by kvc_device_status(): a bounded wait inside a
+ *                          kernel gave up (the kernel then skipped its remaining work)
+ *     KVC_ERR_POINTER      a tensor pointer is not device (or managed) memory of the
+ *                          current device (e.g. a host pointer)
+ *   An empty problem (batch == 0 or N_e == 0) is valid: KVC_OK, nothing is launched and
+ *   no pointer is dereferenced.
+ * Thread safety.  Calls may be made concurrently from several host threads.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVC_API __attribute__((visibility("default")))
+#else
+#define KVC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvc_status {
+  KVC_OK = 0,
+  KVC_ERR_NULL = 1,
+  KVC_ERR_SHAPE = 2,
+  KVC_ERR_DTYPE = 3,
+  KVC_ERR_ALIGN = 4,
+  KVC_ERR_UNSUPPORTED = 5,
+  KVC_ERR_CUDA = 6,
+  KVC_ERR_TIMEOUT = 7,
+  KVC_ERR_POINTER = 8
+} kvc_status;
+
+typedef enum kvc_dtype { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* kvc_stream;
+
+/* Number of compressed entries of an n-token sequence at ratio m: floor(n / m)
+ * ([CSA] §3 cuts the sequence into floor(n/m) segments; [SC] table
+ * attn-seqcomp-csa-hca: ~n/m entries).  Returns -1 if n < 0 or m < 1. */
+KVC_API int64_t kvc_num_entries(int64_t n, int32_t m);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KVC_API const char* kvc_status_string(kvc_status s);
+
+/* CSA compressor over precomputed streams ([SC] eqs. attn-seqcomp-csa-softmax,
+ * attn-seqcomp-csa-pool, attn-seqcomp-overlap-bound; [CSA] §3).
+ *   Ca, Cb, Za, Zb : streams [batch, n, c], dtype in_dtype (KVC_F32 or KVC_BF16)
+ *   Ba, Bb         : position biases [m, c] fp32
+ *   overlap = 1    : entry i pools the 2m rows a-range(i) of (Ca, Za + Ba) and
+ *                    b-range(i) of (Cb, Zb + Bb) under one joint per-channel softmax;
+ *                    entry 0 has no b-rows (logit -inf, vector 0).
+ *   overlap = 0    : entry i pools its own m rows of (Ca, Za + Ba) only; Cb, Zb and Bb
+ *                    are not read and may be NULL.
+ *   out            : [batch, N_e, c], dtype out_dtype (KVC_F32 or KVC_BF16). */
+KVC_API kvc_status csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                        kvc_dtype in_dtype, const float* Ba, const float* Bb,
+                        int64_t batch, int64_t n, int64_t c, int32_t m, int32_t overlap,
+                        void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* HCA compressor ([SC] eq. attn-seqcomp-hca; [HCA] §2): entry i pools the m rows
+ * [m i, m(i+1)-1] of C under Softmax_row(Z + B), no overlap, single stream.
+ *   C, Z : [batch, n, c] in_dtype;  B : [m, c] fp32;  out : [batch, N_e, c] out_dtype.
+ *   m is the compression ratio m' (128 on the pages); windows of up to 320 rows are
+ *   supported (KVC_ERR_UNSUPPORTED beyond). */
+KVC_API kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
+                        int64_t batch, int64_t n, int64_t c, int32_t m,
+                        void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* CSA compressor fed by hidden states ([SC] eq. attn-seqcomp-csa-proj followed by the
+ * csa_compress pool): the four streams H W are formed on the tensor cores (bf16 in,
+ * fp32 accumulate) and pooled on chip; they never reach device memory.
+ *   H : [batch*n, d] bf16;  W_kva, W_kvb, W_za, W_zb : [d, c] bf16;  Ba, Bb : [m, c] fp32
+ *   d % 64 == 0, c % 128 == 0;  out : [batch, N_e, c] out_dtype. */
+KVC_API kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, const void* W_kvb,
+                                   const void* W_za, const void* W_zb,
+                                   const float* Ba, const float* Bb,
+                                   int64_t batch, int64_t n, int64_t d, int64_t c,
+                                   int32_t m, int32_t overlap,
+                                   void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* HCA compressor fed by hidden states: C = H W_kv, Z = H W_z on the tensor cores, then
+ * the hca_compress pool in the GEMM epilogue.  Shapes and rules as above. */
+KVC_API kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* W_z,
+                                   const float* B, int64_t batch, int64_t n, int64_t d,
+                                   int64_t c, int32_t m,
+                                   void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* Synchronises `stream`, then reports and clears the device-side error word that
+ * kernels set when a bounded wait gives up: KVC_ERR_TIMEOUT if one did, KVC_ERR_CUDA
+ * if the synchronisation failed, else KVC_OK. */
+KVC_API kvc_status kvc_device_status(kvc_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H */

@@ -1,0 +1,250 @@
+// C ABI of the compressor: host-side validation, then one kernel launch per call.
+// Every check here runs before anything is enqueued; see include/kvc.h for the contract.
+#include <cuda_runtime.h>
+
+#include "../../include/kvc.h"
+#include "kvc_launch.h"
+
+namespace {
+
+using kvc::FusedProblem;
+using kvc::StreamProblem;
+
+constexpr int kMaxWindowRows = 320;  // longest window whose biases fit one CTA's shared memory
+
+bool dtype_ok(kvc_dtype t) { return t == KVC_F32 || t == KVC_BF16; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t* r) { return !__builtin_mul_overflow(a, b, r); }
+
+// Device (or managed) memory of the current device.
+kvc_status check_device_ptr(const void* p) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the error this query leaves for unknown pointers
+    return KVC_ERR_POINTER;
+  }
+  if (at.type == cudaMemoryTypeManaged) return KVC_OK;
+  if (at.type != cudaMemoryTypeDevice || at.device != dev) return KVC_ERR_POINTER;
+  return KVC_OK;
+}
+
+kvc_status check_ptrs(const void* const* ps, int n) {
+  for (int i = 0; i < n; ++i) {
+    kvc_status s = check_device_ptr(ps[i]);
+    if (s != KVC_OK) return s;
+  }
+  return KVC_OK;
+}
+
+// Common shape checks of the streaming calls.  Sets *empty when nothing is to be done.
+kvc_status check_stream_shape(int64_t batch, int64_t n, int64_t c, int32_t m, bool* empty,
+                              int64_t* ne) {
+  *empty = false;
+  if (batch < 0 || n < 0 || c < 0 || m < 1) return KVC_ERR_SHAPE;
+  *ne = n / m;
+  int64_t t = 0;
+  if (!mul_ok(batch, n, &t) || !mul_ok(t, c, &t) || !mul_ok(t, 4, &t)) return KVC_ERR_SHAPE;
+  if (batch == 0 || *ne == 0 || c == 0) {
+    *empty = true;
+    return KVC_OK;
+  }
+  if (c % 8 != 0) return KVC_ERR_SHAPE;
+  return KVC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t kvc_num_entries(int64_t n, int32_t m) {
+  if (n < 0 || m < 1) return -1;
+  return n / m;
+}
+
+const char* kvc_status_string(kvc_status s) {
+  switch (s) {
+    case KVC_OK: return "KVC_OK";
+    case KVC_ERR_NULL: return "KVC_ERR_NULL: a required pointer is NULL";
+    case KVC_ERR_SHAPE: return "KVC_ERR_SHAPE: invalid size or shape";
+    case KVC_ERR_DTYPE: return "KVC_ERR_DTYPE: unknown or unsupported dtype";
+    case KVC_ERR_ALIGN: return "KVC_ERR_ALIGN: misaligned pointer";
+    case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED: valid but not implemented";
+    case KVC_ERR_CUDA: return "KVC_ERR_CUDA: CUDA launch or query failed";
+    case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT: a bounded wait in a kernel gave up";
+    case KVC_ERR_POINTER: return "KVC_ERR_POINTER: not device memory of the current device";
+  }
+  return "KVC_ERR_UNKNOWN";
+}
+
+kvc_status csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                        kvc_dtype in_dtype, const float* Ba, const float* Bb, int64_t batch,
+                        int64_t n, int64_t c, int32_t m, int32_t overlap, void* out,
+                        kvc_dtype out_dtype, kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (!Ca || !Za || !Ba || !out) return KVC_ERR_NULL;
+  if (overlap && (!Cb || !Zb || !Bb)) return KVC_ERR_NULL;
+  if (!aligned(Ca, 16) || !aligned(Za, 16) || !aligned(out, 16) || !aligned(Ba, 4))
+    return KVC_ERR_ALIGN;
+  if (overlap && (!aligned(Cb, 16) || !aligned(Zb, 16) || !aligned(Bb, 4))) return KVC_ERR_ALIGN;
+  const bool small = (m == 1 || m == 2 || m == 4);
+  const int rows = overlap ? 2 * m : m;
+  if (!small && rows > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  {
+    const void* ps[7] = {Ca, Za, Ba, out, Cb, Zb, Bb};
+    s = check_ptrs(ps, overlap ? 7 : 4);
+    if (s != KVC_OK) return s;
+  }
+  StreamProblem p{};
+  p.C0 = Ca;
+  p.Z0 = Za;
+  p.B0 = Ba;
+  p.C1 = overlap ? Cb : nullptr;
+  p.Z1 = overlap ? Zb : nullptr;
+  p.B1 = overlap ? Bb : nullptr;
+  p.batch = batch;
+  p.n = n;
+  p.c = c;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = overlap != 0;
+  p.small_window_kernel = true;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
+                        int64_t batch, int64_t n, int64_t c, int32_t m, void* out,
+                        kvc_dtype out_dtype, kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (!C || !Z || !B || !out) return KVC_ERR_NULL;
+  if (!aligned(C, 16) || !aligned(Z, 16) || !aligned(out, 16) || !aligned(B, 4))
+    return KVC_ERR_ALIGN;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  {
+    const void* ps[4] = {C, Z, B, out};
+    s = check_ptrs(ps, 4);
+    if (s != KVC_OK) return s;
+  }
+  StreamProblem p{};
+  p.C0 = C;
+  p.Z0 = Z;
+  p.B0 = B;
+  p.batch = batch;
+  p.n = n;
+  p.c = c;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = false;
+  p.small_window_kernel = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static kvc_status fused_common(FusedProblem* p, const void* H, const void* const* W, int nw,
+                               const float* B0, const float* B1, bool need_b1, int64_t batch,
+                               int64_t n, int64_t d, int64_t c, int32_t m, void* out,
+                               kvc_dtype out_dtype, bool* empty) {
+  *empty = false;
+  if (!dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  if (batch < 0 || n < 0 || d < 0 || c < 0 || m < 1) return KVC_ERR_SHAPE;
+  int64_t t = 0;
+  if (!mul_ok(batch, n, &t) || !mul_ok(t, d > c ? d : c, &t) || !mul_ok(t, 4, &t))
+    return KVC_ERR_SHAPE;
+  const int64_t ne = n / m;
+  if (batch == 0 || ne == 0 || c == 0) {
+    *empty = true;
+    return KVC_OK;
+  }
+  if (d == 0 || d % 64 != 0 || c % 128 != 0) return KVC_ERR_SHAPE;
+  if (!H || !out || !B0 || (need_b1 && !B1)) return KVC_ERR_NULL;
+  for (int i = 0; i < nw; ++i)
+    if (!W[i]) return KVC_ERR_NULL;
+  if (!aligned(H, 16) || !aligned(out, 16) || !aligned(B0, 4)) return KVC_ERR_ALIGN;
+  for (int i = 0; i < nw; ++i)
+    if (!aligned(W[i], 16)) return KVC_ERR_ALIGN;
+  if (need_b1 && !aligned(B1, 4)) return KVC_ERR_ALIGN;
+  const void* ps[3] = {H, out, B0};
+  kvc_status s = check_ptrs(ps, 3);
+  if (s == KVC_OK) s = check_ptrs(W, nw);
+  if (s == KVC_OK && need_b1) s = check_device_ptr(B1);
+  if (s != KVC_OK) return s;
+  p->H = H;
+  p->B0 = B0;
+  p->B1 = need_b1 ? B1 : nullptr;
+  p->batch = batch;
+  p->n = n;
+  p->d = d;
+  p->c = c;
+  p->ne = ne;
+  p->m = m;
+  p->out_bf16 = out_dtype == KVC_BF16;
+  p->out = out;
+  return KVC_OK;
+}
+
+kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, const void* W_kvb,
+                                   const void* W_za, const void* W_zb, const float* Ba,
+                                   const float* Bb, int64_t batch, int64_t n, int64_t d,
+                                   int64_t c, int32_t m, int32_t overlap, void* out,
+                                   kvc_dtype out_dtype, kvc_stream stream) {
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  FusedProblem p{};
+  bool empty = false;
+  kvc_status s;
+  if (overlap) {
+    const void* W[4] = {W_kva, W_kvb, W_za, W_zb};
+    s = fused_common(&p, H, W, 4, Ba, Bb, true, batch, n, d, c, m, out, out_dtype, &empty);
+    for (int i = 0; i < 4; ++i) p.W[i] = W[i];
+  } else {  // a-streams only
+    const void* W[2] = {W_kva, W_za};
+    s = fused_common(&p, H, W, 2, Ba, nullptr, false, batch, n, d, c, m, out, out_dtype, &empty);
+    p.W[0] = W_kva;
+    p.W[1] = nullptr;
+    p.W[2] = W_za;
+    p.W[3] = nullptr;
+  }
+  if (s != KVC_OK || empty) return s;
+  p.csa = true;
+  p.overlap = overlap != 0;
+  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* W_z,
+                                   const float* B, int64_t batch, int64_t n, int64_t d,
+                                   int64_t c, int32_t m, void* out, kvc_dtype out_dtype,
+                                   kvc_stream stream) {
+  FusedProblem p{};
+  bool empty = false;
+  const void* W[2] = {W_kv, W_z};
+  kvc_status s =
+      fused_common(&p, H, W, 2, B, nullptr, false, batch, n, d, c, m, out, out_dtype, &empty);
+  if (s != KVC_OK || empty) return s;
+  p.W[0] = W_kv;
+  p.W[1] = W_z;
+  p.csa = false;
+  p.overlap = false;
+  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status kvc_device_status(kvc_stream stream) {
+  return kvc::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

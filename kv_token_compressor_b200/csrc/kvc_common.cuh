@@ -1,0 +1,89 @@
+// Shared device helpers of the sm_100a compressor kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/kvc.h"
+
+namespace kvc {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 16-byte streaming load: read once, no L1 allocation, 256-byte L2 prefetch.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// Streaming (evict-first) stores.
+__device__ __forceinline__ void st_stream16(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_stream8(void* p, uint2 v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// Element j of a 16-byte vector holding 8 bf16 or 4 fp32 values, widened to fp32.
+template <typename T>
+__device__ __forceinline__ float vec_elem(const uint4& v, int j);
+
+template <>
+__device__ __forceinline__ float vec_elem<__nv_bfloat16>(const uint4& v, int j) {
+  const uint32_t w = (j >> 1) == 0 ? v.x : (j >> 1) == 1 ? v.y : (j >> 1) == 2 ? v.z : v.w;
+  return __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+template <>
+__device__ __forceinline__ float vec_elem<float>(const uint4& v, int j) {
+  const uint32_t w = j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+  return __uint_as_float(w);
+}
+
+// Channels carried by one 16-byte vector of T.
+template <typename T>
+struct VecInfo {
+  static constexpr int kChannels = 16 / sizeof(T);
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Store CPT consecutive fp32 results as OutT (fp32 or bf16, RNE) with streaming stores.
+template <typename OutT, int CPT>
+__device__ __forceinline__ void store_out(OutT* dst, const float (&v)[CPT]) {
+  if constexpr (sizeof(OutT) == 2) {
+    static_assert(CPT == 8 || CPT == 4, "bf16 output vector");
+    if constexpr (CPT == 8) {
+      st_stream16(dst, make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                  pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
+    } else {
+      st_stream8(dst, make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3])));
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q)
+      st_stream16(dst + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                          __float_as_uint(v[4 * q + 2]),
+                                          __float_as_uint(v[4 * q + 3])));
+  }
+}
+
+// Store one fp32 result as OutT.
+template <typename OutT>
+__device__ __forceinline__ void store_scalar(OutT* dst, float v) {
+  if constexpr (sizeof(OutT) == 2) {
+    *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
+  } else {
+    *dst = v;
+  }
+}
+
+}  // namespace kvc

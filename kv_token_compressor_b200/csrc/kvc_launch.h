@@ -1,0 +1,51 @@
+// Internal launch interface between the C ABI (kvc_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kvc.h"
+
+namespace kvc {
+
+// A validated streaming problem.  Segment 0 = (C0, Z0, B0): the a-range of CSA or the
+// HCA segment; segment 1 = (C1, Z1, B1): the b-range of CSA with overlap.
+struct StreamProblem {
+  const void* C0;
+  const void* Z0;
+  const void* C1;
+  const void* Z1;
+  const float* B0;
+  const float* B1;
+  int64_t batch, n, c, ne;
+  int m;
+  bool two_segments;         // CSA with overlap
+  bool small_window_kernel;  // allow the one-thread-per-entry kernel for m in {1,2,4}
+  bool in_bf16, out_bf16;
+  void* out;
+};
+
+kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st);
+size_t window_kernel_smem_bytes(bool bf16_in, bool two_segments, int m);
+
+// A validated fused problem: H [batch*n, d] bf16, W_s [d, c] bf16 (s = streams).
+struct FusedProblem {
+  const void* H;
+  const void* W[4];  // CSA: kv_a, kv_b, z_a, z_b;  HCA: kv, z
+  const float* B0;
+  const float* B1;
+  int64_t batch, n, d, c, ne;
+  int m;
+  bool csa;      // true: CSA (4 streams), false: HCA (2 streams)
+  bool overlap;  // CSA only
+  bool out_bf16;
+  void* out;
+};
+
+kvc_status launch_fused(const FusedProblem& p, cudaStream_t st);
+
+// Device error word set by kernels whose bounded waits give up.
+kvc_status read_and_clear_device_error(cudaStream_t st);
+
+}  // namespace kvc

@@ -1,0 +1,419 @@
+// Streaming softmax-pool kernels over precomputed C/Z streams (sm_100a).
+//
+// What they compute ("序列压缩注意力", eqs. attn-seqcomp-csa-softmax, attn-seqcomp-csa-pool,
+// attn-seqcomp-overlap-bound, attn-seqcomp-hca; "Ch 04 · CSA" §3; "Ch 05 · HCA" §2):
+// for every entry i and channel ch, a softmax over the window's logit rows
+// (Z + B per channel) and the weighted sum of the matching C rows.
+//
+// Memory behaviour.  The work is HBM-bound: every stream byte is needed exactly once
+// (CSA: the a-block of entry i is read only by entry i, the b-block of entry i-1 only
+// by entry i; HCA: segments are disjoint).  Both kernels therefore stream the inputs
+// with 16-byte read-once loads straight into registers, issue all loads of a window
+// before using any, and keep the biases (pre-scaled by log2 e) in shared memory.
+// Softmax is exact two-pass per window in registers for the small CSA windows
+// (one exp2 per element), and chunked online (max, sum, acc) with a shared-memory
+// merge across row groups for long windows (HCA m' = 128).
+#include "kvc_common.cuh"
+#include "kvc_launch.h"
+
+#include <math.h>
+
+#include <mutex>
+
+namespace kvc {
+
+// ---------------------------------------------------------------------------------
+// CSA, small m (1, 2, 4): one thread = one entry x one 16-byte channel vector.
+// ---------------------------------------------------------------------------------
+struct CsaSmallArgs {
+  const void* Ca;
+  const void* Cb;
+  const void* Za;
+  const void* Zb;
+  const float* Ba;
+  const float* Bb;
+  int64_t batch, n, c, ne;
+  void* out;
+};
+
+template <typename InT, typename OutT, int M, bool OVERLAP>
+__global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int NB = OVERLAP ? 2 * M : M;  // bias rows: B^a rows then B^b rows
+  extern __shared__ float4 smem_f4[];
+  float* sb = reinterpret_cast<float*>(smem_f4);  // [NB][SC], pre-scaled by log2 e
+
+  const int SC = blockDim.x * CPT;
+  const int64_t ch_base = static_cast<int64_t>(blockIdx.x) * SC;
+  const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+  const int nthr = blockDim.x * blockDim.y;
+  for (int idx = tid; idx < NB * SC; idx += nthr) {
+    const int k = idx / SC;
+    const int64_t ch = ch_base + (idx - k * SC);
+    float v = 0.f;
+    if (ch < a.c) v = (k < M ? a.Ba[k * a.c + ch] : a.Bb[(k - M) * a.c + ch]) * kLog2e;
+    sb[idx] = v;
+  }
+  __syncthreads();
+
+  const int sc0 = threadIdx.x * CPT;
+  const int64_t ch0 = ch_base + sc0;
+  if (ch0 >= a.c) return;
+
+  const InT* Ca = static_cast<const InT*>(a.Ca);
+  const InT* Za = static_cast<const InT*>(a.Za);
+  const InT* Cb = static_cast<const InT*>(a.Cb);
+  const InT* Zb = static_cast<const InT*>(a.Zb);
+  OutT* out = static_cast<OutT*>(a.out);
+  // Boundary rows of entry 0 (eq. attn-seqcomp-overlap-bound): logit -inf, vector 0.
+  const uint32_t neg_inf_bits = sizeof(InT) == 2 ? 0xFF80FF80u : 0xFF800000u;
+  const uint4 z_boundary = make_uint4(neg_inf_bits, neg_inf_bits, neg_inf_bits, neg_inf_bits);
+  const uint4 c_boundary = make_uint4(0u, 0u, 0u, 0u);
+
+  const int64_t istep = static_cast<int64_t>(gridDim.y) * blockDim.y;
+  for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; i < a.ne;
+         i += istep) {
+      const int64_t rowA = b * a.n + static_cast<int64_t>(M) * i;  // a-range(i) start
+      uint4 za[M], ca[M], zb[M], cb[M];
+#pragma unroll
+      for (int k = 0; k < M; ++k) {
+        za[k] = ld_stream16(Za + (rowA + k) * a.c + ch0);
+        ca[k] = ld_stream16(Ca + (rowA + k) * a.c + ch0);
+      }
+      if constexpr (OVERLAP) {
+        if (i > 0) {  // b-range(i) = a-range(i-1)
+#pragma unroll
+          for (int k = 0; k < M; ++k) {
+            zb[k] = ld_stream16(Zb + (rowA - M + k) * a.c + ch0);
+            cb[k] = ld_stream16(Cb + (rowA - M + k) * a.c + ch0);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < M; ++k) {
+            zb[k] = z_boundary;
+            cb[k] = c_boundary;
+          }
+        }
+      }
+      float res[CPT];
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        float la[M], lb[M];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+          la[k] = fmaf(vec_elem<InT>(za[k], j), kLog2e, sb[k * SC + sc0 + j]);
+          mx = fmaxf(mx, la[k]);
+        }
+        if constexpr (OVERLAP) {
+#pragma unroll
+          for (int k = 0; k < M; ++k) {
+            lb[k] = fmaf(vec_elem<InT>(zb[k], j), kLog2e, sb[(M + k) * SC + sc0 + j]);
+            mx = fmaxf(mx, lb[k]);
+          }
+        }
+        float s = 0.f, acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+          const float w = exp2f(la[k] - mx);
+          s += w;
+          acc = fmaf(w, vec_elem<InT>(ca[k], j), acc);
+        }
+        if constexpr (OVERLAP) {
+#pragma unroll
+          for (int k = 0; k < M; ++k) {
+            const float w = exp2f(lb[k] - mx);
+            s += w;
+            acc = fmaf(w, vec_elem<InT>(cb[k], j), acc);
+          }
+        }
+        res[j] = __fdividef(acc, s);
+      }
+      store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Any window length: HCA (one segment of m rows), CSA with overlap for other m (the
+// a-segment then the b-segment), CSA without overlap.  One CTA = one entry x a slab
+// of SC channels at a time; its 16 row groups split the window's rows, each keeps an
+// online (max, sum, acc) per channel, and the partials merge through shared memory.
+// ---------------------------------------------------------------------------------
+struct WinArgs {
+  const void* C0;  // segment 0 streams (a-range / the HCA segment)
+  const void* Z0;
+  const void* C1;  // segment 1 streams (b-range), TWO_SEG only
+  const void* Z1;
+  const float* B0;  // [m, c]
+  const float* B1;  // [m, c], TWO_SEG only
+  int64_t batch, n, c, ne;
+  int m;
+  void* out;
+};
+
+constexpr int kWinCG = 16;  // channel vectors per CTA
+constexpr int kWinRG = 16;  // row groups per CTA
+constexpr int kWinU = 8;    // rows per thread per chunk (all loads in flight)
+
+template <typename InT>
+constexpr int win_slab() {
+  return kWinCG * VecInfo<InT>::kChannels;
+}
+
+template <typename InT, bool TWO_SEG>
+size_t win_smem_bytes(int m) {
+  const int rows = TWO_SEG ? 2 * m : m;
+  return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + 3 * kWinRG * win_slab<InT>());
+}
+
+template <typename InT, typename OutT, bool TWO_SEG>
+__global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int SC = win_slab<InT>();
+  constexpr int CG = kWinCG, RG = kWinRG, U = kWinU;
+  extern __shared__ float4 smem_f4[];
+  const int nb = TWO_SEG ? 2 * a.m : a.m;
+  float* sb = reinterpret_cast<float*>(smem_f4);  // [nb][SC] biases * log2 e
+  float* pm = sb + static_cast<size_t>(nb) * SC;  // [RG][SC] partial max
+  float* ps = pm + RG * SC;                        // [RG][SC] partial sum
+  float* pa = ps + RG * SC;                        // [RG][SC] partial weighted sum
+
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int tid = ty * CG + tx;
+  const int64_t ch_base = static_cast<int64_t>(blockIdx.x) * SC;
+  for (int idx = tid; idx < nb * SC; idx += CG * RG) {
+    const int k = idx / SC;
+    const int64_t ch = ch_base + (idx - k * SC);
+    float v = 0.f;
+    if (ch < a.c) v = (k < a.m ? a.B0[k * a.c + ch] : a.B1[(k - a.m) * a.c + ch]) * kLog2e;
+    sb[idx] = v;
+  }
+  __syncthreads();
+
+  const int sc0 = tx * CPT;
+  const int64_t ch0 = ch_base + sc0;
+  const bool active = ch0 < a.c;
+  const InT* C0 = static_cast<const InT*>(a.C0);
+  const InT* Z0 = static_cast<const InT*>(a.Z0);
+  const InT* C1 = static_cast<const InT*>(a.C1);
+  const InT* Z1 = static_cast<const InT*>(a.Z1);
+  OutT* out = static_cast<OutT*>(a.out);
+  const int m = a.m;
+
+  for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
+    for (int64_t i = blockIdx.y; i < a.ne; i += gridDim.y) {
+      const int64_t row0 = b * a.n + static_cast<int64_t>(m) * i;
+      const int rows_i = (TWO_SEG && i > 0) ? 2 * m : m;
+      float M[CPT], S[CPT], A[CPT];
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        M[j] = -INFINITY;
+        S[j] = 0.f;
+        A[j] = 0.f;
+      }
+      if (active) {
+        for (int v0 = ty; v0 < rows_i; v0 += RG * U) {
+          uint4 z[U], cv[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * RG;
+            if (v < rows_i) {
+              const bool seg1 = TWO_SEG && v >= m;
+              const int64_t row = seg1 ? row0 - m + (v - m) : row0 + v;
+              z[u] = ld_stream16((seg1 ? Z1 : Z0) + row * a.c + ch0);
+              cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) {
+            float l[U];
+            float cm = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int v = v0 + u * RG;
+              l[u] = v < rows_i ? fmaf(vec_elem<InT>(z[u], j), kLog2e, sb[v * SC + sc0 + j])
+                                : -INFINITY;
+              cm = fmaxf(cm, l[u]);
+            }
+            const float nm = fmaxf(M[j], cm);  // finite: row v0 < rows_i is valid
+            const float scale = exp2f(M[j] - nm);
+            float s = S[j] * scale, acc = A[j] * scale;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int v = v0 + u * RG;
+              if (v < rows_i) {
+                const float w = exp2f(l[u] - nm);
+                s += w;
+                acc = fmaf(w, vec_elem<InT>(cv[u], j), acc);
+              }
+            }
+            M[j] = nm;
+            S[j] = s;
+            A[j] = acc;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        pm[ty * SC + sc0 + j] = M[j];
+        ps[ty * SC + sc0 + j] = S[j];
+        pa[ty * SC + sc0 + j] = A[j];
+      }
+      __syncthreads();
+      if (tid < SC && ch_base + tid < a.c) {
+        float gm = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) gm = fmaxf(gm, pm[r * SC + tid]);
+        float s = 0.f, acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < RG; ++r) {
+          const float f = exp2f(pm[r * SC + tid] - gm);  // 0 for empty row groups
+          s = fmaf(ps[r * SC + tid], f, s);
+          acc = fmaf(pa[r * SC + tid], f, acc);
+        }
+        store_scalar<OutT>(out + (b * a.ne + i) * a.c + ch_base + tid, __fdividef(acc, s));
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------------
+namespace {
+
+struct DeviceInfo {
+  int sms = 0;
+  size_t smem_optin = 0;
+};
+
+DeviceInfo device_info(int dev) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return DeviceInfo{};
+  if (cache[dev].sms == 0) {
+    int sms = 0, optin = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return DeviceInfo{};
+    cache[dev].sms = sms;
+    cache[dev].smem_optin = static_cast<size_t>(optin);
+  }
+  return cache[dev];
+}
+
+template <typename Kernel>
+int resident_blocks(Kernel k, int threads, size_t smem) {
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return 0;
+  }
+  int blocks = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, threads, smem) != cudaSuccess)
+    return 0;
+  return blocks;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+template <typename InT, typename OutT, int M, bool OVERLAP>
+kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  const int64_t G = p.c / CPT;  // channel vectors
+  const int cg = static_cast<int>(G < 64 ? G : 64);
+  const int ey = 256 / cg;
+  const dim3 block(cg, ey);
+  const size_t smem = sizeof(float) * (OVERLAP ? 2 * M : M) * cg * CPT;
+  auto kern = csa_small_m_kernel<InT, OutT, M, OVERLAP>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  const int occ = resident_blocks(kern, cg * ey, smem);
+  if (di.sms == 0 || occ == 0) return KVC_ERR_CUDA;
+  const int64_t gx = ceil_div(G, cg);
+  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
+  int64_t want = static_cast<int64_t>(di.sms) * occ;  // one resident wave
+  int64_t gy = want / (gx * gz);
+  if (gy < 1) gy = 1;
+  const int64_t need = ceil_div(p.ne, ey);
+  if (gy > need) gy = need;
+  if (gy > 65535) gy = 65535;
+  // Balance: every CTA row gets the same number of entry iterations (+-1).
+  gy = ceil_div(need, ceil_div(need, gy));
+  CsaSmallArgs args{p.C0, p.C1, p.Z0, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.out};
+  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
+         block, smem, st>>>(args);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+template <typename InT, typename OutT, bool TWO_SEG>
+kvc_status launch_window(const StreamProblem& p, cudaStream_t st) {
+  constexpr int SC = win_slab<InT>();
+  const size_t smem = win_smem_bytes<InT, TWO_SEG>(p.m);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (di.sms == 0) return KVC_ERR_CUDA;
+  if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
+  auto kern = window_pool_kernel<InT, OutT, TWO_SEG>;
+  const int occ = resident_blocks(kern, kWinCG * kWinRG, smem);
+  if (occ == 0) return KVC_ERR_CUDA;
+  const int64_t gx = ceil_div(p.c, SC);
+  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
+  int64_t gy = static_cast<int64_t>(di.sms) * occ / (gx * gz);
+  if (gy < 1) gy = 1;
+  if (gy > p.ne) gy = p.ne;
+  if (gy > 65535) gy = 65535;
+  gy = ceil_div(p.ne, ceil_div(p.ne, gy));
+  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
+  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
+         dim3(kWinCG, kWinRG), smem, st>>>(args);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+template <typename InT, typename OutT>
+kvc_status dispatch_stream(const StreamProblem& p, cudaStream_t st) {
+  if (p.two_segments) {
+    switch (p.m) {
+      case 1: return launch_csa_small<InT, OutT, 1, true>(p, st);
+      case 2: return launch_csa_small<InT, OutT, 2, true>(p, st);
+      case 4: return launch_csa_small<InT, OutT, 4, true>(p, st);
+      default: return launch_window<InT, OutT, true>(p, st);
+    }
+  }
+  if (p.small_window_kernel) {
+    switch (p.m) {
+      case 1: return launch_csa_small<InT, OutT, 1, false>(p, st);
+      case 2: return launch_csa_small<InT, OutT, 2, false>(p, st);
+      case 4: return launch_csa_small<InT, OutT, 4, false>(p, st);
+      default: break;
+    }
+  }
+  return launch_window<InT, OutT, false>(p, st);
+}
+
+}  // namespace
+
+size_t window_kernel_smem_bytes(bool bf16_in, bool two_segments, int m) {
+  if (bf16_in)
+    return two_segments ? win_smem_bytes<__nv_bfloat16, true>(m)
+                        : win_smem_bytes<__nv_bfloat16, false>(m);
+  return two_segments ? win_smem_bytes<float, true>(m) : win_smem_bytes<float, false>(m);
+}
+
+kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st) {
+  if (p.in_bf16) {
+    return p.out_bf16 ? dispatch_stream<__nv_bfloat16, __nv_bfloat16>(p, st)
+                      : dispatch_stream<__nv_bfloat16, float>(p, st);
+  }
+  return p.out_bf16 ? dispatch_stream<float, __nv_bfloat16>(p, st)
+                    : dispatch_stream<float, float>(p, st);
+}
+
+}  // namespace kvc

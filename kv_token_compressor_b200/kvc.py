@@ -1,0 +1,184 @@
+"""Thin Python binding of the C ABI in include/kvc.h (ctypes).
+
+Argument marshalling only: tensors are checked for device, dtype and contiguity, their
+device pointers and the current CUDA stream are passed to libkvc.so, and a non-OK status
+raises :class:`KvcError`.  Every step of the compressor runs in the library's kernels;
+there is no fallback: if libkvc.so is missing this module raises on first use.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvc.so")
+
+# kvc_status
+KVC_OK = 0
+KVC_ERR_NULL = 1
+KVC_ERR_SHAPE = 2
+KVC_ERR_DTYPE = 3
+KVC_ERR_ALIGN = 4
+KVC_ERR_UNSUPPORTED = 5
+KVC_ERR_CUDA = 6
+KVC_ERR_TIMEOUT = 7
+KVC_ERR_POINTER = 8
+# kvc_dtype
+KVC_F32 = 0
+KVC_BF16 = 1
+
+# Every entry point the header declares, with its ctypes signature.
+_i64, _i32, _p = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
+SIGNATURES = {
+    "kvc_num_entries": (_i64, [_i64, _i32]),
+    "kvc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "csa_compress": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64, _i64, _i32,
+                                    _i32, _p, ctypes.c_int, _p]),
+    "hca_compress": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i32, _p,
+                                    ctypes.c_int, _p]),
+    "csa_compress_fused_proj": (ctypes.c_int, [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64,
+                                               _i32, _i32, _p, ctypes.c_int, _p]),
+    "hca_compress_fused_proj": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32, _p,
+                                               ctypes.c_int, _p]),
+    "kvc_device_status": (ctypes.c_int, [_p]),
+}
+
+_lib = None
+
+
+class KvcError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libkvc.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m kv_token_compressor_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().kvc_status_string(status).decode()
+
+
+def num_entries(n: int, m: int) -> int:
+    return int(lib().kvc_num_entries(n, m))
+
+
+def _check(status: int, where: str):
+    if status != KVC_OK:
+        raise KvcError(status, where)
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dtype_code(dt) -> int:
+    torch = _torch()
+    if dt == torch.float32:
+        return KVC_F32
+    if dt == torch.bfloat16:
+        return KVC_BF16
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _out(out, shape, dtype, like):
+    torch = _torch()
+    if out is None:
+        return torch.empty(shape, dtype=dtype, device=like.device)
+    if tuple(out.shape) != tuple(shape) or out.dtype != dtype:
+        raise ValueError(f"out must be {tuple(shape)} {dtype}")
+    return out
+
+
+def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, m: int = 4, overlap: bool = True, out=None,
+                 out_dtype=None, stream=None):
+    """CSA compressor over precomputed streams [batch, n, c] (bf16 or fp32) with fp32
+    biases [m, c].  Returns [batch, n // m, c] in ``out_dtype`` (default: input dtype)."""
+    batch, n, c = Ca.shape
+    out_dtype = Ca.dtype if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, Ca)
+    st = lib().csa_compress(_ptr(Ca), _ptr(Cb) if overlap else None, _ptr(Za),
+                            _ptr(Zb) if overlap else None, _dtype_code(Ca.dtype), _ptr(Ba),
+                            _ptr(Bb) if overlap else None, batch, n, c, m, int(bool(overlap)),
+                            _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "csa_compress")
+    return out
+
+
+def hca_compress(C, Z, B, m: int = 128, out=None, out_dtype=None, stream=None):
+    """HCA compressor over precomputed streams C, Z [batch, n, c] with bias B [m, c]."""
+    batch, n, c = C.shape
+    out_dtype = C.dtype if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, C)
+    st = lib().hca_compress(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
+                            _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "hca_compress")
+    return out
+
+
+def csa_compress_fused_proj(H, W_kva, W_kvb, W_za, W_zb, Ba, Bb, batch: int, n: int, m: int = 4,
+                            overlap: bool = True, out=None, out_dtype=None, stream=None):
+    """CSA compressor fed by hidden states H [batch*n, d] bf16 and W's [d, c] bf16."""
+    torch = _torch()
+    d = H.shape[1]
+    c = W_kva.shape[1]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, H)
+    st = lib().csa_compress_fused_proj(
+        _ptr(H), _ptr(W_kva), _ptr(W_kvb) if overlap else None, _ptr(W_za),
+        _ptr(W_zb) if overlap else None, _ptr(Ba), _ptr(Bb) if overlap else None,
+        batch, n, d, c, m, int(bool(overlap)), _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "csa_compress_fused_proj")
+    return out
+
+
+def hca_compress_fused_proj(H, W_kv, W_z, B, batch: int, n: int, m: int = 128, out=None,
+                            out_dtype=None, stream=None):
+    """HCA compressor fed by hidden states H [batch*n, d] bf16 and W's [d, c] bf16."""
+    torch = _torch()
+    d = H.shape[1]
+    c = W_kv.shape[1]
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, H)
+    st = lib().hca_compress_fused_proj(_ptr(H), _ptr(W_kv), _ptr(W_z), _ptr(B), batch, n, d, c, m,
+                                       _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "hca_compress_fused_proj")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the kernels' device error status."""
+    return int(lib().kvc_device_status(_stream(stream)))

@@ -1,0 +1,184 @@
+"""The C-ABI library on the host: it loads, exports every entry point that
+include/kvc.h declares, and rejects bad arguments before touching the GPU.
+
+Only argument errors that the library detects before its first CUDA call are
+exercised here (no device is needed and no pointer is ever dereferenced)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from kv_token_compressor_b200 import kvc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvc.h")
+
+# Fake, never-dereferenced device addresses (16-byte aligned unless stated).
+A = 0x7F0000000000
+MIS = A + 8
+
+
+def header_entry_points():
+    src = open(HEADER).read()
+    return re.findall(r"KVC_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from kv_token_compressor_b200 import build
+
+    build.build()
+    return kvc.lib()
+
+
+def test_header_declares_the_boundary():
+    names = set(header_entry_points())
+    assert {"csa_compress", "hca_compress", "csa_compress_fused_proj", "hca_compress_fused_proj",
+            "kvc_num_entries", "kvc_status_string", "kvc_device_status"} <= names
+
+
+def test_every_declared_symbol_is_exported(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", kvc.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for name in header_entry_points():
+        assert name in exported, name
+        assert hasattr(L, name)
+    assert set(kvc.SIGNATURES) == set(header_entry_points())
+
+
+def test_num_entries_bit_exact(L):
+    for n in list(range(0, 300)) + [1 << 20, 10**6, (1 << 40) + 3]:
+        for m in (1, 2, 3, 4, 7, 8, 128, 1000):
+            assert L.kvc_num_entries(n, m) == n // m
+    assert L.kvc_num_entries(-1, 4) == -1
+    assert L.kvc_num_entries(10, 0) == -1
+    assert L.kvc_num_entries(10, -4) == -1
+
+
+def test_status_strings(L):
+    for code in range(9):
+        s = kvc.status_string(code)
+        assert s.startswith("KVC_")
+    assert kvc.status_string(99) == "KVC_ERR_UNKNOWN"
+
+
+def csa(L, **kw):
+    a = dict(Ca=A, Cb=A, Za=A, Zb=A, in_dt=kvc.KVC_BF16, Ba=A, Bb=A, batch=1, n=1024, c=512, m=4,
+             overlap=1, out=A, out_dt=kvc.KVC_BF16)
+    a.update(kw)
+    return L.csa_compress(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["in_dt"], a["Ba"], a["Bb"],
+                          a["batch"], a["n"], a["c"], a["m"], a["overlap"], a["out"], a["out_dt"],
+                          None)
+
+
+def hca(L, **kw):
+    a = dict(C=A, Z=A, in_dt=kvc.KVC_BF16, B=A, batch=1, n=65536, c=512, m=128, out=A,
+             out_dt=kvc.KVC_BF16)
+    a.update(kw)
+    return L.hca_compress(a["C"], a["Z"], a["in_dt"], a["B"], a["batch"], a["n"], a["c"], a["m"],
+                          a["out"], a["out_dt"], None)
+
+
+def fused_csa(L, **kw):
+    a = dict(H=A, Wa=A, Wb=A, Za=A, Zb=A, Ba=A, Bb=A, batch=1, n=4096, d=7168, c=512, m=4,
+             overlap=1, out=A, out_dt=kvc.KVC_BF16)
+    a.update(kw)
+    return L.csa_compress_fused_proj(a["H"], a["Wa"], a["Wb"], a["Za"], a["Zb"], a["Ba"], a["Bb"],
+                                     a["batch"], a["n"], a["d"], a["c"], a["m"], a["overlap"],
+                                     a["out"], a["out_dt"], None)
+
+
+def fused_hca(L, **kw):
+    a = dict(H=A, Wk=A, Wz=A, B=A, batch=1, n=4096, d=4096, c=512, m=128, out=A,
+             out_dt=kvc.KVC_BF16)
+    a.update(kw)
+    return L.hca_compress_fused_proj(a["H"], a["Wk"], a["Wz"], a["B"], a["batch"], a["n"], a["d"],
+                                     a["c"], a["m"], a["out"], a["out_dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dt=7), kvc.KVC_ERR_DTYPE),
+    (dict(out_dt=-1), kvc.KVC_ERR_DTYPE),
+    (dict(n=-1), kvc.KVC_ERR_SHAPE),
+    (dict(batch=-2), kvc.KVC_ERR_SHAPE),
+    (dict(c=-8), kvc.KVC_ERR_SHAPE),
+    (dict(c=500), kvc.KVC_ERR_SHAPE),
+    (dict(m=0), kvc.KVC_ERR_SHAPE),
+    (dict(overlap=2), kvc.KVC_ERR_SHAPE),
+    (dict(batch=1 << 40, n=1 << 20, c=1 << 10), kvc.KVC_ERR_SHAPE),
+    (dict(Ca=None), kvc.KVC_ERR_NULL),
+    (dict(Zb=None), kvc.KVC_ERR_NULL),
+    (dict(Bb=None), kvc.KVC_ERR_NULL),
+    (dict(out=None), kvc.KVC_ERR_NULL),
+    (dict(Ca=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(Zb=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(out=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(Ba=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(m=200), kvc.KVC_ERR_UNSUPPORTED),
+])
+def test_csa_rejects_before_launch(L, kw, status):
+    assert csa(L, **kw) == status
+
+
+def test_csa_overlap_off_ignores_b_pointers(L):
+    # With overlap = 0 the b-stream pointers may be NULL: validation passes them.
+    st = csa(L, overlap=0, Cb=None, Zb=None, Bb=None, Ca=MIS)
+    assert st == kvc.KVC_ERR_ALIGN  # it got as far as checking the a-stream pointer
+
+
+@pytest.mark.parametrize("kw", [dict(n=3), dict(n=0), dict(batch=0), dict(c=0)])
+def test_csa_empty_problem_is_ok_and_touches_nothing(L, kw):
+    assert csa(L, Ca=None, Cb=None, Za=None, Zb=None, Ba=None, Bb=None, out=None, **kw) == kvc.KVC_OK
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dt=2), kvc.KVC_ERR_DTYPE),
+    (dict(n=-5), kvc.KVC_ERR_SHAPE),
+    (dict(c=12), kvc.KVC_ERR_SHAPE),
+    (dict(m=0), kvc.KVC_ERR_SHAPE),
+    (dict(Z=None), kvc.KVC_ERR_NULL),
+    (dict(B=None), kvc.KVC_ERR_NULL),
+    (dict(C=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(m=321), kvc.KVC_ERR_UNSUPPORTED),
+])
+def test_hca_rejects_before_launch(L, kw, status):
+    assert hca(L, **kw) == status
+
+
+def test_hca_empty(L):
+    assert hca(L, n=127, C=None, Z=None, B=None, out=None) == kvc.KVC_OK
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(out_dt=5), kvc.KVC_ERR_DTYPE),
+    (dict(d=7160), kvc.KVC_ERR_SHAPE),
+    (dict(c=448), kvc.KVC_ERR_SHAPE),
+    (dict(m=0), kvc.KVC_ERR_SHAPE),
+    (dict(overlap=3), kvc.KVC_ERR_SHAPE),
+    (dict(H=None), kvc.KVC_ERR_NULL),
+    (dict(Zb=None), kvc.KVC_ERR_NULL),
+    (dict(Bb=None), kvc.KVC_ERR_NULL),
+    (dict(H=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(Wb=MIS), kvc.KVC_ERR_ALIGN),
+])
+def test_fused_csa_rejects_before_launch(L, kw, status):
+    assert fused_csa(L, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=100), kvc.KVC_ERR_SHAPE),
+    (dict(c=200), kvc.KVC_ERR_SHAPE),
+    (dict(Wz=None), kvc.KVC_ERR_NULL),
+    (dict(Wk=MIS), kvc.KVC_ERR_ALIGN),
+])
+def test_fused_hca_rejects_before_launch(L, kw, status):
+    assert fused_hca(L, **kw) == status
+
+
+def test_fused_empty(L):
+    assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
+    assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK

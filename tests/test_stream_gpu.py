@@ -1,0 +1,242 @@
+"""GPU parity of the streaming compressor (csa_compress / hca_compress through the C ABI)
+against the fp64 oracle on the same seeded inputs."""
+
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import check_close, dev, host64, tdtype
+from kv_token_compressor_b200 import kvc, synth
+from oracle import compressor as O
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_csa(d, m, overlap, in_dt, out_dt):
+    t = {k: dev(v, in_dt) if k in ("Ca", "Cb", "Za", "Zb") else dev(v, "f32") for k, v in d.items()}
+    out = kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=m,
+                           overlap=overlap, out_dtype=tdtype(out_dt))
+    torch.cuda.synchronize()
+    return out
+
+
+def _run_hca(d, m, in_dt, out_dt):
+    out = kvc.hca_compress(dev(d["C"], in_dt), dev(d["Z"], in_dt), dev(d["B"], "f32"), m=m,
+                           out_dtype=tdtype(out_dt))
+    torch.cuda.synchronize()
+    return out
+
+
+# ------------------------------------------------------------------ the named workloads
+
+def test_csa_f32_n1024_workload():
+    w = synth.WORKLOADS["csa_f32_n1024"]
+    d = synth.stream_inputs("csa", w["batch"], w["n"], w["c"], w["m"], "f32", seed=0)
+    out = _run_csa(d, 4, True, "f32", "f32")
+    ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], 4, True)
+    assert out.shape == (1, 256, 512)
+    check_close(out, ref, "f32", "csa n=1024 fp32")
+
+
+def test_hca_bf16_n65536_workload():
+    w = synth.WORKLOADS["hca_bf16_n65536"]
+    d = synth.stream_inputs("hca", w["batch"], w["n"], w["c"], w["m"], "bf16", seed=0)
+    out = _run_hca(d, 128, "bf16", "bf16")
+    ref = O.hca_compress(d["C"], d["Z"], d["B"], 128)
+    assert out.shape == (1, 512, 512)
+    check_close(out, ref, "bf16", "hca n=65536 bf16")
+
+
+# ------------------------------------------------------------------ ragged / edge shapes
+
+CSA_CASES = [
+    # batch, n, c, m, overlap
+    (3, 4 * 37 + 3, 136, 4, True),
+    (2, 4 * 70, 512, 4, True),
+    (1, 4 * 5, 8, 4, True),
+    (2, 50, 24, 1, True),
+    (2, 51, 24, 2, True),
+    (2, 4 * 33 + 1, 520, 4, False),
+    (2, 8 * 21 + 5, 72, 8, True),
+    (1, 3 * 40 + 2, 16, 3, True),
+    (2, 16 * 9, 64, 16, True),
+    (2, 5 * 30 + 4, 40, 5, False),
+    (1, 160 * 3, 24, 160, True),
+]
+
+
+@pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("bf16", "f32"),
+                                          ("f32", "bf16")])
+@pytest.mark.parametrize("batch,n,c,m,overlap", CSA_CASES)
+def test_csa_shapes(batch, n, c, m, overlap, in_dt, out_dt):
+    d = synth.stream_inputs("csa", batch, n, c, m, in_dt, seed=batch * 1000 + n + c + m)
+    out = _run_csa(d, m, overlap, in_dt, out_dt)
+    if overlap:
+        ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], m, True)
+    else:
+        ref = O.csa_compress(d["Ca"], None, d["Za"], None, d["Ba"], None, m, False)
+    assert out.shape == (batch, n // m, c)
+    check_close(out, ref, out_dt, f"csa {batch}x{n}x{c} m={m} ov={overlap}")
+
+
+HCA_CASES = [
+    (2, 128 * 5 + 17, 520, 128),
+    (1, 128 * 3, 8, 128),
+    (3, 64 * 7 + 63, 136, 64),
+    (1, 40, 24, 1),
+    (2, 160 * 4, 256, 160),
+    (1, 320 * 2 + 5, 16, 320),
+    (1, 7 * 11, 512, 7),
+]
+
+
+@pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("bf16", "f32"),
+                                          ("f32", "bf16")])
+@pytest.mark.parametrize("batch,n,c,m", HCA_CASES)
+def test_hca_shapes(batch, n, c, m, in_dt, out_dt):
+    d = synth.stream_inputs("hca", batch, n, c, m, in_dt, seed=7 + n + c + m)
+    out = _run_hca(d, m, in_dt, out_dt)
+    ref = O.hca_compress(d["C"], d["Z"], d["B"], m)
+    assert out.shape == (batch, n // m, c)
+    check_close(out, ref, out_dt, f"hca {batch}x{n}x{c} m={m}")
+
+
+def test_wide_logit_range():
+    """Row offsets of +-30 on the logits: the max subtraction must keep exp2 finite."""
+    d = synth.stream_inputs("csa", 2, 4 * 64, 64, 4, "f32", seed=3, z_row_offset=30.0)
+    out = _run_csa(d, 4, True, "f32", "f32")
+    ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], 4, True)
+    check_close(out, ref, "f32", "csa wide logits")
+    h = synth.stream_inputs("hca", 1, 512, 64, 128, "f32", seed=4, z_row_offset=30.0)
+    out = _run_hca(h, 128, "f32", "f32")
+    check_close(out, O.hca_compress(h["C"], h["Z"], h["B"], 128), "f32", "hca wide logits")
+
+
+def test_boundary_and_mean_on_gpu():
+    """Closed forms on the kernel itself: entry 0 ignores the b-streams; constant logits
+    with zero bias give the mean of the window (1/8 and 1/4 weights are exact)."""
+    d = synth.stream_inputs("csa", 1, 64, 32, 4, "f32", seed=5)
+    d["Za"][:] = 0.25
+    d["Zb"][:] = 0.25
+    d["Ba"][:] = 0
+    d["Bb"][:] = 0
+    out = host64(_run_csa(d, 4, True, "f32", "f32"))[0]
+    assert np.allclose(out[0], d["Ca"][0, :4].astype(np.float64).mean(0), rtol=0, atol=2e-6)
+    for i in (1, 7, 15):
+        w = np.vstack([d["Ca"][0, 4 * i:4 * i + 4], d["Cb"][0, 4 * i - 4:4 * i]]).astype(np.float64)
+        assert np.allclose(out[i], w.mean(0), rtol=0, atol=2e-6)
+    d2 = {k: v.copy() for k, v in d.items()}
+    d2["Cb"][:] = 1e6
+    out2 = host64(_run_csa(d2, 4, True, "f32", "f32"))[0]
+    assert np.array_equal(out2[0], out[0])
+
+
+def test_empty_problem_returns_empty():
+    x = torch.zeros((2, 3, 64), device="cuda", dtype=torch.bfloat16)
+    b = torch.zeros((4, 64), device="cuda")
+    out = kvc.csa_compress(x, x, x, x, b, b, m=4)
+    assert out.shape == (2, 0, 64)
+    out = kvc.hca_compress(x, x, torch.zeros((128, 64), device="cuda"), m=128)
+    assert out.shape == (2, 0, 64)
+
+
+def test_host_pointer_is_rejected():
+    """A host buffer handed to the ABI is refused on the host, never dereferenced."""
+    L = kvc.lib()
+    host = torch.zeros((1, 64, 64), dtype=torch.float32).pin_memory()
+    dv = torch.zeros((1, 64, 64), device="cuda")
+    b = torch.zeros((4, 64), device="cuda")
+    out = torch.empty((1, 16, 64), device="cuda")
+    plain = np.zeros(64 * 64 + 16, np.float32)
+    hp = plain.ctypes.data + (-plain.ctypes.data) % 16
+    for bad in (hp,):
+        st = L.csa_compress(bad, dv.data_ptr(), dv.data_ptr(), dv.data_ptr(), kvc.KVC_F32,
+                            b.data_ptr(), b.data_ptr(), 1, 64, 64, 4, 1, out.data_ptr(), kvc.KVC_F32,
+                            None)
+        assert st == kvc.KVC_ERR_POINTER
+    st = L.hca_compress(dv.data_ptr(), dv.data_ptr(), kvc.KVC_F32, b.data_ptr(), 1, 64, 64, 4,
+                        host.data_ptr(), kvc.KVC_F32, None)
+    assert st == kvc.KVC_ERR_POINTER
+    assert kvc.device_status() == kvc.KVC_OK
+
+
+# ------------------------------------------------------------------ full size, sampled
+
+def _sample_entries(ne, count, seed):
+    rng = np.random.default_rng(seed)
+    s = set(rng.choice(ne, size=min(count, ne), replace=False).tolist())
+    s |= {0, 1, 2, ne // 2, ne - 2, ne - 1}
+    return sorted(i for i in s if 0 <= i < ne)
+
+
+def _rows(t, rows):
+    idx = torch.as_tensor(rows, device=t.device, dtype=torch.long)
+    return t[0].index_select(0, idx).float().cpu().numpy()
+
+
+@pytest.fixture(scope="module")
+def long_inputs():
+    w = synth.WORKLOADS["csa_long_n1048576"]
+    t = synth.stream_inputs_torch("csa", 1, w["n"], w["c"], 4, "bf16", seed=0,
+                                  z_row_offset=w["z_row_offset"])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1)
+    t["B_hca"] = torch.randn((128, w["c"]), generator=g, device="cuda") * float(np.sqrt(0.1))
+    yield t
+    del t
+    torch.cuda.empty_cache()
+
+
+def test_csa_long_n1048576_sampled(long_inputs):
+    t = long_inputs
+    out = kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=4,
+                           out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ne = (1 << 20) // 4
+    assert out.shape == (1, ne, 512)
+    ents = _sample_entries(ne, 400, 0)
+    Ba, Bb = host64(t["Ba"]), host64(t["Bb"])
+    got = host64(out[0, torch.as_tensor(ents, device="cuda")])
+    refs = []
+    for i in ents:
+        lo = 4 * (i - 1) if i > 0 else 0
+        rows = list(range(lo, 4 * i + 4))
+        mini = {k: _rows(t[k], rows)[None] for k in ("Ca", "Cb", "Za", "Zb")}
+        j = 1 if i > 0 else 0  # entry i of the sequence is entry j of the mini sequence
+        refs.append(O.csa_compress(mini["Ca"], mini["Cb"], mini["Za"], mini["Zb"], Ba, Bb, 4, True,
+                                   entries=[(0, j)])[0])
+    check_close(torch.from_numpy(got), np.array(refs), "bf16", "csa n=2^20 sampled")
+
+
+def test_hca_long_n1048576_sampled(long_inputs):
+    t = long_inputs
+    out = kvc.hca_compress(t["Ca"], t["Za"], t["B_hca"], m=128, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ne = (1 << 20) // 128
+    assert out.shape == (1, ne, 512)
+    ents = _sample_entries(ne, 200, 1)
+    B = host64(t["B_hca"])
+    got = host64(out[0, torch.as_tensor(ents, device="cuda")])
+    refs = []
+    for i in ents:
+        rows = list(range(128 * i, 128 * i + 128))
+        refs.append(O.hca_compress(_rows(t["Ca"], rows)[None], _rows(t["Za"], rows)[None], B, 128)[0, 0])
+    check_close(torch.from_numpy(got), np.array(refs), "bf16", "hca n=2^20 sampled")
+
+
+def test_long_weights_sum_to_one(long_inputs):
+    """Property at full size: with every value row equal to 1 the output is 1 everywhere
+    (weights of each (entry, channel) sum to one, entry 0 included)."""
+    t = long_inputs
+    ones = torch.ones_like(t["Ca"])
+    out = kvc.csa_compress(ones, ones, t["Za"], t["Zb"], t["Ba"], t["Bb"], m=4,
+                           out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.max(torch.abs(out - 1.0)).item() < 2e-6
+    out = kvc.hca_compress(ones, t["Za"], t["B_hca"], m=128, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.max(torch.abs(out - 1.0)).item() < 2e-6
