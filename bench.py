@@ -363,6 +363,44 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_profile_case(kind: str, launches: int = 3):
+    """A small case of one kernel for Nsight Compute captures (inputs still larger than
+    L2 for the streaming kernels; a few hundred MB on the device at most).  Prints one
+    line; not a bench value."""
+    import torch
+
+    from kv_token_compressor_b200 import kvc, synth
+
+    torch.cuda.set_device(0)
+    if kind in ("csa", "hca"):
+        n = 1 << 18
+        t = synth.stream_inputs_torch("csa", 1, n, C, M_CSA, "bf16", seed=0, z_row_offset=Z_OFF)
+        Bh = torch.randn((M_HCA, C), device="cuda") * float(np.sqrt(0.1))
+        for _ in range(launches):
+            if kind == "csa":
+                kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=M_CSA)
+            else:
+                kvc.hca_compress(t["Ca"], t["Za"], Bh, m=M_HCA)
+    elif kind == "csa_fused":
+        n, d = 4096, 7168
+        f = synth.fused_inputs_torch("csa", 1, n, d, C, M_CSA, seed=0)
+        for _ in range(launches):
+            kvc.csa_compress_fused_proj(f["H"], f["W_kva"], f["W_kvb"], f["W_za"], f["W_zb"],
+                                        f["Ba"], f["Bb"], 1, n)
+    elif kind == "hca_fused":
+        n, d = 16384, 4096
+        f = synth.fused_inputs_torch("hca", 1, n, d, C, M_HCA, seed=0)
+        for _ in range(launches):
+            kvc.hca_compress_fused_proj(f["H"], f["W_kv"], f["W_z"], f["B"], 1, n)
+    else:
+        raise SystemExit(f"unknown profile case {kind}")
+    torch.cuda.synchronize()
+    st = kvc.device_status()
+    print(json.dumps({"profile_case": kind, "launches": launches, "device_status": st}))
+    if st != kvc.KVC_OK:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -370,8 +408,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["csa", "hca", "csa_fused", "hca_fused"],
+                    help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -137,9 +137,13 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
 
 // ---------------------------------------------------------------------------------
 // Any window length: HCA (one segment of m rows), CSA with overlap for other m (the
-// a-segment then the b-segment), CSA without overlap.  One CTA = one entry x a slab
-// of SC channels at a time; its 16 row groups split the window's rows, each keeps an
-// online (max, sum, acc) per channel, and the partials merge through shared memory.
+// a-segment then the b-segment), CSA without overlap.  A CTA covers a slab of SC
+// channels (16 vectors of 16 bytes) and 16 thread rows; thread row ty = (entry es, row
+// group rg) with RG row groups per entry.  Each thread walks rows rg, rg+RG, ... of its
+// entry in chunks of U rows (all 2U loads in flight), keeping an online (max, sum, acc)
+// per channel: per chunk one exp2 per element plus one rescale.  With RG = 1 a thread
+// owns a whole window and stores its result directly; with RG > 1 (few entries) the
+// row-group partials merge through shared memory.
 // ---------------------------------------------------------------------------------
 struct WinArgs {
   const void* C0;  // segment 0 streams (a-range / the HCA segment)
@@ -154,8 +158,8 @@ struct WinArgs {
 };
 
 constexpr int kWinCG = 16;  // channel vectors per CTA
-constexpr int kWinRG = 16;  // row groups per CTA
-constexpr int kWinU = 8;    // rows per thread per chunk (all loads in flight)
+constexpr int kWinTY = 16;  // thread rows per CTA
+constexpr int kWinU = 8;    // rows per thread per chunk
 
 template <typename InT>
 constexpr int win_slab() {
@@ -163,27 +167,30 @@ constexpr int win_slab() {
 }
 
 template <typename InT, bool TWO_SEG>
-size_t win_smem_bytes(int m) {
+size_t win_smem_bytes(int m, int rg) {
   const int rows = TWO_SEG ? 2 * m : m;
-  return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + 3 * kWinRG * win_slab<InT>());
+  const size_t partial = rg > 1 ? 3 * kWinTY * win_slab<InT>() : 0;
+  return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + partial);
 }
 
-template <typename InT, typename OutT, bool TWO_SEG>
+template <typename InT, typename OutT, bool TWO_SEG, int RG>
 __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
   constexpr int CPT = VecInfo<InT>::kChannels;
   constexpr int SC = win_slab<InT>();
-  constexpr int CG = kWinCG, RG = kWinRG, U = kWinU;
+  constexpr int EY = kWinTY / RG;  // entries per CTA iteration
+  constexpr int U = kWinU;
   extern __shared__ float4 smem_f4[];
   const int nb = TWO_SEG ? 2 * a.m : a.m;
   float* sb = reinterpret_cast<float*>(smem_f4);  // [nb][SC] biases * log2 e
-  float* pm = sb + static_cast<size_t>(nb) * SC;  // [RG][SC] partial max
-  float* ps = pm + RG * SC;                        // [RG][SC] partial sum
-  float* pa = ps + RG * SC;                        // [RG][SC] partial weighted sum
+  float* pm = sb + static_cast<size_t>(nb) * SC;  // RG > 1: [16][SC] partial max
+  float* ps = pm + kWinTY * SC;                    //         partial sum
+  float* pa = ps + kWinTY * SC;                    //         partial weighted sum
 
   const int tx = threadIdx.x, ty = threadIdx.y;
-  const int tid = ty * CG + tx;
+  const int tid = ty * kWinCG + tx;
+  const int es = ty / RG, rg = ty - (ty / RG) * RG;
   const int64_t ch_base = static_cast<int64_t>(blockIdx.x) * SC;
-  for (int idx = tid; idx < nb * SC; idx += CG * RG) {
+  for (int idx = tid; idx < nb * SC; idx += kWinCG * kWinTY) {
     const int k = idx / SC;
     const int64_t ch = ch_base + (idx - k * SC);
     float v = 0.f;
@@ -203,7 +210,10 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
   const int m = a.m;
 
   for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
-    for (int64_t i = blockIdx.y; i < a.ne; i += gridDim.y) {
+    for (int64_t i0 = static_cast<int64_t>(blockIdx.y) * EY; i0 < a.ne;
+         i0 += static_cast<int64_t>(gridDim.y) * EY) {
+      const int64_t i = i0 + es;
+      const bool live = active && i < a.ne;
       const int64_t row0 = b * a.n + static_cast<int64_t>(m) * i;
       const int rows_i = (TWO_SEG && i > 0) ? 2 * m : m;
       float M[CPT], S[CPT], A[CPT];
@@ -213,8 +223,8 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
         S[j] = 0.f;
         A[j] = 0.f;
       }
-      if (active) {
-        for (int v0 = ty; v0 < rows_i; v0 += RG * U) {
+      if (live) {
+        for (int v0 = rg; v0 < rows_i; v0 += RG * U) {
           uint4 z[U], cv[U];
 #pragma unroll
           for (int u = 0; u < U; ++u) {
@@ -226,56 +236,94 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
               cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
             }
           }
+          // pass 1: chunk max per channel (bias rows read as float4 from shared memory)
+          float cm[CPT];
 #pragma unroll
-          for (int j = 0; j < CPT; ++j) {
-            float l[U];
-            float cm = -INFINITY;
+          for (int j = 0; j < CPT; ++j) cm[j] = -INFINITY;
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-              const int v = v0 + u * RG;
-              l[u] = v < rows_i ? fmaf(vec_elem<InT>(z[u], j), kLog2e, sb[v * SC + sc0 + j])
-                                : -INFINITY;
-              cm = fmaxf(cm, l[u]);
-            }
-            const float nm = fmaxf(M[j], cm);  // finite: row v0 < rows_i is valid
-            const float scale = exp2f(M[j] - nm);
-            float s = S[j] * scale, acc = A[j] * scale;
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * RG;
+            if (v < rows_i) {
+              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-              const int v = v0 + u * RG;
-              if (v < rows_i) {
-                const float w = exp2f(l[u] - nm);
-                s += w;
-                acc = fmaf(w, vec_elem<InT>(cv[u], j), acc);
+              for (int q = 0; q < CPT / 4; ++q) {
+                const float4 bq = bp[q];
+                cm[4 * q + 0] = fmaxf(cm[4 * q + 0], fmaf(vec_elem<InT>(z[u], 4 * q + 0), kLog2e, bq.x));
+                cm[4 * q + 1] = fmaxf(cm[4 * q + 1], fmaf(vec_elem<InT>(z[u], 4 * q + 1), kLog2e, bq.y));
+                cm[4 * q + 2] = fmaxf(cm[4 * q + 2], fmaf(vec_elem<InT>(z[u], 4 * q + 2), kLog2e, bq.z));
+                cm[4 * q + 3] = fmaxf(cm[4 * q + 3], fmaf(vec_elem<InT>(z[u], 4 * q + 3), kLog2e, bq.w));
               }
             }
+          }
+          // rescale the running state once per chunk
+#pragma unroll
+          for (int j = 0; j < CPT; ++j) {
+            const float nm = fmaxf(M[j], cm[j]);  // finite: row v0 < rows_i is valid
+            const float sc = exp2f(M[j] - nm);
+            S[j] *= sc;
+            A[j] *= sc;
             M[j] = nm;
-            S[j] = s;
-            A[j] = acc;
+          }
+          // pass 2: one exp2 per element
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * RG;
+            if (v < rows_i) {
+              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+#pragma unroll
+              for (int q = 0; q < CPT / 4; ++q) {
+                const float4 bq = bp[q];
+                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int j = 4 * q + e;
+                  const float w = exp2f(fmaf(vec_elem<InT>(z[u], j), kLog2e, bb[e]) - M[j]);
+                  S[j] += w;
+                  A[j] = fmaf(w, vec_elem<InT>(cv[u], j), A[j]);
+                }
+              }
+            }
           }
         }
       }
+      if constexpr (RG == 1) {
+        if (live) {
+          float res[CPT];
 #pragma unroll
-      for (int j = 0; j < CPT; ++j) {
-        pm[ty * SC + sc0 + j] = M[j];
-        ps[ty * SC + sc0 + j] = S[j];
-        pa[ty * SC + sc0 + j] = A[j];
-      }
-      __syncthreads();
-      if (tid < SC && ch_base + tid < a.c) {
-        float gm = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < RG; ++r) gm = fmaxf(gm, pm[r * SC + tid]);
-        float s = 0.f, acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < RG; ++r) {
-          const float f = exp2f(pm[r * SC + tid] - gm);  // 0 for empty row groups
-          s = fmaf(ps[r * SC + tid], f, s);
-          acc = fmaf(pa[r * SC + tid], f, acc);
+          for (int j = 0; j < CPT; ++j) res[j] = __fdividef(A[j], S[j]);
+          store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
         }
-        store_scalar<OutT>(out + (b * a.ne + i) * a.c + ch_base + tid, __fdividef(acc, s));
+      } else {
+#pragma unroll
+        for (int q = 0; q < CPT / 4; ++q) {
+          reinterpret_cast<float4*>(pm + ty * SC + sc0)[q] =
+              make_float4(M[4 * q], M[4 * q + 1], M[4 * q + 2], M[4 * q + 3]);
+          reinterpret_cast<float4*>(ps + ty * SC + sc0)[q] =
+              make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+          reinterpret_cast<float4*>(pa + ty * SC + sc0)[q] =
+              make_float4(A[4 * q], A[4 * q + 1], A[4 * q + 2], A[4 * q + 3]);
+        }
+        __syncthreads();
+        for (int item = tid; item < EY * SC; item += kWinCG * kWinTY) {
+          const int e2 = item / SC, sc = item - (item / SC) * SC;
+          const int64_t i2 = i0 + e2;
+          const int64_t ch = ch_base + sc;
+          if (i2 < a.ne && ch < a.c) {
+            float gm = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < RG; ++r) gm = fmaxf(gm, pm[(e2 * RG + r) * SC + sc]);
+            float s = 0.f, acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+              const float f = exp2f(pm[(e2 * RG + r) * SC + sc] - gm);  // 0 for empty groups
+              s = fmaf(ps[(e2 * RG + r) * SC + sc], f, s);
+              acc = fmaf(pa[(e2 * RG + r) * SC + sc], f, acc);
+            }
+            store_scalar<OutT>(out + (b * a.ne + i2) * a.c + ch, __fdividef(acc, s));
+          }
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
 }
@@ -352,29 +400,45 @@ kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
+template <typename InT, typename OutT, bool TWO_SEG, int RG>
+kvc_status launch_window_rg(const StreamProblem& p, cudaStream_t st, const DeviceInfo& di) {
+  constexpr int SC = win_slab<InT>();
+  constexpr int EY = kWinTY / RG;
+  const size_t smem = win_smem_bytes<InT, TWO_SEG>(p.m, RG);
+  if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
+  auto kern = window_pool_kernel<InT, OutT, TWO_SEG, RG>;
+  const int occ = resident_blocks(kern, kWinCG * kWinTY, smem);
+  if (occ == 0) return KVC_ERR_CUDA;
+  const int64_t gx = ceil_div(p.c, SC);
+  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
+  const int64_t need = ceil_div(p.ne, EY);
+  int64_t gy = static_cast<int64_t>(di.sms) * occ / (gx * gz);
+  if (gy < 1) gy = 1;
+  if (gy > need) gy = need;
+  if (gy > 65535) gy = 65535;
+  gy = ceil_div(need, ceil_div(need, gy));
+  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
+  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
+         dim3(kWinCG, kWinTY), smem, st>>>(args);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+// Row groups per entry: the fewest that still give every resident CTA slot a few
+// iterations (one window per thread needs no merge at all).
 template <typename InT, typename OutT, bool TWO_SEG>
 kvc_status launch_window(const StreamProblem& p, cudaStream_t st) {
   constexpr int SC = win_slab<InT>();
-  const size_t smem = win_smem_bytes<InT, TWO_SEG>(p.m);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
   const DeviceInfo di = device_info(dev);
   if (di.sms == 0) return KVC_ERR_CUDA;
-  if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
-  auto kern = window_pool_kernel<InT, OutT, TWO_SEG>;
-  const int occ = resident_blocks(kern, kWinCG * kWinRG, smem);
-  if (occ == 0) return KVC_ERR_CUDA;
-  const int64_t gx = ceil_div(p.c, SC);
-  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
-  int64_t gy = static_cast<int64_t>(di.sms) * occ / (gx * gz);
-  if (gy < 1) gy = 1;
-  if (gy > p.ne) gy = p.ne;
-  if (gy > 65535) gy = 65535;
-  gy = ceil_div(p.ne, ceil_div(p.ne, gy));
-  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
-  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
-         dim3(kWinCG, kWinRG), smem, st>>>(args);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  const int64_t tasks = p.batch * p.ne * ceil_div(p.c, SC);  // (entry, slab) pairs
+  const int64_t slots = static_cast<int64_t>(di.sms) * 2;
+  const int rows = TWO_SEG ? 2 * p.m : p.m;
+  if (tasks >= 3 * slots * kWinTY || rows <= kWinU)
+    return launch_window_rg<InT, OutT, TWO_SEG, 1>(p, st, di);
+  if (tasks >= 3 * slots * (kWinTY / 4)) return launch_window_rg<InT, OutT, TWO_SEG, 4>(p, st, di);
+  return launch_window_rg<InT, OutT, TWO_SEG, 16>(p, st, di);
 }
 
 template <typename InT, typename OutT>
@@ -402,9 +466,9 @@ kvc_status dispatch_stream(const StreamProblem& p, cudaStream_t st) {
 
 size_t window_kernel_smem_bytes(bool bf16_in, bool two_segments, int m) {
   if (bf16_in)
-    return two_segments ? win_smem_bytes<__nv_bfloat16, true>(m)
-                        : win_smem_bytes<__nv_bfloat16, false>(m);
-  return two_segments ? win_smem_bytes<float, true>(m) : win_smem_bytes<float, false>(m);
+    return two_segments ? win_smem_bytes<__nv_bfloat16, true>(m, 16)
+                        : win_smem_bytes<__nv_bfloat16, false>(m, 16);
+  return two_segments ? win_smem_bytes<float, true>(m, 16) : win_smem_bytes<float, false>(m, 16);
 }
 
 kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st) {

@@ -1,0 +1,85 @@
+"""Multi-rank path on the CPU: the shard plan covers every entry exactly once, and two
+gloo ranks that each compress only their planned rows (halo included) reproduce the
+single-process result when their outputs are gathered."""
+
+from __future__ import annotations
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from kv_token_compressor_b200 import shard, synth
+
+
+@pytest.mark.parametrize("n,m,world,overlap", [(1024, 4, 2, True), (1027, 4, 3, True), (50, 4, 8, True),
+                                               (640, 128, 3, False), (9, 4, 4, True), (4, 4, 2, True)])
+def test_plan_covers_entries_once(n, m, world, overlap):
+    p = shard.plan(n, m, world, overlap)
+    assert [s.rank for s in p] == list(range(world))
+    covered = [e for s in p for e in range(s.e0, s.e1)]
+    assert covered == list(range(n // m))
+    for s in p:
+        if s.entries == 0:
+            continue
+        # the rank reads exactly the rows its entries' windows name, nothing else
+        need = set()
+        for e in range(s.e0, s.e1):
+            need |= set(range(m * e, m * e + m))
+            if overlap and e > 0:
+                need |= set(range(m * (e - 1), m * e))
+        assert set(range(s.row0, s.row1)) == need
+        assert s.drop_first == (overlap and s.e0 > 0)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, n, m, q):
+    from oracle import compressor as O
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        d = synth.stream_inputs("csa", 1, n, 16, m, "f32", seed=5)  # every rank draws the same
+        s = shard.plan(n, m, world, True)[rank]
+        loc = {k: (v[:, s.row0:s.row1] if v.ndim == 3 else v) for k, v in d.items()}
+        part = O.csa_compress(loc["Ca"], loc["Cb"], loc["Za"], loc["Zb"], loc["Ba"], loc["Bb"], m, True)[0]
+        if s.drop_first:
+            part = part[1:]
+        assert part.shape[0] == s.entries
+        # ranks own unequal entry counts: pad to the largest, gather, then trim
+        sizes = [None] * world
+        dist.all_gather_object(sizes, int(part.shape[0]))
+        t = torch.zeros((max(sizes), 16), dtype=torch.float64)
+        t[:part.shape[0]] = torch.from_numpy(np.ascontiguousarray(part))
+        gathered = [torch.zeros_like(t) for _ in range(world)]
+        dist.all_gather(gathered, t)
+        if rank == 0:
+            full = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], m, True)[0]
+            got = torch.cat([g[:k] for g, k in zip(gathered, sizes)]).numpy()
+            q.put(bool(got.shape == full.shape and np.array_equal(got, full)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("n", [4 * 61 + 2, 64])
+def test_two_gloo_ranks_match_single_process(n):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, n, 4, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    assert q.get(timeout=5) is True

@@ -240,3 +240,21 @@ def test_long_weights_sum_to_one(long_inputs):
     out = kvc.hca_compress(ones, t["Za"], t["B_hca"], m=128, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.max(torch.abs(out - 1.0)).item() < 2e-6
+
+
+def test_shard_plan_on_gpu_is_bit_exact():
+    """Each rank's planned rows (one-block halo included), compressed on their own with
+    the halo entry dropped, give exactly the full run's entries."""
+    from kv_token_compressor_b200 import shard
+
+    n, c = 4 * 1000 + 3, 512
+    d = synth.stream_inputs("csa", 1, n, c, 4, "bf16", seed=21)
+    t = {k: dev(v, "bf16") if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+    full = kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=4)
+    parts = []
+    for s in shard.plan(n, 4, 3, True):
+        loc = {k: (v[:, s.row0:s.row1].contiguous() if v.dim() == 3 else v) for k, v in t.items()}
+        o = kvc.csa_compress(loc["Ca"], loc["Cb"], loc["Za"], loc["Zb"], loc["Ba"], loc["Bb"], m=4)
+        parts.append(o[:, 1:] if s.drop_first else o)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts, dim=1), full)
