@@ -373,7 +373,7 @@ def run_profile_case(kind: str, launches: int = 3):
 
     torch.cuda.set_device(0)
     if kind in ("csa", "hca"):
-        n = 1 << 18
+        n = 1 << 18 if kind == "csa" else 1 << 19  # HCA: enough windows for one per thread
         t = synth.stream_inputs_torch("csa", 1, n, C, M_CSA, "bf16", seed=0, z_row_offset=Z_OFF)
         Bh = torch.randn((M_HCA, C), device="cuda") * float(np.sqrt(0.1))
         for _ in range(launches):

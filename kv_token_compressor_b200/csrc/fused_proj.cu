@@ -43,16 +43,21 @@ __device__ unsigned int g_device_error = 0;
 namespace fused {
 
 constexpr int kCh = 128;         // channels per tile (MMA M, TMEM lanes)
-constexpr int kBK = 64;          // K per pipeline stage: one 128-byte swizzle row of bf16
 constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
-template <int NS>
+// NS streams; BK = K per pipeline stage: 64 (H rows of 128 bytes, 128-byte swizzle) or
+// 32 (H rows of 64 bytes, 64-byte swizzle; half the stage size, twice the stages).
+template <int NS, int BK_>
 struct Cfg {
+  static constexpr int BK = BK_;
   static constexpr int TN = 512 / NS;               // tokens per tile (MMA N)
-  static constexpr int A_BOX = kBK * 64 * 2;        // one [64 k x 64 ch] bf16 W box
+  static constexpr int A_BOX = BK * 64 * 2;         // one [BK k x 64 ch] bf16 W box
   static constexpr int A_BYTES = NS * 2 * A_BOX;    // NS streams x 2 boxes (128 channels)
-  static constexpr int B_BYTES = TN * kBK * 2;      // H tile [TN tokens x 64 k]
+  static constexpr int B_BYTES = TN * BK * 2;       // H tile [TN tokens x BK k]
+  static constexpr uint32_t B_SBO = BK * 2 * 8;     // 8 H rows
+  static constexpr uint64_t B_LAYOUT = BK == 64 ? 2 : 4;  // SWIZZLE_128B / SWIZZLE_64B
+  static_assert(BK == 64 || BK == 32, "stage K");
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE + 256;
@@ -120,15 +125,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: start >> 4 at
-// [0,14), leading byte offset >> 4 at [16,30), stride byte offset >> 4 at [32,46),
-// version 1 at [46,48), layout type 2 = SWIZZLE_128B at [61,64)).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor (tcgen05 format: start >> 4 at [0,14), leading byte
+// offset >> 4 at [16,30), stride byte offset >> 4 at [32,46), version 1 at [46,48),
+// layout type at [61,64): 2 = SWIZZLE_128B, 4 = SWIZZLE_64B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint64_t layout) {
   uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
   d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;
-  d |= 2ull << 61;
+  d |= layout << 61;
   return d;
 }
 
@@ -233,7 +239,7 @@ __device__ __forceinline__ HcaTile hca_tile(const Args& a, int64_t t) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <bool CSA, typename OutT>
+template <bool CSA, int BK, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_pool_kernel(const __grid_constant__ CUtensorMap tmH,
                       const __grid_constant__ CUtensorMap tmW0,
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmW2,
                       const __grid_constant__ CUtensorMap tmW3, const Args a) {
   constexpr int NS = CSA ? 4 : 2;
-  using C = Cfg<NS>;
+  using C = Cfg<NS, BK>;
   constexpr int TN = C::TN;
   constexpr uint32_t IDESC = idesc_bf16(TN);
 
@@ -317,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* st = smem + stage * C::STAGE;
             mbar_arrive_expect_tx(&full[stage], C::STAGE);
             pending_parity[stage] = static_cast<int>(phase);
-            const int x = kstep * kBK;
+            const int x = kstep * BK;
             tma_load_2d(smem_u32(st + C::A_BYTES), &tmH, &full[stage], x, y);
             const CUtensorMap* maps[4] = {&tmW0, &tmW1, &tmW2, &tmW3};
 #pragma unroll
@@ -369,14 +375,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int s = 0; s < NS; ++s) {
 #pragma unroll
-              for (int ks = 0; ks < kBK / 16; ++ks) {
-                // A: W tile of stream s, MN-major: 64-channel blocks A_BOX apart (LBO),
-                // 8-row k groups 1024 B apart (SBO); k-slice ks starts 16 rows in.
+              for (int ks = 0; ks < BK / 16; ++ks) {
+                // A: W tile of stream s, MN-major, 128-byte swizzle: 64-channel blocks
+                // A_BOX apart (LBO), 8-row k groups 1024 B apart (SBO); k-slice ks starts
+                // 16 rows in.
                 const uint64_t ad =
-                    smem_desc_sw128(st + (2 * s) * C::A_BOX + ks * 16 * 128, C::A_BOX, 1024);
-                // B: H tile, K-major: token rows of 128 B, 8-row groups 1024 B apart;
+                    smem_desc(st + (2 * s) * C::A_BOX + ks * 16 * 128, C::A_BOX, 1024, 2);
+                // B: H tile, K-major: token rows of 2*BK bytes, 8-row groups B_SBO apart;
                 // k-slice ks starts 32 bytes into the swizzled row.
-                const uint64_t bd = smem_desc_sw128(st + C::A_BYTES + ks * 32, 16, 1024);
+                const uint64_t bd =
+                    smem_desc(st + C::A_BYTES + ks * 32, 16, C::B_SBO, C::B_LAYOUT);
                 umma_bf16(tmem_base + s * TN, ad, bd, IDESC, (kstep | ks) != 0 ? 1u : 0u);
               }
             }
@@ -557,34 +565,39 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 row-major [rows, cols] tensor map with a [box_rows, 64] box, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D bf16 row-major [rows, cols] tensor map with a [box_rows, box_cols] box; the
+// swizzle span equals the box row (box_cols * 2 bytes: 128 or 64).
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              uint32_t box_cols) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw =
+      box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool CSA, typename OutT>
+template <bool CSA, int BK, typename OutT>
 kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   constexpr int NS = CSA ? 4 : 2;
-  using C = Cfg<NS>;
+  using C = Cfg<NS, BK>;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return KVC_ERR_CUDA;
   if (p.batch * p.n > (int64_t(1) << 31) - 1 - C::TN) return KVC_ERR_UNSUPPORTED;  // TMA y: int32
   CUtensorMap mh, mw[4];
-  if (!make_map(&mh, p.H, static_cast<uint64_t>(p.batch * p.n), static_cast<uint64_t>(p.d), C::TN))
+  if (!make_map(&mh, p.H, static_cast<uint64_t>(p.batch * p.n), static_cast<uint64_t>(p.d), C::TN,
+                BK))
     return KVC_ERR_CUDA;
   for (int s = 0; s < 4; ++s) {
     const void* w = CSA ? p.W[s] : p.W[s < 2 ? s : 0];
-    if (!make_map(&mw[s], w, static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.c), kBK))
+    if (!make_map(&mw[s], w, static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.c), BK, 64))
       return KVC_ERR_CUDA;
   }
   Args a{};
@@ -596,7 +609,7 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   a.c = p.c;
   a.ne = p.ne;
   a.ncg = static_cast<int>(p.c / kCh);
-  a.nk = static_cast<int>(p.d / kBK);
+  a.nk = static_cast<int>(p.d / BK);
   int64_t grid;
   if constexpr (CSA) {
     const int64_t seq_units = p.batch * a.ncg;
@@ -610,7 +623,7 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
     a.units = p.batch * ((p.ne * 128 + C::TN - 1) / C::TN) * a.ncg;
   }
   grid = a.units < sms ? a.units : sms;
-  auto kern = fused_pool_kernel<CSA, OutT>;
+  auto kern = fused_pool_kernel<CSA, BK, OutT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(C::SMEM)) != cudaSuccess)
     return KVC_ERR_CUDA;
@@ -620,15 +633,22 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
 
 }  // namespace fused
 
+// Stage K per mode.  64-deep stages: CSA 80 KB (two fit), HCA 64 KB (three).  32-deep
+// stages (CSA: five of 40 KB) measured slower on B200 (0.84 vs 0.79 ms on the n = 32768,
+// d = 7168 workload): the CSA tile is bound by shared-memory bandwidth (N = 128 operand
+// reads plus TMA writes), not by pipeline depth.
+constexpr int kBkCsa = 64;
+constexpr int kBkHca = 64;
+
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st) {
   if (p.csa) {
     if (p.m != 4 || !p.overlap) return KVC_ERR_UNSUPPORTED;
-    return p.out_bf16 ? fused::launch_impl<true, __nv_bfloat16>(p, st)
-                      : fused::launch_impl<true, float>(p, st);
+    return p.out_bf16 ? fused::launch_impl<true, kBkCsa, __nv_bfloat16>(p, st)
+                      : fused::launch_impl<true, kBkCsa, float>(p, st);
   }
   if (p.m != 128) return KVC_ERR_UNSUPPORTED;
-  return p.out_bf16 ? fused::launch_impl<false, __nv_bfloat16>(p, st)
-                    : fused::launch_impl<false, float>(p, st);
+  return p.out_bf16 ? fused::launch_impl<false, kBkHca, __nv_bfloat16>(p, st)
+                    : fused::launch_impl<false, kBkHca, float>(p, st);
 }
 
 kvc_status read_and_clear_device_error(cudaStream_t st) {

@@ -160,6 +160,7 @@ struct WinArgs {
 constexpr int kWinCG = 16;  // channel vectors per CTA
 constexpr int kWinTY = 16;  // thread rows per CTA
 constexpr int kWinU = 8;    // rows per thread per chunk
+constexpr bool kWinPrefetch = false;  // load chunk k+1 before folding chunk k
 
 template <typename InT>
 constexpr int win_slab() {
@@ -223,67 +224,88 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
         S[j] = 0.f;
         A[j] = 0.f;
       }
+      // Issue the 2U loads of the chunk whose first row is v0.
+      auto load_chunk = [&](uint4 (&z)[U], uint4 (&cv)[U], int v0) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * RG;
+          if (v < rows_i) {
+            const bool seg1 = TWO_SEG && v >= m;
+            const int64_t row = seg1 ? row0 - m + (v - m) : row0 + v;
+            z[u] = ld_stream16((seg1 ? Z1 : Z0) + row * a.c + ch0);
+            cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
+          }
+        }
+      };
+      // Fold one loaded chunk into the running (M, S, A).
+      auto consume_chunk = [&](const uint4 (&z)[U], const uint4 (&cv)[U], int v0) {
+        // pass 1: chunk max per channel (bias rows read as float4 from shared memory)
+        float cm[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) cm[j] = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * RG;
+          if (v < rows_i) {
+            const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+#pragma unroll
+            for (int q = 0; q < CPT / 4; ++q) {
+              const float4 bq = bp[q];
+              cm[4 * q + 0] = fmaxf(cm[4 * q + 0], fmaf(vec_elem<InT>(z[u], 4 * q + 0), kLog2e, bq.x));
+              cm[4 * q + 1] = fmaxf(cm[4 * q + 1], fmaf(vec_elem<InT>(z[u], 4 * q + 1), kLog2e, bq.y));
+              cm[4 * q + 2] = fmaxf(cm[4 * q + 2], fmaf(vec_elem<InT>(z[u], 4 * q + 2), kLog2e, bq.z));
+              cm[4 * q + 3] = fmaxf(cm[4 * q + 3], fmaf(vec_elem<InT>(z[u], 4 * q + 3), kLog2e, bq.w));
+            }
+          }
+        }
+        // rescale the running state once per chunk
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+          const float nm = fmaxf(M[j], cm[j]);  // finite: row v0 < rows_i is valid
+          const float sc = exp2f(M[j] - nm);
+          S[j] *= sc;
+          A[j] *= sc;
+          M[j] = nm;
+        }
+        // pass 2: one exp2 per element
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * RG;
+          if (v < rows_i) {
+            const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+#pragma unroll
+            for (int q = 0; q < CPT / 4; ++q) {
+              const float4 bq = bp[q];
+              const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = 4 * q + e;
+                const float w = exp2f(fmaf(vec_elem<InT>(z[u], j), kLog2e, bb[e]) - M[j]);
+                S[j] += w;
+                A[j] = fmaf(w, vec_elem<InT>(cv[u], j), A[j]);
+              }
+            }
+          }
+        }
+      };
       if (live) {
-        for (int v0 = rg; v0 < rows_i; v0 += RG * U) {
-          uint4 z[U], cv[U];
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int v = v0 + u * RG;
-            if (v < rows_i) {
-              const bool seg1 = TWO_SEG && v >= m;
-              const int64_t row = seg1 ? row0 - m + (v - m) : row0 + v;
-              z[u] = ld_stream16((seg1 ? Z1 : Z0) + row * a.c + ch0);
-              cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
-            }
-          }
-          // pass 1: chunk max per channel (bias rows read as float4 from shared memory)
-          float cm[CPT];
-#pragma unroll
-          for (int j = 0; j < CPT; ++j) cm[j] = -INFINITY;
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int v = v0 + u * RG;
-            if (v < rows_i) {
-              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
-#pragma unroll
-              for (int q = 0; q < CPT / 4; ++q) {
-                const float4 bq = bp[q];
-                cm[4 * q + 0] = fmaxf(cm[4 * q + 0], fmaf(vec_elem<InT>(z[u], 4 * q + 0), kLog2e, bq.x));
-                cm[4 * q + 1] = fmaxf(cm[4 * q + 1], fmaf(vec_elem<InT>(z[u], 4 * q + 1), kLog2e, bq.y));
-                cm[4 * q + 2] = fmaxf(cm[4 * q + 2], fmaf(vec_elem<InT>(z[u], 4 * q + 2), kLog2e, bq.z));
-                cm[4 * q + 3] = fmaxf(cm[4 * q + 3], fmaf(vec_elem<InT>(z[u], 4 * q + 3), kLog2e, bq.w));
-              }
-            }
-          }
-          // rescale the running state once per chunk
-#pragma unroll
-          for (int j = 0; j < CPT; ++j) {
-            const float nm = fmaxf(M[j], cm[j]);  // finite: row v0 < rows_i is valid
-            const float sc = exp2f(M[j] - nm);
-            S[j] *= sc;
-            A[j] *= sc;
-            M[j] = nm;
-          }
-          // pass 2: one exp2 per element
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int v = v0 + u * RG;
-            if (v < rows_i) {
-              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
-#pragma unroll
-              for (int q = 0; q < CPT / 4; ++q) {
-                const float4 bq = bp[q];
-                const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int j = 4 * q + e;
-                  const float w = exp2f(fmaf(vec_elem<InT>(z[u], j), kLog2e, bb[e]) - M[j]);
-                  S[j] += w;
-                  A[j] = fmaf(w, vec_elem<InT>(cv[u], j), A[j]);
-                }
-              }
-            }
-          }
+        // Two register buffers: with kWinPrefetch the next chunk's loads are in flight
+        // while the current one is folded in.
+        uint4 zA[U], cA[U], zB[U], cB[U];
+        int v0 = rg;
+        load_chunk(zA, cA, v0);
+        while (true) {
+          const int v1 = v0 + RG * U;
+          if (kWinPrefetch && v1 < rows_i) load_chunk(zB, cB, v1);
+          consume_chunk(zA, cA, v0);
+          if (v1 >= rows_i) break;
+          if (!kWinPrefetch) load_chunk(zB, cB, v1);
+          const int v2 = v1 + RG * U;
+          if (kWinPrefetch && v2 < rows_i) load_chunk(zA, cA, v2);
+          consume_chunk(zB, cB, v1);
+          if (v2 >= rows_i) break;
+          if (!kWinPrefetch) load_chunk(zA, cA, v2);
+          v0 = v2;
         }
       }
       if constexpr (RG == 1) {
