@@ -45,6 +45,62 @@ __device__ __forceinline__ float vec_elem<float>(const uint4& v, int j) {
   return __uint_as_float(w);
 }
 
+// 2^x on the special-function unit, flushing subnormal results to zero (weights below
+// 2^-126 of the window maximum are negligible next to the maximum's weight of 1;
+// 2^-inf = +0, which the entry-0 boundary relies on).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes of math).
+__device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2_max(float2 a, float2 b) {
+  return make_float2(fmaxf(a.x, b.x), fmaxf(a.y, b.y));
+}
+__device__ __forceinline__ float2 f2_ex2(float2 a) { return make_float2(ex2_ftz(a.x), ex2_ftz(a.y)); }
+
+// Channel pair p (channels 2p, 2p+1) of a 16-byte vector of T, widened to fp32.
+template <typename T>
+__device__ __forceinline__ float2 vec_pair(const uint4& v, int p);
+template <>
+__device__ __forceinline__ float2 vec_pair<__nv_bfloat16>(const uint4& v, int p) {
+  const uint32_t w = p == 0 ? v.x : p == 1 ? v.y : p == 2 ? v.z : v.w;
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <>
+__device__ __forceinline__ float2 vec_pair<float>(const uint4& v, int p) {
+  return p == 0 ? make_float2(__uint_as_float(v.x), __uint_as_float(v.y))
+                : make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+
 // Channels carried by one 16-byte vector of T.
 template <typename T>
 struct VecInfo {

@@ -39,7 +39,9 @@ struct CsaSmallArgs {
 template <typename InT, typename OutT, int M, bool OVERLAP>
 __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
   constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int NP = CPT / 2;              // channel pairs per thread
   constexpr int NB = OVERLAP ? 2 * M : M;  // bias rows: B^a rows then B^b rows
+  const float2 kL2e2 = make_float2(kLog2e, kLog2e);
   extern __shared__ float4 smem_f4[];
   float* sb = reinterpret_cast<float*>(smem_f4);  // [NB][SC], pre-scaled by log2 e
 
@@ -98,37 +100,42 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
       }
       float res[CPT];
 #pragma unroll
-      for (int j = 0; j < CPT; ++j) {
-        float la[M], lb[M];
-        float mx = -INFINITY;
+      for (int p = 0; p < NP; ++p) {
+        const float2 ba_k0 = *reinterpret_cast<const float2*>(sb + sc0 + 2 * p);  // row 0
+        float2 la[M], lb[M];
+        float2 mx = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
         for (int k = 0; k < M; ++k) {
-          la[k] = fmaf(vec_elem<InT>(za[k], j), kLog2e, sb[k * SC + sc0 + j]);
-          mx = fmaxf(mx, la[k]);
+          const float2 bk = k == 0 ? ba_k0 : *reinterpret_cast<const float2*>(sb + k * SC + sc0 + 2 * p);
+          la[k] = f2_fma(vec_pair<InT>(za[k], p), kL2e2, bk);
+          mx = f2_max(mx, la[k]);
         }
         if constexpr (OVERLAP) {
 #pragma unroll
           for (int k = 0; k < M; ++k) {
-            lb[k] = fmaf(vec_elem<InT>(zb[k], j), kLog2e, sb[(M + k) * SC + sc0 + j]);
-            mx = fmaxf(mx, lb[k]);
+            const float2 bk = *reinterpret_cast<const float2*>(sb + (M + k) * SC + sc0 + 2 * p);
+            lb[k] = f2_fma(vec_pair<InT>(zb[k], p), kL2e2, bk);
+            mx = f2_max(mx, lb[k]);
           }
         }
-        float s = 0.f, acc = 0.f;
+        const float2 negm = make_float2(-mx.x, -mx.y);
+        float2 s = make_float2(0.f, 0.f), acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < M; ++k) {
-          const float w = exp2f(la[k] - mx);
-          s += w;
-          acc = fmaf(w, vec_elem<InT>(ca[k], j), acc);
+          const float2 w = f2_ex2(f2_add(la[k], negm));
+          s = f2_add(s, w);
+          acc = f2_fma(w, vec_pair<InT>(ca[k], p), acc);
         }
         if constexpr (OVERLAP) {
 #pragma unroll
           for (int k = 0; k < M; ++k) {
-            const float w = exp2f(lb[k] - mx);
-            s += w;
-            acc = fmaf(w, vec_elem<InT>(cb[k], j), acc);
+            const float2 w = f2_ex2(f2_add(lb[k], negm));
+            s = f2_add(s, w);
+            acc = f2_fma(w, vec_pair<InT>(cb[k], p), acc);
           }
         }
-        res[j] = __fdividef(acc, s);
+        res[2 * p] = __fdividef(acc.x, s.x);
+        res[2 * p + 1] = __fdividef(acc.y, s.y);
       }
       store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
     }
@@ -160,7 +167,6 @@ struct WinArgs {
 constexpr int kWinCG = 16;  // channel vectors per CTA
 constexpr int kWinTY = 16;  // thread rows per CTA
 constexpr int kWinU = 8;    // rows per thread per chunk
-constexpr bool kWinPrefetch = false;  // load chunk k+1 before folding chunk k
 
 template <typename InT>
 constexpr int win_slab() {
@@ -180,6 +186,8 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
   constexpr int SC = win_slab<InT>();
   constexpr int EY = kWinTY / RG;  // entries per CTA iteration
   constexpr int U = kWinU;
+  constexpr int NP = CPT / 2;      // channel pairs per thread
+  const float2 kL2e2 = make_float2(kLog2e, kLog2e);
   extern __shared__ float4 smem_f4[];
   const int nb = TWO_SEG ? 2 * a.m : a.m;
   float* sb = reinterpret_cast<float*>(smem_f4);  // [nb][SC] biases * log2 e
@@ -217,113 +225,98 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
       const bool live = active && i < a.ne;
       const int64_t row0 = b * a.n + static_cast<int64_t>(m) * i;
       const int rows_i = (TWO_SEG && i > 0) ? 2 * m : m;
-      float M[CPT], S[CPT], A[CPT];
+      float2 M[NP], S[NP], A[NP];  // per channel pair: running max, sum, weighted sum
 #pragma unroll
-      for (int j = 0; j < CPT; ++j) {
-        M[j] = -INFINITY;
-        S[j] = 0.f;
-        A[j] = 0.f;
+      for (int p = 0; p < NP; ++p) {
+        M[p] = make_float2(-INFINITY, -INFINITY);
+        S[p] = make_float2(0.f, 0.f);
+        A[p] = make_float2(0.f, 0.f);
       }
-      // Issue the 2U loads of the chunk whose first row is v0.
-      auto load_chunk = [&](uint4 (&z)[U], uint4 (&cv)[U], int v0) {
+      if (live) {
+        for (int v0 = rg; v0 < rows_i; v0 += RG * U) {
+          uint4 z[U], cv[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + u * RG;
-          if (v < rows_i) {
-            const bool seg1 = TWO_SEG && v >= m;
-            const int64_t row = seg1 ? row0 - m + (v - m) : row0 + v;
-            z[u] = ld_stream16((seg1 ? Z1 : Z0) + row * a.c + ch0);
-            cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
-          }
-        }
-      };
-      // Fold one loaded chunk into the running (M, S, A).
-      auto consume_chunk = [&](const uint4 (&z)[U], const uint4 (&cv)[U], int v0) {
-        // pass 1: chunk max per channel (bias rows read as float4 from shared memory)
-        float cm[CPT];
-#pragma unroll
-        for (int j = 0; j < CPT; ++j) cm[j] = -INFINITY;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + u * RG;
-          if (v < rows_i) {
-            const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
-#pragma unroll
-            for (int q = 0; q < CPT / 4; ++q) {
-              const float4 bq = bp[q];
-              cm[4 * q + 0] = fmaxf(cm[4 * q + 0], fmaf(vec_elem<InT>(z[u], 4 * q + 0), kLog2e, bq.x));
-              cm[4 * q + 1] = fmaxf(cm[4 * q + 1], fmaf(vec_elem<InT>(z[u], 4 * q + 1), kLog2e, bq.y));
-              cm[4 * q + 2] = fmaxf(cm[4 * q + 2], fmaf(vec_elem<InT>(z[u], 4 * q + 2), kLog2e, bq.z));
-              cm[4 * q + 3] = fmaxf(cm[4 * q + 3], fmaf(vec_elem<InT>(z[u], 4 * q + 3), kLog2e, bq.w));
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * RG;
+            if (v < rows_i) {
+              const bool seg1 = TWO_SEG && v >= m;
+              const int64_t row = seg1 ? row0 - m + (v - m) : row0 + v;
+              z[u] = ld_stream16((seg1 ? Z1 : Z0) + row * a.c + ch0);
+              cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
             }
           }
-        }
-        // rescale the running state once per chunk
+          // pass 1: chunk max per channel (bias rows read as float4 from shared memory)
+          float2 cm[NP];
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) {
-          const float nm = fmaxf(M[j], cm[j]);  // finite: row v0 < rows_i is valid
-          const float sc = exp2f(M[j] - nm);
-          S[j] *= sc;
-          A[j] *= sc;
-          M[j] = nm;
-        }
-        // pass 2: one exp2 per element
+          for (int p = 0; p < NP; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int v = v0 + u * RG;
-          if (v < rows_i) {
-            const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * RG;
+            if (v < rows_i) {
+              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
 #pragma unroll
-            for (int q = 0; q < CPT / 4; ++q) {
-              const float4 bq = bp[q];
-              const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = 4 * q + e;
-                const float w = exp2f(fmaf(vec_elem<InT>(z[u], j), kLog2e, bb[e]) - M[j]);
-                S[j] += w;
-                A[j] = fmaf(w, vec_elem<InT>(cv[u], j), A[j]);
+              for (int q = 0; q < NP / 2; ++q) {
+                const float4 bq = bp[q];
+                cm[2 * q] = f2_max(cm[2 * q], f2_fma(vec_pair<InT>(z[u], 2 * q), kL2e2,
+                                                     make_float2(bq.x, bq.y)));
+                cm[2 * q + 1] = f2_max(cm[2 * q + 1], f2_fma(vec_pair<InT>(z[u], 2 * q + 1),
+                                                             kL2e2, make_float2(bq.z, bq.w)));
               }
             }
           }
-        }
-      };
-      if (live) {
-        // Two register buffers: with kWinPrefetch the next chunk's loads are in flight
-        // while the current one is folded in.
-        uint4 zA[U], cA[U], zB[U], cB[U];
-        int v0 = rg;
-        load_chunk(zA, cA, v0);
-        while (true) {
-          const int v1 = v0 + RG * U;
-          if (kWinPrefetch && v1 < rows_i) load_chunk(zB, cB, v1);
-          consume_chunk(zA, cA, v0);
-          if (v1 >= rows_i) break;
-          if (!kWinPrefetch) load_chunk(zB, cB, v1);
-          const int v2 = v1 + RG * U;
-          if (kWinPrefetch && v2 < rows_i) load_chunk(zA, cA, v2);
-          consume_chunk(zB, cB, v1);
-          if (v2 >= rows_i) break;
-          if (!kWinPrefetch) load_chunk(zA, cA, v2);
-          v0 = v2;
+          // rescale the running state once per chunk
+          float2 negm[NP];
+#pragma unroll
+          for (int p = 0; p < NP; ++p) {
+            const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 < rows_i is valid
+            const float2 sc = make_float2(ex2_ftz(M[p].x - nm.x), ex2_ftz(M[p].y - nm.y));
+            S[p] = f2_mul(S[p], sc);
+            A[p] = f2_mul(A[p], sc);
+            M[p] = nm;
+            negm[p] = make_float2(-nm.x, -nm.y);
+          }
+          // pass 2: one exp2 per element, packed pair arithmetic
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * RG;
+            if (v < rows_i) {
+              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+#pragma unroll
+              for (int q = 0; q < NP / 2; ++q) {
+                const float4 bq = bp[q];
+                const float2 b2[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int pp = 2 * q + e;
+                  const float2 l = f2_fma(vec_pair<InT>(z[u], pp), kL2e2, f2_add(b2[e], negm[pp]));
+                  const float2 w = f2_ex2(l);
+                  S[pp] = f2_add(S[pp], w);
+                  A[pp] = f2_fma(w, vec_pair<InT>(cv[u], pp), A[pp]);
+                }
+              }
+            }
+          }
         }
       }
       if constexpr (RG == 1) {
         if (live) {
           float res[CPT];
 #pragma unroll
-          for (int j = 0; j < CPT; ++j) res[j] = __fdividef(A[j], S[j]);
+          for (int p = 0; p < NP; ++p) {
+            res[2 * p] = __fdividef(A[p].x, S[p].x);
+            res[2 * p + 1] = __fdividef(A[p].y, S[p].y);
+          }
           store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < CPT / 4; ++q) {
+        for (int q = 0; q < NP / 2; ++q) {
           reinterpret_cast<float4*>(pm + ty * SC + sc0)[q] =
-              make_float4(M[4 * q], M[4 * q + 1], M[4 * q + 2], M[4 * q + 3]);
+              make_float4(M[2 * q].x, M[2 * q].y, M[2 * q + 1].x, M[2 * q + 1].y);
           reinterpret_cast<float4*>(ps + ty * SC + sc0)[q] =
-              make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+              make_float4(S[2 * q].x, S[2 * q].y, S[2 * q + 1].x, S[2 * q + 1].y);
           reinterpret_cast<float4*>(pa + ty * SC + sc0)[q] =
-              make_float4(A[4 * q], A[4 * q + 1], A[4 * q + 2], A[4 * q + 3]);
+              make_float4(A[2 * q].x, A[2 * q].y, A[2 * q + 1].x, A[2 * q + 1].y);
         }
         __syncthreads();
         for (int item = tid; item < EY * SC; item += kWinCG * kWinTY) {
@@ -337,7 +330,7 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
             float s = 0.f, acc = 0.f;
 #pragma unroll
             for (int r = 0; r < RG; ++r) {
-              const float f = exp2f(pm[(e2 * RG + r) * SC + sc] - gm);  // 0 for empty groups
+              const float f = ex2_ftz(pm[(e2 * RG + r) * SC + sc] - gm);  // 0 for empty groups
               s = fmaf(ps[(e2 * RG + r) * SC + sc], f, s);
               acc = fmaf(pa[(e2 * RG + r) * SC + sc], f, acc);
             }
