@@ -363,6 +363,167 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------------------ other paths
+
+def _peak(kind):
+    """Measured roofline denominators (MEASURED_PEAKS.json), else the recipe's fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return (float(d["hbm_gbs"]) if kind == "hbm" else float(d["bf16_tflops"])), "measured"
+    return (FALLBACK_HBM_GBS if kind == "hbm" else 1590.0), "fallback"
+
+
+def _workload(name, dev):
+    """Inputs, launch function, outputs and roofline units of one named workload."""
+    import torch
+
+    from kv_token_compressor_b200 import kvc, synth
+
+    bf = torch.bfloat16
+    if name in ("fused_csa", "fused_indexer_keys"):
+        n, d, c = 32768, 7168, (512 if name == "fused_csa" else 128)
+        t = synth.fused_inputs_torch("csa", 1, n, d, c, 4, seed=0, device=dev)
+        out = torch.empty((1, n // 4, c), device=dev, dtype=bf)
+
+        def launch(x, st):
+            kvc.csa_compress_fused_proj(x["H"], x["W_kva"], x["W_kvb"], x["W_za"], x["W_zb"],
+                                        x["Ba"], x["Bb"], 1, n, m=4, out=out, stream=st)
+        return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // 4,
+                    bound="tensor", units=2.0 * n * d * 4 * c, flush=False,
+                    kernel="fused_pool_kernel<CSA>",
+                    config={"workload": f"CSA fused projection + pool: H [{n}, {d}] bf16, 4 W "
+                                        f"[{d}, {c}] bf16, m=4 overlap, bf16 out", "n": n,
+                            "d": d, "c": c, "m": 4})
+    if name == "fused_hca":
+        b, n, d, c = 4, 131072, 4096, 512
+        t = synth.fused_inputs_torch("hca", b, n, d, c, 128, seed=0, device=dev)
+        out = torch.empty((b, n // 128, c), device=dev, dtype=bf)
+
+        def launch(x, st):
+            kvc.hca_compress_fused_proj(x["H"], x["W_kv"], x["W_z"], x["B"], b, n, m=128,
+                                        out=out, stream=st)
+        return dict(inputs=t, launch=launch, outputs=[out], tokens=b * n, entries=b * n // 128,
+                    bound="tensor", units=2.0 * b * n * d * 2 * c, flush=False,
+                    kernel="fused_pool_kernel<HCA>",
+                    config={"workload": f"HCA fused projection + pool: batch {b}, n={n}, H d={d} "
+                                        f"bf16, W_kv, W_z [{d}, {c}], m'=128, bf16 out",
+                            "batch": b, "n": n, "d": d, "c": c, "m": 128})
+    if name in ("hca_n65536", "csa_f32_n1024", "indexer_keys"):
+        if name == "hca_n65536":
+            mode, n, c, m, dt = "hca", 65536, 512, 128, "bf16"
+        elif name == "csa_f32_n1024":
+            mode, n, c, m, dt = "csa", 1024, 512, 4, "f32"
+        else:
+            mode, n, c, m, dt = "csa", 1 << 20, 128, 4, "bf16"
+        t = synth.stream_inputs_torch(mode, 1, n, c, m, dt, seed=0, device=dev)
+        tdt = bf if dt == "bf16" else torch.float32
+        out = torch.empty((1, n // m, c), device=dev, dtype=tdt)
+        es = 2 if dt == "bf16" else 4
+        if mode == "hca":
+            def launch(x, st):
+                kvc.hca_compress(x["C"], x["Z"], x["B"], m=m, out=out, stream=st)
+            nbytes = 2 * n * c * es + m * c * 4 + (n // m) * c * es
+        else:
+            def launch(x, st):
+                kvc.csa_compress(x["Ca"], x["Cb"], x["Za"], x["Zb"], x["Ba"], x["Bb"], m=m,
+                                 out=out, stream=st)
+            ne = n // m
+            nbytes = (2 * ne * m + 2 * (ne - 1) * m) * c * es + 2 * m * c * 4 + ne * c * es
+        return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // m,
+                    bound="hbm", units=float(nbytes), flush=nbytes < 4 * (126 << 20),
+                    kernel="csa_small_m_kernel" if mode == "csa" else "window_pool_kernel",
+                    config={"workload": f"{mode.upper()} streams: batch 1, n={n}, c={c}, m={m}, "
+                                        f"{dt} in/out", "n": n, "c": c, "m": m})
+    raise SystemExit(f"unknown workload {name}")
+
+
+def run_workload(args):
+    """One JSON line for a named workload other than the default step (1 GPU, or weak
+    replicas under torchrun); the kernel is timed per launch with CUDA events, L2 flushed
+    between launches when the inputs are not far larger than L2."""
+    import torch
+
+    from kv_token_compressor_b200 import kvc
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    w = _workload(args.workload, dev)
+    st = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if w["flush"] else None
+    for _ in range(max(args.warmup, 3)):
+        w["launch"](w["inputs"], st)
+    torch.cuda.synchronize()
+    if kvc.device_status(st) != kvc.KVC_OK:
+        raise SystemExit("device error during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for a, b in evs:
+        if flush is not None:
+            flush.zero_()
+        a.record(st)
+        w["launch"](w["inputs"], st)
+        b.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), world)
+    if kvc.device_status(st) != kvc.KVC_OK:
+        raise SystemExit("device error in the timed region")
+    # e2e: pinned host inputs -> device, the call, outputs -> pinned host
+    host = {k: v.cpu().pin_memory() for k, v in w["inputs"].items()}
+    houts = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in w["outputs"]]
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(o.numel() * o.element_size() for o in houts)
+
+    def e2e():
+        dv = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        w["launch"](dv, st)
+        for ho, o in zip(houts, w["outputs"]):
+            ho.copy_(o, non_blocking=True)
+
+    e2e()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = 3
+    e0.record(st)
+    for _ in range(n_e2e):
+        e2e()
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
+    peak, kind = _peak(w["bound"])
+    if w["bound"] == "tensor":
+        ach, unit = w["units"] / (ms * 1e-3) / 1e12, "TFLOP/s"
+    else:
+        ach, unit = w["units"] / (ms * 1e-3) / 1e9, "GB/s"
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * w["tokens"] / (ms * 1e-3), "unit": "tokens/s",
+            "entries_per_s": world * w["entries"] / (ms * 1e-3), "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": dict(w["config"], l2="flushed between launches" if w["flush"]
+                           else "inputs larger than L2"),
+            "roofline": {"bound": w["bound"], "kernel": w["kernel"], "achieved": ach,
+                         "peak": peak, "unit": unit, "frac": ach / peak, "peak_kind": kind,
+                         "traffic": None,
+                         ("algorithmic_flops" if w["bound"] == "tensor" else "algorithmic_bytes"):
+                             w["units"]},
+            "gpu_launches": args.steps,
+            "e2e": {"value": world * w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def run_profile_case(kind: str, launches: int = 3):
     """A small case of one kernel for Nsight Compute captures (inputs still larger than
     L2 for the streaming kernels; a few hundred MB on the device at most).  Prints one
@@ -408,6 +569,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="long",
+                    choices=["long", "fused_csa", "fused_hca", "hca_n65536", "csa_f32_n1024",
+                             "indexer_keys", "fused_indexer_keys"],
+                    help="long (default): CSA + HCA over the 2^20-token streams; the others "
+                         "time one kernel on its own workload")
     ap.add_argument("--profile-case", choices=["csa", "hca", "csa_fused", "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
@@ -416,7 +582,7 @@ def main():
     elif args.impl == "reference":
         run_reference(args)
     else:
-        run_ours(args)
+        run_ours(args) if args.workload == "long" else run_workload(args)
 
 
 if __name__ == "__main__":
