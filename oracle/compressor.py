@@ -48,6 +48,10 @@ __all__ = [
     "project",
     "csa_compress_fused",
     "hca_compress_fused",
+    "csa_entry_scalar",
+    "csa_compress_scalar",
+    "hca_entry_scalar",
+    "hca_compress_scalar",
 ]
 
 
@@ -249,3 +253,63 @@ def hca_compress_fused(H, W_kv, W_z, B, batch: int, n: int, m: int = 128, entrie
     if entries is None:
         return out.reshape(batch, ne, c)
     return out
+
+
+# --------------------------------------------------------------------------------------
+# Scalar-logit form.  "Ch 04 · CSA" §3's symbol table reads the same equations with one
+# score per token and stream (Z^a, Z^b of dimension n), an m-dimensional bias B^a, B^b,
+# and S_j a scalar that multiplies the whole vector C_j; "Ch 05 · HCA" §2 likewise gives
+# B as m'-dimensional.  The softmax is still joint over the window's rows.
+# --------------------------------------------------------------------------------------
+
+def csa_entry_scalar(Ca, Cb, za, zb, ba, bb, i: int, m: int, overlap: bool = True):
+    """C^Comp_i of one sequence with scalar logits: za, zb are [n], ba, bb are [m]."""
+    a_rows, b_rows = entry_rows(i, m)
+    la = _f64(za[a_rows.start:a_rows.stop]) + _f64(ba)
+    va = _f64(Ca[a_rows.start:a_rows.stop])
+    if overlap:
+        if i == 0:
+            lb = np.full(m, -np.inf)                 # Z^b_{-m:-1} = -inf
+            vb = np.zeros((m, np.shape(Ca)[1]))      # C^b_{-m:-1} = 0
+        else:
+            lb = _f64(zb[b_rows.start:b_rows.stop]) + _f64(bb)
+            vb = _f64(Cb[b_rows.start:b_rows.stop])
+        L = np.concatenate([la, lb])
+        V = np.concatenate([va, vb], axis=0)
+    else:
+        L, V = la, va
+    w = np.exp(L - np.max(L))
+    s = w / np.sum(w)                                # one weight per row, shared by channels
+    return np.sum(s[:, None] * V, axis=0)
+
+
+def csa_compress_scalar(Ca, Cb, za, zb, ba, bb, m: int = 4, overlap: bool = True, entries=None):
+    """CSA compressor with scalar logits.  Ca, Cb: [batch, n, c]; za, zb: [batch, n];
+    ba, bb: [m].  Output as in :func:`csa_compress`."""
+    batch, n, c = np.shape(Ca)
+    ne = num_entries(n, m)
+    todo = _entry_list(batch, ne, entries)
+    rows = [csa_entry_scalar(Ca[b], None if Cb is None else Cb[b], za[b],
+                             None if zb is None else zb[b], ba, bb, i, m, overlap)
+            for b, i in todo]
+    res = np.array(rows, dtype=np.float64).reshape(len(todo), c)
+    return res.reshape(batch, ne, c) if entries is None else res
+
+
+def hca_entry_scalar(C, z, bvec, i: int, m: int):
+    """HCA segment i with scalar logits z [n] and bias bvec [m]."""
+    lo, hi = m * i, m * (i + 1)
+    L = _f64(z[lo:hi]) + _f64(bvec)
+    w = np.exp(L - np.max(L))
+    s = w / np.sum(w)
+    return np.sum(s[:, None] * _f64(C[lo:hi]), axis=0)
+
+
+def hca_compress_scalar(C, z, bvec, m: int = 128, entries=None):
+    """HCA compressor with scalar logits: C [batch, n, c], z [batch, n], bvec [m]."""
+    batch, n, c = np.shape(C)
+    ne = num_entries(n, m)
+    todo = _entry_list(batch, ne, entries)
+    rows = [hca_entry_scalar(C[b], z[b], bvec, i, m) for b, i in todo]
+    res = np.array(rows, dtype=np.float64).reshape(len(todo), c)
+    return res.reshape(batch, ne, c) if entries is None else res

@@ -410,4 +410,87 @@ def pin_fused_selection(O):
     assert np.allclose(ent, ref[0, [4, 0]], rtol=1e-13, atol=1e-13)
 
 
+# --------------------------------------------------------------------------------------
+# Scalar-logit form ("Ch 04 · CSA" §3 symbol table: one score per token, S_j a scalar)
+# --------------------------------------------------------------------------------------
+
+def _rand_scalar(rng, batch, n, c, m):
+    f = lambda *s: rng.standard_normal(s)
+    return dict(Ca=f(batch, n, c), Cb=f(batch, n, c), za=2 * f(batch, n), zb=2 * f(batch, n),
+                ba=0.3 * f(m), bb=0.3 * f(m))
+
+
+def pin_scalar_is_channel_constant_case(O):
+    """Scalar logits are the per-channel form with Z and B constant across channels (a
+    special case of the pinned per-channel definition)."""
+    rng = np.random.default_rng(31)
+    m, c = 4, 5
+    d = _rand_scalar(rng, 2, 4 * 7 + 2, c, m)
+    out = O.csa_compress_scalar(d["Ca"], d["Cb"], d["za"], d["zb"], d["ba"], d["bb"], m, True)
+    rep = lambda z: np.repeat(z[..., None], c, axis=-1)
+    ref = O.csa_compress(d["Ca"], d["Cb"], rep(d["za"]), rep(d["zb"]), rep(d["ba"]), rep(d["bb"]), m, True)
+    assert np.allclose(out, ref, rtol=1e-13, atol=1e-13)
+    C = rng.standard_normal((1, 256, c))
+    z = rng.standard_normal((1, 256)) * 3
+    b = rng.standard_normal(128)
+    assert np.allclose(O.hca_compress_scalar(C, z, b, 128), O.hca_compress(C, rep(z), rep(b), 128),
+                       rtol=1e-13, atol=1e-13)
+
+
+def pin_scalar_weights_via_unit_rows(O):
+    """With the window's value rows set to unit vectors the entry IS the weight vector:
+    it must equal scipy's softmax of [z^a + b^a; z^b + b^b] (entry 0: a-rows only)."""
+    from scipy.special import softmax
+
+    rng = np.random.default_rng(32)
+    m, ne = 4, 5
+    n = m * ne
+    d = _rand_scalar(rng, 1, n, 2 * m, m)
+    for i in range(ne):
+        Ca = np.zeros((1, n, 2 * m))
+        Cb = np.zeros((1, n, 2 * m))
+        for k in range(m):
+            Ca[0, m * i + k, k] = 1.0
+            if i > 0:
+                Cb[0, m * (i - 1) + k, m + k] = 1.0
+        out = O.csa_compress_scalar(Ca, Cb, d["za"], d["zb"], d["ba"], d["bb"], m, True,
+                                    entries=[(0, i)])[0]
+        La = d["za"][0, m * i:m * i + m] + d["ba"]
+        if i == 0:
+            ref = np.concatenate([softmax(La), np.zeros(m)])
+        else:
+            ref = softmax(np.concatenate([La, d["zb"][0, m * (i - 1):m * i] + d["bb"]]))
+        assert np.allclose(out, ref, rtol=1e-13, atol=1e-14), i
+
+
+def pin_scalar_one_hot_and_logistic(O):
+    rng = np.random.default_rng(33)
+    m, ne, c = 4, 4, 3
+    n = m * ne
+    d = _rand_scalar(rng, 1, n, c, m)
+    for r in range(n):
+        for zs, cs, target in (("za", "Ca", r // m), ("zb", "Cb", r // m + 1)):
+            if target >= ne:
+                continue
+            d2 = {k: v.copy() for k, v in d.items()}
+            d2[zs][0, r] += 60.0
+            out = O.csa_compress_scalar(d2["Ca"], d2["Cb"], d2["za"], d2["zb"], d2["ba"], d2["bb"], m,
+                                        True, entries=[(0, target)])
+            assert np.allclose(out[0], d[cs][0, r], rtol=1e-12, atol=1e-12), (zs, r)
+    e = _rand_scalar(rng, 1, 7, c, 1)
+    out = O.csa_compress_scalar(e["Ca"], e["Cb"], e["za"], e["zb"], e["ba"], e["bb"], 1, True)
+    for i in range(1, 7):
+        x = e["za"][0, i] + e["ba"][0] - e["zb"][0, i - 1] - e["bb"][0]
+        s = 1.0 / (1.0 + math.exp(-x))
+        assert np.allclose(out[0, i], s * e["Ca"][0, i] + (1 - s) * e["Cb"][0, i - 1], rtol=1e-13, atol=1e-13)
+    assert np.allclose(out[0, 0], e["Ca"][0, 0], rtol=0, atol=1e-15)
+    # HCA: bias one-hot selects in-segment position k
+    C = rng.standard_normal((1, 256, c))
+    z = rng.standard_normal((1, 256))
+    b = np.zeros(128)
+    b[77] = 60.0
+    out = O.hca_compress_scalar(C, z, b, 128)
+    assert np.allclose(out[0, 1], C[0, 128 + 77], rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -32,12 +32,23 @@ MUTANTS = [
      "    return pool_window(L, V)"),
     ("normaliser_dropped", "return w / np.sum(w, axis=0, keepdims=True)", "return w"),
     ("hca_bias_dropped", "L = _f64(Z[lo:hi]) + _f64(B)", "L = _f64(Z[lo:hi])"),
-    ("hca_segment_shift", "lo, hi = m * i, m * (i + 1)", "lo, hi = m * i + 1, m * (i + 1) + 1"),
+    ("hca_segment_shift", "lo, hi = m * i, m * (i + 1)\n    L = _f64(Z[lo:hi])",
+     "lo, hi = m * i + 1, m * (i + 1) + 1\n    L = _f64(Z[lo:hi])"),
+    ("scalar_hca_segment_shift", "lo, hi = m * i, m * (i + 1)\n    L = _f64(z[lo:hi])",
+     "lo, hi = m * i + 1, m * (i + 1) + 1\n    L = _f64(z[lo:hi])"),
     ("entries_ceil", "    return n // m", "    return -(-n // m)"),
     ("projection_transposed", "return _f64(H) @ _f64(W)", "return _f64(H) @ _f64(W).T"),
     ("projection_k_misaligned", "return _f64(H) @ _f64(W)", "return _f64(H) @ _f64(W)[::-1]"),
     ("fused_streams_swapped", "Ca, Za = stream(W_kva), stream(W_za)", "Ca, Za = stream(W_za), stream(W_kva)"),
     ("fused_b_streams_swapped", "Cb = stream(W_kvb) if overlap else None", "Cb = stream(W_zb) if overlap else None"),
+    ("scalar_a_bias_dropped", "la = _f64(za[a_rows.start:a_rows.stop]) + _f64(ba)",
+     "la = _f64(za[a_rows.start:a_rows.stop])"),
+    ("scalar_b_rows_from_a_block", "lb = _f64(zb[b_rows.start:b_rows.stop]) + _f64(bb)",
+     "lb = _f64(zb[a_rows.start:a_rows.stop]) + _f64(bb)"),
+    ("scalar_boundary_zero_logit", "lb = np.full(m, -np.inf)", "lb = np.zeros(m)"),
+    ("scalar_separately_normalised", "    w = np.exp(L - np.max(L))\n    s = w / np.sum(w)                                # one",
+     "    w = np.exp(L - np.max(L))\n    s = w / (np.sum(w[:m]) if len(w) == m else np.sum(w[m:]) + 0 * np.sum(w[:m]))  # one"),
+    ("scalar_hca_bias_dropped", "L = _f64(z[lo:hi]) + _f64(bvec)", "L = _f64(z[lo:hi])"),
     ("fused_hca_streams_swapped", "C = project(Hs, W_kv)\n        Z = project(Hs, W_z)",
      "C = project(Hs, W_z)\n        Z = project(Hs, W_kv)"),
 ]
