@@ -44,6 +44,9 @@
  *                          kernel gave up (the kernel then skipped its remaining work)
  *     KVC_ERR_POINTER      a tensor pointer is not device (or managed) memory of the
  *                          current device (e.g. a host pointer)
+ *     KVC_ERR_INDEX        reported by kvc_device_status(): an entry list read from device
+ *                          memory named a window outside its sequence or the streams (that
+ *                          entry was skipped and its output row left unwritten)
  *   An empty problem (batch == 0 or N_e == 0) is valid: KVC_OK, nothing is launched and
  *   no pointer is dereferenced.
  * Thread safety.  Calls may be made concurrently from several host threads.
@@ -72,7 +75,8 @@ typedef enum kvc_status {
   KVC_ERR_UNSUPPORTED = 5,
   KVC_ERR_CUDA = 6,
   KVC_ERR_TIMEOUT = 7,
-  KVC_ERR_POINTER = 8
+  KVC_ERR_POINTER = 8,
+  KVC_ERR_INDEX = 9
 } kvc_status;
 
 typedef enum kvc_dtype { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
@@ -111,6 +115,57 @@ KVC_API kvc_status csa_compress(const void* Ca, const void* Cb, const void* Za, 
 KVC_API kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
                         int64_t batch, int64_t n, int64_t c, int32_t m,
                         void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* Scalar-logit CSA compressor ([CSA] §3 symbol table: one score per token and stream,
+ * an m-dimensional position bias, and a scalar weight S_j on the whole vector C_j).
+ *   Ca, Cb : [batch, n, c] in_dtype (16-byte aligned);  za, zb : [batch, n] in_dtype
+ *   (element aligned);  ba, bb : [m] fp32;  out : [batch, N_e, c] out_dtype.
+ *   Entry i: w = softmax over the 2m scalars [za[mi..m(i+1)-1] + ba ; zb[m(i-1)..mi-1] + bb]
+ *   (entry 0: its m a-rows only), C^Comp_i = sum_j w_j C_j, the same w for every
+ *   channel.  overlap = 0: a-rows only; Cb, zb and bb are not read and may be NULL.
+ *   Windows of up to 320 rows. */
+KVC_API kvc_status csa_compress_scalar_logits(const void* Ca, const void* Cb, const void* za,
+                                              const void* zb, kvc_dtype in_dtype,
+                                              const float* ba, const float* bb, int64_t batch,
+                                              int64_t n, int64_t c, int32_t m, int32_t overlap,
+                                              void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* Scalar-logit HCA compressor ([HCA] §2 with an m'-dimensional bias): entry i pools the
+ * m rows of segment i of C with w = softmax(z[mi..m(i+1)-1] + b).
+ *   C : [batch, n, c] in_dtype;  z : [batch, n] in_dtype;  b : [m] fp32. */
+KVC_API kvc_status hca_compress_scalar_logits(const void* C, const void* z, kvc_dtype in_dtype,
+                                              const float* b, int64_t batch, int64_t n,
+                                              int64_t c, int32_t m, void* out,
+                                              kvc_dtype out_dtype, kvc_stream stream);
+
+/* Entry lists: the CSA compressor for an arbitrary set of entries of sequences packed
+ * one after another in the streams (decode: each sequence that just completed a block
+ * emits its new entry; ragged prefill: every entry of sequences of different lengths).
+ *   Ca, Cb, Za, Zb : packed streams [total_rows, c] in_dtype;  Ba, Bb : [m, c] fp32
+ *   seq_start, seq_len, entry : device int64 arrays [num]: listed entry k is entry
+ *     entry[k] of the sequence occupying rows [seq_start[k], seq_start[k] + seq_len[k]);
+ *     it reads rows seq_start[k] + m*entry[k] .. +m-1 (a) and the m rows before them (b,
+ *     when entry[k] > 0), exactly as csa_compress does for that sequence.
+ *   out : [num, c] out_dtype, row k = listed entry k.
+ * The lists live in device memory and are not read on the host: each listed window is
+ * checked on the device (0 <= seq_start, seq_start + seq_len <= total_rows,
+ * 0 <= entry < seq_len / m); a failing entry is skipped, its output row is left
+ * unwritten, and kvc_device_status() then reports KVC_ERR_INDEX. */
+KVC_API kvc_status csa_compress_entries(const void* Ca, const void* Cb, const void* Za,
+                                        const void* Zb, kvc_dtype in_dtype, const float* Ba,
+                                        const float* Bb, int64_t total_rows, int64_t c,
+                                        int32_t m, int32_t overlap, const int64_t* seq_start,
+                                        const int64_t* seq_len, const int64_t* entry,
+                                        int64_t num, void* out, kvc_dtype out_dtype,
+                                        kvc_stream stream);
+
+/* Entry lists for the HCA compressor: listed entry k pools rows
+ * seq_start[k] + m*entry[k] .. +m-1 of the packed C, Z ([total_rows, c]); B : [m, c]. */
+KVC_API kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype in_dtype,
+                                        const float* B, int64_t total_rows, int64_t c, int32_t m,
+                                        const int64_t* seq_start, const int64_t* seq_len,
+                                        const int64_t* entry, int64_t num, void* out,
+                                        kvc_dtype out_dtype, kvc_stream stream);
 
 /* CSA compressor fed by hidden states ([SC] eq. attn-seqcomp-csa-proj followed by the
  * csa_compress pool): the four streams H W are formed on the tensor cores (bf16 in,

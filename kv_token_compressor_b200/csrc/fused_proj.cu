@@ -658,7 +658,11 @@ kvc_status read_and_clear_device_error(cudaStream_t st) {
   if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return KVC_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
     return KVC_ERR_CUDA;
-  return v ? KVC_ERR_TIMEOUT : KVC_OK;
+  bool failed = false;
+  const bool index_error = read_and_clear_index_error(&failed);
+  if (failed) return KVC_ERR_CUDA;
+  if (v) return KVC_ERR_TIMEOUT;
+  return index_error ? KVC_ERR_INDEX : KVC_OK;
 }
 
 }  // namespace kvc

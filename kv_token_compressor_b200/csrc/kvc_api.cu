@@ -76,6 +76,7 @@ const char* kvc_status_string(kvc_status s) {
     case KVC_ERR_CUDA: return "KVC_ERR_CUDA: CUDA launch or query failed";
     case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT: a bounded wait in a kernel gave up";
     case KVC_ERR_POINTER: return "KVC_ERR_POINTER: not device memory of the current device";
+    case KVC_ERR_INDEX: return "KVC_ERR_INDEX: a listed entry was out of range and skipped";
   }
   return "KVC_ERR_UNKNOWN";
 }
@@ -149,6 +150,179 @@ kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const 
   p.c = c;
   p.ne = ne;
   p.m = m;
+  p.two_segments = false;
+  p.small_window_kernel = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status csa_compress_scalar_logits(const void* Ca, const void* Cb, const void* za,
+                                      const void* zb, kvc_dtype in_dtype, const float* ba,
+                                      const float* bb, int64_t batch, int64_t n, int64_t c,
+                                      int32_t m, int32_t overlap, void* out, kvc_dtype out_dtype,
+                                      kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (!Ca || !za || !ba || !out) return KVC_ERR_NULL;
+  if (overlap && (!Cb || !zb || !bb)) return KVC_ERR_NULL;
+  const uintptr_t es = in_dtype == KVC_BF16 ? 2 : 4;
+  if (!aligned(Ca, 16) || !aligned(out, 16) || !aligned(za, es) || !aligned(ba, 4))
+    return KVC_ERR_ALIGN;
+  if (overlap && (!aligned(Cb, 16) || !aligned(zb, es) || !aligned(bb, 4))) return KVC_ERR_ALIGN;
+  if ((overlap ? 2 * m : m) > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  {
+    const void* ps[7] = {Ca, za, ba, out, Cb, zb, bb};
+    s = check_ptrs(ps, overlap ? 7 : 4);
+    if (s != KVC_OK) return s;
+  }
+  StreamProblem p{};
+  p.C0 = Ca;
+  p.Z0 = za;
+  p.B0 = ba;
+  p.C1 = overlap ? Cb : nullptr;
+  p.Z1 = overlap ? zb : nullptr;
+  p.B1 = overlap ? bb : nullptr;
+  p.batch = batch;
+  p.n = n;
+  p.c = c;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = overlap != 0;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_scalar_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_scalar_logits(const void* C, const void* z, kvc_dtype in_dtype,
+                                      const float* b, int64_t batch, int64_t n, int64_t c,
+                                      int32_t m, void* out, kvc_dtype out_dtype,
+                                      kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (!C || !z || !b || !out) return KVC_ERR_NULL;
+  const uintptr_t es = in_dtype == KVC_BF16 ? 2 : 4;
+  if (!aligned(C, 16) || !aligned(out, 16) || !aligned(z, es) || !aligned(b, 4))
+    return KVC_ERR_ALIGN;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  {
+    const void* ps[4] = {C, z, b, out};
+    s = check_ptrs(ps, 4);
+    if (s != KVC_OK) return s;
+  }
+  StreamProblem p{};
+  p.C0 = C;
+  p.Z0 = z;
+  p.B0 = b;
+  p.batch = batch;
+  p.n = n;
+  p.c = c;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_scalar_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Common checks of the entry-list calls; fills the list fields of p.
+static kvc_status check_list(StreamProblem* p, int64_t total_rows, int64_t c, int32_t m,
+                             const int64_t* seq_start, const int64_t* seq_len,
+                             const int64_t* entry, int64_t num, bool* empty) {
+  *empty = false;
+  if (total_rows < 0 || c < 0 || m < 1 || num < 0) return KVC_ERR_SHAPE;
+  int64_t t = 0;
+  if (!mul_ok(total_rows, c, &t) || !mul_ok(t, 4, &t) || !mul_ok(num, c, &t)) return KVC_ERR_SHAPE;
+  if (num == 0 || c == 0) {
+    *empty = true;
+    return KVC_OK;
+  }
+  if (c % 8 != 0) return KVC_ERR_SHAPE;
+  if (!seq_start || !seq_len || !entry) return KVC_ERR_NULL;
+  if (!aligned(seq_start, 8) || !aligned(seq_len, 8) || !aligned(entry, 8)) return KVC_ERR_ALIGN;
+  p->listed = true;
+  p->seq_start = seq_start;
+  p->seq_len = seq_len;
+  p->entry = entry;
+  p->num = num;
+  p->total_rows = total_rows;
+  p->batch = 1;
+  p->n = total_rows;
+  p->c = c;
+  p->ne = num;
+  p->m = m;
+  return KVC_OK;
+}
+
+kvc_status csa_compress_entries(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                                kvc_dtype in_dtype, const float* Ba, const float* Bb,
+                                int64_t total_rows, int64_t c, int32_t m, int32_t overlap,
+                                const int64_t* seq_start, const int64_t* seq_len,
+                                const int64_t* entry, int64_t num, void* out,
+                                kvc_dtype out_dtype, kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  StreamProblem p{};
+  bool empty = false;
+  kvc_status s = check_list(&p, total_rows, c, m, seq_start, seq_len, entry, num, &empty);
+  if (s != KVC_OK || empty) return s;
+  if (!Ca || !Za || !Ba || !out) return KVC_ERR_NULL;
+  if (overlap && (!Cb || !Zb || !Bb)) return KVC_ERR_NULL;
+  if (!aligned(Ca, 16) || !aligned(Za, 16) || !aligned(out, 16) || !aligned(Ba, 4))
+    return KVC_ERR_ALIGN;
+  if (overlap && (!aligned(Cb, 16) || !aligned(Zb, 16) || !aligned(Bb, 4))) return KVC_ERR_ALIGN;
+  const bool small = (m == 1 || m == 2 || m == 4);
+  if (!small && (overlap ? 2 * m : m) > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  {
+    const void* ps[10] = {Ca, Za, Ba, out, seq_start, seq_len, entry, Cb, Zb, Bb};
+    s = check_ptrs(ps, overlap ? 10 : 7);
+    if (s != KVC_OK) return s;
+  }
+  p.C0 = Ca;
+  p.Z0 = Za;
+  p.B0 = Ba;
+  p.C1 = overlap ? Cb : nullptr;
+  p.Z1 = overlap ? Zb : nullptr;
+  p.B1 = overlap ? Bb : nullptr;
+  p.two_segments = overlap != 0;
+  p.small_window_kernel = true;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
+                                int64_t total_rows, int64_t c, int32_t m, const int64_t* seq_start,
+                                const int64_t* seq_len, const int64_t* entry, int64_t num,
+                                void* out, kvc_dtype out_dtype, kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  StreamProblem p{};
+  bool empty = false;
+  kvc_status s = check_list(&p, total_rows, c, m, seq_start, seq_len, entry, num, &empty);
+  if (s != KVC_OK || empty) return s;
+  if (!C || !Z || !B || !out) return KVC_ERR_NULL;
+  if (!aligned(C, 16) || !aligned(Z, 16) || !aligned(out, 16) || !aligned(B, 4))
+    return KVC_ERR_ALIGN;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  {
+    const void* ps[7] = {C, Z, B, out, seq_start, seq_len, entry};
+    s = check_ptrs(ps, 7);
+    if (s != KVC_OK) return s;
+  }
+  p.C0 = C;
+  p.Z0 = Z;
+  p.B0 = B;
   p.two_segments = false;
   p.small_window_kernel = false;
   p.in_bf16 = in_dtype == KVC_BF16;

@@ -1,0 +1,52 @@
+// Host-side launch helpers shared by the kernel files (device attributes, occupancy).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <mutex>
+
+namespace kvc {
+
+struct DeviceInfo {
+  int sms = 0;
+  size_t smem_optin = 0;
+};
+
+// Multiprocessor count and opt-in shared memory of a device, queried once per device.
+inline DeviceInfo device_info(int dev) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return DeviceInfo{};
+  if (cache[dev].sms == 0) {
+    int sms = 0, optin = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return DeviceInfo{};
+    cache[dev].sms = sms;
+    cache[dev].smem_optin = static_cast<size_t>(optin);
+  }
+  return cache[dev];
+}
+
+// Resident CTAs per SM of kernel k at this block size and dynamic shared memory (0 on
+// error); raises the kernel's dynamic shared-memory limit when needed.
+template <typename Kernel>
+int resident_blocks(Kernel k, int threads, size_t smem) {
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return 0;
+  }
+  int blocks = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, threads, smem) != cudaSuccess)
+    return 0;
+  return blocks;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace kvc

@@ -24,9 +24,19 @@ struct StreamProblem {
   bool small_window_kernel;  // allow the one-thread-per-entry kernel for m in {1,2,4}
   bool in_bf16, out_bf16;
   void* out;
+  // Entry list (csa_compress_entries / hca_compress_entries): when `listed`, the kernel
+  // compresses entry entry[k] of the sequence at rows [seq_start[k], +seq_len[k]) of the
+  // packed streams (total_rows rows) into output row k, k < num; batch, n, ne unused.
+  bool listed;
+  const int64_t* seq_start;
+  const int64_t* seq_len;
+  const int64_t* entry;
+  int64_t num, total_rows;
 };
 
 kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st);
+// Scalar-logit form: Z0 / Z1 point at [batch, n] logits, B0 / B1 at [m] biases.
+kvc_status launch_scalar_pool(const StreamProblem& p, cudaStream_t st);
 size_t window_kernel_smem_bytes(bool bf16_in, bool two_segments, int m);
 
 // A validated fused problem: H [batch*n, d] bf16, W_s [d, c] bf16 (s = streams).
@@ -45,7 +55,10 @@ struct FusedProblem {
 
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st);
 
-// Device error word set by kernels whose bounded waits give up.
+// Device error words: bounded waits that gave up (fused kernels) and listed entries out
+// of range (streaming kernels).  Synchronises the stream first.
 kvc_status read_and_clear_device_error(cudaStream_t st);
+// Reads and clears the listed-entry error word (no synchronisation); true if it was set.
+bool read_and_clear_index_error(bool* failed);
 
 }  // namespace kvc

@@ -1,0 +1,174 @@
+// Scalar-logit compressor kernels (sm_100a).
+//
+// What they compute ("Ch 04 · CSA" §3, symbol table: one score per token and stream,
+// an m-dimensional position bias, S_j a scalar weight on the whole vector C_j; "Ch 05 ·
+// HCA" §2 likewise with an m'-dimensional bias): for entry i the window's logits are
+// [z^a_{mi..m(i+1)-1} + b^a ; z^b_{m(i-1)..mi-1} + b^b] (HCA: z + b over the segment),
+// one softmax over them, and C^Comp_i = sum_j S_j C_j with the same weights for every
+// channel.  Entry 0 has no b-rows (eq. attn-seqcomp-overlap-bound of "序列压缩注意力").
+//
+// One warp = one entry x a slab of 32 channel vectors (256 bf16 / 128 fp32 channels).
+// The warp first turns the window's scalar logits into weights (lanes split the rows;
+// shuffle max and sum; one exp2 per row), keeps them in shared memory, then every lane
+// streams its 16-byte vector of each window row (8 rows in flight) and accumulates the
+// weighted sum with packed f32x2 FMAs.  HBM-bound: the value streams are read once.
+#include "kvc_common.cuh"
+#include "kvc_host.h"
+#include "kvc_launch.h"
+
+namespace kvc {
+
+namespace {
+
+struct ScalarArgs {
+  const void* C0;  // value stream of segment 0 (C^a / the HCA stream)
+  const void* Z0;  // scalar logits of segment 0 [batch, n]
+  const void* C1;  // segment 1 (b-rows), TWO_SEG only
+  const void* Z1;
+  const float* B0;  // [m]
+  const float* B1;  // [m], TWO_SEG only
+  int64_t batch, n, c, ne;
+  int m;
+  void* out;
+};
+
+constexpr int kScWarps = 8;  // warps per CTA
+constexpr int kScU = 8;      // rows in flight per lane
+
+template <typename T>
+__device__ __forceinline__ float load_scalar(const T* p);
+template <>
+__device__ __forceinline__ float load_scalar<float>(const float* p) {
+  return __ldg(p);
+}
+template <>
+__device__ __forceinline__ float load_scalar<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+template <typename InT, typename OutT, bool TWO_SEG>
+__global__ void __launch_bounds__(kScWarps * 32) scalar_pool_kernel(ScalarArgs a) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int NP = CPT / 2;
+  extern __shared__ float smem_w[];  // [kScWarps][window rows] weights
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = a.m;
+  const int wmax = TWO_SEG ? 2 * m : m;
+  float* wts = smem_w + warp * wmax;
+  const InT* C0 = static_cast<const InT*>(a.C0);
+  const InT* Z0 = static_cast<const InT*>(a.Z0);
+  const InT* C1 = static_cast<const InT*>(a.C1);
+  const InT* Z1 = static_cast<const InT*>(a.Z1);
+  OutT* out = static_cast<OutT*>(a.out);
+  const int64_t G = a.c / CPT;               // channel vectors per row
+  const int64_t slabs = (G + 31) / 32;
+  const int64_t tasks = a.batch * a.ne * slabs;
+
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kScWarps + warp; t < tasks;
+       t += static_cast<int64_t>(gridDim.x) * kScWarps) {
+    const int64_t slab = t % slabs;
+    const int64_t e = t / slabs;
+    const int64_t b = e / a.ne, i = e - (e / a.ne) * a.ne;
+    const int64_t row0 = b * a.n + static_cast<int64_t>(m) * i;  // a-range(i) start
+    const int rows = (TWO_SEG && i > 0) ? 2 * m : m;
+
+    // weights of the window's rows (row v < m: segment 0; v >= m: segment 1)
+    float mx = -INFINITY;
+    for (int v = lane; v < rows; v += 32) {
+      const bool seg1 = TWO_SEG && v >= m;
+      const float z = seg1 ? load_scalar<InT>(Z1 + row0 - m + (v - m)) : load_scalar<InT>(Z0 + row0 + v);
+      const float l = fmaf(z, kLog2e, (seg1 ? a.B1[v - m] : a.B0[v]) * kLog2e);
+      wts[v] = l;
+      mx = fmaxf(mx, l);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+    for (int v = lane; v < rows; v += 32) {
+      const float w = ex2_ftz(wts[v] - mx);
+      wts[v] = w;
+      sum += w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.0f / sum;
+    __syncwarp();
+
+    const int64_t vec = slab * 32 + lane;
+    if (vec < G) {
+      const int64_t ch0 = vec * CPT;
+      float2 A[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) A[p] = make_float2(0.f, 0.f);
+      for (int v0 = 0; v0 < rows; v0 += kScU) {
+        uint4 cv[kScU];
+#pragma unroll
+        for (int u = 0; u < kScU; ++u) {
+          const int v = v0 + u;
+          if (v < rows) {
+            const bool seg1 = TWO_SEG && v >= m;
+            const int64_t row = seg1 ? row0 - m + (v - m) : row0 + v;
+            cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kScU; ++u) {
+          const int v = v0 + u;
+          if (v < rows) {
+            const float w = wts[v];
+            const float2 w2 = make_float2(w, w);
+#pragma unroll
+            for (int p = 0; p < NP; ++p) A[p] = f2_fma(w2, vec_pair<InT>(cv[u], p), A[p]);
+          }
+        }
+      }
+      float res[CPT];
+      const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const float2 r = f2_mul(A[p], inv2);
+        res[2 * p] = r.x;
+        res[2 * p + 1] = r.y;
+      }
+      store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
+    }
+    __syncwarp();  // the next task overwrites this warp's weights
+  }
+}
+
+template <typename InT, typename OutT, bool TWO_SEG>
+kvc_status launch(const StreamProblem& p, cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (di.sms == 0) return KVC_ERR_CUDA;
+  const size_t smem = sizeof(float) * kScWarps * (TWO_SEG ? 2 * p.m : p.m);
+  auto kern = scalar_pool_kernel<InT, OutT, TWO_SEG>;
+  const int occ = resident_blocks(kern, kScWarps * 32, smem);
+  if (occ == 0) return KVC_ERR_CUDA;
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  const int64_t tasks = p.batch * p.ne * ceil_div(p.c / CPT, 32);
+  int64_t grid = static_cast<int64_t>(di.sms) * occ;
+  const int64_t need = ceil_div(tasks, kScWarps);
+  if (grid > need) grid = need;
+  ScalarArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
+  kern<<<static_cast<unsigned>(grid), kScWarps * 32, smem, st>>>(args);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+template <typename InT, typename OutT>
+kvc_status dispatch(const StreamProblem& p, cudaStream_t st) {
+  return p.two_segments ? launch<InT, OutT, true>(p, st) : launch<InT, OutT, false>(p, st);
+}
+
+}  // namespace
+
+kvc_status launch_scalar_pool(const StreamProblem& p, cudaStream_t st) {
+  if (p.in_bf16) {
+    return p.out_bf16 ? dispatch<__nv_bfloat16, __nv_bfloat16>(p, st)
+                      : dispatch<__nv_bfloat16, float>(p, st);
+  }
+  return p.out_bf16 ? dispatch<float, __nv_bfloat16>(p, st) : dispatch<float, float>(p, st);
+}
+
+}  // namespace kvc

@@ -14,17 +14,41 @@
 // (one exp2 per element), and chunked online (max, sum, acc) with a shared-memory
 // merge across row groups for long windows (HCA m' = 128).
 #include "kvc_common.cuh"
+#include "kvc_host.h"
 #include "kvc_launch.h"
 
 #include <math.h>
 
-#include <mutex>
 
 namespace kvc {
 
 // ---------------------------------------------------------------------------------
 // CSA, small m (1, 2, 4): one thread = one entry x one 16-byte channel vector.
 // ---------------------------------------------------------------------------------
+// Set when an entry list read from device memory names a window outside its sequence or
+// the streams (that entry is skipped); read and cleared by kvc_device_status().
+__device__ unsigned int g_index_error = 0;
+
+// Entry lists (decode / ragged batches): entry k reads the sequence whose rows start at
+// seq_start[k] (seq_len[k] rows) and is that sequence's entry entry[k]; its output row is k.
+struct EntryList {
+  const int64_t* seq_start;
+  const int64_t* seq_len;
+  const int64_t* entry;
+  int64_t num, total_rows;
+};
+
+// Checks one listed entry against its sequence and the streams; on success gives the first
+// a-row and whether it is the sequence's entry 0.
+__device__ __forceinline__ bool listed_entry(const EntryList& L, int64_t k, int m, int64_t* rowA,
+                                             bool* first) {
+  const int64_t s0 = L.seq_start[k], len = L.seq_len[k], e = L.entry[k];
+  if (!(s0 >= 0 && len >= 0 && s0 <= L.total_rows - len && e >= 0 && e < len / m)) return false;
+  *rowA = s0 + static_cast<int64_t>(m) * e;
+  *first = e == 0;
+  return true;
+}
+
 struct CsaSmallArgs {
   const void* Ca;
   const void* Cb;
@@ -34,9 +58,10 @@ struct CsaSmallArgs {
   const float* Bb;
   int64_t batch, n, c, ne;
   void* out;
+  EntryList list;
 };
 
-template <typename InT, typename OutT, int M, bool OVERLAP>
+template <typename InT, typename OutT, int M, bool OVERLAP, bool LISTED>
 __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
   constexpr int CPT = VecInfo<InT>::kChannels;
   constexpr int NP = CPT / 2;              // channel pairs per thread
@@ -73,10 +98,24 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
   const uint4 c_boundary = make_uint4(0u, 0u, 0u, 0u);
 
   const int64_t istep = static_cast<int64_t>(gridDim.y) * blockDim.y;
+  const int64_t lim = LISTED ? a.list.num : a.ne;
   for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
-    for (int64_t i = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; i < a.ne;
+    for (int64_t i = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; i < lim;
          i += istep) {
-      const int64_t rowA = b * a.n + static_cast<int64_t>(M) * i;  // a-range(i) start
+      int64_t rowA;  // a-range start of the entry
+      bool first;    // entry 0 of its sequence: no b-rows
+      int64_t orow;  // output row
+      if constexpr (LISTED) {
+        if (!listed_entry(a.list, i, M, &rowA, &first)) {
+          if (threadIdx.x == 0) atomicOr(&g_index_error, 1u);
+          continue;
+        }
+        orow = i;
+      } else {
+        rowA = b * a.n + static_cast<int64_t>(M) * i;
+        first = i == 0;
+        orow = b * a.ne + i;
+      }
       uint4 za[M], ca[M], zb[M], cb[M];
 #pragma unroll
       for (int k = 0; k < M; ++k) {
@@ -84,7 +123,7 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
         ca[k] = ld_stream16(Ca + (rowA + k) * a.c + ch0);
       }
       if constexpr (OVERLAP) {
-        if (i > 0) {  // b-range(i) = a-range(i-1)
+        if (!first) {  // b-range(i) = a-range(i-1)
 #pragma unroll
           for (int k = 0; k < M; ++k) {
             zb[k] = ld_stream16(Zb + (rowA - M + k) * a.c + ch0);
@@ -137,7 +176,7 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
         res[2 * p] = __fdividef(acc.x, s.x);
         res[2 * p + 1] = __fdividef(acc.y, s.y);
       }
-      store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
+      store_out<OutT, CPT>(out + orow * a.c + ch0, res);
     }
   }
 }
@@ -162,6 +201,7 @@ struct WinArgs {
   int64_t batch, n, c, ne;
   int m;
   void* out;
+  EntryList list;
 };
 
 constexpr int kWinCG = 16;  // channel vectors per CTA
@@ -180,8 +220,9 @@ size_t win_smem_bytes(int m, int rg) {
   return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + partial);
 }
 
-template <typename InT, typename OutT, bool TWO_SEG, int RG>
+template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED>
 __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
+  static_assert(!LISTED || RG == 1, "entry lists use one window per thread");
   constexpr int CPT = VecInfo<InT>::kChannels;
   constexpr int SC = win_slab<InT>();
   constexpr int EY = kWinTY / RG;  // entries per CTA iteration
@@ -219,12 +260,28 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
   const int m = a.m;
 
   for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
-    for (int64_t i0 = static_cast<int64_t>(blockIdx.y) * EY; i0 < a.ne;
+    const int64_t lim = LISTED ? a.list.num : a.ne;
+    for (int64_t i0 = static_cast<int64_t>(blockIdx.y) * EY; i0 < lim;
          i0 += static_cast<int64_t>(gridDim.y) * EY) {
       const int64_t i = i0 + es;
-      const bool live = active && i < a.ne;
-      const int64_t row0 = b * a.n + static_cast<int64_t>(m) * i;
-      const int rows_i = (TWO_SEG && i > 0) ? 2 * m : m;
+      bool live = active && i < lim;
+      int64_t row0 = 0;    // first row of the entry's own segment
+      bool first = false;  // entry 0 of its sequence
+      int64_t orow = 0;    // output row
+      if constexpr (LISTED) {
+        if (i < lim) {
+          if (!listed_entry(a.list, i, m, &row0, &first)) {
+            if (tx == 0) atomicOr(&g_index_error, 1u);
+            live = false;
+          }
+          orow = i;
+        }
+      } else {
+        row0 = b * a.n + static_cast<int64_t>(m) * i;
+        first = i == 0;
+        orow = b * a.ne + i;
+      }
+      const int rows_i = (TWO_SEG && !first) ? 2 * m : m;
       float2 M[NP], S[NP], A[NP];  // per channel pair: running max, sum, weighted sum
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
@@ -306,7 +363,7 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
             res[2 * p] = __fdividef(A[p].x, S[p].x);
             res[2 * p + 1] = __fdividef(A[p].y, S[p].y);
           }
-          store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
+          store_out<OutT, CPT>(out + orow * a.c + ch0, res);
         }
       } else {
 #pragma unroll
@@ -348,44 +405,11 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
 // ---------------------------------------------------------------------------------
 namespace {
 
-struct DeviceInfo {
-  int sms = 0;
-  size_t smem_optin = 0;
-};
-
-DeviceInfo device_info(int dev) {
-  static std::mutex mu;
-  static DeviceInfo cache[64];
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev < 0 || dev >= 64) return DeviceInfo{};
-  if (cache[dev].sms == 0) {
-    int sms = 0, optin = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-            cudaSuccess)
-      return DeviceInfo{};
-    cache[dev].sms = sms;
-    cache[dev].smem_optin = static_cast<size_t>(optin);
-  }
-  return cache[dev];
+EntryList entry_list(const StreamProblem& p) {
+  return EntryList{p.seq_start, p.seq_len, p.entry, p.num, p.total_rows};
 }
 
-template <typename Kernel>
-int resident_blocks(Kernel k, int threads, size_t smem) {
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return 0;
-  }
-  int blocks = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, threads, smem) != cudaSuccess)
-    return 0;
-  return blocks;
-}
-
-int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
-template <typename InT, typename OutT, int M, bool OVERLAP>
+template <typename InT, typename OutT, int M, bool OVERLAP, bool LISTED>
 kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
   constexpr int CPT = VecInfo<InT>::kChannels;
   const int64_t G = p.c / CPT;  // channel vectors
@@ -393,46 +417,50 @@ kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
   const int ey = 256 / cg;
   const dim3 block(cg, ey);
   const size_t smem = sizeof(float) * (OVERLAP ? 2 * M : M) * cg * CPT;
-  auto kern = csa_small_m_kernel<InT, OutT, M, OVERLAP>;
+  auto kern = csa_small_m_kernel<InT, OutT, M, OVERLAP, LISTED>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
   const DeviceInfo di = device_info(dev);
   const int occ = resident_blocks(kern, cg * ey, smem);
   if (di.sms == 0 || occ == 0) return KVC_ERR_CUDA;
   const int64_t gx = ceil_div(G, cg);
-  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
+  const int64_t batch = LISTED ? 1 : p.batch;
+  const int64_t gz = batch < 65535 ? batch : 65535;
   int64_t want = static_cast<int64_t>(di.sms) * occ;  // one resident wave
   int64_t gy = want / (gx * gz);
   if (gy < 1) gy = 1;
-  const int64_t need = ceil_div(p.ne, ey);
+  const int64_t need = ceil_div(LISTED ? p.num : p.ne, ey);
   if (gy > need) gy = need;
   if (gy > 65535) gy = 65535;
   // Balance: every CTA row gets the same number of entry iterations (+-1).
   gy = ceil_div(need, ceil_div(need, gy));
-  CsaSmallArgs args{p.C0, p.C1, p.Z0, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.out};
+  CsaSmallArgs args{p.C0, p.C1, p.Z0, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.out,
+                    entry_list(p)};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
          block, smem, st>>>(args);
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
-template <typename InT, typename OutT, bool TWO_SEG, int RG>
+template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED>
 kvc_status launch_window_rg(const StreamProblem& p, cudaStream_t st, const DeviceInfo& di) {
   constexpr int SC = win_slab<InT>();
   constexpr int EY = kWinTY / RG;
   const size_t smem = win_smem_bytes<InT, TWO_SEG>(p.m, RG);
   if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
-  auto kern = window_pool_kernel<InT, OutT, TWO_SEG, RG>;
+  auto kern = window_pool_kernel<InT, OutT, TWO_SEG, RG, LISTED>;
   const int occ = resident_blocks(kern, kWinCG * kWinTY, smem);
   if (occ == 0) return KVC_ERR_CUDA;
   const int64_t gx = ceil_div(p.c, SC);
-  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
-  const int64_t need = ceil_div(p.ne, EY);
+  const int64_t batch = LISTED ? 1 : p.batch;
+  const int64_t gz = batch < 65535 ? batch : 65535;
+  const int64_t need = ceil_div(LISTED ? p.num : p.ne, EY);
   int64_t gy = static_cast<int64_t>(di.sms) * occ / (gx * gz);
   if (gy < 1) gy = 1;
   if (gy > need) gy = need;
   if (gy > 65535) gy = 65535;
   gy = ceil_div(need, ceil_div(need, gy));
-  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
+  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.m, p.out,
+               entry_list(p)};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
          dim3(kWinCG, kWinTY), smem, st>>>(args);
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
@@ -440,41 +468,51 @@ kvc_status launch_window_rg(const StreamProblem& p, cudaStream_t st, const Devic
 
 // Row groups per entry: the fewest that still give every resident CTA slot a few
 // iterations (one window per thread needs no merge at all).
-template <typename InT, typename OutT, bool TWO_SEG>
+template <typename InT, typename OutT, bool TWO_SEG, bool LISTED>
 kvc_status launch_window(const StreamProblem& p, cudaStream_t st) {
   constexpr int SC = win_slab<InT>();
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
   const DeviceInfo di = device_info(dev);
   if (di.sms == 0) return KVC_ERR_CUDA;
-  const int64_t tasks = p.batch * p.ne * ceil_div(p.c, SC);  // (entry, slab) pairs
-  const int64_t slots = static_cast<int64_t>(di.sms) * 2;
-  const int rows = TWO_SEG ? 2 * p.m : p.m;
-  if (tasks >= 3 * slots * kWinTY || rows <= kWinU)
-    return launch_window_rg<InT, OutT, TWO_SEG, 1>(p, st, di);
-  if (tasks >= 3 * slots * (kWinTY / 4)) return launch_window_rg<InT, OutT, TWO_SEG, 4>(p, st, di);
-  return launch_window_rg<InT, OutT, TWO_SEG, 16>(p, st, di);
+  if constexpr (LISTED) {
+    return launch_window_rg<InT, OutT, TWO_SEG, 1, true>(p, st, di);
+  } else {
+    const int64_t tasks = p.batch * p.ne * ceil_div(p.c, SC);  // (entry, slab) pairs
+    const int64_t slots = static_cast<int64_t>(di.sms) * 2;
+    const int rows = TWO_SEG ? 2 * p.m : p.m;
+    if (tasks >= 3 * slots * kWinTY || rows <= kWinU)
+      return launch_window_rg<InT, OutT, TWO_SEG, 1, false>(p, st, di);
+    if (tasks >= 3 * slots * (kWinTY / 4))
+      return launch_window_rg<InT, OutT, TWO_SEG, 4, false>(p, st, di);
+    return launch_window_rg<InT, OutT, TWO_SEG, 16, false>(p, st, di);
+  }
 }
 
-template <typename InT, typename OutT>
+template <typename InT, typename OutT, bool LISTED>
 kvc_status dispatch_stream(const StreamProblem& p, cudaStream_t st) {
   if (p.two_segments) {
     switch (p.m) {
-      case 1: return launch_csa_small<InT, OutT, 1, true>(p, st);
-      case 2: return launch_csa_small<InT, OutT, 2, true>(p, st);
-      case 4: return launch_csa_small<InT, OutT, 4, true>(p, st);
-      default: return launch_window<InT, OutT, true>(p, st);
+      case 1: return launch_csa_small<InT, OutT, 1, true, LISTED>(p, st);
+      case 2: return launch_csa_small<InT, OutT, 2, true, LISTED>(p, st);
+      case 4: return launch_csa_small<InT, OutT, 4, true, LISTED>(p, st);
+      default: return launch_window<InT, OutT, true, LISTED>(p, st);
     }
   }
   if (p.small_window_kernel) {
     switch (p.m) {
-      case 1: return launch_csa_small<InT, OutT, 1, false>(p, st);
-      case 2: return launch_csa_small<InT, OutT, 2, false>(p, st);
-      case 4: return launch_csa_small<InT, OutT, 4, false>(p, st);
+      case 1: return launch_csa_small<InT, OutT, 1, false, LISTED>(p, st);
+      case 2: return launch_csa_small<InT, OutT, 2, false, LISTED>(p, st);
+      case 4: return launch_csa_small<InT, OutT, 4, false, LISTED>(p, st);
       default: break;
     }
   }
-  return launch_window<InT, OutT, false>(p, st);
+  return launch_window<InT, OutT, false, LISTED>(p, st);
+}
+
+template <typename InT, typename OutT>
+kvc_status dispatch_listed(const StreamProblem& p, cudaStream_t st) {
+  return p.listed ? dispatch_stream<InT, OutT, true>(p, st) : dispatch_stream<InT, OutT, false>(p, st);
 }
 
 }  // namespace
@@ -488,11 +526,20 @@ size_t window_kernel_smem_bytes(bool bf16_in, bool two_segments, int m) {
 
 kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st) {
   if (p.in_bf16) {
-    return p.out_bf16 ? dispatch_stream<__nv_bfloat16, __nv_bfloat16>(p, st)
-                      : dispatch_stream<__nv_bfloat16, float>(p, st);
+    return p.out_bf16 ? dispatch_listed<__nv_bfloat16, __nv_bfloat16>(p, st)
+                      : dispatch_listed<__nv_bfloat16, float>(p, st);
   }
-  return p.out_bf16 ? dispatch_stream<float, __nv_bfloat16>(p, st)
-                    : dispatch_stream<float, float>(p, st);
+  return p.out_bf16 ? dispatch_listed<float, __nv_bfloat16>(p, st)
+                    : dispatch_listed<float, float>(p, st);
+}
+
+bool read_and_clear_index_error(bool* failed) {
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  *failed = cudaMemcpyFromSymbol(&v, g_index_error, sizeof(v)) != cudaSuccess;
+  if (!*failed && v != 0)
+    *failed = cudaMemcpyToSymbol(g_index_error, &zero, sizeof(zero)) != cudaSuccess;
+  return v != 0;
 }
 
 }  // namespace kvc

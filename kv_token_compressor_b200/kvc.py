@@ -24,6 +24,7 @@ KVC_ERR_UNSUPPORTED = 5
 KVC_ERR_CUDA = 6
 KVC_ERR_TIMEOUT = 7
 KVC_ERR_POINTER = 8
+KVC_ERR_INDEX = 9
 # kvc_dtype
 KVC_F32 = 0
 KVC_BF16 = 1
@@ -42,6 +43,14 @@ SIGNATURES = {
     "hca_compress_fused_proj": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32, _p,
                                                ctypes.c_int, _p]),
     "kvc_device_status": (ctypes.c_int, [_p]),
+    "csa_compress_scalar_logits": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64,
+                                                  _i64, _i32, _i32, _p, ctypes.c_int, _p]),
+    "hca_compress_scalar_logits": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i32,
+                                                  _p, ctypes.c_int, _p]),
+    "csa_compress_entries": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64, _i32,
+                                            _i32, _p, _p, _p, _i64, _p, ctypes.c_int, _p]),
+    "hca_compress_entries": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i32, _p, _p, _p,
+                                            _i64, _p, ctypes.c_int, _p]),
 }
 
 _lib = None
@@ -146,6 +155,75 @@ def hca_compress(C, Z, B, m: int = 128, out=None, out_dtype=None, stream=None):
     st = lib().hca_compress(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
                             _ptr(out), _dtype_code(out_dtype), _stream(stream))
     _check(st, "hca_compress")
+    return out
+
+
+def csa_compress_scalar_logits(Ca, Cb, za, zb, ba, bb, m: int = 4, overlap: bool = True, out=None,
+                               out_dtype=None, stream=None):
+    """Scalar-logit CSA: streams Ca, Cb [batch, n, c], logits za, zb [batch, n] (same dtype),
+    fp32 biases ba, bb [m].  Returns [batch, n // m, c]."""
+    batch, n, c = Ca.shape
+    if tuple(za.shape) != (batch, n) or za.dtype != Ca.dtype:
+        raise ValueError("za must be [batch, n] with the streams' dtype")
+    out_dtype = Ca.dtype if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, Ca)
+    st = lib().csa_compress_scalar_logits(
+        _ptr(Ca), _ptr(Cb) if overlap else None, _ptr(za), _ptr(zb) if overlap else None,
+        _dtype_code(Ca.dtype), _ptr(ba), _ptr(bb) if overlap else None, batch, n, c, m,
+        int(bool(overlap)), _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "csa_compress_scalar_logits")
+    return out
+
+
+def hca_compress_scalar_logits(C, z, b, m: int = 128, out=None, out_dtype=None, stream=None):
+    """Scalar-logit HCA: C [batch, n, c], logits z [batch, n], fp32 bias b [m]."""
+    batch, n, c = C.shape
+    if tuple(z.shape) != (batch, n) or z.dtype != C.dtype:
+        raise ValueError("z must be [batch, n] with C's dtype")
+    out_dtype = C.dtype if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, C)
+    st = lib().hca_compress_scalar_logits(_ptr(C), _ptr(z), _dtype_code(C.dtype), _ptr(b), batch, n,
+                                          c, m, _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "hca_compress_scalar_logits")
+    return out
+
+
+def _index(t, num):
+    torch = _torch()
+    if t.dtype != torch.int64 or tuple(t.shape) != (num,):
+        raise ValueError("index arrays must be int64 [num]")
+    return _ptr(t)
+
+
+def csa_compress_entries(Ca, Cb, Za, Zb, Ba, Bb, seq_start, seq_len, entry, m: int = 4,
+                         overlap: bool = True, out=None, out_dtype=None, stream=None):
+    """CSA entries listed by device int64 arrays (seq_start, seq_len, entry) over packed
+    streams [total_rows, c].  Returns [num, c]; row k is entry entry[k] of its sequence."""
+    total_rows, c = Ca.shape
+    num = entry.shape[0]
+    out_dtype = Ca.dtype if out_dtype is None else out_dtype
+    out = _out(out, (num, c), out_dtype, Ca)
+    st = lib().csa_compress_entries(
+        _ptr(Ca), _ptr(Cb) if overlap else None, _ptr(Za), _ptr(Zb) if overlap else None,
+        _dtype_code(Ca.dtype), _ptr(Ba), _ptr(Bb) if overlap else None, total_rows, c, m,
+        int(bool(overlap)), _index(seq_start, num), _index(seq_len, num), _index(entry, num), num,
+        _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "csa_compress_entries")
+    return out
+
+
+def hca_compress_entries(C, Z, B, seq_start, seq_len, entry, m: int = 128, out=None,
+                         out_dtype=None, stream=None):
+    """HCA entries listed by device int64 arrays over packed streams [total_rows, c]."""
+    total_rows, c = C.shape
+    num = entry.shape[0]
+    out_dtype = C.dtype if out_dtype is None else out_dtype
+    out = _out(out, (num, c), out_dtype, C)
+    st = lib().hca_compress_entries(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), total_rows, c,
+                                    m, _index(seq_start, num), _index(seq_len, num),
+                                    _index(entry, num), num, _ptr(out), _dtype_code(out_dtype),
+                                    _stream(stream))
+    _check(st, "hca_compress_entries")
     return out
 
 

@@ -31,6 +31,8 @@ __all__ = [
     "fused_inputs",
     "stream_inputs_torch",
     "fused_inputs_torch",
+    "scalar_inputs",
+    "scalar_inputs_torch",
     "WORKLOADS",
 ]
 
@@ -138,6 +140,43 @@ def fused_inputs_torch(mode: str, batch: int, n: int, d: int, c: int, m: int, se
                   * float(1.0 / np.sqrt(d))).to(torch.bfloat16)
     for k in (("Ba", "Bb") if mode == "csa" else ("B",)):
         out[k] = torch.randn((m, c), generator=g, device=device, dtype=torch.float32) * float(np.sqrt(bias_var))
+    return out
+
+
+def scalar_inputs(mode: str, batch: int, n: int, c: int, m: int, dtype: str = "f32", seed: int = 0,
+                  z_scale: float = 2.0, bias_var: float = 0.1):
+    """Host inputs for the scalar-logit form: value streams [batch, n, c] N(0, 1), one logit
+    per token and stream [batch, n] N(0, z_scale^2), biases [m] N(0, bias_var).
+    mode "csa": Ca, Cb, za, zb, ba, bb;  mode "hca": C, z, b."""
+    rng = np.random.default_rng(seed)
+    vals = ("Ca", "Cb") if mode == "csa" else ("C",)
+    logs = ("za", "zb") if mode == "csa" else ("z",)
+    out = {k: _normal(rng, (batch, n, c)) for k in vals}
+    for k in logs:
+        out[k] = (_normal(rng, (batch, n)) * np.float32(z_scale)).astype(np.float32)
+    if dtype == "bf16":
+        for k in vals + logs:
+            out[k] = round_to_bf16(out[k])
+    for k in (("ba", "bb") if mode == "csa" else ("b",)):
+        out[k] = _normal(rng, (m,), bias_var)
+    return out
+
+
+def scalar_inputs_torch(mode: str, batch: int, n: int, c: int, m: int, dtype: str, seed: int = 0,
+                        z_scale: float = 2.0, bias_var: float = 0.1, device="cuda"):
+    """Same distributions as :func:`scalar_inputs`, generated on ``device``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    vals = ("Ca", "Cb") if mode == "csa" else ("C",)
+    logs = ("za", "zb") if mode == "csa" else ("z",)
+    out = {k: torch.randn((batch, n, c), generator=g, device=device).to(tdt) for k in vals}
+    for k in logs:
+        out[k] = (torch.randn((batch, n), generator=g, device=device) * z_scale).to(tdt)
+    for k in (("ba", "bb") if mode == "csa" else ("b",)):
+        out[k] = torch.randn((m,), generator=g, device=device) * float(np.sqrt(bias_var))
     return out
 
 

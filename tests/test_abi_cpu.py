@@ -60,7 +60,7 @@ def test_num_entries_bit_exact(L):
 
 
 def test_status_strings(L):
-    for code in range(9):
+    for code in range(10):
         s = kvc.status_string(code)
         assert s.startswith("KVC_")
     assert kvc.status_string(99) == "KVC_ERR_UNKNOWN"
@@ -182,3 +182,41 @@ def test_fused_hca_rejects_before_launch(L, kw, status):
 def test_fused_empty(L):
     assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
     assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK
+
+
+def csa_sc(L, **kw):
+    a = dict(Ca=A, Cb=A, za=A, zb=A, in_dt=kvc.KVC_BF16, ba=A, bb=A, batch=1, n=1024, c=512, m=4,
+             overlap=1, out=A, out_dt=kvc.KVC_BF16)
+    a.update(kw)
+    return L.csa_compress_scalar_logits(a["Ca"], a["Cb"], a["za"], a["zb"], a["in_dt"], a["ba"], a["bb"],
+                                        a["batch"], a["n"], a["c"], a["m"], a["overlap"], a["out"],
+                                        a["out_dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dt=9), kvc.KVC_ERR_DTYPE),
+    (dict(n=-1), kvc.KVC_ERR_SHAPE),
+    (dict(c=12), kvc.KVC_ERR_SHAPE),
+    (dict(overlap=5), kvc.KVC_ERR_SHAPE),
+    (dict(za=None), kvc.KVC_ERR_NULL),
+    (dict(bb=None), kvc.KVC_ERR_NULL),
+    (dict(Ca=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(za=A + 1), kvc.KVC_ERR_ALIGN),
+    (dict(in_dt=kvc.KVC_F32, za=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(m=161), kvc.KVC_ERR_UNSUPPORTED),
+])
+def test_csa_scalar_rejects_before_launch(L, kw, status):
+    assert csa_sc(L, **kw) == status
+
+
+def test_scalar_logit_misc(L):
+    # za may sit at any 2-byte offset for bf16 (no 16-byte rule for the logits)
+    assert csa_sc(L, za=A + 2, Ca=MIS) == kvc.KVC_ERR_ALIGN  # fails on Ca, not on za
+    assert csa_sc(L, overlap=0, Cb=None, zb=None, bb=None, out=MIS) == kvc.KVC_ERR_ALIGN
+    assert csa_sc(L, n=2, Ca=None, za=None, out=None) == kvc.KVC_OK
+    assert L.hca_compress_scalar_logits(A, None, kvc.KVC_BF16, A, 1, 256, 512, 128, A, kvc.KVC_BF16,
+                                        None) == kvc.KVC_ERR_NULL
+    assert L.hca_compress_scalar_logits(A, A, kvc.KVC_BF16, A, 1, 1024, 512, 400, A, kvc.KVC_BF16,
+                                        None) == kvc.KVC_ERR_UNSUPPORTED
+    assert L.hca_compress_scalar_logits(A, A, kvc.KVC_BF16, A, 1, 100, 512, 128, A, kvc.KVC_BF16,
+                                        None) == kvc.KVC_OK
