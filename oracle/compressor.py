@@ -52,6 +52,9 @@ __all__ = [
     "csa_compress_scalar",
     "hca_entry_scalar",
     "hca_compress_scalar",
+    "round_e4m3",
+    "rope_pairs",
+    "cache_format",
 ]
 
 
@@ -313,3 +316,58 @@ def hca_compress_scalar(C, z, bvec, m: int = 128, entries=None):
     rows = [hca_entry_scalar(C[b], z[b], bvec, i, m) for b, i in todo]
     res = np.array(rows, dtype=np.float64).reshape(len(todo), c)
     return res.reshape(batch, ne, c) if entries is None else res
+
+
+# --------------------------------------------------------------------------------------
+# Cache-format epilogue.  "Ch 05 · HCA" §4 (2): RoPE acts on the last r = 64 dimensions
+# of each entry only, rotating adjacent pairs of dimensions by a position-dependent angle,
+# the other c - r stay position-free; the segment position is carried approximately by
+# the rope dimensions (segment-centre RoPE).  The CSA/HCA comparison article (section
+# 三.4, mixed-precision storage) stores the RoPE part in BF16 and the other KV values in
+# FP8.  Readings (the pages fix neither): the caller supplies the inverse frequencies of
+# the r/2 pairs and the entry position pos_i = pos_offset + pos_stride * i; FP8 is
+# E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
+# finite 448), round to nearest even, saturating, after multiplying by a caller scale.
+# --------------------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x):
+    """Nearest FP8 E4M3 value (ties to even), saturating to +-448, as float64."""
+    x = _f64(x)
+    a = np.abs(x)
+    mant, expo = np.frexp(a)                 # a = mant * 2^expo, mant in [0.5, 1)
+    lead = expo - 1                          # exponent of the leading bit
+    quantum = np.ldexp(1.0, np.maximum(lead, -6) - 3)   # 3 mantissa bits; subnormal step 2^-9
+    q = np.round(a / quantum) * quantum      # numpy rounds half to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.where(a == 0, 0.0, np.copysign(q, x))
+
+
+def rope_pairs(x, pos, inv_freq):
+    """Rotate adjacent pairs (2j, 2j+1) of x [..., r] by angle pos * inv_freq[j]."""
+    x = _f64(x)
+    r = x.shape[-1]
+    ang = np.multiply.outer(_f64(pos), _f64(inv_freq))          # [..., r/2]
+    z = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * ang)  # one complex number per pair
+    out = np.empty_like(x)
+    out[..., 0::2] = z.real
+    out[..., 1::2] = z.imag
+    assert out.shape[-1] == r
+    return out
+
+
+def cache_format(entries, r: int, inv_freq, pos_stride: float, pos_offset: float,
+                 scale: float = 1.0):
+    """Split compressed entries [batch, N_e, c] into the cache layout: the first c - r
+    dimensions times `scale` rounded to E4M3, and the last r dimensions rotated at
+    pos_i = pos_offset + pos_stride * i (i = entry index in its sequence), float64."""
+    entries = _f64(entries)
+    c = entries.shape[-1]
+    ne = entries.shape[-2]
+    pos = pos_offset + pos_stride * np.arange(ne, dtype=np.float64)
+    pos = np.broadcast_to(pos, entries.shape[:-1])
+    nope = round_e4m3(entries[..., :c - r] * scale)
+    rope = rope_pairs(entries[..., c - r:], pos, inv_freq)
+    return nope, rope

@@ -493,4 +493,70 @@ def pin_scalar_one_hot_and_logistic(O):
     assert np.allclose(out[0, 1], C[0, 128 + 77], rtol=1e-12, atol=1e-12)
 
 
+# --------------------------------------------------------------------------------------
+# Cache-format epilogue: FP8 E4M3 rounding and pair-wise RoPE
+# --------------------------------------------------------------------------------------
+
+def _e4m3_codes():
+    """All finite non-negative E4M3 values decoded from the bit fields of the format
+    (4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 is subnormal;
+    exponent 15 with mantissa 7 is NaN), in code order."""
+    vals = []
+    for e in range(16):
+        for mm in range(8):
+            if e == 15 and mm == 7:
+                continue
+            vals.append(mm / 8 * 2.0 ** -6 if e == 0 else (1 + mm / 8) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def pin_e4m3_rounding(O):
+    v = _e4m3_codes()
+    assert v[-1] == 448.0 and v[1] == 2.0 ** -9
+    assert np.array_equal(O.round_e4m3(v), v) and np.array_equal(O.round_e4m3(-v), -v)
+    mids = (v[:-1] + v[1:]) / 2
+    got = O.round_e4m3(mids)
+    for k, g in enumerate(got):       # ties go to the even code
+        assert g == (v[k] if k % 2 == 0 else v[k + 1]), (k, mids[k], g)
+    inside = (v[:-1] + 0.49 * (v[1:] - v[:-1]))
+    assert np.array_equal(O.round_e4m3(inside), v[:-1])
+    assert np.all(O.round_e4m3(np.array([449.0, 1e6, -5e3])) == np.array([448.0, 448.0, -448.0]))
+    import torch  # library cast (saturation excluded: torch maps overflow to NaN)
+    x = np.random.default_rng(40).standard_normal(20000) * 40
+    x = np.clip(x, -448, 448)
+    t = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(O.round_e4m3(x), t)
+
+
+def pin_rope_closed_forms(O):
+    rng = np.random.default_rng(41)
+    r = 8
+    inv = 10000.0 ** (-np.arange(r // 2) * 2 / r)
+    x = rng.standard_normal((5, r))
+    assert np.allclose(O.rope_pairs(x, np.zeros(5), inv), x, rtol=0, atol=1e-15)
+    pos = rng.uniform(0, 5000, 5)
+    y = O.rope_pairs(x, pos, inv)
+    for t in range(5):
+        for j in range(r // 2):
+            a = pos[t] * inv[j]
+            ref = (x[t, 2 * j] * math.cos(a) - x[t, 2 * j + 1] * math.sin(a),
+                   x[t, 2 * j] * math.sin(a) + x[t, 2 * j + 1] * math.cos(a))
+            assert abs(y[t, 2 * j] - ref[0]) < 1e-12 and abs(y[t, 2 * j + 1] - ref[1]) < 1e-12
+    p2 = rng.uniform(0, 100, 5)
+    assert np.allclose(O.rope_pairs(y, p2, inv), O.rope_pairs(x, pos + p2, inv), rtol=1e-10, atol=1e-10)
+
+
+def pin_cache_format_layout(O):
+    rng = np.random.default_rng(42)
+    e = rng.standard_normal((2, 6, 24)) * 3
+    r = 8
+    inv = rng.uniform(0, 1, r // 2)
+    nope, rope = O.cache_format(e, r, inv, pos_stride=4.0, pos_offset=1.5, scale=2.0)
+    assert nope.shape == (2, 6, 16) and rope.shape == (2, 6, 8)
+    assert np.array_equal(nope, O.round_e4m3(e[..., :16] * 2.0))
+    for i in range(6):
+        a = (1.5 + 4.0 * i) * inv[1]
+        assert abs(rope[1, i, 2] - (e[1, i, 18] * math.cos(a) - e[1, i, 19] * math.sin(a))) < 1e-12
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

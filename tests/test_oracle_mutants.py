@@ -49,6 +49,14 @@ MUTANTS = [
     ("scalar_separately_normalised", "    w = np.exp(L - np.max(L))\n    s = w / np.sum(w)                                # one",
      "    w = np.exp(L - np.max(L))\n    s = w / (np.sum(w[:m]) if len(w) == m else np.sum(w[m:]) + 0 * np.sum(w[:m]))  # one"),
     ("scalar_hca_bias_dropped", "L = _f64(z[lo:hi]) + _f64(bvec)", "L = _f64(z[lo:hi])"),
+    ("e4m3_two_mantissa_bits", "np.maximum(lead, -6) - 3)", "np.maximum(lead, -6) - 2)"),
+    ("e4m3_subnormal_boundary", "np.maximum(lead, -6) - 3)", "np.maximum(lead, -7) - 3)"),
+    ("e4m3_no_saturation", "    q = np.minimum(q, E4M3_MAX)\n", "\n"),
+    ("rope_angle_sign", "np.exp(1j * ang)", "np.exp(-1j * ang)"),
+    ("rope_pairs_halves", "z = (x[..., 0::2] + 1j * x[..., 1::2])", "z = (x[..., :r // 2] + 1j * x[..., r // 2:])"),
+    ("cache_position_shift", "pos = pos_offset + pos_stride * np.arange(ne, dtype=np.float64)",
+     "pos = pos_offset + pos_stride * np.arange(1, ne + 1, dtype=np.float64)"),
+    ("cache_scale_dropped", "nope = round_e4m3(entries[..., :c - r] * scale)", "nope = round_e4m3(entries[..., :c - r])"),
     ("fused_hca_streams_swapped", "C = project(Hs, W_kv)\n        Z = project(Hs, W_z)",
      "C = project(Hs, W_z)\n        Z = project(Hs, W_kv)"),
 ]
