@@ -429,6 +429,27 @@ def _workload(name, dev):
                     units=float(nbytes), flush=False, kernel="scalar_pool_kernel",
                     config={"workload": f"scalar-logit CSA: batch 1, n={n}, c={c}, m=4 overlap, "
                                         "bf16 streams and logits", "n": n, "c": c, "m": m})
+    if name == "cache_long":
+        n, c, m, r = 1 << 20, 512, 4, 64
+        t = synth.stream_inputs_torch("csa", 1, n, c, m, "bf16", seed=0, z_row_offset=Z_OFF,
+                                      device=dev)
+        t["inv_freq"] = (10000.0 ** (-torch.arange(r // 2, device=dev, dtype=torch.float64)
+                                     * 2 / r)).float()
+        ne = n // m
+        nope = torch.empty((ne, c - r), device=dev, dtype=torch.uint8)
+        rope = torch.empty((ne, r), device=dev, dtype=bf)
+
+        def launch(x, st):
+            kvc.csa_compress_cache(x["Ca"], x["Cb"], x["Za"], x["Zb"], x["Ba"], x["Bb"], r,
+                                   x["inv_freq"], 4.0, 1.5, 1.0, m=m, out_nope=nope,
+                                   out_rope=rope, stream=st)
+        nbytes = (2 * ne * m + 2 * (ne - 1) * m) * c * 2 + 2 * m * c * 4 + ne * ((c - r) + 2 * r)
+        return dict(inputs=t, launch=launch, outputs=[nope, rope], tokens=n, entries=ne,
+                    bound="hbm", units=float(nbytes), flush=False,
+                    kernel="csa_small_m_kernel (cache layout)",
+                    config={"workload": f"CSA n={n}, c={c}, m=4, bf16 streams, entries written "
+                                        f"as E4M3 [c-{r}] + RoPE'd bf16 [{r}]", "n": n, "c": c,
+                            "m": m, "r": r})
     if name == "decode_entries":
         seqs, c, m = 4096, 512, 4
         g = torch.Generator(device=dev)
@@ -621,7 +642,7 @@ def main():
     ap.add_argument("--workload", default="long",
                     choices=["long", "fused_csa", "fused_hca", "hca_n65536", "csa_f32_n1024",
                              "indexer_keys", "fused_indexer_keys", "scalar_long",
-                             "decode_entries"],
+                             "decode_entries", "cache_long"],
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "
                          "time one kernel on its own workload")
     ap.add_argument("--profile-case", choices=["csa", "hca", "csa_fused", "hca_fused"],

@@ -167,6 +167,44 @@ KVC_API kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype 
                                         const int64_t* entry, int64_t num, void* out,
                                         kvc_dtype out_dtype, kvc_stream stream);
 
+/* Cache layout ([HCA] §4 (2): RoPE on the last r dimensions of each entry only, rotating
+ * adjacent pairs of dimensions; the CSA/HCA comparison article's mixed-precision storage:
+ * BF16 for the RoPE part, FP8 for the other KV values).  Instead of `out`, the entries are
+ * written as
+ *   out_nope : [rows, c - r] FP8 E4M3 bytes = entry[:c-r] * fp8_scale, rounded to nearest
+ *              even, saturating at +-448 (16-byte aligned; unused when r == c)
+ *   out_rope : [rows, r] bf16 = entry[c-r:] with pair j (dimensions 2j, 2j+1 of the slice)
+ *              rotated by the angle pos * inv_freq[j], pos = pos_offset + pos_stride * i,
+ *              i = the entry's index within its sequence (16-byte aligned; unused when r == 0)
+ *   inv_freq : [r / 2] fp32 device array (the pages fix neither the frequencies nor the
+ *              position a pooled entry takes: both are the caller's);  r % 8 == 0, 0 <= r <= c.
+ * rows = batch * N_e for the dense calls, num for the entry-list calls.  The angle is
+ * formed and reduced modulo 2 pi in fp64, its sine and cosine taken in fp32. */
+KVC_API kvc_status csa_compress_cache(const void* Ca, const void* Cb, const void* Za,
+                                      const void* Zb, kvc_dtype in_dtype, const float* Ba,
+                                      const float* Bb, int64_t batch, int64_t n, int64_t c,
+                                      int32_t m, int32_t overlap, int32_t r,
+                                      const float* inv_freq, double pos_stride,
+                                      double pos_offset, float fp8_scale, void* out_nope,
+                                      void* out_rope, kvc_stream stream);
+KVC_API kvc_status hca_compress_cache(const void* C, const void* Z, kvc_dtype in_dtype,
+                                      const float* B, int64_t batch, int64_t n, int64_t c,
+                                      int32_t m, int32_t r, const float* inv_freq,
+                                      double pos_stride, double pos_offset, float fp8_scale,
+                                      void* out_nope, void* out_rope, kvc_stream stream);
+/* Entry lists written in the cache layout (decode-time cache insertion). */
+KVC_API kvc_status csa_compress_entries_cache(
+    const void* Ca, const void* Cb, const void* Za, const void* Zb, kvc_dtype in_dtype,
+    const float* Ba, const float* Bb, int64_t total_rows, int64_t c, int32_t m, int32_t overlap,
+    const int64_t* seq_start, const int64_t* seq_len, const int64_t* entry, int64_t num,
+    int32_t r, const float* inv_freq, double pos_stride, double pos_offset, float fp8_scale,
+    void* out_nope, void* out_rope, kvc_stream stream);
+KVC_API kvc_status hca_compress_entries_cache(
+    const void* C, const void* Z, kvc_dtype in_dtype, const float* B, int64_t total_rows,
+    int64_t c, int32_t m, const int64_t* seq_start, const int64_t* seq_len,
+    const int64_t* entry, int64_t num, int32_t r, const float* inv_freq, double pos_stride,
+    double pos_offset, float fp8_scale, void* out_nope, void* out_rope, kvc_stream stream);
+
 /* CSA compressor fed by hidden states ([SC] eq. attn-seqcomp-csa-proj followed by the
  * csa_compress pool): the four streams H W are formed on the tensor cores (bf16 in,
  * fp32 accumulate) and pooled on chip; they never reach device memory.

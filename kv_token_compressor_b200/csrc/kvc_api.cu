@@ -331,6 +331,183 @@ kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype in_dtype
   return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Checks and records the cache-layout arguments (after the problem's own checks).
+static kvc_status set_cache(StreamProblem* p, int32_t r, const float* inv_freq, double pos_stride,
+                           double pos_offset, float fp8_scale, void* out_nope, void* out_rope) {
+  if (r < 0 || r > p->c || r % 8 != 0) return KVC_ERR_SHAPE;
+  if (!(fp8_scale == fp8_scale) || !(pos_stride == pos_stride) || !(pos_offset == pos_offset))
+    return KVC_ERR_SHAPE;  // NaN arguments
+  const bool has_nope = p->c - r > 0, has_rope = r > 0;
+  if ((has_nope && !out_nope) || (has_rope && (!out_rope || !inv_freq))) return KVC_ERR_NULL;
+  if ((has_nope && !aligned(out_nope, 16)) || (has_rope && !aligned(out_rope, 16)) ||
+      (has_rope && !aligned(inv_freq, 4)))
+    return KVC_ERR_ALIGN;
+  const void* ps[3];
+  int np = 0;
+  if (has_nope) ps[np++] = out_nope;
+  if (has_rope) {
+    ps[np++] = out_rope;
+    ps[np++] = inv_freq;
+  }
+  kvc_status s = check_ptrs(ps, np);
+  if (s != KVC_OK) return s;
+  p->cache = true;
+  p->out_nope = out_nope;
+  p->out_rope = out_rope;
+  p->inv_freq = inv_freq;
+  p->r = r;
+  p->pos_stride = pos_stride;
+  p->pos_offset = pos_offset;
+  p->fp8_scale = fp8_scale;
+  return KVC_OK;
+}
+
+kvc_status csa_compress_cache(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                              kvc_dtype in_dtype, const float* Ba, const float* Bb, int64_t batch,
+                              int64_t n, int64_t c, int32_t m, int32_t overlap, int32_t r,
+                              const float* inv_freq, double pos_stride, double pos_offset,
+                              float fp8_scale, void* out_nope, void* out_rope, kvc_stream stream) {
+  if (!dtype_ok(in_dtype)) return KVC_ERR_DTYPE;
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (!Ca || !Za || !Ba) return KVC_ERR_NULL;
+  if (overlap && (!Cb || !Zb || !Bb)) return KVC_ERR_NULL;
+  if (!aligned(Ca, 16) || !aligned(Za, 16) || !aligned(Ba, 4)) return KVC_ERR_ALIGN;
+  if (overlap && (!aligned(Cb, 16) || !aligned(Zb, 16) || !aligned(Bb, 4))) return KVC_ERR_ALIGN;
+  const bool small = (m == 1 || m == 2 || m == 4);
+  if (!small && (overlap ? 2 * m : m) > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  StreamProblem p{};
+  p.c = c;
+  s = set_cache(&p, r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope);
+  if (s != KVC_OK) return s;
+  {
+    const void* ps[6] = {Ca, Za, Ba, Cb, Zb, Bb};
+    s = check_ptrs(ps, overlap ? 6 : 3);
+    if (s != KVC_OK) return s;
+  }
+  p.C0 = Ca;
+  p.Z0 = Za;
+  p.B0 = Ba;
+  p.C1 = overlap ? Cb : nullptr;
+  p.Z1 = overlap ? Zb : nullptr;
+  p.B1 = overlap ? Bb : nullptr;
+  p.batch = batch;
+  p.n = n;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = overlap != 0;
+  p.small_window_kernel = true;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_cache(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
+                              int64_t batch, int64_t n, int64_t c, int32_t m, int32_t r,
+                              const float* inv_freq, double pos_stride, double pos_offset,
+                              float fp8_scale, void* out_nope, void* out_rope, kvc_stream stream) {
+  if (!dtype_ok(in_dtype)) return KVC_ERR_DTYPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (!C || !Z || !B) return KVC_ERR_NULL;
+  if (!aligned(C, 16) || !aligned(Z, 16) || !aligned(B, 4)) return KVC_ERR_ALIGN;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  StreamProblem p{};
+  p.c = c;
+  s = set_cache(&p, r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope);
+  if (s != KVC_OK) return s;
+  {
+    const void* ps[3] = {C, Z, B};
+    s = check_ptrs(ps, 3);
+    if (s != KVC_OK) return s;
+  }
+  p.C0 = C;
+  p.Z0 = Z;
+  p.B0 = B;
+  p.batch = batch;
+  p.n = n;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = false;
+  p.small_window_kernel = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status csa_compress_entries_cache(const void* Ca, const void* Cb, const void* Za,
+                                      const void* Zb, kvc_dtype in_dtype, const float* Ba,
+                                      const float* Bb, int64_t total_rows, int64_t c, int32_t m,
+                                      int32_t overlap, const int64_t* seq_start,
+                                      const int64_t* seq_len, const int64_t* entry, int64_t num,
+                                      int32_t r, const float* inv_freq, double pos_stride,
+                                      double pos_offset, float fp8_scale, void* out_nope,
+                                      void* out_rope, kvc_stream stream) {
+  if (!dtype_ok(in_dtype)) return KVC_ERR_DTYPE;
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  StreamProblem p{};
+  bool empty = false;
+  kvc_status s = check_list(&p, total_rows, c, m, seq_start, seq_len, entry, num, &empty);
+  if (s != KVC_OK || empty) return s;
+  if (!Ca || !Za || !Ba) return KVC_ERR_NULL;
+  if (overlap && (!Cb || !Zb || !Bb)) return KVC_ERR_NULL;
+  if (!aligned(Ca, 16) || !aligned(Za, 16) || !aligned(Ba, 4)) return KVC_ERR_ALIGN;
+  if (overlap && (!aligned(Cb, 16) || !aligned(Zb, 16) || !aligned(Bb, 4))) return KVC_ERR_ALIGN;
+  const bool small = (m == 1 || m == 2 || m == 4);
+  if (!small && (overlap ? 2 * m : m) > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  s = set_cache(&p, r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope);
+  if (s != KVC_OK) return s;
+  {
+    const void* ps[9] = {Ca, Za, Ba, seq_start, seq_len, entry, Cb, Zb, Bb};
+    s = check_ptrs(ps, overlap ? 9 : 6);
+    if (s != KVC_OK) return s;
+  }
+  p.C0 = Ca;
+  p.Z0 = Za;
+  p.B0 = Ba;
+  p.C1 = overlap ? Cb : nullptr;
+  p.Z1 = overlap ? Zb : nullptr;
+  p.B1 = overlap ? Bb : nullptr;
+  p.two_segments = overlap != 0;
+  p.small_window_kernel = true;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_entries_cache(const void* C, const void* Z, kvc_dtype in_dtype,
+                                      const float* B, int64_t total_rows, int64_t c, int32_t m,
+                                      const int64_t* seq_start, const int64_t* seq_len,
+                                      const int64_t* entry, int64_t num, int32_t r,
+                                      const float* inv_freq, double pos_stride, double pos_offset,
+                                      float fp8_scale, void* out_nope, void* out_rope,
+                                      kvc_stream stream) {
+  if (!dtype_ok(in_dtype)) return KVC_ERR_DTYPE;
+  StreamProblem p{};
+  bool empty = false;
+  kvc_status s = check_list(&p, total_rows, c, m, seq_start, seq_len, entry, num, &empty);
+  if (s != KVC_OK || empty) return s;
+  if (!C || !Z || !B) return KVC_ERR_NULL;
+  if (!aligned(C, 16) || !aligned(Z, 16) || !aligned(B, 4)) return KVC_ERR_ALIGN;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  s = set_cache(&p, r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope);
+  if (s != KVC_OK) return s;
+  {
+    const void* ps[6] = {C, Z, B, seq_start, seq_len, entry};
+    s = check_ptrs(ps, 6);
+    if (s != KVC_OK) return s;
+  }
+  p.C0 = C;
+  p.Z0 = Z;
+  p.B0 = B;
+  p.two_segments = false;
+  p.small_window_kernel = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 static kvc_status fused_common(FusedProblem* p, const void* H, const void* const* W, int nw,
                                const float* B0, const float* B1, bool need_b1, int64_t batch,
                                int64_t n, int64_t d, int64_t c, int32_t m, void* out,

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "../../include/kvc.h"
@@ -73,6 +74,15 @@ __device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
 __device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
   float2 d;
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
@@ -139,6 +149,63 @@ __device__ __forceinline__ void store_scalar(OutT* dst, float v) {
     *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
   } else {
     *dst = v;
+  }
+}
+
+// Cache layout of an entry ("Ch 05 · HCA" §4 (2): RoPE on the last r dimensions only,
+// rotating adjacent pairs; the comparison article's storage split: BF16 for the RoPE part,
+// FP8 for the rest).  nope: [rows, c - r] E4M3 bytes = entry[:c-r] * scale, round to
+// nearest even, saturating; rope: [rows, r] bf16 = entry[c-r:] with pair j rotated by
+// (pos_offset + pos_stride * i) * inv_freq[j], i = the entry's index in its sequence.
+struct CacheFmt {
+  uint8_t* nope;
+  __nv_bfloat16* rope;
+  const float* inv_freq;  // [r / 2]
+  int64_t cn, r;          // c - r, r
+  double pos_stride, pos_offset;
+  float scale;
+};
+struct NoCache {};
+
+// Store the CPT results of channels [ch0, ch0 + CPT) of entry `entry` (output row orow)
+// in the cache layout.  A thread's vector lies wholly in one part (r % 8 == 0).
+template <int CPT>
+__device__ __forceinline__ void store_cache(const CacheFmt& cf, int64_t orow, int64_t ch0,
+                                            int64_t entry, const float (&v)[CPT]) {
+  if (ch0 < cf.cn) {
+    uint32_t w[CPT / 4];
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q) {
+      const uint32_t lo = __nv_cvt_float2_to_fp8x2(
+          make_float2(v[4 * q] * cf.scale, v[4 * q + 1] * cf.scale), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+          make_float2(v[4 * q + 2] * cf.scale, v[4 * q + 3] * cf.scale), __NV_SATFINITE, __NV_E4M3);
+      w[q] = lo | (hi << 16);
+    }
+    uint8_t* dst = cf.nope + orow * cf.cn + ch0;
+    if constexpr (CPT == 8) {
+      st_stream8(dst, make_uint2(w[0], w[1]));
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = w[0];
+    }
+  } else {
+    const int64_t off = ch0 - cf.cn;  // channel offset inside the rope part (even)
+    const double pos = cf.pos_offset + cf.pos_stride * static_cast<double>(entry);
+    float rot[CPT];
+#pragma unroll
+    for (int p = 0; p < CPT / 2; ++p) {
+      // angle in fp64 (the product of two fp32 values is exact), reduced by a multiple of
+      // 2 pi in fp64, then the fp32 sine and cosine of the remainder (|red| <= pi)
+      const double ang = pos * static_cast<double>(cf.inv_freq[off / 2 + p]);
+      const double turns = rint(ang * 0.15915494309189535);
+      const float red = static_cast<float>(fma(-turns, 6.283185307179586, ang));
+      float sn, cs;
+      sincosf(red, &sn, &cs);
+      const float x = v[2 * p], y = v[2 * p + 1];
+      rot[2 * p] = fmaf(x, cs, -y * sn);
+      rot[2 * p + 1] = fmaf(x, sn, y * cs);
+    }
+    store_out<__nv_bfloat16, CPT>(cf.rope + orow * cf.r + off, rot);
   }
 }
 

@@ -32,6 +32,15 @@ struct StreamProblem {
   const int64_t* seq_len;
   const int64_t* entry;
   int64_t num, total_rows;
+  // Cache layout (csa_compress_cache / hca_compress_cache): when `cache`, the entries go to
+  // out_nope ([rows, c - r] E4M3) and out_rope ([rows, r] bf16) instead of `out`.
+  bool cache;
+  void* out_nope;
+  void* out_rope;
+  const float* inv_freq;
+  int64_t r;
+  double pos_stride, pos_offset;
+  float fp8_scale;
 };
 
 kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st);

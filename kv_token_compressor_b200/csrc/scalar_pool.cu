@@ -7,7 +7,8 @@
 // one softmax over them, and C^Comp_i = sum_j S_j C_j with the same weights for every
 // channel.  Entry 0 has no b-rows (eq. attn-seqcomp-overlap-bound of "序列压缩注意力").
 //
-// One warp = one entry x a slab of 32 channel vectors (256 bf16 / 128 fp32 channels).
+// Small CSA windows (m <= 4): one thread per entry and 16-byte channel vector (below).
+// Other windows: one warp = one entry x a slab of 32 channel vectors (256 bf16 / 128 fp32).
 // The warp first turns the window's scalar logits into weights (lanes split the rows;
 // shuffle max and sum; one exp2 per row), keeps them in shared memory, then every lane
 // streams its 16-byte vector of each window row (8 rows in flight) and accumulates the
@@ -136,6 +137,106 @@ __global__ void __launch_bounds__(kScWarps * 32) scalar_pool_kernel(ScalarArgs a
   }
 }
 
+// Small windows (m in {1, 2, 4}): one thread = one entry x one 16-byte channel vector,
+// the same shape as the per-channel CSA kernel.  The thread loads its window's 2m scalar
+// logits (the same addresses for every thread of the entry, served by broadcast), forms
+// the 2m weights itself, issues all value loads before using any, and pools.
+template <typename InT, typename OutT, int M, bool OVERLAP>
+__global__ void __launch_bounds__(256) scalar_small_m_kernel(ScalarArgs a) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int NP = CPT / 2;
+  constexpr int NR = OVERLAP ? 2 * M : M;
+  const InT* C0 = static_cast<const InT*>(a.C0);
+  const InT* Z0 = static_cast<const InT*>(a.Z0);
+  const InT* C1 = static_cast<const InT*>(a.C1);
+  const InT* Z1 = static_cast<const InT*>(a.Z1);
+  OutT* out = static_cast<OutT*>(a.out);
+  float b2[NR];
+#pragma unroll
+  for (int k = 0; k < NR; ++k) b2[k] = (k < M ? a.B0[k] : a.B1[k - M]) * kLog2e;
+  const int64_t ch0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * CPT;
+  if (ch0 >= a.c) return;
+  const int64_t istep = static_cast<int64_t>(gridDim.y) * blockDim.y;
+  for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; i < a.ne;
+         i += istep) {
+      const int64_t rowA = b * a.n + static_cast<int64_t>(M) * i;
+      const bool has_b = OVERLAP && i > 0;
+      uint4 cv[NR];
+      float l[NR];
+#pragma unroll
+      for (int k = 0; k < M; ++k) {
+        cv[k] = ld_stream16(C0 + (rowA + k) * a.c + ch0);
+        l[k] = fmaf(load_scalar<InT>(Z0 + rowA + k), kLog2e, b2[k]);
+      }
+      if constexpr (OVERLAP) {
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+          if (has_b) {
+            cv[M + k] = ld_stream16(C1 + (rowA - M + k) * a.c + ch0);
+            l[M + k] = fmaf(load_scalar<InT>(Z1 + rowA - M + k), kLog2e, b2[M + k]);
+          } else {
+            cv[M + k] = make_uint4(0u, 0u, 0u, 0u);  // entry 0: vector 0, logit -inf
+            l[M + k] = -INFINITY;
+          }
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < NR; ++k) mx = fmaxf(mx, l[k]);
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        l[k] = ex2_ftz(l[k] - mx);
+        sum += l[k];
+      }
+      const float inv = 1.0f / sum;
+      float2 A[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) A[p] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const float2 w2 = make_float2(l[k] * inv, l[k] * inv);
+#pragma unroll
+        for (int p = 0; p < NP; ++p) A[p] = f2_fma(w2, vec_pair<InT>(cv[k], p), A[p]);
+      }
+      float res[CPT];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        res[2 * p] = A[p].x;
+        res[2 * p + 1] = A[p].y;
+      }
+      store_out<OutT, CPT>(out + (b * a.ne + i) * a.c + ch0, res);
+    }
+  }
+}
+
+template <typename InT, typename OutT, int M, bool OVERLAP>
+kvc_status launch_small(const StreamProblem& p, cudaStream_t st) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  const int64_t G = p.c / CPT;
+  const int cg = static_cast<int>(G < 64 ? G : 64);
+  const int ey = 256 / cg;
+  auto kern = scalar_small_m_kernel<InT, OutT, M, OVERLAP>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  const int occ = resident_blocks(kern, cg * ey, 0);
+  if (di.sms == 0 || occ == 0) return KVC_ERR_CUDA;
+  const int64_t gx = ceil_div(G, cg);
+  const int64_t gz = p.batch < 65535 ? p.batch : 65535;
+  int64_t gy = static_cast<int64_t>(di.sms) * occ / (gx * gz);
+  if (gy < 1) gy = 1;
+  const int64_t need = ceil_div(p.ne, ey);
+  if (gy > need) gy = need;
+  if (gy > 65535) gy = 65535;
+  gy = ceil_div(need, ceil_div(need, gy));
+  ScalarArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
+  kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
+         dim3(cg, ey), 0, st>>>(args);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
 template <typename InT, typename OutT, bool TWO_SEG>
 kvc_status launch(const StreamProblem& p, cudaStream_t st) {
   int dev = 0;
@@ -158,7 +259,15 @@ kvc_status launch(const StreamProblem& p, cudaStream_t st) {
 
 template <typename InT, typename OutT>
 kvc_status dispatch(const StreamProblem& p, cudaStream_t st) {
-  return p.two_segments ? launch<InT, OutT, true>(p, st) : launch<InT, OutT, false>(p, st);
+  if (p.two_segments) {
+    switch (p.m) {
+      case 1: return launch_small<InT, OutT, 1, true>(p, st);
+      case 2: return launch_small<InT, OutT, 2, true>(p, st);
+      case 4: return launch_small<InT, OutT, 4, true>(p, st);
+      default: return launch<InT, OutT, true>(p, st);
+    }
+  }
+  return launch<InT, OutT, false>(p, st);
 }
 
 }  // namespace

@@ -19,6 +19,8 @@
 
 #include <math.h>
 
+#include <type_traits>
+
 
 namespace kvc {
 
@@ -41,13 +43,18 @@ struct EntryList {
 // Checks one listed entry against its sequence and the streams; on success gives the first
 // a-row and whether it is the sequence's entry 0.
 __device__ __forceinline__ bool listed_entry(const EntryList& L, int64_t k, int m, int64_t* rowA,
-                                             bool* first) {
+                                             bool* first, int64_t* e_out) {
   const int64_t s0 = L.seq_start[k], len = L.seq_len[k], e = L.entry[k];
   if (!(s0 >= 0 && len >= 0 && s0 <= L.total_rows - len && e >= 0 && e < len / m)) return false;
   *rowA = s0 + static_cast<int64_t>(m) * e;
   *first = e == 0;
+  *e_out = e;
   return true;
 }
+
+// Extra kernel argument of the cache-layout instantiations (empty otherwise).
+template <bool CACHE>
+using CacheArg = typename std::conditional<CACHE, CacheFmt, NoCache>::type;
 
 struct CsaSmallArgs {
   const void* Ca;
@@ -58,11 +65,11 @@ struct CsaSmallArgs {
   const float* Bb;
   int64_t batch, n, c, ne;
   void* out;
-  EntryList list;
 };
 
-template <typename InT, typename OutT, int M, bool OVERLAP, bool LISTED>
-__global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
+template <typename InT, typename OutT, int M, bool OVERLAP, bool LISTED, bool CACHE>
+__global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a, const EntryList list,
+                                                             const CacheArg<CACHE> cf) {
   constexpr int CPT = VecInfo<InT>::kChannels;
   constexpr int NP = CPT / 2;              // channel pairs per thread
   constexpr int NB = OVERLAP ? 2 * M : M;  // bias rows: B^a rows then B^b rows
@@ -98,15 +105,16 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
   const uint4 c_boundary = make_uint4(0u, 0u, 0u, 0u);
 
   const int64_t istep = static_cast<int64_t>(gridDim.y) * blockDim.y;
-  const int64_t lim = LISTED ? a.list.num : a.ne;
+  const int64_t lim = LISTED ? list.num : a.ne;
   for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
     for (int64_t i = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y; i < lim;
          i += istep) {
       int64_t rowA;  // a-range start of the entry
       bool first;    // entry 0 of its sequence: no b-rows
       int64_t orow;  // output row
+      int64_t eidx;  // entry index within its sequence
       if constexpr (LISTED) {
-        if (!listed_entry(a.list, i, M, &rowA, &first)) {
+        if (!listed_entry(list, i, M, &rowA, &first, &eidx)) {
           if (threadIdx.x == 0) atomicOr(&g_index_error, 1u);
           continue;
         }
@@ -115,6 +123,7 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
         rowA = b * a.n + static_cast<int64_t>(M) * i;
         first = i == 0;
         orow = b * a.ne + i;
+        eidx = i;
       }
       uint4 za[M], ca[M], zb[M], cb[M];
 #pragma unroll
@@ -176,7 +185,11 @@ __global__ void __launch_bounds__(256, 2) csa_small_m_kernel(CsaSmallArgs a) {
         res[2 * p] = __fdividef(acc.x, s.x);
         res[2 * p + 1] = __fdividef(acc.y, s.y);
       }
-      store_out<OutT, CPT>(out + orow * a.c + ch0, res);
+      if constexpr (CACHE) {
+        store_cache<CPT>(cf, orow, ch0, eidx, res);
+      } else {
+        store_out<OutT, CPT>(out + orow * a.c + ch0, res);
+      }
     }
   }
 }
@@ -201,7 +214,6 @@ struct WinArgs {
   int64_t batch, n, c, ne;
   int m;
   void* out;
-  EntryList list;
 };
 
 constexpr int kWinCG = 16;  // channel vectors per CTA
@@ -220,9 +232,10 @@ size_t win_smem_bytes(int m, int rg) {
   return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + partial);
 }
 
-template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED>
-__global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
-  static_assert(!LISTED || RG == 1, "entry lists use one window per thread");
+template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED, bool CACHE>
+__global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const EntryList list,
+                                                             const CacheArg<CACHE> cf) {
+  static_assert(!(LISTED || CACHE) || RG == 1, "entry lists and the cache layout use one window per thread");
   constexpr int CPT = VecInfo<InT>::kChannels;
   constexpr int SC = win_slab<InT>();
   constexpr int EY = kWinTY / RG;  // entries per CTA iteration
@@ -260,27 +273,19 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
   const int m = a.m;
 
   for (int64_t b = blockIdx.z; b < a.batch; b += gridDim.z) {
-    const int64_t lim = LISTED ? a.list.num : a.ne;
+    const int64_t lim = LISTED ? list.num : a.ne;
     for (int64_t i0 = static_cast<int64_t>(blockIdx.y) * EY; i0 < lim;
          i0 += static_cast<int64_t>(gridDim.y) * EY) {
       const int64_t i = i0 + es;
-      bool live = active && i < lim;
-      int64_t row0 = 0;    // first row of the entry's own segment
-      bool first = false;  // entry 0 of its sequence
-      int64_t orow = 0;    // output row
+      int64_t row0 = b * a.n + static_cast<int64_t>(m) * i;  // first row of its own segment
+      bool first = i == 0;                                      // no b-rows
+      bool ok = true;
+      int64_t eidx = i;                                         // index within its sequence
       if constexpr (LISTED) {
-        if (i < lim) {
-          if (!listed_entry(a.list, i, m, &row0, &first)) {
-            if (tx == 0) atomicOr(&g_index_error, 1u);
-            live = false;
-          }
-          orow = i;
-        }
-      } else {
-        row0 = b * a.n + static_cast<int64_t>(m) * i;
-        first = i == 0;
-        orow = b * a.ne + i;
+        ok = i < lim && listed_entry(list, i, m, &row0, &first, &eidx);
+        if (i < lim && !ok && tx == 0) atomicOr(&g_index_error, 1u);
       }
+      const bool live = active && i < lim && ok;
       const int rows_i = (TWO_SEG && !first) ? 2 * m : m;
       float2 M[NP], S[NP], A[NP];  // per channel pair: running max, sum, weighted sum
 #pragma unroll
@@ -322,7 +327,6 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
             }
           }
           // rescale the running state once per chunk
-          float2 negm[NP];
 #pragma unroll
           for (int p = 0; p < NP; ++p) {
             const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 < rows_i is valid
@@ -330,7 +334,6 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
             S[p] = f2_mul(S[p], sc);
             A[p] = f2_mul(A[p], sc);
             M[p] = nm;
-            negm[p] = make_float2(-nm.x, -nm.y);
           }
           // pass 2: one exp2 per element, packed pair arithmetic
 #pragma unroll
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                   const int pp = 2 * q + e;
-                  const float2 l = f2_fma(vec_pair<InT>(z[u], pp), kL2e2, f2_add(b2[e], negm[pp]));
+                  const float2 l = f2_fma(vec_pair<InT>(z[u], pp), kL2e2, f2_sub(b2[e], M[pp]));
                   const float2 w = f2_ex2(l);
                   S[pp] = f2_add(S[pp], w);
                   A[pp] = f2_fma(w, vec_pair<InT>(cv[u], pp), A[pp]);
@@ -363,7 +366,11 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a) {
             res[2 * p] = __fdividef(A[p].x, S[p].x);
             res[2 * p + 1] = __fdividef(A[p].y, S[p].y);
           }
-          store_out<OutT, CPT>(out + orow * a.c + ch0, res);
+          if constexpr (CACHE) {
+            store_cache<CPT>(cf, LISTED ? i : b * a.ne + i, ch0, eidx, res);
+          } else {
+            store_out<OutT, CPT>(out + (LISTED ? i : b * a.ne + i) * a.c + ch0, res);
+          }
         }
       } else {
 #pragma unroll
@@ -409,7 +416,17 @@ EntryList entry_list(const StreamProblem& p) {
   return EntryList{p.seq_start, p.seq_len, p.entry, p.num, p.total_rows};
 }
 
-template <typename InT, typename OutT, int M, bool OVERLAP, bool LISTED>
+template <bool CACHE>
+CacheArg<CACHE> cache_arg(const StreamProblem& p) {
+  if constexpr (CACHE) {
+    return CacheFmt{static_cast<uint8_t*>(p.out_nope), static_cast<__nv_bfloat16*>(p.out_rope),
+                    p.inv_freq, p.c - p.r, p.r, p.pos_stride, p.pos_offset, p.fp8_scale};
+  } else {
+    return NoCache{};
+  }
+}
+
+template <typename InT, typename OutT, int M, bool OVERLAP, bool LISTED, bool CACHE>
 kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
   constexpr int CPT = VecInfo<InT>::kChannels;
   const int64_t G = p.c / CPT;  // channel vectors
@@ -417,7 +434,7 @@ kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
   const int ey = 256 / cg;
   const dim3 block(cg, ey);
   const size_t smem = sizeof(float) * (OVERLAP ? 2 * M : M) * cg * CPT;
-  auto kern = csa_small_m_kernel<InT, OutT, M, OVERLAP, LISTED>;
+  auto kern = csa_small_m_kernel<InT, OutT, M, OVERLAP, LISTED, CACHE>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
   const DeviceInfo di = device_info(dev);
@@ -434,20 +451,19 @@ kvc_status launch_csa_small(const StreamProblem& p, cudaStream_t st) {
   if (gy > 65535) gy = 65535;
   // Balance: every CTA row gets the same number of entry iterations (+-1).
   gy = ceil_div(need, ceil_div(need, gy));
-  CsaSmallArgs args{p.C0, p.C1, p.Z0, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.out,
-                    entry_list(p)};
+  CsaSmallArgs args{p.C0, p.C1, p.Z0, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.out};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
-         block, smem, st>>>(args);
+         block, smem, st>>>(args, entry_list(p), cache_arg<CACHE>(p));
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
-template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED>
+template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED, bool CACHE>
 kvc_status launch_window_rg(const StreamProblem& p, cudaStream_t st, const DeviceInfo& di) {
   constexpr int SC = win_slab<InT>();
   constexpr int EY = kWinTY / RG;
   const size_t smem = win_smem_bytes<InT, TWO_SEG>(p.m, RG);
   if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
-  auto kern = window_pool_kernel<InT, OutT, TWO_SEG, RG, LISTED>;
+  auto kern = window_pool_kernel<InT, OutT, TWO_SEG, RG, LISTED, CACHE>;
   const int occ = resident_blocks(kern, kWinCG * kWinTY, smem);
   if (occ == 0) return KVC_ERR_CUDA;
   const int64_t gx = ceil_div(p.c, SC);
@@ -459,60 +475,68 @@ kvc_status launch_window_rg(const StreamProblem& p, cudaStream_t st, const Devic
   if (gy > need) gy = need;
   if (gy > 65535) gy = 65535;
   gy = ceil_div(need, ceil_div(need, gy));
-  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.m, p.out,
-               entry_list(p)};
+  // The entry list is its own parameter: inside WinArgs it made ptxas spill the dense path.
+  WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.m, p.out};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
-         dim3(kWinCG, kWinTY), smem, st>>>(args);
+         dim3(kWinCG, kWinTY), smem, st>>>(args, entry_list(p), cache_arg<CACHE>(p));
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
 // Row groups per entry: the fewest that still give every resident CTA slot a few
 // iterations (one window per thread needs no merge at all).
-template <typename InT, typename OutT, bool TWO_SEG, bool LISTED>
+template <typename InT, typename OutT, bool TWO_SEG, bool LISTED, bool CACHE>
 kvc_status launch_window(const StreamProblem& p, cudaStream_t st) {
   constexpr int SC = win_slab<InT>();
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
   const DeviceInfo di = device_info(dev);
   if (di.sms == 0) return KVC_ERR_CUDA;
-  if constexpr (LISTED) {
-    return launch_window_rg<InT, OutT, TWO_SEG, 1, true>(p, st, di);
+  if constexpr (LISTED || CACHE) {
+    return launch_window_rg<InT, OutT, TWO_SEG, 1, LISTED, CACHE>(p, st, di);
   } else {
     const int64_t tasks = p.batch * p.ne * ceil_div(p.c, SC);  // (entry, slab) pairs
     const int64_t slots = static_cast<int64_t>(di.sms) * 2;
     const int rows = TWO_SEG ? 2 * p.m : p.m;
     if (tasks >= 3 * slots * kWinTY || rows <= kWinU)
-      return launch_window_rg<InT, OutT, TWO_SEG, 1, false>(p, st, di);
+      return launch_window_rg<InT, OutT, TWO_SEG, 1, false, false>(p, st, di);
     if (tasks >= 3 * slots * (kWinTY / 4))
-      return launch_window_rg<InT, OutT, TWO_SEG, 4, false>(p, st, di);
-    return launch_window_rg<InT, OutT, TWO_SEG, 16, false>(p, st, di);
+      return launch_window_rg<InT, OutT, TWO_SEG, 4, false, false>(p, st, di);
+    return launch_window_rg<InT, OutT, TWO_SEG, 16, false, false>(p, st, di);
   }
 }
 
-template <typename InT, typename OutT, bool LISTED>
+template <typename InT, typename OutT, bool LISTED, bool CACHE>
 kvc_status dispatch_stream(const StreamProblem& p, cudaStream_t st) {
   if (p.two_segments) {
     switch (p.m) {
-      case 1: return launch_csa_small<InT, OutT, 1, true, LISTED>(p, st);
-      case 2: return launch_csa_small<InT, OutT, 2, true, LISTED>(p, st);
-      case 4: return launch_csa_small<InT, OutT, 4, true, LISTED>(p, st);
-      default: return launch_window<InT, OutT, true, LISTED>(p, st);
+      case 1: return launch_csa_small<InT, OutT, 1, true, LISTED, CACHE>(p, st);
+      case 2: return launch_csa_small<InT, OutT, 2, true, LISTED, CACHE>(p, st);
+      case 4: return launch_csa_small<InT, OutT, 4, true, LISTED, CACHE>(p, st);
+      default: return launch_window<InT, OutT, true, LISTED, CACHE>(p, st);
     }
   }
   if (p.small_window_kernel) {
     switch (p.m) {
-      case 1: return launch_csa_small<InT, OutT, 1, false, LISTED>(p, st);
-      case 2: return launch_csa_small<InT, OutT, 2, false, LISTED>(p, st);
-      case 4: return launch_csa_small<InT, OutT, 4, false, LISTED>(p, st);
+      case 1: return launch_csa_small<InT, OutT, 1, false, LISTED, CACHE>(p, st);
+      case 2: return launch_csa_small<InT, OutT, 2, false, LISTED, CACHE>(p, st);
+      case 4: return launch_csa_small<InT, OutT, 4, false, LISTED, CACHE>(p, st);
       default: break;
     }
   }
-  return launch_window<InT, OutT, false, LISTED>(p, st);
+  return launch_window<InT, OutT, false, LISTED, CACHE>(p, st);
 }
 
 template <typename InT, typename OutT>
 kvc_status dispatch_listed(const StreamProblem& p, cudaStream_t st) {
-  return p.listed ? dispatch_stream<InT, OutT, true>(p, st) : dispatch_stream<InT, OutT, false>(p, st);
+  return p.listed ? dispatch_stream<InT, OutT, true, false>(p, st)
+                  : dispatch_stream<InT, OutT, false, false>(p, st);
+}
+
+// Cache layout: the output type is fixed by the layout (E4M3 + bf16).
+template <typename InT>
+kvc_status dispatch_cache(const StreamProblem& p, cudaStream_t st) {
+  return p.listed ? dispatch_stream<InT, __nv_bfloat16, true, true>(p, st)
+                  : dispatch_stream<InT, __nv_bfloat16, false, true>(p, st);
 }
 
 }  // namespace
@@ -525,6 +549,8 @@ size_t window_kernel_smem_bytes(bool bf16_in, bool two_segments, int m) {
 }
 
 kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st) {
+  if (p.cache)
+    return p.in_bf16 ? dispatch_cache<__nv_bfloat16>(p, st) : dispatch_cache<float>(p, st);
   if (p.in_bf16) {
     return p.out_bf16 ? dispatch_listed<__nv_bfloat16, __nv_bfloat16>(p, st)
                       : dispatch_listed<__nv_bfloat16, float>(p, st);

@@ -31,6 +31,7 @@ KVC_BF16 = 1
 
 # Every entry point the header declares, with its ctypes signature.
 _i64, _i32, _p = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
+_d, _f = ctypes.c_double, ctypes.c_float
 SIGNATURES = {
     "kvc_num_entries": (_i64, [_i64, _i32]),
     "kvc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -51,6 +52,15 @@ SIGNATURES = {
                                             _i32, _p, _p, _p, _i64, _p, ctypes.c_int, _p]),
     "hca_compress_entries": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i32, _p, _p, _p,
                                             _i64, _p, ctypes.c_int, _p]),
+    "csa_compress_cache": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64, _i64, _i32,
+                                          _i32, _i32, _p, _d, _d, _f, _p, _p, _p]),
+    "hca_compress_cache": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i32, _i32, _p,
+                                          _d, _d, _f, _p, _p, _p]),
+    "csa_compress_entries_cache": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64,
+                                                  _i32, _i32, _p, _p, _p, _i64, _i32, _p, _d, _d, _f,
+                                                  _p, _p, _p]),
+    "hca_compress_entries_cache": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i32, _p, _p,
+                                                  _p, _i64, _i32, _p, _d, _d, _f, _p, _p, _p]),
 }
 
 _lib = None
@@ -225,6 +235,87 @@ def hca_compress_entries(C, Z, B, seq_start, seq_len, entry, m: int = 128, out=N
                                     _stream(stream))
     _check(st, "hca_compress_entries")
     return out
+
+
+def _cache_outs(rows, c, r, like, out_nope, out_rope):
+    # sizes are clamped so that an invalid r reaches the library, which reports it
+    torch = _torch()
+    cn, rr = max(c - r, 0), max(min(r, c), 0)
+    if out_nope is None:
+        out_nope = torch.empty((rows, cn), dtype=torch.uint8, device=like.device)
+    if out_rope is None:
+        out_rope = torch.empty((rows, rr), dtype=torch.bfloat16, device=like.device)
+    if out_nope.dtype not in (torch.uint8, torch.float8_e4m3fn) or out_nope.numel() != rows * cn:
+        raise ValueError("out_nope must hold rows x (c - r) E4M3 bytes")
+    if out_rope.dtype != torch.bfloat16 or out_rope.numel() != rows * rr:
+        raise ValueError("out_rope must be rows x r bf16")
+    return out_nope, out_rope
+
+
+def _cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope, c):
+    return (r, _ptr(inv_freq) if r > 0 else None, float(pos_stride), float(pos_offset),
+            float(fp8_scale), _ptr(out_nope) if c - r > 0 else None, _ptr(out_rope) if r > 0 else None)
+
+
+def csa_compress_cache(Ca, Cb, Za, Zb, Ba, Bb, r, inv_freq, pos_stride=4.0, pos_offset=1.5,
+                       fp8_scale=1.0, m: int = 4, overlap: bool = True, out_nope=None,
+                       out_rope=None, stream=None):
+    """CSA entries in the cache layout: E4M3 bytes [batch, N_e, c - r] and RoPE'd bf16
+    [batch, N_e, r].  The default position is the centre of the entry's own m-block."""
+    batch, n, c = Ca.shape
+    ne = n // m
+    nope, rope = _cache_outs(batch * ne, c, r, Ca, out_nope, out_rope)
+    st = lib().csa_compress_cache(
+        _ptr(Ca), _ptr(Cb) if overlap else None, _ptr(Za), _ptr(Zb) if overlap else None,
+        _dtype_code(Ca.dtype), _ptr(Ba), _ptr(Bb) if overlap else None, batch, n, c, m,
+        int(bool(overlap)), *_cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, nope, rope, c),
+        _stream(stream))
+    _check(st, "csa_compress_cache")
+    return nope.view(batch, ne, max(c - r, 0)), rope.view(batch, ne, max(min(r, c), 0))
+
+
+def hca_compress_cache(C, Z, B, r, inv_freq, pos_stride=128.0, pos_offset=63.5, fp8_scale=1.0,
+                       m: int = 128, out_nope=None, out_rope=None, stream=None):
+    """HCA entries in the cache layout (default position: the segment centre)."""
+    batch, n, c = C.shape
+    ne = n // m
+    nope, rope = _cache_outs(batch * ne, c, r, C, out_nope, out_rope)
+    st = lib().hca_compress_cache(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
+                                  *_cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, nope,
+                                               rope, c), _stream(stream))
+    _check(st, "hca_compress_cache")
+    return nope.view(batch, ne, max(c - r, 0)), rope.view(batch, ne, max(min(r, c), 0))
+
+
+def csa_compress_entries_cache(Ca, Cb, Za, Zb, Ba, Bb, seq_start, seq_len, entry, r, inv_freq,
+                               pos_stride=4.0, pos_offset=1.5, fp8_scale=1.0, m: int = 4,
+                               overlap: bool = True, out_nope=None, out_rope=None, stream=None):
+    """Listed CSA entries (decode-time cache insertion) in the cache layout."""
+    total_rows, c = Ca.shape
+    num = entry.shape[0]
+    nope, rope = _cache_outs(num, c, r, Ca, out_nope, out_rope)
+    st = lib().csa_compress_entries_cache(
+        _ptr(Ca), _ptr(Cb) if overlap else None, _ptr(Za), _ptr(Zb) if overlap else None,
+        _dtype_code(Ca.dtype), _ptr(Ba), _ptr(Bb) if overlap else None, total_rows, c, m,
+        int(bool(overlap)), _index(seq_start, num), _index(seq_len, num), _index(entry, num), num,
+        *_cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, nope, rope, c), _stream(stream))
+    _check(st, "csa_compress_entries_cache")
+    return nope.view(num, max(c - r, 0)), rope.view(num, max(min(r, c), 0))
+
+
+def hca_compress_entries_cache(C, Z, B, seq_start, seq_len, entry, r, inv_freq, pos_stride=128.0,
+                               pos_offset=63.5, fp8_scale=1.0, m: int = 128, out_nope=None,
+                               out_rope=None, stream=None):
+    """Listed HCA entries in the cache layout."""
+    total_rows, c = C.shape
+    num = entry.shape[0]
+    nope, rope = _cache_outs(num, c, r, C, out_nope, out_rope)
+    st = lib().hca_compress_entries_cache(
+        _ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), total_rows, c, m, _index(seq_start, num),
+        _index(seq_len, num), _index(entry, num), num,
+        *_cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, nope, rope, c), _stream(stream))
+    _check(st, "hca_compress_entries_cache")
+    return nope.view(num, max(c - r, 0)), rope.view(num, max(min(r, c), 0))
 
 
 def csa_compress_fused_proj(H, W_kva, W_kvb, W_za, W_zb, Ba, Bb, batch: int, n: int, m: int = 4,

@@ -220,3 +220,45 @@ def test_scalar_logit_misc(L):
                                         None) == kvc.KVC_ERR_UNSUPPORTED
     assert L.hca_compress_scalar_logits(A, A, kvc.KVC_BF16, A, 1, 100, 512, 128, A, kvc.KVC_BF16,
                                         None) == kvc.KVC_OK
+
+
+def csa_cache(L, **kw):
+    a = dict(Ca=A, Cb=A, Za=A, Zb=A, in_dt=kvc.KVC_BF16, Ba=A, Bb=A, batch=1, n=1024, c=512, m=4,
+             overlap=1, r=64, inv=A, ps=4.0, po=1.5, sc=1.0, nope=A, rope=A)
+    a.update(kw)
+    return L.csa_compress_cache(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["in_dt"], a["Ba"], a["Bb"],
+                                a["batch"], a["n"], a["c"], a["m"], a["overlap"], a["r"], a["inv"],
+                                a["ps"], a["po"], a["sc"], a["nope"], a["rope"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dt=4), kvc.KVC_ERR_DTYPE),
+    (dict(r=12), kvc.KVC_ERR_SHAPE),
+    (dict(r=-8), kvc.KVC_ERR_SHAPE),
+    (dict(r=520), kvc.KVC_ERR_SHAPE),
+    (dict(sc=float("nan")), kvc.KVC_ERR_SHAPE),
+    (dict(po=float("nan")), kvc.KVC_ERR_SHAPE),
+    (dict(inv=None), kvc.KVC_ERR_NULL),
+    (dict(rope=None), kvc.KVC_ERR_NULL),
+    (dict(nope=None), kvc.KVC_ERR_NULL),
+    (dict(nope=A + 8), kvc.KVC_ERR_ALIGN),
+    (dict(rope=A + 4), kvc.KVC_ERR_ALIGN),
+    (dict(inv=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(Ca=MIS), kvc.KVC_ERR_ALIGN),
+])
+def test_csa_cache_rejects_before_launch(L, kw, status):
+    assert csa_cache(L, **kw) == status
+
+
+def test_cache_layout_optional_parts(L):
+    # r == 0: no rope part, so rope / inv_freq may be NULL (stops at the next check)
+    assert csa_cache(L, r=0, rope=None, inv=None, nope=A + 8) == kvc.KVC_ERR_ALIGN
+    # r == c: no nope part
+    assert csa_cache(L, r=512, nope=None, rope=A + 4) == kvc.KVC_ERR_ALIGN
+    assert csa_cache(L, n=3, Ca=None, nope=None) == kvc.KVC_OK  # empty problem
+    assert L.hca_compress_cache(A, A, kvc.KVC_BF16, A, 1, 1024, 512, 128, 64, None, 128.0, 63.5, 1.0,
+                                A, A, None) == kvc.KVC_ERR_NULL
+    assert L.csa_compress_entries_cache(A, A, A, A, kvc.KVC_BF16, A, A, 1024, 512, 4, 1, A, A, A, 8,
+                                        12, A, 4.0, 1.5, 1.0, A, A, None) == kvc.KVC_ERR_SHAPE
+    assert L.hca_compress_entries_cache(A, A, kvc.KVC_BF16, A, 1024, 512, 128, A, A, A, 0, 64, A,
+                                        128.0, 63.5, 1.0, A, A, None) == kvc.KVC_OK  # empty list
