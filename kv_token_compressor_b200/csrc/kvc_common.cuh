@@ -111,6 +111,27 @@ __device__ __forceinline__ float2 vec_pair<float>(const uint4& v, int p) {
                 : make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
 }
 
+// Lane-wise maximum of two 16-byte vectors of T, in T (bf16: max.bf16x2, two lanes per
+// instruction; exact, since a maximum only selects).
+template <typename T>
+__device__ __forceinline__ uint4 vec_max(const uint4& a, const uint4& b);
+template <>
+__device__ __forceinline__ uint4 vec_max<__nv_bfloat16>(const uint4& a, const uint4& b) {
+  uint4 r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r.x) : "r"(a.x), "r"(b.x));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r.y) : "r"(a.y), "r"(b.y));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r.z) : "r"(a.z), "r"(b.z));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r.w) : "r"(a.w), "r"(b.w));
+  return r;
+}
+template <>
+__device__ __forceinline__ uint4 vec_max<float>(const uint4& a, const uint4& b) {
+  return make_uint4(__float_as_uint(fmaxf(__uint_as_float(a.x), __uint_as_float(b.x))),
+                    __float_as_uint(fmaxf(__uint_as_float(a.y), __uint_as_float(b.y))),
+                    __float_as_uint(fmaxf(__uint_as_float(a.z), __uint_as_float(b.z))),
+                    __float_as_uint(fmaxf(__uint_as_float(a.w), __uint_as_float(b.w))));
+}
+
 // Channels carried by one 16-byte vector of T.
 template <typename T>
 struct VecInfo {

@@ -225,11 +225,24 @@ constexpr int win_slab() {
   return kWinCG * VecInfo<InT>::kChannels;
 }
 
+// Largest per-channel spread of the (log2 e-scaled) bias rows for which a chunk's maximum
+// logit may be bounded by max(z) * log2 e + max(b) instead of taken row by row.
+constexpr float kMaxBiasSpread = 64.f;
+
+// Position of slab channel sc in a shared-memory bias row: float4 q of thread group g at
+// (q * kWinCG + g) * 4.
+template <int CPT>
+__device__ __forceinline__ int win_bias_pos(int sc) {
+  const int g = sc / CPT, j = sc - (sc / CPT) * CPT;
+  return ((j >> 2) * kWinCG + g) * 4 + (j & 3);
+}
+
 template <typename InT, bool TWO_SEG>
 size_t win_smem_bytes(int m, int rg) {
   const int rows = TWO_SEG ? 2 * m : m;
   const size_t partial = rg > 1 ? 3 * kWinTY * win_slab<InT>() : 0;
-  return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + partial);
+  const size_t extra = win_slab<InT>() + 2 * kWinCG * kWinTY;  // bias maxima, spread partials
+  return sizeof(float) * (static_cast<size_t>(rows) * win_slab<InT>() + extra + partial);
 }
 
 template <typename InT, typename OutT, bool TWO_SEG, int RG, bool LISTED, bool CACHE>
@@ -244,8 +257,12 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const En
   const float2 kL2e2 = make_float2(kLog2e, kLog2e);
   extern __shared__ float4 smem_f4[];
   const int nb = TWO_SEG ? 2 * a.m : a.m;
-  float* sb = reinterpret_cast<float*>(smem_f4);  // [nb][SC] biases * log2 e
-  float* pm = sb + static_cast<size_t>(nb) * SC;  // RG > 1: [16][SC] partial max
+  // Bias rows pre-scaled by log2 e, as [nb][CPT/4][kWinCG] float4: the q-th float4 of
+  // every thread group of a row is contiguous, so a warp's reads of it hit no bank twice.
+  float* sb = reinterpret_cast<float*>(smem_f4);
+  float* bmx = sb + static_cast<size_t>(nb) * SC;  // [SC] per-channel largest bias, same order
+  float* red = bmx + SC;                           // [2][256] bias max / min partials
+  float* pm = red + 2 * kWinCG * kWinTY;           // RG > 1: [16][SC] partial max
   float* ps = pm + kWinTY * SC;                    //         partial sum
   float* pa = ps + kWinTY * SC;                    //         partial weighted sum
 
@@ -253,14 +270,34 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const En
   const int tid = ty * kWinCG + tx;
   const int es = ty / RG, rg = ty - (ty / RG) * RG;
   const int64_t ch_base = static_cast<int64_t>(blockIdx.x) * SC;
+  // 256 is a multiple of SC, so each thread loads one channel's rows tid/SC, tid/SC + 256/SC, ...
+  float lmax = -INFINITY, lmin = INFINITY;
   for (int idx = tid; idx < nb * SC; idx += kWinCG * kWinTY) {
     const int k = idx / SC;
-    const int64_t ch = ch_base + (idx - k * SC);
+    const int sc = idx - k * SC;
+    const int64_t ch = ch_base + sc;
     float v = 0.f;
     if (ch < a.c) v = (k < a.m ? a.B0[k * a.c + ch] : a.B1[(k - a.m) * a.c + ch]) * kLog2e;
-    sb[idx] = v;
+    sb[k * SC + win_bias_pos<CPT>(sc)] = v;
+    lmax = fmaxf(lmax, v);
+    lmin = fminf(lmin, v);
   }
+  red[tid] = lmax;
+  red[kWinCG * kWinTY + tid] = lmin;
   __syncthreads();
+  // Fast chunk maximum (see pass 1 below) when every channel's bias spread is at most
+  // kMaxBiasSpread; a CTA-uniform choice.
+  bool wide = false;
+  if (tid < SC) {
+    float mx = -INFINITY, mn = INFINITY;
+    for (int j = tid; j < kWinCG * kWinTY; j += SC) {
+      mx = fmaxf(mx, red[j]);
+      mn = fminf(mn, red[kWinCG * kWinTY + j]);
+    }
+    bmx[win_bias_pos<CPT>(tid)] = mx;
+    wide = !(mx - mn <= kMaxBiasSpread);  // also true for infinite or NaN spreads
+  }
+  const bool fast = !__syncthreads_or(wide);
 
   const int sc0 = tx * CPT;
   const int64_t ch0 = ch_base + sc0;
@@ -307,22 +344,40 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const En
               cv[u] = ld_stream16((seg1 ? C1 : C0) + row * a.c + ch0);
             }
           }
-          // pass 1: chunk max per channel (bias rows read as float4 from shared memory)
+          // pass 1: an upper bound M' of the chunk's largest logit per channel.  Fast form:
+          // max_k z_k * log2 e + max_k b_k, the maximum taken in the input type (exact).
+          // M' exceeds the true maximum by at most the bias spread, so the largest weight
+          // exp2(l* - M') stays >= 2^-kMaxBiasSpread: the softmax is unchanged and nothing
+          // underflows.  Otherwise the exact per-row maximum of z * log2 e + b.
           float2 cm[NP];
+          if (fast) {
+            uint4 zm = z[0];
 #pragma unroll
-          for (int p = 0; p < NP; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
+            for (int u = 1; u < U; ++u)
+              if (v0 + u * RG < rows_i) zm = vec_max<InT>(zm, z[u]);
+            const float4* bx = reinterpret_cast<const float4*>(bmx) + tx;
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int v = v0 + u * RG;
-            if (v < rows_i) {
-              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+            for (int q = 0; q < NP / 2; ++q) {
+              const float4 bq = bx[q * kWinCG];
+              cm[2 * q] = f2_fma(vec_pair<InT>(zm, 2 * q), kL2e2, make_float2(bq.x, bq.y));
+              cm[2 * q + 1] = f2_fma(vec_pair<InT>(zm, 2 * q + 1), kL2e2, make_float2(bq.z, bq.w));
+            }
+          } else {
 #pragma unroll
-              for (int q = 0; q < NP / 2; ++q) {
-                const float4 bq = bp[q];
-                cm[2 * q] = f2_max(cm[2 * q], f2_fma(vec_pair<InT>(z[u], 2 * q), kL2e2,
-                                                     make_float2(bq.x, bq.y)));
-                cm[2 * q + 1] = f2_max(cm[2 * q + 1], f2_fma(vec_pair<InT>(z[u], 2 * q + 1),
-                                                             kL2e2, make_float2(bq.z, bq.w)));
+            for (int p = 0; p < NP; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int v = v0 + u * RG;
+              if (v < rows_i) {
+                const float4* bp = reinterpret_cast<const float4*>(sb + v * SC) + tx;
+#pragma unroll
+                for (int q = 0; q < NP / 2; ++q) {
+                  const float4 bq = bp[q * kWinCG];
+                  cm[2 * q] = f2_max(cm[2 * q], f2_fma(vec_pair<InT>(z[u], 2 * q), kL2e2,
+                                                       make_float2(bq.x, bq.y)));
+                  cm[2 * q + 1] = f2_max(cm[2 * q + 1], f2_fma(vec_pair<InT>(z[u], 2 * q + 1),
+                                                               kL2e2, make_float2(bq.z, bq.w)));
+                }
               }
             }
           }
@@ -340,10 +395,10 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const En
           for (int u = 0; u < U; ++u) {
             const int v = v0 + u * RG;
             if (v < rows_i) {
-              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC + sc0);
+              const float4* bp = reinterpret_cast<const float4*>(sb + v * SC) + tx;
 #pragma unroll
               for (int q = 0; q < NP / 2; ++q) {
-                const float4 bq = bp[q];
+                const float4 bq = bp[q * kWinCG];
                 const float2 b2[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {

@@ -116,6 +116,30 @@ def test_wide_logit_range():
     check_close(out, O.hca_compress(h["C"], h["Z"], h["B"], 128), "f32", "hca wide logits")
 
 
+@pytest.mark.parametrize("spread", [38.0, 90.0])
+@pytest.mark.parametrize("mode,batch,n,c,m", [
+    ("hca", 1, 128 * 6 + 5, 136, 128),   # few windows: row groups merged in shared memory
+    ("hca", 1, 16 * 15000, 64, 16),       # many windows: one per thread, several chunks
+    ("csa", 2, 8 * 40 + 3, 72, 8),        # two segments (a then b) in the window kernel
+])
+def test_bias_spread_paths(mode, batch, n, c, m, spread):
+    """Biases uniform in [-spread/2, spread/2] (natural-log units).  38 stays inside the
+    spread (64 in log2 units) where the window kernel bounds each chunk's maximum by
+    max(z) + max(b); 90 is beyond it and takes the exact per-row maximum.  Both must
+    match the oracle, although the bounded maximum leaves weights as small as 2^-55."""
+    rng = np.random.default_rng(int(spread) + m)
+    d = synth.stream_inputs(mode, batch, n, c, m, "f32", seed=int(spread) + n)
+    for k in [k for k in d if k.startswith("B")]:
+        d[k] = rng.uniform(-spread / 2, spread / 2, size=d[k].shape).astype(np.float32)
+    if mode == "hca":
+        out = _run_hca(d, m, "f32", "f32")
+        ref = O.hca_compress(d["C"], d["Z"], d["B"], m)
+    else:
+        out = _run_csa(d, m, True, "f32", "f32")
+        ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], m, True)
+    check_close(out, ref, "f32", f"{mode} m={m} bias spread {spread}")
+
+
 def test_boundary_and_mean_on_gpu():
     """Closed forms on the kernel itself: entry 0 ignores the b-streams; constant logits
     with zero bias give the mean of the window (1/8 and 1/4 weights are exact)."""
