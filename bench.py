@@ -396,7 +396,8 @@ def _workload(name, dev):
                                         x["Ba"], x["Bb"], 1, n, m=4, out=out, stream=st)
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // 4,
                     bound="tensor", units=2.0 * n * d * 4 * c, flush=False,
-                    kernel="fused_pool_kernel<CSA>",
+                    kernel=("fused_pair_kernel<CSA> (CTA pairs, M=256)" if c % 128 == 0
+                            else "fused_pool_kernel<CSA>"),
                     config={"workload": f"CSA fused projection + pool: H [{n}, {d}] bf16, 4 W "
                                         f"[{d}, {c}] bf16, m=4 overlap, bf16 out", "n": n,
                             "d": d, "c": c, "m": 4})
@@ -410,7 +411,7 @@ def _workload(name, dev):
                                         out=out, stream=st)
         return dict(inputs=t, launch=launch, outputs=[out], tokens=b * n, entries=b * n // 128,
                     bound="tensor", units=2.0 * b * n * d * 2 * c, flush=False,
-                    kernel="fused_pool_kernel<HCA>",
+                    kernel="fused_pair_kernel<HCA> (CTA pairs, M=256)",
                     config={"workload": f"HCA fused projection + pool: batch {b}, n={n}, H d={d} "
                                         f"bf16, W_kv, W_z [{d}, {c}], m'=128, bf16 out",
                             "batch": b, "n": n, "d": d, "c": c, "m": 128})

@@ -12,7 +12,12 @@
 // that channel's stream values for consecutive tokens in its own registers, so the
 // softmax over a window is thread-local (no shuffles).
 //
-// Per CTA (persistent, one per SM, 192 threads):
+// Two kernels.  fused_pair_kernel (further down) runs on clusters of two CTAs sharing
+// M = 256 MMAs and is the one launched; fused_pool_kernel below, one CTA per SM, is
+// taken when no CTA pair can be resident, and for HCA when the channel groups of 128 are
+// odd in number (they cannot pair up).
+//
+// fused_pool_kernel, per CTA (persistent, one per SM, 192 threads):
 //   warp 0        TMA producer: H tile [TN tokens x 64] + the W tiles [64 x 128] of
 //                 every stream per pipeline stage (128-byte swizzle, mbarrier tx count)
 //   warp 1        TMEM allocator and MMA issuer (one thread): NS x 4 tcgen05.mma
@@ -181,6 +186,107 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ CTA-pair wrappers
+// (a cluster of two CTAs on two SMs sharing one M = 256 MMA: tcgen05 cta_group::2)
+
+// The same shared-memory variable in CTA `rank` of the cluster (shared::cluster address).
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier of either CTA; release orders this thread's earlier writes
+// (including remote shared-memory stores) before the arrival, at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+// try_wait on a local barrier whose arrivals may come from the other CTA (acquire at
+// cluster scope, so the other CTA's released writes are visible afterwards).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Named barrier `id` over `nthreads` threads that also ANDs a predicate across them, so
+// that a decision taken after per-thread bounded waits is the same in every thread.
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q, o;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred o, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, o;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(p)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_named(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Generic-proxy shared-memory writes of this thread become visible to async copies.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Arm a barrier of either CTA with an arrival plus `bytes` of expected transfer.
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   cluster_bar),
+               "r"(bytes)
+               : "memory");
+}
+// Bulk copy of `bytes` from this CTA's shared memory into the other CTA's, counted on a
+// barrier there (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_cta,
+                                                     uint32_t bytes, uint32_t cluster_bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src_cta), "r"(bytes), "r"(cluster_bar)
+      : "memory");
+}
+// All threads of both CTAs.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Tile load into this CTA's shared memory whose completion is counted on the pair
+// leader's barrier (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+      : "memory");
+}
+// M = 256 MMA over the pair: A rows 0..127 from the leader's shared memory, 128..255 from
+// the peer's (same offsets); B columns split in halves the same way; each CTA's TMEM
+// receives its own 128 rows.  Issued by one leader thread.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Arrive on a barrier (of either CTA, cluster address) once this thread's pair MMAs finish.
+__device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   cluster_bar)
+               : "memory");
 }
 
 // ------------------------------------------------------------------ work schedules
@@ -544,6 +650,564 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ==================================================================================
+// CTA-pair kernel (cluster of 2, tcgen05 cta_group::2, M = 256, N <= 256 tokens)
+//
+// Why: in the single-CTA CSA kernel every token tile of N = 128 re-reads the H tile for
+// four MMAs and re-streams the W tiles of four streams, which asks ~206 B/clk of shared
+// memory per SM against 128 available.  A pair of CTAs shares each M = 256 MMA: every SM
+// reads only its own half of A and of B per MMA and loads W for two streams per 256
+// tokens, ~111 B/clk at full tensor rate.
+//
+// Split of the M = 256 rows over the pair:
+//   CSA  the streams: the leader (rank 0) accumulates C^a, Z^a of 128 channels, the peer
+//        (rank 1) C^b, Z^b of the same channels, both for the same N tokens.  Entry i needs
+//        the a-block i (leader) and the b-block i-1 (peer): the peer reduces each block to
+//        a softmax partial per channel, (L, mean) = (max + log2 sum of exp2, weighted
+//        mean), and copies them into the leader's shared memory; the leader merges each
+//        with its a-block and stores the entry.
+//   HCA  the channels: the leader owns channel group 2g, the peer 2g + 1, each with both
+//        streams C and Z; windows stay inside each CTA, nothing is exchanged.
+// TMEM of each CTA: stream 0 (C) in columns [0, 256), stream 1 (Z) in [256, 512).
+//
+// Per CTA: warp 0 TMA (its own halves: H rows [y, y + N/2) or [y + N/2, y + N), W tiles of
+// its two streams), warp 1 TMEM allocation (both CTAs) and MMA issue (leader only),
+// warps 2..17 epilogue.  Stage completion is counted on the leader's barrier; the leader's
+// commits arrive on both CTAs' barriers.  Every wait is bounded as in the kernel above,
+// and a CTA that gives up also raises the other CTA's abort flag.
+//
+// Epilogue.  TMEM is full during it (the MMAs of the next tile wait), so its latency is
+// what costs: 16 warps in 4 groups, group g taking tokens [64 g, 64 g + 64) of the tile
+// (4 warps = the 4 TMEM lane quarters).  CSA tiles advance by 63 blocks (252 rows), so the
+// first block of a tile repeats the last block of the one before and only serves as the
+// b-block of the next entry: no softmax state crosses tiles.  Each CSA group has its own
+// 2-slot ring; a slot holds, per channel, the partials of the 4 blocks preceding the
+// chunk's 4 entries (the first one the peer group carries from its previous chunk, or
+// loads once per tile), so the groups never wait on one another.  An HCA window is split
+// over two groups whose (max, sum, acc) states merge through shared memory.
+// ==================================================================================
+namespace pair {
+
+constexpr int kGroups = 4;             // epilogue groups of 4 warps
+constexpr int kThreads = 64 + kGroups * 128;
+constexpr int kSlotsPerGroup = 2;      // CSA exchange ring per group
+constexpr int kXFloats = 8;            // per channel and chunk: 4 partials x (L, mean)
+constexpr uint32_t kSlotBytes = 128 * kXFloats * 4;  // one exchange slot, 4 KB
+
+struct Cfg {
+  static constexpr int BK = 64;
+  static constexpr int A_BOX = BK * 64 * 2;          // [64 k x 64 ch] bf16, 8 KB
+  static constexpr int A_BYTES = 2 * 2 * A_BOX;      // 2 streams x 128 channels
+  static constexpr int B_BYTES = 128 * BK * 2;       // this CTA's 128 H rows
+  static constexpr int STAGE = A_BYTES + B_BYTES;    // 48 KB
+  static constexpr int STAGES = 4;
+  // CSA exchange slots; HCA uses the same space for its half-window states
+  static constexpr int XBUF = kGroups * kSlotsPerGroup * static_cast<int>(kSlotBytes);  // 32 KB
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE + XBUF + 512;
+  static_assert(STAGE % 1024 == 0 && A_BYTES % 1024 == 0, "1024-byte swizzle atoms");
+  static_assert(SMEM <= 232448, "shared memory per CTA");
+  static_assert(2 * 2 * 128 * 3 * 4 <= XBUF, "HCA half-window states fit the exchange space");
+};
+
+// Bounded wait, as wait_phase, for barriers that the other CTA of the pair may arrive on
+// (acquire at cluster scope).  On giving up it raises both CTAs' abort flags.
+__device__ __noinline__ bool wait_pair(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       uint32_t peer_abort, bool honour_abort = true) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (honour_abort && *abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      st_cluster_u32(peer_abort, 1u);
+      atomicOr(&g_device_error, 1u);
+      return false;
+    }
+  }
+}
+
+// One unit of work of a cluster: `ntiles` token tiles, tile t starting at H row
+// row0 + t * stride and holding tile_tokens(t) <= 256 tokens; the channel group of this CTA.
+struct Unit {
+  int b, cg;              // sequence; channel group of this CTA (128 channels)
+  int64_t row0;           // first H row of tile 0
+  int64_t e0, e1, first_block;  // CSA: entries [e0, e1); blocks from first_block
+  int64_t j;              // HCA: token tile index within the sequence
+  int64_t rows;           // rows covered by the unit
+  int64_t stride;         // rows between tile starts
+  int ntiles;
+};
+
+// CSA: unit u = (sequence, channel group, entry range).  The a.units pieces are spread
+// over the G = batch x channel-group sequences as evenly as integers allow (group g owns
+// pieces [g U / G, (g + 1) U / G)), so every resident pair gets one piece of about equal
+// size.  A piece covers blocks [first_block, e1); tile t covers its blocks
+// [63 t, 63 t + 64), the last tile shortened to the remaining rows (multiple of 16).
+__device__ __forceinline__ Unit csa_unit(const Args& a, int64_t u) {
+  Unit q;
+  const int64_t G = a.batch * a.ncg, U = a.units;
+  const int64_t g = ((u + 1) * G + U - 1) / U - 1;
+  const int64_t start = g * U / G;
+  const int64_t P = (g + 1) * U / G - start, r = u - start;
+  q.b = static_cast<int>(g / a.ncg);
+  q.cg = static_cast<int>(g - static_cast<int64_t>(q.b) * a.ncg);
+  q.e0 = (r * a.ne) / P;
+  q.e1 = ((r + 1) * a.ne) / P;
+  q.first_block = q.e0 > 0 ? q.e0 - 1 : 0;
+  const int64_t nblocks = q.e1 - q.first_block;
+  q.rows = 4 * nblocks;
+  q.stride = 252;
+  q.ntiles = q.e1 > q.e0 ? (nblocks <= 64 ? 1 : 1 + static_cast<int>((nblocks - 64 + 62) / 63)) : 0;
+  q.row0 = static_cast<int64_t>(q.b) * a.n + 4 * q.first_block;
+  q.j = 0;
+  return q;
+}
+// HCA: unit u = (sequence, 256-token tile, channel-group pair), pair fastest; the leader
+// takes group 2p, the peer 2p + 1.  A tile holding one window is 128 tokens.
+__device__ __forceinline__ Unit hca_unit(const Args& a, int64_t u, uint32_t rank) {
+  Unit h;
+  const int npairs = a.ncg / 2;
+  const int64_t tiles_per_seq = (a.ne + 1) / 2;
+  const int p = static_cast<int>(u % npairs);
+  const int64_t r = u / npairs;
+  h.b = static_cast<int>(r / tiles_per_seq);
+  h.j = r - static_cast<int64_t>(h.b) * tiles_per_seq;
+  h.cg = 2 * p + static_cast<int>(rank);
+  h.row0 = static_cast<int64_t>(h.b) * a.n + h.j * 256;
+  const int64_t wins = a.ne - 2 * h.j < 2 ? a.ne - 2 * h.j : 2;
+  h.rows = 128 * wins;
+  h.stride = 256;
+  h.ntiles = 1;
+  h.e0 = h.e1 = h.first_block = 0;
+  return h;
+}
+// Tokens of tile t (MMA N): 256, or the rest of the unit rounded up to 16.
+__device__ __forceinline__ int tile_tokens(const Unit& q, int t) {
+  const int64_t left = q.rows - static_cast<int64_t>(t) * q.stride;
+  return left >= 256 ? 256 : static_cast<int>((left + 15) & ~int64_t(15));
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Softmax partial of one 4-row b-block for one channel: L = max + log2(sum of exp2) and
+// the weighted mean of the C rows (the block's whole contribution to a joint softmax).
+__device__ __forceinline__ void block_partial(const float* z, const float* cv, const float* b2,
+                                              float* L, float* mean) {
+  float l[4], mx = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    l[k] = fmaf(z[k], kLog2e, b2[k]);
+    mx = fmaxf(mx, l[k]);
+  }
+  float s = 0.f, acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float w = ex2_ftz(l[k] - mx);
+    s += w;
+    acc = fmaf(w, cv[k], acc);
+  }
+  *L = mx + lg2_approx(s);  // s >= 1: the largest term is exp2(0)
+  *mean = __fdividef(acc, s);
+}
+
+// Instruction descriptor of the pair MMA: as idesc_bf16 with M = 256.
+__host__ __device__ constexpr uint32_t idesc_pair(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (static_cast<uint32_t>(n >> 3) << 17) |
+         (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+}  // namespace pair
+
+// W maps: CSA W0 = W^{KV_a}, W1 = W^{KV_b}, W2 = W^{Z_a}, W3 = W^{Z_b} (the leader loads
+// W0/W2, the peer W1/W3); HCA W0 = W^{KV}, W1 = W^{Z} (both CTAs).
+template <bool CSA, typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
+    fused_pair_kernel(const __grid_constant__ CUtensorMap tmH,
+                      const __grid_constant__ CUtensorMap tmW0,
+                      const __grid_constant__ CUtensorMap tmW1,
+                      const __grid_constant__ CUtensorMap tmW2,
+                      const __grid_constant__ CUtensorMap tmW3, const Args a) {
+  using C = pair::Cfg;
+  constexpr int S = C::STAGES;
+  constexpr int R = pair::kGroups * pair::kSlotsPerGroup;  // exchange slots (CSA)
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // [R][128][8] CSA partials: the peer stages a slot here, then copies it to the same
+  // place in the leader.  HCA: [2 windows][128][3] half-window states.
+  float* xbuf = reinterpret_cast<float*>(smem + S * C::STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE + C::XBUF);
+  uint64_t* full = bars;                   // [S] leader: both CTAs' bytes of a stage
+  uint64_t* empty = bars + S;              // [S] each CTA: the leader's MMAs freed the stage
+  uint64_t* tmem_full = bars + 2 * S;      // each CTA: accumulators of a tile complete
+  uint64_t* tmem_empty = tmem_full + 1;    // leader: every epilogue group drained TMEM
+  uint64_t* final_bar = tmem_full + 2;     // each CTA: every MMA of the leader finished
+  uint64_t* xfull = tmem_full + 3;         // [R] leader: a slot arrived (1 + its bytes)
+  uint64_t* xempty = xfull + R;            // [R] peer: the leader has read a slot (1)
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(xempty + R);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(xempty + R + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = blockIdx.x & 1u;  // clusters of two consecutive CTAs along x
+  const uint32_t peer = rank ^ 1u;
+  const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const uint32_t peer_abort = cluster_addr(smem_u32(const_cast<int*>(abort_flag)), peer);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, 2 * pair::kGroups);  // one arrival per epilogue group and CTA
+    mbar_init(final_bar, 1);
+    for (int r = 0; r < R; ++r) {
+      mbar_init(&xfull[r], 1);
+      mbar_init(&xempty[r], 1);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  cluster_sync_all();  // barriers and flags of both CTAs exist before any remote arrival
+  if (warp == 1) {     // one warp of each CTA allocates the pair's 512 columns
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(const_cast<uint32_t*>(tmem_slot))),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t units = a.units;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both)
+    if (lane == 0) {
+      const CUtensorMap* mA0 = CSA ? (rank ? &tmW1 : &tmW0) : &tmW0;
+      const CUtensorMap* mA1 = CSA ? (rank ? &tmW3 : &tmW2) : &tmW1;
+      int stage = 0;
+      uint32_t phase = 0;
+      int pending_parity[S];
+      for (int s = 0; s < S; ++s) pending_parity[s] = -1;
+      bool ok = true;
+      for (int64_t u = cid; u < units && ok; u += ncl) {
+        const pair::Unit q = CSA ? pair::csa_unit(a, u) : pair::hca_unit(a, u, rank);
+        for (int t = 0; t < q.ntiles && ok; ++t) {
+          const int nt = pair::tile_tokens(q, t);
+          const int y = static_cast<int>(q.row0 + static_cast<int64_t>(t) * q.stride +
+                                         static_cast<int64_t>(rank) * (nt / 2));
+          for (int kstep = 0; kstep < a.nk; ++kstep) {
+            if (!pair::wait_pair(&empty[stage], phase ^ 1u, abort_flag, peer_abort)) {
+              ok = false;
+              break;
+            }
+            if (rank == 0) {  // the leader arms its barrier for both CTAs' bytes
+              mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE);
+              pending_parity[stage] = static_cast<int>(phase);
+            }
+            const uint32_t lbar = cluster_addr(smem_u32(&full[stage]), 0);
+            uint8_t* st = smem + stage * C::STAGE;
+            const int x = kstep * C::BK;
+            tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tmH, lbar, x, y);
+            tma_load_2d_pair(smem_u32(st + 0 * C::A_BOX), mA0, lbar, q.cg * kCh, x);
+            tma_load_2d_pair(smem_u32(st + 1 * C::A_BOX), mA0, lbar, q.cg * kCh + 64, x);
+            tma_load_2d_pair(smem_u32(st + 2 * C::A_BOX), mA1, lbar, q.cg * kCh, x);
+            tma_load_2d_pair(smem_u32(st + 3 * C::A_BOX), mA1, lbar, q.cg * kCh + 64, x);
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+      if (!ok && rank == 0) {  // drain the stages this CTA armed before giving up
+        for (int s = 0; s < S; ++s)
+          if (pending_parity[s] >= 0)
+            pair::wait_pair(&full[s], static_cast<uint32_t>(pending_parity[s]), abort_flag,
+                            peer_abort, false);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0) {
+      if (rank == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t acc_phase = 0;
+        bool ok = true;
+        for (int64_t u = cid; u < units && ok; u += ncl) {
+          const pair::Unit q = CSA ? pair::csa_unit(a, u) : pair::hca_unit(a, u, 0);
+          for (int t = 0; t < q.ntiles && ok; ++t) {
+            const uint32_t idesc = pair::idesc_pair(pair::tile_tokens(q, t));
+            if (!pair::wait_pair(tmem_empty, acc_phase ^ 1u, abort_flag, peer_abort)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int kstep = 0; kstep < a.nk; ++kstep) {
+              if (!pair::wait_pair(&full[stage], phase, abort_flag, peer_abort)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t st = smem_u32(smem + stage * C::STAGE);
+#pragma unroll
+              for (int s = 0; s < 2; ++s) {
+#pragma unroll
+                for (int ks = 0; ks < C::BK / 16; ++ks) {
+                  // same operand layouts as the single-CTA kernel, per CTA half
+                  const uint64_t ad = smem_desc(st + (2 * s) * C::A_BOX + ks * 16 * 128,
+                                                C::A_BOX, 1024, 2);
+                  const uint64_t bd = smem_desc(st + C::A_BYTES + ks * 32, 16, 1024, 2);
+                  umma_bf16_pair(tmem_base + s * 256, ad, bd, idesc, (kstep | ks) != 0 ? 1u : 0u);
+                }
+              }
+              umma_commit_pair(cluster_addr(smem_u32(&empty[stage]), 0));
+              umma_commit_pair(cluster_addr(smem_u32(&empty[stage]), 1));
+              if (++stage == S) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+            if (!ok) break;
+            umma_commit_pair(cluster_addr(smem_u32(tmem_full), 0));
+            umma_commit_pair(cluster_addr(smem_u32(tmem_full), 1));
+            acc_phase ^= 1u;
+          }
+        }
+        // both CTAs learn when every MMA (which reads and writes both) has finished
+        umma_commit_pair(cluster_addr(smem_u32(final_bar), 0));
+        umma_commit_pair(cluster_addr(smem_u32(final_bar), 1));
+      }
+      pair::wait_pair(final_bar, 0, abort_flag, peer_abort, false);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..17)
+    const int eg = (warp - 2) >> 2;         // group: tokens [64 eg, 64 eg + 64) of a tile
+    const int qw = warp & 3;                // TMEM lane quarter this warp may access
+    const int row = qw * 32 + lane;         // TMEM lane = channel within the CTA's group
+    const bool elected = ((warp - 2) & 3) == 0 && lane == 0;  // one thread per group
+    const int gbar = 1 + eg;                // the group's named barrier (128 threads)
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(qw * 32) << 16);
+    const uint32_t leader_tmem_empty = cluster_addr(smem_u32(tmem_empty), 0);
+    OutT* out = static_cast<OutT*>(a.out);
+    uint32_t acc_phase = 0;
+    uint32_t xcount = 0;  // CSA: exchange chunks of this group so far
+    bool ok = true;
+    for (int64_t u = cid; u < units && ok; u += ncl) {
+      if constexpr (CSA) {
+        const pair::Unit pc = pair::csa_unit(a, u);
+        const int64_t ch = static_cast<int64_t>(pc.cg) * kCh + row;
+        const float* Bsrc = rank == 0 ? a.B0 : a.B1;  // B^a (leader) or B^b (peer)
+        float b2[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) b2[k] = __ldg(Bsrc + k * a.c + ch) * kLog2e;
+        for (int t = 0; t < pc.ntiles && ok; ++t) {
+          const int nch = pair::tile_tokens(pc, t) / 16;
+          const int c_lo = 4 * eg, c_hi = 4 * eg + 4 < nch ? 4 * eg + 4 : nch;
+          // one decision for the group's four warps (they meet at named barriers below)
+          if (!bar_and(gbar, 128, pair::wait_pair(tmem_full, acc_phase, abort_flag, peer_abort))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int64_t kb_tile = pc.first_block + static_cast<int64_t>(t) * 63;
+          if (rank == 1) {
+            // partial of the block before the group's first chunk: block 16 eg - 1 of the
+            // tile (none for group 0: its block 0 is a repeat or the sequence's entry 0)
+            float pL = -INFINITY, pmean = 0.f;
+            if (eg > 0 && c_lo < nch) {
+              float cv[16], zv[16];
+              tmem_ld16(lane_addr + (c_lo - 1) * 16, cv);
+              tmem_ld16(lane_addr + 256 + (c_lo - 1) * 16, zv);
+              tmem_wait_ld();
+              pair::block_partial(zv + 12, cv + 12, b2, &pL, &pmean);
+            }
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; ++c, ++xcount) {
+              float cv[16], zv[16];
+              tmem_ld16(lane_addr + c * 16, cv);
+              tmem_ld16(lane_addr + 256 + c * 16, zv);
+              tmem_wait_ld();
+              float L[4], mean[4];
+#pragma unroll
+              for (int blk = 0; blk < 4; ++blk)
+                pair::block_partial(zv + 4 * blk, cv + 4 * blk, b2, &L[blk], &mean[blk]);
+              const uint32_t slot = eg * pair::kSlotsPerGroup + xcount % pair::kSlotsPerGroup;
+              const uint32_t xpar = (xcount / pair::kSlotsPerGroup) & 1u;
+              if (!bar_and(gbar, 128, pair::wait_pair(&xempty[slot], xpar ^ 1u, abort_flag,
+                                                      peer_abort))) {
+                ok = false;
+                break;
+              }
+              // entry 4c + j of the tile takes the partial of block 4c + j - 1
+              float4* xs = reinterpret_cast<float4*>(xbuf + (slot * 128 + row) * pair::kXFloats);
+              xs[0] = make_float4(pL, pmean, L[0], mean[0]);
+              xs[1] = make_float4(L[1], mean[1], L[2], mean[2]);
+              fence_proxy_async_smem();
+              bar_named(gbar, 128);
+              if (elected) {  // one thread moves the slot to the same place in the leader
+                const uint32_t src = smem_u32(xbuf + slot * 128 * pair::kXFloats);
+                const uint32_t lbar = cluster_addr(smem_u32(&xfull[slot]), 0);
+                mbar_arrive_expect_tx_cluster(lbar, pair::kSlotBytes);
+                bulk_copy_to_cluster(cluster_addr(src, 0), src, pair::kSlotBytes, lbar);
+              }
+              pL = L[3];
+              pmean = mean[3];
+            }
+          } else {
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; ++c, ++xcount) {
+              float cv[16], zv[16];
+              tmem_ld16(lane_addr + c * 16, cv);
+              tmem_ld16(lane_addr + 256 + c * 16, zv);
+              tmem_wait_ld();
+              const uint32_t slot = eg * pair::kSlotsPerGroup + xcount % pair::kSlotsPerGroup;
+              const uint32_t xpar = (xcount / pair::kSlotsPerGroup) & 1u;
+              if (!bar_and(gbar, 128, pair::wait_pair(&xfull[slot], xpar, abort_flag, peer_abort))) {
+                ok = false;
+                break;
+              }
+              const float4* xs =
+                  reinterpret_cast<const float4*>(xbuf + (slot * 128 + row) * pair::kXFloats);
+              const float4 x0 = xs[0], x1 = xs[1];
+              bar_named(gbar, 128);  // every thread of the group has read the slot
+              if (elected) mbar_arrive_cluster(cluster_addr(smem_u32(&xempty[slot]), 1));
+              const float pl[4] = {x0.x, x0.z, x1.x, x1.z};
+              const float pm[4] = {x0.y, x0.w, x1.y, x1.w};
+#pragma unroll
+              for (int blk = 0; blk < 4; ++blk) {
+                const int lb = 4 * c + blk;  // block within the tile
+                const int64_t kb = kb_tile + lb;
+                // entry kb: a-rows of block kb here, b-rows of block kb - 1 as (L, mean);
+                // block 0 of a later tile repeats the last block of the one before
+                if (kb >= pc.e0 && kb < pc.e1 && (t == 0 || lb > 0)) {
+                  float l[4], mx = pl[blk];
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    l[k] = fmaf(zv[4 * blk + k], kLog2e, b2[k]);
+                    mx = fmaxf(mx, l[k]);
+                  }
+                  float s = 0.f, acc = 0.f;
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) {
+                    const float w = ex2_ftz(l[k] - mx);
+                    s += w;
+                    acc = fmaf(w, cv[4 * blk + k], acc);
+                  }
+                  const float f = ex2_ftz(pl[blk] - mx);  // 0 when there are no b-rows
+                  s += f;
+                  acc = fmaf(pm[blk], f, acc);
+                  store_scalar<OutT>(out + (static_cast<int64_t>(pc.b) * a.ne + kb) * a.c + ch,
+                                     __fdividef(acc, s));
+                }
+              }
+            }
+          }
+          if (!ok) break;
+          tc_fence_before();
+          bar_named(gbar, 128);  // the group's TMEM reads of this tile are done
+          if (elected) {
+            if (rank == 0) {
+              mbar_arrive(tmem_empty);
+            } else {
+              mbar_arrive_cluster(leader_tmem_empty);
+            }
+          }
+          acc_phase ^= 1u;
+        }
+      } else {
+        const pair::Unit h = pair::hca_unit(a, u, rank);
+        const int64_t ch = static_cast<int64_t>(h.cg) * kCh + row;
+        const int wins = static_cast<int>(h.rows / 128);
+        const int w = eg >> 1, half = eg & 1;  // window of the tile, rows [64 half, +64) of it
+        const bool active = w < wins;
+        const int wbar = 5 + w;  // the window's two groups (256 threads)
+        const bool got = pair::wait_pair(tmem_full, acc_phase, abort_flag, peer_abort);
+        if (!(active ? bar_and(wbar, 256, got) : bar_and(gbar, 128, got))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (active) {
+          float M = -INFINITY, Ssum = 0.f, A = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            const int cc = 4 * half + c;  // chunk within the window
+            float cv[16], zv[16];
+            const uint32_t col = static_cast<uint32_t>(w * 128 + cc * 16);
+            tmem_ld16(lane_addr + col, cv);
+            tmem_ld16(lane_addr + 256 + col, zv);
+            tmem_wait_ld();
+            float cmx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float b2 = __ldg(a.B0 + (cc * 16 + k) * a.c + ch) * kLog2e;
+              zv[k] = fmaf(zv[k], kLog2e, b2);
+              cmx = fmaxf(cmx, zv[k]);
+            }
+            const float nm = fmaxf(M, cmx);
+            const float sc = ex2_ftz(M - nm);
+            Ssum *= sc;
+            A *= sc;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float wgt = ex2_ftz(zv[k] - nm);
+              Ssum += wgt;
+              A = fmaf(wgt, cv[k], A);
+            }
+            M = nm;
+          }
+          // the second half's state goes through shared memory to the first half
+          float* hs = xbuf + (w * 128 + row) * 3;
+          if (half == 1) {
+            hs[0] = M;
+            hs[1] = Ssum;
+            hs[2] = A;
+          }
+          bar_named(wbar, 256);
+          if (half == 0) {
+            const float M1 = hs[0], S1 = hs[1], A1 = hs[2];
+            const float nm = fmaxf(M, M1);
+            const float f0 = ex2_ftz(M - nm), f1 = ex2_ftz(M1 - nm);
+            Ssum = fmaf(S1, f1, Ssum * f0);
+            A = fmaf(A1, f1, A * f0);
+            store_scalar<OutT>(out + (static_cast<int64_t>(h.b) * a.ne + h.j * 2 + w) * a.c + ch,
+                               __fdividef(A, Ssum));
+          }
+        }
+        tc_fence_before();
+        bar_named(gbar, 128);
+        if (elected) {
+          if (rank == 0) {
+            mbar_arrive(tmem_empty);
+          } else {
+            mbar_arrive_cluster(leader_tmem_empty);
+          }
+        }
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no remote access of either CTA is still in flight
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(512));
+  }
+  cluster_sync_all();
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -631,6 +1295,66 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
+// CTA-pair launch (fused_pair_kernel): clusters of two CTAs, as many as can be resident.
+template <bool CSA, typename OutT>
+kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
+  using C = pair::Cfg;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  if (p.batch * p.n > (int64_t(1) << 31) - 1 - 256) return KVC_ERR_UNSUPPORTED;  // TMA y: int32
+  CUtensorMap mh, mw[4];
+  if (!make_map(&mh, p.H, static_cast<uint64_t>(p.batch * p.n), static_cast<uint64_t>(p.d), 128,
+                C::BK))
+    return KVC_ERR_CUDA;
+  for (int s = 0; s < 4; ++s) {
+    const void* w = CSA ? p.W[s] : p.W[s < 2 ? s : 0];
+    if (!make_map(&mw[s], w, static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.c), C::BK, 64))
+      return KVC_ERR_CUDA;
+  }
+  auto kern = fused_pair_kernel<CSA, OutT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(C::SMEM)) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  int clusters = 0;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+    cfg.blockDim = dim3(pair::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+      (void)cudaGetLastError();
+      return KVC_ERR_UNSUPPORTED;  // no resident pair: the caller takes the single-CTA kernel
+    }
+  }
+  Args a{};
+  a.B0 = p.B0;
+  a.B1 = p.B1;
+  a.out = p.out;
+  a.batch = p.batch;
+  a.n = p.n;
+  a.c = p.c;
+  a.ne = p.ne;
+  a.ncg = static_cast<int>(p.c / kCh);
+  a.nk = static_cast<int>(p.d / C::BK);
+  a.pieces_per_unit = 1;
+  if constexpr (CSA) {
+    const int64_t groups = p.batch * a.ncg;  // (sequence, channel group) pairs
+    int64_t U = clusters;                    // one piece per resident pair ...
+    if (U < groups) U = groups;              // ... but at least one per group
+    if (U > groups * p.ne) U = groups * p.ne;  // and at least one entry per piece
+    a.units = U;
+  } else {
+    a.units = p.batch * ((p.ne + 1) / 2) * (a.ncg / 2);
+  }
+  const int64_t ncl = a.units < clusters ? a.units : clusters;
+  kern<<<static_cast<unsigned>(2 * ncl), pair::kThreads, C::SMEM, st>>>(mh, mw[0], mw[1], mw[2], mw[3],
+                                                                   a);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
 }  // namespace fused
 
 // Stage K per mode.  64-deep stages: CSA 80 KB (two fit), HCA 64 KB (three).  32-deep
@@ -643,10 +1367,18 @@ constexpr int kBkHca = 64;
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st) {
   if (p.csa) {
     if (p.m != 4 || !p.overlap) return KVC_ERR_UNSUPPORTED;
+    const kvc_status r = p.out_bf16 ? fused::launch_pair<true, __nv_bfloat16>(p, st)
+                                    : fused::launch_pair<true, float>(p, st);
+    if (r != KVC_ERR_UNSUPPORTED) return r;
     return p.out_bf16 ? fused::launch_impl<true, kBkCsa, __nv_bfloat16>(p, st)
                       : fused::launch_impl<true, kBkCsa, float>(p, st);
   }
   if (p.m != 128) return KVC_ERR_UNSUPPORTED;
+  if ((p.c / fused::kCh) % 2 == 0) {  // channel groups pair up over the CTA pair
+    const kvc_status r = p.out_bf16 ? fused::launch_pair<false, __nv_bfloat16>(p, st)
+                                    : fused::launch_pair<false, float>(p, st);
+    if (r != KVC_ERR_UNSUPPORTED) return r;
+  }
   return p.out_bf16 ? fused::launch_impl<false, kBkHca, __nv_bfloat16>(p, st)
                     : fused::launch_impl<false, kBkHca, float>(p, st);
 }

@@ -29,6 +29,8 @@ CSA_CASES = [
     (3, 517, 192, 128),
     (2, 4 * 700 + 2, 64, 384),
     (1, 36, 512, 128),
+    # every entry of several pieces and 256-row tiles (shortened last tiles), 4 groups
+    (2, 4 * 2000 + 3, 256, 512),
 ]
 
 
@@ -52,6 +54,8 @@ HCA_CASES = [
     (2, 128 * 5 + 17, 256, 256),
     (3, 128 * 3, 64, 384),
     (1, 128 * 40, 448, 128),
+    # channel groups in pairs over a CTA pair; an odd entry count ends in a half tile
+    (2, 128 * 9 + 5, 128, 512),
 ]
 
 
@@ -111,8 +115,10 @@ def _sampled_check(mode, w, ents_per_seq, seed):
     for b in range(batch):
         pick = set(rng.choice(ne, size=min(ents_per_seq, ne), replace=False).tolist())
         pick |= {0, 1, ne - 1}
-        # tile and piece boundaries: every 31st / 32nd entry region
-        pick |= {min(ne - 1, 31 * k) for k in range(1, 6)} | {min(ne - 1, 32 * k) for k in range(1, 6)}
+        # tile boundaries (32 and 64 entries per tile) and piece boundaries
+        pick |= {min(ne - 1, 32 * k + d) for k in range(1, 9) for d in (-1, 0, 1)}
+        pick |= {min(ne - 1, (ne * r) // P + d) for P in (18, 37, 74) for r in range(1, 4)
+                 for d in (-1, 0, 1)}
         entries += [(b, i) for i in sorted(pick)]
     Ws = {k: host64(v) for k, v in t.items() if k.startswith("W") or k.startswith("B")}
     refs, got = [], []
