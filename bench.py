@@ -613,6 +613,12 @@ def run_profile_case(kind: str, launches: int = 3):
                 kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=M_CSA)
             else:
                 kvc.hca_compress(t["Ca"], t["Za"], Bh, m=M_HCA)
+    elif kind == "hca_n65536":  # the 65536-token HCA workload itself (134 MB, few windows)
+        t = synth.stream_inputs_torch("hca", 1, 65536, C, M_HCA, "bf16", seed=0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        for _ in range(launches):
+            flush.zero_()
+            kvc.hca_compress(t["C"], t["Z"], t["B"], m=M_HCA)
     elif kind == "csa_fused":
         n, d = 4096, 7168
         f = synth.fused_inputs_torch("csa", 1, n, d, C, M_CSA, seed=0)
@@ -646,7 +652,7 @@ def main():
                              "decode_entries", "cache_long"],
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "
                          "time one kernel on its own workload")
-    ap.add_argument("--profile-case", choices=["csa", "hca", "csa_fused", "hca_fused"],
+    ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "csa_fused", "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
     if args.profile_case:
