@@ -498,7 +498,9 @@ def _workload(name, dev):
             nbytes = (2 * ne * m + 2 * (ne - 1) * m) * c * es + 2 * m * c * 4 + ne * c * es
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // m,
                     bound="hbm", units=float(nbytes), flush=nbytes < 4 * (126 << 20),
-                    kernel="csa_small_m_kernel" if mode == "csa" else "window_pool_kernel",
+                    kernel=("csa_small_m_kernel" if mode == "csa" else
+                            "window_pipe_kernel (8 row groups)" if n == 65536 else
+                            "window_pool_kernel"),
                     config={"workload": f"{mode.upper()} streams: batch 1, n={n}, c={c}, m={m}, "
                                         f"{dt} in/out", "n": n, "c": c, "m": m})
     raise SystemExit(f"unknown workload {name}")

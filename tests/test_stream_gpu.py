@@ -91,6 +91,10 @@ HCA_CASES = [
     (2, 160 * 4, 256, 160),
     (1, 320 * 2 + 5, 16, 320),
     (1, 7 * 11, 512, 7),
+    # mid-size window counts: 8 row groups per window; m = 100 leaves the row groups
+    # uneven numbers of rows
+    (1, 32 * 200, 256, 32),
+    (1, 100 * 300 + 7, 136, 100),
 ]
 
 
