@@ -415,6 +415,38 @@ def _workload(name, dev):
                     config={"workload": f"HCA fused projection + pool: batch {b}, n={n}, H d={d} "
                                         f"bf16, W_kv, W_z [{d}, {c}], m'=128, bf16 out",
                             "batch": b, "n": n, "d": d, "c": c, "m": 128})
+    if name == "indexer_decode":
+        T, H, S, k = 8, 64, 1 << 18, 1024
+        t = synth.indexer_inputs_torch(T, H, T * S, seed=0, device=dev)
+        t["key_start"] = torch.arange(T, dtype=torch.int64, device=dev) * S
+        t["n_visible"] = torch.full((T,), S, dtype=torch.int64, device=dev)
+        scores = torch.empty((T, S), dtype=torch.float32, device=dev)
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        val = torch.empty((T, k), dtype=torch.float32, device=dev)
+
+        def score(x, st):
+            kvc.lightning_indexer_scores(x["q"], x["w"], x["K"], x["key_start"], x["n_visible"],
+                                         S, scores=scores, stream=st)
+
+        def select(x, st):
+            kvc.indexer_topk(scores, x["n_visible"], k, S, out_idx=idx, out_score=val, stream=st)
+
+        def launch(x, st):
+            score(x, st)
+            select(x, st)
+        score_bytes = float(T * S * 128 * 2 + T * S * 4 + T * H * 128 * 2 + T * H * 4)
+        topk_bytes = float(T * S * 4 + T * k * 8)
+        return dict(inputs=t, launch=launch, outputs=[idx, val], tokens=T * S * 4, entries=T * S,
+                    bound="hbm", units=score_bytes, flush=False, resident=("K",),
+                    kernel="indexer_score_kernel (tcgen05, keys on M, heads on N)",
+                    parts=[dict(name="indexer_score_kernel", launch=score, units=score_bytes,
+                                bound="hbm"),
+                           dict(name="indexer_topk_kernel", launch=select, units=topk_bytes,
+                                bound="hbm")],
+                    config={"workload": f"lightning-indexer decode step: {T} sequences of 2^20 "
+                                        f"tokens ({S} compressed indexer keys each, 128 wide, "
+                                        f"bf16), one {H}-head query per sequence, top-{k}",
+                            "queries": T, "keys_per_query": S, "heads": H, "k": k})
     if name == "scalar_long":
         n, c, m = 1 << 20, 512, 4
         t = synth.scalar_inputs_torch("csa", 1, n, c, m, "bf16", seed=0, device=dev)
@@ -539,6 +571,21 @@ def run_workload(args):
     ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), world)
     if kvc.device_status(st) != kvc.KVC_OK:
         raise SystemExit("device error in the timed region")
+    # workloads made of several kernels: time each on its own as well (same loop)
+    part_ms = {}
+    for part in w.get("parts", ()):
+        pev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in pev:
+            if flush is not None:
+                flush.zero_()
+            a.record(st)
+            part["launch"](w["inputs"], st)
+            b.record(st)
+        torch.cuda.synchronize()
+        part_ms[part["name"]] = max_over_ranks(
+            statistics.median(a.elapsed_time(b) for a, b in pev), world)
     # e2e: pinned host inputs -> device, the call, outputs -> pinned host
     # inputs the workload keeps resident in device memory (a decode step's KV streams) are
     # not copied; everything else is
@@ -566,10 +613,12 @@ def run_workload(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
     peak, kind = _peak(w["bound"])
+    # the roofline is the dominant kernel's: its own time when the step has several
+    rms = part_ms[w["parts"][0]["name"]] if w.get("parts") else ms
     if w["bound"] == "tensor":
-        ach, unit = w["units"] / (ms * 1e-3) / 1e12, "TFLOP/s"
+        ach, unit = w["units"] / (rms * 1e-3) / 1e12, "TFLOP/s"
     else:
-        ach, unit = w["units"] / (ms * 1e-3) / 1e9, "GB/s"
+        ach, unit = w["units"] / (rms * 1e-3) / 1e9, "GB/s"
     if rank == 0:
         line = {
             "metric": METRIC, "value": world * w["tokens"] / (ms * 1e-3), "unit": "tokens/s",
@@ -586,10 +635,17 @@ def run_workload(args):
                          "traffic": None,
                          ("algorithmic_flops" if w["bound"] == "tensor" else "algorithmic_bytes"):
                              w["units"]},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * max(1, len(w.get("parts", ()))),
             "e2e": {"value": world * w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         }
+        if w.get("parts"):
+            line["kernels"] = {}
+            for part in w["parts"]:
+                pm = part_ms[part["name"]]
+                pk, _ = _peak(part["bound"])
+                a_ = part["units"] / (pm * 1e-3) / 1e9
+                line["kernels"][part["name"]] = {"ms": pm, "GB/s": a_, "frac": a_ / pk}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -621,6 +677,15 @@ def run_profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             flush.zero_()
             kvc.hca_compress(t["C"], t["Z"], t["B"], m=M_HCA)
+    elif kind == "indexer":  # 4 queries x 131072 keys (K 128 MB), top-1024
+        T, S = 4, 1 << 17
+        t = synth.indexer_inputs_torch(T, 64, T * S, seed=0)
+        ks = torch.arange(T, dtype=torch.int64, device="cuda") * S
+        nv = torch.full((T,), S, dtype=torch.int64, device="cuda")
+        sc = torch.empty((T, S), dtype=torch.float32, device="cuda")
+        for _ in range(launches):
+            kvc.lightning_indexer_scores(t["q"], t["w"], t["K"], ks, nv, S, scores=sc)
+            kvc.indexer_topk(sc, nv, 1024, S)
     elif kind == "csa_fused":
         n, d = 4096, 7168
         f = synth.fused_inputs_torch("csa", 1, n, d, C, M_CSA, seed=0)
@@ -651,10 +716,10 @@ def main():
     ap.add_argument("--workload", default="long",
                     choices=["long", "fused_csa", "fused_hca", "hca_n65536", "csa_f32_n1024",
                              "indexer_keys", "fused_indexer_keys", "scalar_long",
-                             "decode_entries", "cache_long"],
+                             "decode_entries", "cache_long", "indexer_decode"],
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "
                          "time one kernel on its own workload")
-    ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "csa_fused", "hca_fused"],
+    ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "indexer", "csa_fused", "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
     if args.profile_case:

@@ -224,6 +224,48 @@ KVC_API kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, cons
                                    int64_t c, int32_t m,
                                    void* out, kvc_dtype out_dtype, kvc_stream stream);
 
+/* ---------------------------------------------------------------- lightning indexer
+ * [CSA] §4 (Lightning Indexer) and §5: CSA attends only to the compressed entries that
+ * its indexer ranks highest.  Query t's score for compressed indexer key s is
+ *     I[t, s] = sum_h w[t, h] * max(0, q[t, h] . K[s])
+ * (one key per entry, shared by all indexer heads; 64 heads of width 128 on the page),
+ * and the selected entries are those with the k largest scores (k = 1024 / 512).  The
+ * keys are the compressed entries of an indexer compressor (csa_compress with c = 128).
+ * Candidates.  Query t scores the n_visible[t] keys K[key_start[t] .. key_start[t] +
+ *   n_visible[t] - 1] (its own sequence in a packed key array): a decode step passes all
+ *   of its sequence's entries, a prefill query only the complete blocks before it.
+ * Check on the device.  A query whose window leaves [0, key_rows) or whose n_visible
+ *   exceeds max_visible is skipped (its rows untouched) and reported by
+ *   kvc_device_status() as KVC_ERR_INDEX. */
+
+/* Scores: scores[t * ld + s] = I[t, s] (fp32) for s < n_visible[t]; the rest of each
+ * row is left untouched.
+ *   q [T, H, D] bf16 with D == 128 and H a multiple of 16 in [16, 128];
+ *   w [T, H] fp32 (4-byte aligned); K [key_rows, D] bf16;
+ *   key_start, n_visible [T] int64 (8-byte aligned); scores [T, ld] fp32, ld >= max_visible;
+ *   max_visible (host) an upper bound of every n_visible[t] (it sizes the launch).
+ * q, K and scores are 16-byte aligned.  Dot products accumulate in fp32 on the tensor
+ * cores (bf16 products are exact in fp32); ReLU and the head-weighted sum in fp32. */
+KVC_API kvc_status lightning_indexer_scores(const void* q, const float* w, const void* K,
+                                    const int64_t* key_start, const int64_t* n_visible,
+                                    int64_t T, int32_t H, int32_t D, int64_t key_rows,
+                                    int64_t max_visible, float* scores, int64_t ld,
+                                    kvc_stream stream);
+
+/* Top-k of each score row over its first n_visible[t] entries:
+ *   out_idx[t * k + j] (int32), j < k: the entry indices in descending score order,
+ *   equal scores by ascending index (-0.0 counts as 0.0); -1 for j >= n_visible[t].
+ *   out_score[t * k + j] (fp32, may be NULL): the matching scores, -inf past the end.
+ * 1 <= k <= 2048; max_visible <= kvc_topk_max_candidates(); scores [T, ld] fp32,
+ * 16-byte aligned with ld a multiple of 4; n_visible as above.  The result is exact
+ * for the given scores (no NaN among them). */
+KVC_API kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* n_visible,
+                                int64_t T, int64_t max_visible, int32_t k, int32_t* out_idx,
+                                float* out_score, kvc_stream stream);
+
+/* The largest n_visible indexer_topk accepts (its candidates stay on chip). */
+KVC_API int64_t kvc_topk_max_candidates(void);
+
 /* Synchronises `stream`, then reports and clears the device-side error word that
  * kernels set when a bounded wait gives up: KVC_ERR_TIMEOUT if one did, KVC_ERR_CUDA
  * if the synchronisation failed, else KVC_OK. */

@@ -594,6 +594,57 @@ kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* 
   return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+kvc_status lightning_indexer_scores(const void* q, const float* w, const void* K,
+                                    const int64_t* key_start, const int64_t* n_visible,
+                                    int64_t T, int32_t H, int32_t D, int64_t key_rows,
+                                    int64_t max_visible, float* scores, int64_t ld,
+                                    kvc_stream stream) {
+  if (T < 0 || key_rows < 0 || max_visible < 0 || ld < 0) return KVC_ERR_SHAPE;
+  if (D != 128 || H < 16 || H > 128 || H % 16 != 0) return KVC_ERR_UNSUPPORTED;
+  if (ld < max_visible) return KVC_ERR_SHAPE;
+  int64_t tmp = 0;
+  if (!mul_ok(T, ld, &tmp) || !mul_ok(tmp, 4, &tmp) || !mul_ok(T, H, &tmp) ||
+      !mul_ok(key_rows, D * 2, &tmp))
+    return KVC_ERR_SHAPE;
+  if (T * H > (int64_t(1) << 31) - 1 || key_rows > (int64_t(1) << 31) - 1 - 256)
+    return KVC_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  if (T == 0 || max_visible == 0) return KVC_OK;
+  if (!q || !w || !K || !key_start || !n_visible || !scores) return KVC_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(scores, 16) || !aligned(w, 4) ||
+      !aligned(key_start, 8) || !aligned(n_visible, 8))
+    return KVC_ERR_ALIGN;
+  const void* ps[] = {q, w, K, key_start, n_visible, scores};
+  kvc_status s = check_ptrs(ps, 6);
+  if (s != KVC_OK) return s;
+  kvc::IndexerProblem p{q, w, K, key_start, n_visible, T, key_rows, max_visible, ld, H, scores};
+  return kvc::launch_indexer_scores(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* n_visible, int64_t T,
+                        int64_t max_visible, int32_t k, int32_t* out_idx, float* out_score,
+                        kvc_stream stream) {
+  if (T < 0 || max_visible < 0 || ld < 0 || k < 1) return KVC_ERR_SHAPE;
+  if (k > 2048 || max_visible > kvc::topk_max_candidates()) return KVC_ERR_UNSUPPORTED;
+  if (ld < max_visible || ld % 4 != 0) return KVC_ERR_SHAPE;
+  int64_t tmp = 0;
+  if (!mul_ok(T, ld, &tmp) || !mul_ok(tmp, 4, &tmp) || !mul_ok(T, k, &tmp) ||
+      T > ((int64_t(1) << 31) - 1) / 8)
+    return KVC_ERR_SHAPE;
+  if (T == 0) return KVC_OK;
+  if (!scores || !n_visible || !out_idx) return KVC_ERR_NULL;
+  if (!aligned(scores, 16) || !aligned(n_visible, 8) || !aligned(out_idx, 4) ||
+      (out_score && !aligned(out_score, 4)))
+    return KVC_ERR_ALIGN;
+  const void* ps[] = {scores, n_visible, out_idx};
+  kvc_status s = check_ptrs(ps, 3);
+  if (s == KVC_OK && out_score) s = check_device_ptr(out_score);
+  if (s != KVC_OK) return s;
+  kvc::TopkProblem p{scores, n_visible, T, max_visible, ld, k, out_idx, out_score};
+  return kvc::launch_indexer_topk(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int64_t kvc_topk_max_candidates(void) { return kvc::topk_max_candidates(); }
+
 kvc_status kvc_device_status(kvc_stream stream) {
   return kvc::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));
 }

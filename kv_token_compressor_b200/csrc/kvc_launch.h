@@ -64,6 +64,34 @@ struct FusedProblem {
 
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st);
 
+// A validated lightning-indexer scoring problem (lightning_indexer_scores).
+struct IndexerProblem {
+  const void* q;  // [T, H, 128] bf16
+  const float* w;  // [T, H]
+  const void* K;  // [key_rows, 128] bf16
+  const int64_t* key_start;
+  const int64_t* n_visible;
+  int64_t T, key_rows, max_visible, ld;
+  int H;
+  float* scores;  // [T, ld]
+};
+kvc_status launch_indexer_scores(const IndexerProblem& p, cudaStream_t st);
+
+// A validated top-k problem (indexer_topk).
+struct TopkProblem {
+  const float* scores;  // [T, ld]
+  const int64_t* n_visible;
+  int64_t T, max_visible, ld;
+  int k;
+  int32_t* out_idx;   // [T, k]
+  float* out_score;   // [T, k] or nullptr
+};
+kvc_status launch_indexer_topk(const TopkProblem& p, cudaStream_t st);
+int64_t topk_max_candidates();
+// Reads and clears the indexer kernels' error word (no synchronisation): bit 0 a bounded
+// wait gave up, bit 1 a query's candidate window was out of range.
+unsigned int read_and_clear_indexer_error(bool* failed);
+
 // Device error words: bounded waits that gave up (fused kernels) and listed entries out
 // of range (streaming kernels).  Synchronises the stream first.
 kvc_status read_and_clear_device_error(cudaStream_t st);

@@ -61,6 +61,10 @@ SIGNATURES = {
                                                   _p, _p, _p]),
     "hca_compress_entries_cache": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i32, _p, _p,
                                                   _p, _i64, _i32, _p, _d, _d, _f, _p, _p, _p]),
+    "lightning_indexer_scores": (ctypes.c_int, [_p, _p, _p, _p, _p, _i64, _i32, _i32, _i64, _i64, _p,
+                                                _i64, _p]),
+    "indexer_topk": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i32, _p, _p, _p]),
+    "kvc_topk_max_candidates": (_i64, []),
 }
 
 _lib = None
@@ -346,6 +350,47 @@ def hca_compress_fused_proj(H, W_kv, W_z, B, batch: int, n: int, m: int = 128, o
                                        _ptr(out), _dtype_code(out_dtype), _stream(stream))
     _check(st, "hca_compress_fused_proj")
     return out
+
+
+def lightning_indexer_scores(q, w, K, key_start, n_visible, max_visible: int, scores=None,
+                             stream=None):
+    """Lightning-indexer scores: q [T, H, 128] bf16, w [T, H] fp32, K [rows, 128] bf16,
+    key_start / n_visible device int64 [T]; max_visible bounds n_visible.  Returns (or
+    fills) scores [T, ld] fp32 with scores[t, s] = sum_h w[t, h] relu(q[t, h] . K[key_start[t]
+    + s]) for s < n_visible[t] (the rest of each row untouched)."""
+    torch = _torch()
+    T, H, D = q.shape
+    if scores is None:
+        ld = max(4, -(-int(max_visible) // 4) * 4)
+        scores = torch.zeros((T, ld), dtype=torch.float32, device=q.device)
+    if scores.dim() != 2 or scores.shape[0] != T or scores.dtype != torch.float32:
+        raise ValueError("scores must be fp32 [T, ld]")
+    st = lib().lightning_indexer_scores(_ptr(q), _ptr(w), _ptr(K), _index(key_start, T),
+                                        _index(n_visible, T), T, H, D, K.shape[0], int(max_visible),
+                                        _ptr(scores), scores.shape[1], _stream(stream))
+    _check(st, "lightning_indexer_scores")
+    return scores
+
+
+def indexer_topk(scores, n_visible, k: int, max_visible: int, out_idx=None, out_score=None,
+                 want_scores: bool = True, stream=None):
+    """Top-k of every score row over its first n_visible[t] entries: (idx int32 [T, k],
+    scores fp32 [T, k] or None), descending, equal scores by ascending index, -1 / -inf
+    past n_visible[t]."""
+    torch = _torch()
+    T, ld = scores.shape
+    out_idx = _out(out_idx, (T, k), torch.int32, scores)
+    if want_scores:
+        out_score = _out(out_score, (T, k), torch.float32, scores)
+    st = lib().indexer_topk(_ptr(scores), ld, _index(n_visible, T), T, int(max_visible), k,
+                            _ptr(out_idx), _ptr(out_score) if want_scores else None,
+                            _stream(stream))
+    _check(st, "indexer_topk")
+    return out_idx, (out_score if want_scores else None)
+
+
+def topk_max_candidates() -> int:
+    return int(lib().kvc_topk_max_candidates())
 
 
 def device_status(stream=None) -> int:

@@ -13,7 +13,10 @@ Distributions (N(mu, var) notation, second argument = variance):
   independently for Z^a and Z^b, added to all c channels of that row in fp32 before the
   bf16 rounding (the long-context workload, lo = 4, stresses the softmax range);
 * position biases B^a, B^b (m x c) and B (m' x c): N(0, 0.1), fp32;
-* hidden states H: N(0, 1) -> bf16; projections W (d x c): N(0, 1/d) -> bf16.
+* hidden states H: N(0, 1) -> bf16; projections W (d x c): N(0, 1/d) -> bf16;
+* lightning indexer: queries q [T, H, 128] and compressed indexer keys K [rows, 128]
+  N(0, 1) -> bf16, head weights w [T, H] N(0, 1/H) fp32 (the pages give no
+  distributions; these keep every head's dot product O(sqrt(128)) and the scores O(1)).
 
 Draw order for a given seed (numpy ``default_rng(seed)``): the streams in the order
 listed in the returned dict, then the offsets, then the biases.  Large workloads can be
@@ -33,6 +36,8 @@ __all__ = [
     "fused_inputs_torch",
     "scalar_inputs",
     "scalar_inputs_torch",
+    "indexer_inputs",
+    "indexer_inputs_torch",
     "WORKLOADS",
 ]
 
@@ -178,6 +183,28 @@ def scalar_inputs_torch(mode: str, batch: int, n: int, c: int, m: int, dtype: st
     for k in (("ba", "bb") if mode == "csa" else ("b",)):
         out[k] = torch.randn((m,), generator=g, device=device) * float(np.sqrt(bias_var))
     return out
+
+
+def indexer_inputs(T: int, H: int, rows: int, D: int = 128, seed: int = 0):
+    """Host inputs of the lightning indexer: q [T, H, D], w [T, H], K [rows, D] (fp32
+    arrays holding bf16 values for q and K).  Draw order: q, K, w."""
+    rng = np.random.default_rng(seed)
+    q = round_to_bf16(_normal(rng, (T, H, D)))
+    K = round_to_bf16(_normal(rng, (rows, D)))
+    w = _normal(rng, (T, H), 1.0 / H)
+    return dict(q=q, K=K, w=w)
+
+
+def indexer_inputs_torch(T: int, H: int, rows: int, D: int = 128, seed: int = 0, device="cuda"):
+    """Same distributions as :func:`indexer_inputs`, generated on ``device``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    q = torch.randn((T, H, D), generator=g, device=device).to(torch.bfloat16)
+    K = torch.randn((rows, D), generator=g, device=device).to(torch.bfloat16)
+    w = torch.randn((T, H), generator=g, device=device) * float(np.sqrt(1.0 / H))
+    return dict(q=q, K=K, w=w)
 
 
 # The five workloads, named by what they are.

@@ -262,3 +262,65 @@ def test_cache_layout_optional_parts(L):
                                         12, A, 4.0, 1.5, 1.0, A, A, None) == kvc.KVC_ERR_SHAPE
     assert L.hca_compress_entries_cache(A, A, kvc.KVC_BF16, A, 1024, 512, 128, A, A, A, 0, 64, A,
                                         128.0, 63.5, 1.0, A, A, None) == kvc.KVC_OK  # empty list
+
+
+# ------------------------------------------------------------------ lightning indexer
+
+def ix_scores(L, q=A, w=A, K=A, ks=A, nv=A, T=8, H=64, D=128, rows=1 << 20, mv=262144,
+              sc=A, ld=262144):
+    return L.lightning_indexer_scores(q, w, K, ks, nv, T, H, D, rows, mv, sc, ld, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=-1), kvc.KVC_ERR_SHAPE),
+    (dict(rows=-1), kvc.KVC_ERR_SHAPE),
+    (dict(mv=-1), kvc.KVC_ERR_SHAPE),
+    (dict(ld=1000), kvc.KVC_ERR_SHAPE),            # ld < max_visible
+    (dict(D=64), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(H=8), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(H=136), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(H=72), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(rows=1 << 31), kvc.KVC_ERR_UNSUPPORTED),  # TMA rows are 32-bit
+    (dict(q=None), kvc.KVC_ERR_NULL),
+    (dict(nv=None), kvc.KVC_ERR_NULL),
+    (dict(sc=None), kvc.KVC_ERR_NULL),
+    (dict(q=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(K=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(sc=A + 4), kvc.KVC_ERR_ALIGN),
+    (dict(w=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(ks=A + 4), kvc.KVC_ERR_ALIGN),
+])
+def test_indexer_scores_rejects_before_launch(L, kw, status):
+    assert ix_scores(L, **kw) == status
+
+
+def test_indexer_scores_empty(L):
+    assert ix_scores(L, T=0, q=None, K=None) == kvc.KVC_OK
+    assert ix_scores(L, mv=0, ld=0, q=None) == kvc.KVC_OK
+
+
+def ix_topk(L, sc=A, ld=262144, nv=A, T=8, mv=262144, k=1024, idx=A, val=A):
+    return L.indexer_topk(sc, ld, nv, T, mv, k, idx, val, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), kvc.KVC_ERR_SHAPE),
+    (dict(k=2049), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(mv=327681, ld=327684), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(ld=262146), kvc.KVC_ERR_SHAPE),          # ld not a multiple of 4
+    (dict(ld=1000), kvc.KVC_ERR_SHAPE),
+    (dict(T=-1), kvc.KVC_ERR_SHAPE),
+    (dict(sc=None), kvc.KVC_ERR_NULL),
+    (dict(idx=None), kvc.KVC_ERR_NULL),
+    (dict(sc=A + 4), kvc.KVC_ERR_ALIGN),
+    (dict(nv=A + 4), kvc.KVC_ERR_ALIGN),
+    (dict(idx=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(val=A + 2), kvc.KVC_ERR_ALIGN),
+])
+def test_indexer_topk_rejects_before_launch(L, kw, status):
+    assert ix_topk(L, **kw) == status
+
+
+def test_indexer_topk_limits(L):
+    assert L.kvc_topk_max_candidates() == 8 * 40960
+    assert ix_topk(L, T=0, sc=None, idx=None) == kvc.KVC_OK

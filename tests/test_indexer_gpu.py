@@ -1,0 +1,155 @@
+"""GPU parity of the lightning indexer (lightning_indexer_scores / indexer_topk through the C
+ABI) against the fp64 oracle on the same seeded inputs.
+
+Scores are fp32 outputs: within 1e-5 of the row's largest |score| of the oracle.  The
+top-k is compared bit for bit with the oracle's selection over the SAME fp32 scores the
+kernel was given (several entries can share a score; the order is fixed by the index), and
+end to end against the oracle's fp64 scores up to the scores' own rounding."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from kv_token_compressor_b200 import kvc, synth
+from oracle import indexer as IX
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(d):
+    return {"q": torch.from_numpy(d["q"]).cuda().to(torch.bfloat16),
+            "K": torch.from_numpy(d["K"]).cuda().to(torch.bfloat16),
+            "w": torch.from_numpy(d["w"]).cuda()}
+
+
+def _i64(xs):
+    return torch.tensor(list(xs), dtype=torch.int64, device="cuda")
+
+
+def _scores(t, ks, nv, max_visible, ld=None, fill=-12345.0):
+    T = t["q"].shape[0]
+    ld = ld or max(4, -(-max_visible // 4) * 4)
+    out = torch.full((T, ld), fill, dtype=torch.float32, device="cuda")
+    kvc.lightning_indexer_scores(t["q"], t["w"], t["K"], _i64(ks), _i64(nv), max_visible, scores=out)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("H", [64, 16, 48, 128])
+def test_scores_windows(H):
+    rows = 3000
+    d = synth.indexer_inputs(5, H, rows, seed=H)
+    t = _dev(d)
+    ks = [0, 100, 2999, 1500, 7]
+    nv = [3000, 1029, 1, 0, 128]
+    out = _scores(t, ks, nv, 3000)
+    assert kvc.device_status() == kvc.KVC_OK
+    ref = IX.indexer_scores(d["q"], d["w"], d["K"], ks, nv)
+    got = out.cpu().numpy()
+    for i in range(5):
+        r = ref[i]
+        if len(r):
+            tol = 1e-5 * max(np.max(np.abs(r)), 1e-30)
+            assert np.max(np.abs(got[i, :nv[i]] - r)) <= tol, (H, i)
+        assert np.all(got[i, nv[i]:3000] == -12345.0), "entries past n_visible were written"
+
+
+def test_scores_bad_window_is_skipped_and_reported():
+    d = synth.indexer_inputs(3, 64, 500, seed=1)
+    t = _dev(d)
+    ks, nv = [0, 450, 10], [300, 100, 20]  # query 1 runs past the keys
+    out = _scores(t, ks, nv, 300)
+    assert kvc.device_status() == kvc.KVC_ERR_INDEX
+    assert kvc.device_status() == kvc.KVC_OK
+    got = out.cpu().numpy()
+    assert np.all(got[1] == -12345.0)
+    ref = IX.indexer_scores(d["q"][[0, 2]], d["w"][[0, 2]], d["K"], [0, 10], [300, 20])
+    assert np.allclose(got[0, :300], ref[0], rtol=0, atol=1e-5 * np.max(np.abs(ref[0])))
+    assert np.allclose(got[2, :20], ref[1], rtol=0, atol=1e-5 * np.max(np.abs(ref[1])))
+    # n_visible above max_visible is refused the same way
+    out2 = torch.full((1, 300), -1.0, device="cuda")
+    tt = {k: v[:1] for k, v in t.items() if k != "K"}
+    kvc.lightning_indexer_scores(tt["q"], tt["w"], t["K"], _i64([0]), _i64([300]), 200, scores=out2)
+    assert kvc.device_status() == kvc.KVC_ERR_INDEX
+    assert torch.all(out2 == -1.0).item()
+
+
+def _topk_gpu(scores, nv, k, max_visible):
+    idx, val = kvc.indexer_topk(scores, _i64(nv), k, max_visible)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), val.cpu().numpy()
+
+
+@pytest.mark.parametrize("k", [1, 7, 512, 1024, 2048])
+@pytest.mark.parametrize("kind", ["ties", "continuous"])
+def test_topk_exact_given_scores(k, kind):
+    rng = np.random.default_rng(k + len(kind))
+    nv = [0, 1, 5, 1000, 4099, 100003, 327680]
+    ld = 327680
+    S = np.full((len(nv), ld), np.nan, dtype=np.float32)  # past n_visible: never read
+    for i, n in enumerate(nv):
+        if kind == "ties":  # few distinct values, many exact zeros (as ReLU makes)
+            v = rng.integers(-2, 5, size=n).astype(np.float32)
+            v[rng.random(n) < 0.5] = 0.0
+        else:
+            v = rng.standard_normal(n).astype(np.float32)
+        S[i, :n] = v
+    idx, val = _topk_gpu(torch.from_numpy(S).cuda(), nv, k, ld)
+    assert kvc.device_status() == kvc.KVC_OK
+    for i, n in enumerate(nv):
+        ref_idx, ref_val = IX.topk_row(S[i, :n].astype(np.float64), k)
+        assert np.array_equal(idx[i], ref_idx), (k, kind, n)
+        assert np.array_equal(val[i].astype(np.float64), ref_val), (k, kind, n)
+
+
+def test_topk_signed_zero_and_negatives():
+    """-0.0 and 0.0 are the same score (ties by index); negative scores order correctly."""
+    v = np.array([0.0, -0.0, -1.5, 2.0, -0.0, 0.0, -3.0, 2.0, -1.5], dtype=np.float32)
+    S = np.zeros((1, 12), dtype=np.float32)
+    S[0, :9] = v
+    idx, val = _topk_gpu(torch.from_numpy(S).cuda(), [9], 7, 9)
+    assert idx[0].tolist() == [3, 7, 0, 1, 4, 5, 2]
+    assert val[0].tolist()[:2] == [2.0, 2.0]
+
+
+def test_topk_row_past_max_visible_is_reported():
+    S = torch.zeros((2, 8), device="cuda")
+    idx = torch.full((2, 4), 77, dtype=torch.int32, device="cuda")
+    kvc.indexer_topk(S, _i64([8, 3]), 4, 4, out_idx=idx)
+    assert kvc.device_status() == kvc.KVC_ERR_INDEX
+    assert idx[0].tolist() == [77] * 4          # skipped row untouched
+    assert idx[1].tolist() == [0, 1, 2, -1]
+
+
+def test_decode_step_end_to_end():
+    """A decode step: 4 sequences of 2^20 tokens (262144 compressed keys each), one query
+    of 64 heads per sequence, k = 1024.  Full score rows against the fp64 oracle, the top-k
+    bit-exact on the kernel's scores, and against the oracle's fp64 scores up to rounding."""
+    T, H, S, k = 4, 64, 262144, 1024
+    t = synth.indexer_inputs_torch(T, H, T * S, seed=5)
+    ks, nv = [i * S for i in range(T)], [S, S - 1, S - 1000, 77777]
+    out = torch.empty((T, S), dtype=torch.float32, device="cuda")
+    kvc.lightning_indexer_scores(t["q"], t["w"], t["K"], _i64(ks), _i64(nv), S, scores=out)
+    idx, val = kvc.indexer_topk(out, _i64(nv), k, S)
+    torch.cuda.synchronize()
+    assert kvc.device_status() == kvc.KVC_OK
+    q = t["q"].float().cpu().numpy()
+    w = t["w"].cpu().numpy()
+    K = t["K"].float().cpu().numpy()
+    got = out.cpu().numpy()
+    gidx = idx.cpu().numpy()
+    for i in range(T):
+        ref = IX.indexer_scores_row(q[i], w[i], K[ks[i]:ks[i] + nv[i]])
+        tol = 1e-5 * np.max(np.abs(ref))
+        assert np.max(np.abs(got[i, :nv[i]] - ref)) <= tol
+        # exact on the kernel's own scores
+        ref_idx, _ = IX.topk_row(got[i, :nv[i]].astype(np.float64), k)
+        assert np.array_equal(gidx[i], ref_idx)
+        # against the fp64 scores: everything clearly above the k-th score is selected,
+        # and nothing selected is clearly below it
+        kth = np.sort(ref)[::-1][k - 1]
+        sel = set(gidx[i].tolist())
+        assert all(j in sel for j in np.nonzero(ref > kth + 2 * tol)[0])
+        assert all(ref[j] >= kth - 2 * tol for j in sel)
