@@ -63,9 +63,8 @@ __host__ __device__ constexpr uint32_t idesc_kk(int n) {
          (static_cast<uint32_t>(kKT >> 4) << 24);
 }
 
-__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          bool honour_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_bounded_slow(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag, bool honour_abort) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -76,6 +75,12 @@ __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+// Bounded wait; a phase that has already completed costs one try_wait and no call.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bounded_slow(bar, parity, abort_flag, honour_abort);
 }
 
 // The candidate window of query t; false (and the error bit) when it is out of range.
@@ -91,6 +96,21 @@ __device__ __forceinline__ Window query_window(const ScoreArgs& a, int64_t t) {
          w.start <= a.key_rows - w.count;
   return w;
 }
+
+// (query t, key tile j) of unit u, advanced one unit at a time (64-bit division once per
+// CTA: in every unit it sat on the MMA thread's critical path).
+struct UnitCursor {
+  int64_t t, j, tiles;
+  __device__ UnitCursor(const ScoreArgs& a, int64_t u)
+      : t(u / a.tiles_per_query), j(u - (u / a.tiles_per_query) * a.tiles_per_query),
+        tiles(a.tiles_per_query) {}
+  __device__ __forceinline__ void next() {
+    if (++j == tiles) {
+      j = 0;
+      ++t;
+    }
+  }
+};
 
 // Units u = (query t, key tile j), t-major; each CTA takes one contiguous range so that
 // consecutive tiles share the query's q tile.  Every role walks the same units and takes
@@ -158,8 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t cur_t = -1;
       Window win{0, 0, false};
       bool ok = true;
-      for (int64_t u = lo; u < hi && ok; ++u) {
-        const int64_t t = u / a.tiles_per_query, j = u - t * a.tiles_per_query;
+      UnitCursor cu(a, lo);
+      for (int64_t u = lo; u < hi && ok; ++u, cu.next()) {
+        const int64_t t = cu.t, j = cu.j;
         if (t != cur_t) {
           win = query_window(a, t);
           if (!win.ok) atomicOr(&g_indexer_error, 2u);  // the query is skipped
@@ -208,9 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       Window win{0, 0, false};
       uint32_t n = 0;  // tiles issued (accumulator rotation)
       const uint32_t idesc = idesc_kk(H);
+      // shared memory stays below 256 KB, so address >> 4 fits the 14-bit field with room
+      // for every offset added to it
+      const uint64_t adesc_base = smem_desc(smem_u32(ktiles), 16, 1024, 2);
+      const uint64_t bdesc_base = smem_desc(smem_u32(qslots), 16, 1024, 2);
       bool ok = true;
-      for (int64_t u = lo; u < hi && ok; ++u) {
-        const int64_t t = u / a.tiles_per_query, j = u - t * a.tiles_per_query;
+      UnitCursor cu(a, lo);
+      for (int64_t u = lo; u < hi && ok; ++u, cu.next()) {
+        const int64_t t = cu.t, j = cu.j;
         if (t != cur_t) win = query_window(a, t);
         if (!win.ok || j * kKT >= win.count) {
           cur_t = t;
@@ -233,16 +259,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t ka = smem_u32(ktiles + stage * kTile);
-        const uint32_t qa = smem_u32(qslots + (qcount & 1) * kQSlot);
+        // both operands K-major, 128-byte swizzle: k-slice ks is 32 bytes into the 128-byte
+        // rows of box ks / 4; 8-row groups 1024 bytes apart.  Only the start-address field
+        // (address >> 4, low bits) changes between slices, so it is added to a base.
+        const uint64_t ad0 = adesc_base + ((stage * kTile) >> 4);
+        const uint64_t bd0 = bdesc_base + (((qcount & 1) * kQSlot) >> 4);
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-          // both operands K-major, 128-byte swizzle: k-slice ks is 32 bytes into the
-          // 128-byte rows of box ks / 4; 8-row groups 1024 bytes apart
-          const uint32_t off = (ks & 3) * 32;
-          const uint64_t ad = smem_desc(ka + (ks >> 2) * kHalf + off, 16, 1024, 2);
-          const uint64_t bd = smem_desc(qa + (ks >> 2) * (kQSlot / 2) + off, 16, 1024, 2);
-          umma_bf16(tmem_base + buf * 128, ad, bd, idesc, ks != 0 ? 1u : 0u);
+          const uint32_t off = ((ks >> 2) * kHalf + (ks & 3) * 32) >> 4;
+          const uint32_t offq = ((ks >> 2) * (kQSlot / 2) + (ks & 3) * 32) >> 4;
+          umma_bf16(tmem_base + buf * 128, ad0 + off, bd0 + offq, idesc, ks != 0 ? 1u : 0u);
         }
         umma_commit(&empty[stage]);
         umma_commit(&tfull[buf]);
@@ -271,8 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     Window win{0, 0, false};
     uint32_t n = 0;
     bool ok = true;
-    for (int64_t u = lo; u < hi && ok; ++u) {
-      const int64_t t = u / a.tiles_per_query, j = u - t * a.tiles_per_query;
+    UnitCursor cu(a, lo);
+    for (int64_t u = lo; u < hi && ok; ++u, cu.next()) {
+      const int64_t t = cu.t, j = cu.j;
       if (t != cur_t) win = query_window(a, t);
       if (!win.ok || j * kKT >= win.count) {
         cur_t = t;
@@ -333,16 +360,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Top-k: one cluster of kCluster CTAs per query row.
+// Top-k: one cluster of CL CTAs per query row (launched with the portable 8).
 // ---------------------------------------------------------------------------------
-constexpr int kCluster = 8;
-constexpr int kTkThreads = 512;
+constexpr int kCluster = 8;   // portable cluster size: the guaranteed capacity
+constexpr int kTkThreads = 1024;
 constexpr int kSlice = 40960;    // scores held on chip per CTA
 constexpr int kMaxK = 2048;
 constexpr int kBins = 256;       // radix digits of 8 bits
 constexpr int kWarps = kTkThreads / 32;
 constexpr size_t kTkSmem =
-    kSlice * 4 + (kWarps + 1) * kBins * 4 + kMaxK * 8 + kTkThreads * 4 + 64 + 2 * kWarps * 4;
+    kSlice * 4 + (kWarps + 1) * kBins * 4 + kMaxK * 8 + kTkThreads * 4 + 64 + 2 * kWarps * 4 + 128;
 
 struct TopkArgs {
   const float* scores;
@@ -407,8 +434,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
   return before;
 }
 
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1)
-    indexer_topk_kernel(const TopkArgs a) {
+template <int CL>
+__global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                      // [kSlice]
   uint32_t* hist = keys + kSlice;                                  // [kWarps][kBins]
@@ -417,9 +444,10 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
   uint32_t* scratch = reinterpret_cast<uint32_t*>(cand + kMaxK);          // [kTkThreads]
   uint32_t* info = scratch + kTkThreads;                                   // [16]
   uint32_t* wcnt = info + 16;                                              // [2][kWarps]
+  uint32_t* runs = wcnt + 2 * kWarps;                                      // [2][16]
 
-  const uint32_t rank = blockIdx.x % kCluster;
-  const int64_t t = blockIdx.x / kCluster;
+  const uint32_t rank = blockIdx.x % CL;
+  const int64_t t = blockIdx.x / CL;
   const int tid = threadIdx.x;
   const int64_t nv = a.n_visible[t];
   // the same decision in every CTA of the cluster: an out-of-range row is skipped whole
@@ -430,7 +458,7 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
   const int k = a.k;
   const int ksel = static_cast<int>(nv < k ? nv : k);
   // this CTA's candidates [lo, lo + cnt), a multiple of 4 apart
-  const int64_t per = ((nv + kCluster - 1) / kCluster + 3) & ~int64_t(3);
+  const int64_t per = ((nv + CL - 1) / CL + 3) & ~int64_t(3);
   const int64_t lo = rank * per;
   const int cnt = static_cast<int>(lo < nv ? (nv - lo < per ? nv - lo : per) : 0);
   const float* row = a.scores + t * a.ld;
@@ -459,11 +487,19 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
       }
     }
     // radix select of the ksel-th largest key: four 8-bit digits, high to low.  Each warp
-    // counts into its own histogram (the keys of a query share few leading bits, so a
-    // shared histogram would serialise on a handful of bins), the CTA sums its warps', and
-    // every CTA sums the cluster's CTA histograms through distributed shared memory.
+    // counts into its own histogram (the keys of a query share few leading bits, so one
+    // shared histogram would serialise all warps on a handful of bins), the CTA sums its
+    // warps', and every CTA sums the cluster's CTA histograms through distributed shared
+    // memory.
     const int warp = tid >> 5, lane = tid & 31;
     uint32_t* whist = hist + warp * kBins;
+    // Warp w owns candidates [w * seg, (w + 1) * seg) in every pass below, its lanes on
+    // consecutive keys (no bank conflicts), so its histogram also gives its own counts of
+    // keys above and at the final threshold.
+    const int seg = ((cnt + kWarps - 1) / kWarps + 31) & ~31;
+    const int s0 = warp * seg;
+    const int s1 = s0 + seg < cnt ? s0 + seg : cnt;
+    uint32_t wgt = 0;  // keys of the segment above the threshold (summed over the passes)
     uint32_t prefix = 0, mask = 0;
     uint32_t kk = static_cast<uint32_t>(ksel);  // rank of the wanted key among the matches
 #pragma unroll 1
@@ -471,21 +507,21 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
       const int shift = 24 - 8 * pass;
       for (int b = tid; b < kWarps * kBins; b += kTkThreads) hist[b] = 0u;
       __syncthreads();
-      for (int base = 0; base < cnt; base += kTkThreads) {  // same trip count in every lane
-        const int i = base + tid;
-        const uint32_t u = i < cnt ? keys[i] : 0u;
-        const bool match = i < cnt && (u & mask) == prefix;
-        const uint32_t active = __ballot_sync(0xffffffffu, match);
-        if (match) {
-          const uint32_t bin = (u >> shift) & (kBins - 1);
-          const int first = __ffs(active) - 1;
-          const uint32_t b0 = __shfl_sync(active, bin, first);
-          if (__ballot_sync(active, bin == b0) == active) {  // the common case: one bin
-            if (lane == first) atomicAdd(&whist[bin], __popc(active));
-          } else {
-            const uint32_t peers = __match_any_sync(active, bin);
-            if (lane == __ffs(peers) - 1) atomicAdd(&whist[bin], __popc(peers));
-          }
+      // four loads in flight per thread; lanes of a warp that hit the same bin are
+      // serialised by the shared-memory atomics (measured cheaper than aggregating them
+      // with __match_any_sync first)
+      for (int i0 = s0 + lane; i0 < s1; i0 += 128) {
+        uint32_t u[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = i0 + 32 * r;
+          u[r] = i < s1 ? keys[i] : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = i0 + 32 * r;
+          if (i < s1 && (u[r] & mask) == prefix)
+            atomicAdd(&whist[(u[r] >> shift) & (kBins - 1)], 1u);
         }
       }
       __syncthreads();
@@ -500,12 +536,12 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
       // counts the keys in higher bins
       uint32_t tot = 0;
       if (tid < kBins) {
-        uint32_t rv[kCluster];
+        uint32_t rv[CL];
 #pragma unroll
-        for (int r = 0; r < kCluster; ++r)  // all remote loads in flight before any use
+        for (int r = 0; r < CL; ++r)  // all remote loads in flight before any use
           rv[r] = ld_cluster_u32(cluster_addr_of(chist + (kBins - 1 - tid), static_cast<uint32_t>(r)));
 #pragma unroll
-        for (int r = 0; r < kCluster; ++r) tot += rv[r];
+        for (int r = 0; r < CL; ++r) tot += rv[r];
       }
       uint32_t all;
       const uint32_t above = block_exclusive_scan(tot, scratch, &all);
@@ -514,38 +550,26 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
         info[1] = kk - above;
       }
       __syncthreads();
-      prefix |= info[0] << shift;
+      const uint32_t digit = info[0];
+      {  // this warp's keys above the chosen digit (they all sort above the threshold)
+        uint32_t c = 0;
+        for (int b = static_cast<int>(digit) + 1 + lane; b < kBins; b += 32) c += whist[b];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        wgt += c;
+      }
+      if (pass == 3 && lane == 0) {  // the warp's counts above and at the threshold
+        wcnt[warp] = wgt;
+        wcnt[kWarps + warp] = whist[digit];
+      }
+      prefix |= digit << shift;
       mask |= static_cast<uint32_t>(kBins - 1) << shift;
       kk = info[1];
       cluster_sync();  // remote reads are done before the next pass rewrites the histograms
     }
     const uint32_t thr = prefix;  // the ksel-th largest key; kk of its copies are taken
-    // Per-warp counts of keys above / at the threshold.  Warp w owns candidates
-    // [w * seg, (w + 1) * seg); its lanes read consecutive keys (no bank conflicts).
-    const int seg = ((cnt + kWarps - 1) / kWarps + 31) & ~31;
-    const int s0 = warp * seg;
-    const int s1 = s0 + seg < cnt ? s0 + seg : cnt;
     const uint32_t lt = (1u << lane) - 1u;
-    uint32_t wgt = 0, weq = 0;
-    for (int i0 = s0; i0 < s1; i0 += 128) {  // four loads in flight, then the ballots
-      uint32_t u[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = i0 + 32 * r + lane;
-        u[r] = i < s1 ? keys[i] : 0u;
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const bool in = i0 + 32 * r + lane < s1;
-        wgt += __popc(__ballot_sync(0xffffffffu, in && u[r] > thr));
-        weq += __popc(__ballot_sync(0xffffffffu, in && u[r] == thr));
-      }
-    }
-    if (lane == 0) {
-      wcnt[warp] = wgt;
-      wcnt[kWarps + warp] = weq;
-    }
-    __syncthreads();
+    __syncthreads();  // every warp's counts are in wcnt
     if (tid == 0) {
       uint32_t g = 0, e = 0;
       for (int w = 0; w < kWarps; ++w) {
@@ -557,13 +581,18 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
     }
     cluster_sync();
     // the copies of the threshold go to the lowest indices: CTAs, then warps, in order
-    uint32_t base = 0, take = 0, eq_before = 0;
-    for (uint32_t r = 0; r < kCluster; ++r) {
+    uint32_t base = 0, take = 0, eq_before = 0, run_base = 0;
+    for (uint32_t r = 0; r < CL; ++r) {
       const uint32_t g = ld_cluster_u32(cluster_addr_of(info + 2, r));
       const uint32_t e = ld_cluster_u32(cluster_addr_of(info + 3, r));
       const uint32_t tk = kk > eq_before ? (kk - eq_before < e ? kk - eq_before : e) : 0u;
       if (r < rank) base += g + tk;
       if (r == rank) take = tk;
+      if (tid == 0) {  // every CTA's run of selected entries: [base, base + length)
+        runs[2 * r] = run_base;
+        runs[2 * r + 1] = g + tk;
+      }
+      run_base += g + tk;
       eq_before += e;
     }
     uint32_t pos = base, wtake = 0, web = 0;
@@ -574,8 +603,8 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
       else wtake = tk;
       web += e;
     }
-    // write the selected entries in index order into CTA 0
-    const uint32_t cbase = cluster_addr_of(cand, 0);
+    // write the selected entries in index order into this CTA's run buffer
+    pos -= base;
     uint32_t er = 0;  // threshold copies of this warp already passed
     for (int i0 = s0; i0 < s1; i0 += 128) {
       uint32_t u[4];
@@ -588,68 +617,63 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
       for (int r = 0; r < 4; ++r) {
         const int i = i0 + 32 * r + lane;
         const bool in = i < s1;
+        if (!__any_sync(0xffffffffu, in && u[r] >= thr)) continue;  // most groups
         const uint32_t eb = __ballot_sync(0xffffffffu, in && u[r] == thr);
         const bool sel = in && (u[r] > thr || (u[r] == thr && er + __popc(eb & lt) < wtake));
         const uint32_t sb = __ballot_sync(0xffffffffu, sel);
         if (sel) {
           const uint32_t index = static_cast<uint32_t>(lo + i);
-          st_cluster_u64(cbase + 8u * (pos + __popc(sb & lt)),
-                         (static_cast<unsigned long long>(u[r]) << 32) | (0xFFFFFFFFu - index));
+          cand[pos + __popc(sb & lt)] =
+              (static_cast<unsigned long long>(u[r]) << 32) | (0xFFFFFFFFu - index);
         }
         pos += __popc(sb);
         er += __popc(eb);
       }
     }
   }
-  cluster_sync();  // every selected entry is in CTA 0
-  if (rank != 0) return;
-  // CTA 0: sort descending (key, then smaller index first) and write the row.  Bitonic
-  // network over P = max(512, 2^ceil(log2 ksel)) entries held in registers, element
-  // e = r * 512 + tid in x[r]: strides up to 16 are lane exchanges (shuffles), 32..256 go
-  // through shared memory, 512 and 1024 are between a thread's own registers.
-  int P = 512;
-  while (P < ksel) P <<= 1;
-  const int E = P / kTkThreads;
-  unsigned long long x[4];
+  __syncthreads();
+  // Each CTA sorts its own run descending (key, then smaller index first): a bitonic
+  // network over P = 2^ceil(log2 n) entries in registers, element e = r * 1024 + tid in
+  // x[r]; strides up to 16 are lane exchanges, 32..512 go through shared memory, 1024 is
+  // between a thread's two registers.  Threads past n hold 0, below every real entry, and
+  // only ever pair with each other.
+  const int nsel = ksel > 0 ? static_cast<int>(runs[2 * rank + 1]) : 0;
+  int P = 1;
+  while (P < nsel) P <<= 1;
+  const int E = P > kTkThreads ? 2 : 1;
+  unsigned long long x[2];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
+  for (int r = 0; r < 2; ++r) {
     const int e = r * kTkThreads + tid;
-    x[r] = (r < E && e < ksel) ? cand[e] : 0ull;  // 0 sorts below every real entry
+    x[r] = (r < E && e < nsel) ? cand[e] : 0ull;
   }
   __syncthreads();
   for (int size = 2; size <= P; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= kTkThreads) {  // partners in this thread's own registers
-        auto cx = [&](unsigned long long& p, unsigned long long& q, int e) {
-          const bool desc = (e & size) == 0;
-          const unsigned long long hi = p > q ? p : q, lo2 = p > q ? q : p;
-          p = desc ? hi : lo2;
-          q = desc ? lo2 : hi;
-        };
-        if (stride == kTkThreads) {
-          cx(x[0], x[1], tid);
-          if (E == 4) cx(x[2], x[3], 2 * kTkThreads + tid);
-        } else {  // 2 * kTkThreads, E == 4
-          cx(x[0], x[2], tid);
-          cx(x[1], x[3], kTkThreads + tid);
-        }
+      if (stride >= kTkThreads) {  // E == 2: the thread's own two registers
+        const bool desc = (tid & size) == 0;
+        const unsigned long long hi = x[0] > x[1] ? x[0] : x[1], lo2 = x[0] > x[1] ? x[1] : x[0];
+        x[0] = desc ? hi : lo2;
+        x[1] = desc ? lo2 : hi;
       } else {
-        unsigned long long y[4];
+        unsigned long long y[2];
         if (stride >= 32) {
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
+          for (int r = 0; r < 2; ++r)
             if (r < E) cand[r * kTkThreads + tid] = x[r];
           __syncthreads();
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
+          for (int r = 0; r < 2; ++r)
             if (r < E) y[r] = cand[(r * kTkThreads + tid) ^ stride];
           __syncthreads();
         } else {
+          // a warp whose entries are all padding (past P) has nothing to exchange
+          if (E == 1 && (tid & ~31) >= P) continue;
 #pragma unroll
-          for (int r = 0; r < 4; ++r) y[r] = __shfl_xor_sync(0xffffffffu, x[r], stride);
+          for (int r = 0; r < 2; ++r) y[r] = __shfl_xor_sync(0xffffffffu, x[r], stride);
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < 2; ++r) {
           if (r < E) {
             const int e = r * kTkThreads + tid;
             const bool lower = (e & stride) == 0, desc = (e & size) == 0;
@@ -661,21 +685,41 @@ __global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kTkThreads, 1
       }
     }
   }
+  // the sorted runs go to CTA 0, in its key space (free once every CTA is past this sync)
+  cluster_sync();
+  unsigned long long* merged = reinterpret_cast<unsigned long long*>(keys);  // [ksel], CTA 0
+  if (nsel > 0) {
+    const uint32_t mbase = cluster_addr_of(merged, 0) + 8u * runs[2 * rank];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int e = r * kTkThreads + tid;
-    if (r < E && e < k) {
-      int32_t id = -1;
-      float sc = -INFINITY;
-      if (e < ksel) {
-        id = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(x[r]));
-        sc = key_value(static_cast<uint32_t>(x[r] >> 32));
-      }
-      a.out_idx[t * k + e] = id;
-      if (a.out_score) a.out_score[t * k + e] = sc;
+    for (int r = 0; r < 2; ++r) {
+      const int e = r * kTkThreads + tid;
+      if (r < E && e < nsel) st_cluster_u64(mbase + 8u * e, x[r]);
     }
   }
-  for (int e = P + tid; e < k; e += kTkThreads) {  // k past the sorted span: padding
+  cluster_sync();
+  if (rank != 0) return;
+  // CTA 0: each entry's place is its position in its run plus, for every other run, the
+  // number of entries there that sort before it (binary search; the entries are distinct)
+  for (int e = tid; e < ksel; e += kTkThreads) {
+    int r0 = 0;
+    while (r0 + 1 < CL && static_cast<uint32_t>(e) >= runs[2 * (r0 + 1)]) ++r0;
+    const unsigned long long v = merged[e];
+    uint32_t place = static_cast<uint32_t>(e) - runs[2 * r0];
+    for (int r = 0; r < CL; ++r) {
+      if (r == r0) continue;
+      const unsigned long long* run = merged + runs[2 * r];
+      int lo_ = 0, hi_ = static_cast<int>(runs[2 * r + 1]);
+      while (lo_ < hi_) {
+        const int mid = (lo_ + hi_) >> 1;
+        if (run[mid] > v) lo_ = mid + 1;
+        else hi_ = mid;
+      }
+      place += static_cast<uint32_t>(lo_);
+    }
+    a.out_idx[t * k + place] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(v));
+    if (a.out_score) a.out_score[t * k + place] = key_value(static_cast<uint32_t>(v >> 32));
+  }
+  for (int e = ksel + tid; e < k; e += kTkThreads) {  // fewer candidates than k: padding
     a.out_idx[t * k + e] = -1;
     if (a.out_score) a.out_score[t * k + e] = -INFINITY;
   }
@@ -722,25 +766,39 @@ kvc_status launch_indexer_topk(const TopkProblem& p, cudaStream_t st) {
   using namespace idx;
   if (p.T == 0) return KVC_OK;
   if (p.k < 1 || p.k > kMaxK || p.max_visible > topk_max_candidates()) return KVC_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(indexer_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kTkSmem)) != cudaSuccess)
-    return KVC_ERR_CUDA;
-  {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kCluster, 1, 1);
-    cfg.blockDim = dim3(kTkThreads, 1, 1);
-    cfg.dynamicSmemBytes = kTkSmem;
-    cfg.stream = st;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, indexer_topk_kernel, &cfg) != cudaSuccess ||
-        clusters < 1) {
+  TopkArgs a{p.scores, p.n_visible, p.out_idx, p.out_score, p.T, p.max_visible, p.ld, p.k};
+  // Clusters of 8 CTAs (16-CTA clusters were measured slower on the decode step).
+  auto try_launch = [&](auto kern, int cl, bool non_portable) -> kvc_status {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kTkSmem)) != cudaSuccess ||
+        (non_portable &&
+         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+             cudaSuccess)) {
       (void)cudaGetLastError();
       return KVC_ERR_UNSUPPORTED;
     }
-  }
-  TopkArgs a{p.scores, p.n_visible, p.out_idx, p.out_score, p.T, p.max_visible, p.ld, p.k};
-  indexer_topk_kernel<<<static_cast<unsigned>(p.T * kCluster), kTkThreads, kTkSmem, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cl), 1, 1);
+    cfg.blockDim = dim3(kTkThreads, 1, 1);
+    cfg.dynamicSmemBytes = kTkSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+      (void)cudaGetLastError();
+      return KVC_ERR_UNSUPPORTED;
+    }
+    cfg.gridDim = dim3(static_cast<unsigned>(p.T * cl), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return KVC_ERR_CUDA;
+    return KVC_OK;
+  };
+  return try_launch(indexer_topk_kernel<kCluster>, kCluster, false);
 }
 
 unsigned int read_and_clear_indexer_error(bool* failed) {
