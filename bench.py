@@ -60,6 +60,15 @@ def algorithmic_bytes(batch=1, n=N_TOK, c=C):
     return csa, hca
 
 
+def _traffic(key):
+    """DRAM bytes per launch of a kernel from the committed ncu summaries (None if absent)."""
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(prof):
+        return None
+    with open(prof) as f:
+        return json.load(f).get(key)
+
+
 class ClockSampler:
     """nvidia-smi sampled every 100 ms while the timed region runs."""
 
@@ -320,11 +329,7 @@ def run_ours(args):
     ms_step = elapsed_ms / args.steps
     tokens_per_s = world * N_TOK / (ms_step * 1e-3)
     entries = N_TOK // M_CSA + N_TOK // M_HCA
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        with open(prof) as f:
-            traffic = json.load(f).get("csa_compress_bf16_n1048576")
+    traffic = _traffic("csa_compress_bf16_n1048576")
     if rank == 0:
         line = {
             "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s",
@@ -346,6 +351,7 @@ def run_ours(args):
                                  "tokens_per_s": N_TOK / (csa_ms * 1e-3),
                                  "entries_per_s": (N_TOK // M_CSA) / (csa_ms * 1e-3)},
                 "hca_compress": {"ms": hca_ms, "GB/s": hca_gbs, "frac": hca_gbs / peak,
+                                 "traffic": _traffic("hca_compress_bf16_n1048576"),
                                  "tokens_per_s": N_TOK / (hca_ms * 1e-3),
                                  "entries_per_s": (N_TOK // M_HCA) / (hca_ms * 1e-3)},
             },
@@ -531,8 +537,8 @@ def _workload(name, dev):
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // m,
                     bound="hbm", units=float(nbytes), flush=nbytes < 4 * (126 << 20),
                     kernel=("csa_small_m_kernel" if mode == "csa" else
-                            "window_pipe_kernel (8 row groups)" if n == 65536 else
-                            "window_pool_kernel"),
+                            "window_tma_kernel (TMA-fed, 8 row groups)"),
+                    traffic_key="hca_compress_bf16_n65536" if mode == "hca" else None,
                     config={"workload": f"{mode.upper()} streams: batch 1, n={n}, c={c}, m={m}, "
                                         f"{dt} in/out", "n": n, "c": c, "m": m})
     raise SystemExit(f"unknown workload {name}")
@@ -558,8 +564,12 @@ def run_workload(args):
         raise SystemExit("device error during warm-up")
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", ""))
+    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0"))
+    sampler.start()
     barrier(world)
     torch.cuda.synchronize()
+    sampler.mark(True)
     for a, b in evs:
         if flush is not None:
             flush.zero_()
@@ -567,7 +577,9 @@ def run_workload(args):
         w["launch"](w["inputs"], st)
         b.record(st)
     torch.cuda.synchronize()
+    sampler.mark(False)
     barrier(world)
+    clocks = sampler.stop()
     ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), world)
     if kvc.device_status(st) != kvc.KVC_OK:
         raise SystemExit("device error in the timed region")
@@ -632,13 +644,14 @@ def run_workload(args):
                          "peak": peak, "unit": unit, "frac": ach / peak, "peak_kind": kind,
                          "frac_of_sustained": (ach / _peak("tensor", True)[0]
                                                if w["bound"] == "tensor" else None),
-                         "traffic": None,
+                         "traffic": _traffic(w["traffic_key"]) if w.get("traffic_key") else None,
                          ("algorithmic_flops" if w["bound"] == "tensor" else "algorithmic_bytes"):
                              w["units"]},
             "gpu_launches": args.steps * max(1, len(w.get("parts", ()))),
             "e2e": {"value": world * w["tokens"] / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         }
+        line["clocks"] = clocks
         if w.get("parts"):
             line["kernels"] = {}
             for part in w["parts"]:

@@ -36,6 +36,7 @@
 #include <cuda.h>
 
 #include "kvc_common.cuh"
+#include "kvc_host.h"
 #include "kvc_launch.h"
 #include "tc_ptx.cuh"
 
@@ -1105,30 +1106,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 // 2-D bf16 row-major [rows, cols] tensor map with a [box_rows, box_cols] box; the
 // swizzle span equals the box row (box_cols * 2 bytes: 128 or 64).
 bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
               uint32_t box_cols) {
-  EncodeTiledFn enc = encode_fn();
+  EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
@@ -1288,8 +1270,9 @@ kvc_status read_and_clear_device_error(cudaStream_t st) {
   bool failed = false;
   const bool index_error = read_and_clear_index_error(&failed);
   const unsigned int ix = read_and_clear_indexer_error(&failed);
+  const unsigned int wx = read_and_clear_window_error(&failed);
   if (failed) return KVC_ERR_CUDA;
-  if (v || (ix & 1u)) return KVC_ERR_TIMEOUT;
+  if (v || (ix & 1u) || (wx & 1u)) return KVC_ERR_TIMEOUT;
   return (index_error || (ix & 2u)) ? KVC_ERR_INDEX : KVC_OK;
 }
 

@@ -92,6 +92,13 @@ int64_t topk_max_candidates();
 // wait gave up, bit 1 a query's candidate window was out of range.
 unsigned int read_and_clear_indexer_error(bool* failed);
 
+// The TMA-fed single-segment window kernel (dense HCA-style problems with m >= 32);
+// KVC_ERR_UNSUPPORTED when the problem or the device does not fit it (the caller then uses
+// the register-staged kernels).
+kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st);
+// Reads and clears its error word (no synchronisation): bit 0 a bounded wait gave up.
+unsigned int read_and_clear_window_error(bool* failed);
+
 // Device error words: bounded waits that gave up (fused kernels) and listed entries out
 // of range (streaming kernels).  Synchronises the stream first.
 kvc_status read_and_clear_device_error(cudaStream_t st);

@@ -16,6 +16,7 @@
 #include "kvc_common.cuh"
 #include "kvc_host.h"
 #include "kvc_launch.h"
+#include "stream_common.cuh"
 
 #include <math.h>
 
@@ -55,47 +56,6 @@ __device__ __forceinline__ bool listed_entry(const EntryList& L, int64_t k, int 
 // Extra kernel argument of the cache-layout instantiations (empty otherwise).
 template <bool CACHE>
 using CacheArg = typename std::conditional<CACHE, CacheFmt, NoCache>::type;
-
-// Stages `nrows` bias rows of a channel slab, pre-scaled by log2 e, into shared memory:
-// row k comes from B0 row k (k < m0) or B1 row k - m0, slab channel sc goes to
-// dst[k * SC + pos(sc)] (channels past c read 0).  The loads are issued kBiasBatch at a
-// time per thread so that they overlap: this stage sits at the start of every CTA, and
-// one dependent L2 round trip per value made it a sizeable part of short launches.
-// Returns this thread's (max, min) over the values it staged.
-constexpr int kBiasBatch = 16;
-
-template <typename PosFn>
-__device__ __forceinline__ float2 stage_bias(float* dst, const float* B0, const float* B1, int m0,
-                                             int nrows, int SC, int64_t ch_base, int64_t c,
-                                             int tid, int nthr, PosFn pos) {
-  float lmax = -INFINITY, lmin = INFINITY;
-  const int total = nrows * SC;
-  for (int base = tid; base < total; base += nthr * kBiasBatch) {
-    float v[kBiasBatch];
-#pragma unroll
-    for (int r = 0; r < kBiasBatch; ++r) {
-      const int idx = base + r * nthr;
-      v[r] = 0.f;
-      if (idx < total) {
-        const int k = idx / SC;
-        const int64_t ch = ch_base + (idx - k * SC);
-        if (ch < c) v[r] = __ldg(k < m0 ? B0 + k * c + ch : B1 + (k - m0) * c + ch);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kBiasBatch; ++r) {
-      const int idx = base + r * nthr;
-      if (idx < total) {
-        const int k = idx / SC;
-        const float x = v[r] * kLog2e;
-        dst[k * SC + pos(idx - k * SC)] = x;
-        lmax = fmaxf(lmax, x);
-        lmin = fminf(lmin, x);
-      }
-    }
-  }
-  return make_float2(lmax, lmin);
-}
 
 struct CsaSmallArgs {
   const void* Ca;
@@ -260,18 +220,6 @@ constexpr int win_slab() {
   return kWinCG * VecInfo<InT>::kChannels;
 }
 
-// Largest per-channel spread of the (log2 e-scaled) bias rows for which a chunk's maximum
-// logit may be bounded by max(z) * log2 e + max(b) instead of taken row by row.
-constexpr float kMaxBiasSpread = 64.f;
-
-// Position of slab channel sc in a shared-memory bias row: float4 q of thread group g at
-// (q * kWinCG + g) * 4.
-template <int CPT>
-__device__ __forceinline__ int win_bias_pos(int sc) {
-  const int g = sc / CPT, j = sc - (sc / CPT) * CPT;
-  return ((j >> 2) * kWinCG + g) * 4 + (j & 3);
-}
-
 template <typename InT, bool TWO_SEG>
 size_t win_smem_bytes(int m, int rg) {
   const int rows = TWO_SEG ? 2 * m : m;
@@ -307,7 +255,7 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const En
   const int64_t ch_base = static_cast<int64_t>(blockIdx.x) * SC;
   // 256 is a multiple of SC, so each thread stages one channel's rows tid/SC, tid/SC + 256/SC, ...
   const float2 mm = stage_bias(sb, a.B0, a.B1, a.m, nb, SC, ch_base, a.c, tid, kWinCG * kWinTY,
-                               [](int sc) { return win_bias_pos<CPT>(sc); });
+                               [](int sc) { return slab_bias_pos<CPT, kWinCG>(sc); });
   red[tid] = mm.x;
   red[kWinCG * kWinTY + tid] = mm.y;
   __syncthreads();
@@ -320,7 +268,7 @@ __global__ void __launch_bounds__(256, 2) window_pool_kernel(WinArgs a, const En
       mx = fmaxf(mx, red[j]);
       mn = fminf(mn, red[kWinCG * kWinTY + j]);
     }
-    bmx[win_bias_pos<CPT>(tid)] = mx;
+    bmx[slab_bias_pos<CPT, kWinCG>(tid)] = mx;
     wide = !(mx - mn <= kMaxBiasSpread);  // also true for infinite or NaN spreads
   }
   const bool fast = !__syncthreads_or(wide);
@@ -610,7 +558,7 @@ __global__ void __launch_bounds__(256, 2) window_pipe_kernel(WinArgs a) {
   const int es = ty / RG, rg = ty - (ty / RG) * RG;
   const int64_t ch_base = static_cast<int64_t>(blockIdx.x) * SC;
   const float2 mm = stage_bias(sb, a.B0, a.B0, m, m, SC, ch_base, a.c, tid, kWinCG * kWinTY,
-                               [](int sc) { return win_bias_pos<CPT>(sc); });
+                               [](int sc) { return slab_bias_pos<CPT, kWinCG>(sc); });
   red[tid] = mm.x;
   red[kWinCG * kWinTY + tid] = mm.y;
   __syncthreads();
@@ -621,7 +569,7 @@ __global__ void __launch_bounds__(256, 2) window_pipe_kernel(WinArgs a) {
       mx = fmaxf(mx, red[j]);
       mn = fminf(mn, red[kWinCG * kWinTY + j]);
     }
-    bmx[win_bias_pos<CPT>(tid)] = mx;
+    bmx[slab_bias_pos<CPT, kWinCG>(tid)] = mx;
     wide = !(mx - mn <= kMaxBiasSpread);
   }
   const bool fast = !__syncthreads_or(wide);
@@ -837,6 +785,10 @@ kvc_status launch_window(const StreamProblem& p, cudaStream_t st) {
   if constexpr (LISTED || CACHE) {
     return launch_window_rg<InT, OutT, TWO_SEG, 1, LISTED, CACHE>(p, st, di);
   } else {
+    if constexpr (!TWO_SEG) {
+      const kvc_status r = launch_window_tma(p, st);
+      if (r != KVC_ERR_UNSUPPORTED) return r;
+    }
     const int64_t tasks = p.batch * p.ne * ceil_div(p.c, SC);  // (entry, slab) pairs
     const int64_t slots = static_cast<int64_t>(di.sms) * 2;
     const int rows = TWO_SEG ? 2 * p.m : p.m;

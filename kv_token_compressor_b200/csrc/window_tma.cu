@@ -1,0 +1,600 @@
+// Single-segment softmax pool over long windows (HCA, m' = 128) fed by TMA (sm_100a).
+//
+// What it computes ("序列压缩注意力", eq. attn-seqcomp-hca; "Ch 05 · HCA" §2): for every
+// entry i and channel ch, the softmax over the window's m rows of Z[i*m + v, ch] + B[v, ch]
+// and the weighted sum of C[i*m + v, ch], exactly as the register-staged window kernel.
+//
+// Why a second kernel.  With loads into registers each warp alternates between waiting on
+// memory and computing, and only the warps that happen to be waiting keep bytes in flight.
+// Here one producer thread streams the windows into a ring of shared-memory stages with
+// 4-D tensor-map copies ([channels, row in window, entry, sequence] boxes), and eight
+// consumer warps pool from shared memory; the copies of the next stages are in flight
+// while the consumers compute, so every SM keeps about 100 KB of reads outstanding.
+//
+// Work split.  A task is (channel slab of 16 vectors, sequence, group of E = 16 / RG
+// entries).  The 16 consumer thread rows are (entry, row group): with RG row groups an
+// entry's rows are dealt round-robin to RG threads, whose partial (max, sum, acc) merge in
+// shared memory at the end of the window.  A stage holds UR = 4 RG rows of each of the
+// group's E entries, so every consumer thread takes four rows per stage whatever RG is,
+// and rescales its running state once per two stages (eight rows).  Tasks are ordered slab
+// first, so a CTA's contiguous range of tasks re-stages the bias rarely.
+#include <cuda.h>
+
+#include "kvc_common.cuh"
+#include "kvc_host.h"
+#include "kvc_launch.h"
+#include "stream_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace kvc {
+
+// Bit 0: a bounded wait of the TMA-fed window kernel gave up (outputs undefined).
+__device__ unsigned int g_window_error = 0;
+
+namespace wtma {
+
+using namespace tcx;
+
+constexpr int kCG = 16;                       // channel vectors per slab (threads along x)
+constexpr int kTY = 16;                       // consumer thread rows
+constexpr int kConsumers = kCG * kTY;         // 256
+constexpr int kThreads = kConsumers + 32;     // + one producer warp
+constexpr int kRowsPerThread = 4;             // rows of each consumer thread per stage
+constexpr int kStages = 4;
+constexpr int kHalf = kTY * kRowsPerThread * 256;  // one stream's stage: 64 rows x 256 B
+constexpr int kStageBytes = 2 * kHalf;             // Z then C
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr int kMinRows = 32;                       // shorter windows use the other kernels
+
+struct Args {
+  const float* B;  // [m, c]
+  void* out;       // [batch, ne, c]
+  int64_t batch, ne, c;
+  int m;
+  int64_t groups;  // entry groups per sequence
+  int64_t tasks;   // slabs * batch * groups
+  int bias_tma;    // the bias rows arrive through mapB (else plain loads)
+};
+
+template <typename InT>
+constexpr int slab() {
+  return kCG * VecInfo<InT>::kChannels;
+}
+
+// Dynamic shared memory: stages, bias rows, per-channel bias maxima, spread partials,
+// row-group partials (RG > 1), barriers (stage full / empty, bias full / free) and the
+// abort flag; 1 KB slack for alignment.
+template <typename InT>
+size_t smem_bytes(int m, int rg) {
+  constexpr int SC = slab<InT>();
+  size_t f = static_cast<size_t>(m) * SC + SC + 2 * kConsumers;
+  if (rg > 1) f += 3 * static_cast<size_t>(kTY) * SC;
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + f * sizeof(float) +
+         (2 * kStages + 2) * sizeof(uint64_t) + 16;
+}
+
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       bool honour_abort) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (honour_abort && *abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(&g_window_error, 1u);
+      return false;
+    }
+  }
+}
+// Bounded wait: true once the phase of `parity` has completed; false after the limit (which
+// raises the CTA's abort flag and the error bit) or, when honoured, once another thread of
+// the CTA has raised the abort flag.
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                     bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, abort_flag, honour_abort);
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// (slab, sequence, entry group) of task t, stepped one task at a time (the divisions once
+// per CTA, not on every task boundary).
+struct Task {
+  int64_t x, b, g;
+  __device__ Task(const Args& a, int64_t t) {
+    const int64_t per_slab = a.batch * a.groups;
+    x = t / per_slab;
+    const int64_t r = t - x * per_slab;
+    b = r / a.groups;
+    g = r - b * a.groups;
+  }
+  __device__ __forceinline__ void next(const Args& a) {
+    if (++g == a.groups) {
+      g = 0;
+      if (++b == a.batch) {
+        b = 0;
+        ++x;
+      }
+    }
+  }
+};
+
+// Order-preserving map of fp32 to uint32 (larger float, larger key) and its inverse, for
+// shared-memory atomic max / min.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+template <typename InT, typename OutT, int RG>
+__global__ void __launch_bounds__(kThreads, 1)
+    window_tma_kernel(const __grid_constant__ CUtensorMap mapZ,
+                      const __grid_constant__ CUtensorMap mapC,
+                      const __grid_constant__ CUtensorMap mapB, const Args a) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int SC = slab<InT>();
+  constexpr int E = kTY / RG;                 // entries per task
+  constexpr int UR = kRowsPerThread * RG;     // rows of each entry per stage
+  constexpr int NP = CPT / 2;                 // channel pairs per thread
+  static_assert(E * UR * SC * sizeof(InT) == kHalf, "stage geometry");
+  const float2 kL2e2 = make_float2(kLog2e, kLog2e);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = base;
+  float* sb = reinterpret_cast<float*>(base + kStages * kStageBytes);  // [m][SC] bias * log2 e
+  float* bmx = sb + static_cast<size_t>(a.m) * SC;                      // [SC] largest bias
+  float* red = bmx + SC;                                                 // [2][256] max / min
+  float* pm = red + 2 * kConsumers;                                      // RG > 1: [16][SC]
+  float* ps = pm + (RG > 1 ? kTY * SC : 0);
+  float* pa = ps + (RG > 1 ? kTY * SC : 0);
+  uint64_t* full = reinterpret_cast<uint64_t*>(pa + (RG > 1 ? kTY * SC : 0));
+  uint64_t* empty = full + kStages;
+  uint64_t* bias_full = empty + kStages;
+  uint64_t* bias_free = bias_full + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bias_free + 1);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  uint32_t* kmax = reinterpret_cast<uint32_t*>(red);  // [SC] bias maxima as order keys
+  uint32_t* kmin = kmax + SC;                          // [SC] minima
+  if (tid < SC) {
+    kmax[tid] = 0u;
+    kmin[tid] = 0xFFFFFFFFu;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers / 32);
+    }
+    mbar_init(bias_full, 1);
+    mbar_init(bias_free, kConsumers / 32);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * a.tasks / gridDim.x;
+  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * a.tasks / gridDim.x;
+  const int nst = (a.m + UR - 1) / UR;  // stages per window
+
+  if (warp == kConsumers / 32) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t used = 0, last_par = 0;  // stages ever filled; parity of their last fill
+      uint32_t nbias = 0;               // bias loads issued
+      int64_t px = -1;
+      bool ok = true;
+      Task k(a, lo);
+      for (int64_t t = lo; t < hi && ok; ++t, k.next(a)) {
+        if (a.bias_tma && k.x != px) {
+          // the slab's bias rows, once the consumers are done with the previous slab's
+          if (nbias > 0 && !wait(bias_free, (nbias - 1) & 1u, abort_flag)) break;
+          mbar_arrive_expect_tx(bias_full, static_cast<uint32_t>(a.m) * SC * 4);
+          tma_load_2d(smem_u32(sb), &mapB, bias_full, static_cast<int>(k.x * SC), 0);
+          ++nbias;
+          px = k.x;
+        }
+        for (int st = 0; st < nst; ++st) {
+          if (!wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          const uint32_t dst = smem_u32(stages + s * kStageBytes);
+          const int x = static_cast<int>(k.x * SC), y = st * UR;
+          const int z = static_cast<int>(k.g * E), w = static_cast<int>(k.b);
+          tma_load_4d(dst, &mapZ, &full[s], x, y, z, w);
+          tma_load_4d(dst + kHalf, &mapC, &full[s], x, y, z, w);
+          used |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // Every copy issued above lands before this thread exits, whatever the consumers did.
+      for (int q = 0; q < kStages; ++q)
+        if (used & (1u << q)) wait(&full[q], (last_par >> q) & 1u, abort_flag, false);
+      if (nbias > 0) wait(bias_full, (nbias - 1) & 1u, abort_flag, false);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers (warps 0..7)
+  const int tx = tid % kCG, ty = tid / kCG;
+  const int e = ty / RG, rg = ty - (ty / RG) * RG;
+  const int sc0 = tx * CPT;  // this thread's CPT channels of the slab
+  int s = 0;
+  uint32_t ph = 0;
+  bool dead = false;
+  bool fast = false;
+  int64_t cur_x = -1;
+  uint32_t nb = 0;  // bias loads consumed
+  OutT* out = static_cast<OutT*>(a.out);
+
+  Task k(a, lo);
+  for (int64_t t = lo; t < hi; ++t, k.next(a)) {
+    if (k.x != cur_x) {  // the same in every consumer thread
+      bool narrow = true;
+      if (a.bias_tma) {
+        if (cur_x >= 0) {  // this warp is done with the old slab's bias
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bias_free);
+        }
+        if (!dead && !wait(bias_full, nb & 1u, abort_flag)) dead = true;
+        ++nb;
+        // The rows arrive in natural channel order.  Scale them by log2 e and move each
+        // float4 to its slot in the consumers' order (whole float4s move: channels 4w..4w+3
+        // go to slab_bias_pos(4w)); the SC / 4 float4s of a row are one warp's, or half of
+        // one for fp32 (whose order is the identity), so reading the whole row before
+        // writing it makes the move safe in place.  This thread always holds float4 w of
+        // a row (256 is a multiple of SC / 4): it folds its rows' maxima and minima
+        // channel by channel and publishes them with one atomic per channel.
+        static_assert(SC / 4 == 32 || SC / 4 == 16, "a row is one warp's (or half)");
+        float4* s4 = reinterpret_cast<float4*>(sb);
+        float4 mx4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        float4 mn4 = make_float4(INFINITY, INFINITY, INFINITY, INFINITY);
+        const int w = tid % (SC / 4);
+        const int slot = slab_bias_pos<CPT, kCG>(4 * w) / 4;
+        for (int f = tid - w; f < a.m * (SC / 4); f += kConsumers) {  // f: the row's start
+          float4 v = s4[f + w];
+          v.x *= kLog2e;
+          v.y *= kLog2e;
+          v.z *= kLog2e;
+          v.w *= kLog2e;
+          if constexpr (CPT == 8) __syncwarp();  // the warp's lanes run this loop alike
+          s4[f + slot] = v;
+          mx4 = make_float4(fmaxf(mx4.x, v.x), fmaxf(mx4.y, v.y), fmaxf(mx4.z, v.z), fmaxf(mx4.w, v.w));
+          mn4 = make_float4(fminf(mn4.x, v.x), fminf(mn4.y, v.y), fminf(mn4.z, v.z), fminf(mn4.w, v.w));
+        }
+        const int w4 = slot * 4;  // position of this thread's four channels in a staged row
+        atomicMax(&kmax[w4], order_key(mx4.x));
+        atomicMax(&kmax[w4 + 1], order_key(mx4.y));
+        atomicMax(&kmax[w4 + 2], order_key(mx4.z));
+        atomicMax(&kmax[w4 + 3], order_key(mx4.w));
+        atomicMin(&kmin[w4], order_key(mn4.x));
+        atomicMin(&kmin[w4 + 1], order_key(mn4.y));
+        atomicMin(&kmin[w4 + 2], order_key(mn4.z));
+        atomicMin(&kmin[w4 + 3], order_key(mn4.w));
+        bar_named(1, kConsumers);
+        if (tid < SC) {  // tid is a position in a staged row here
+          const float mx = key_float(kmax[tid]), mn = key_float(kmin[tid]);
+          kmax[tid] = 0u;  // ready for the next slab (ordered by the barrier below)
+          kmin[tid] = 0xFFFFFFFFu;
+          bmx[tid] = mx;
+          narrow = mx - mn <= kMaxBiasSpread;  // false for infinite or NaN spreads
+        }
+      } else {
+        if (cur_x >= 0) bar_named(1, kConsumers);  // nobody still reads the old slab's bias
+        const float2 mm = stage_bias(sb, a.B, a.B, a.m, a.m, SC, k.x * SC, a.c, tid, kConsumers,
+                                     [](int sc) { return slab_bias_pos<CPT, kCG>(sc); });
+        red[tid] = mm.x;
+        red[kConsumers + tid] = mm.y;
+        bar_named(1, kConsumers);
+        if (tid < SC) {
+          float mx = -INFINITY, mn = INFINITY;
+          for (int j = tid; j < kConsumers; j += SC) {
+            mx = fmaxf(mx, red[j]);
+            mn = fminf(mn, red[kConsumers + j]);
+          }
+          bmx[slab_bias_pos<CPT, kCG>(tid)] = mx;
+          narrow = mx - mn <= kMaxBiasSpread;
+        }
+      }
+      // fast chunk maximum only when every channel's spread is small; also publishes bmx
+      fast = bar_and(1, kConsumers, narrow);
+      cur_x = k.x;
+    }
+    const int64_t i = k.g * E + e;  // entry within its sequence
+    const int64_t ch0 = k.x * SC + sc0;
+    const bool live = i < a.ne && ch0 < a.c;
+
+    float2 M[NP], S[NP], A[NP];  // per channel pair: running max, sum, weighted sum
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      M[p] = make_float2(-INFINITY, -INFINITY);
+      S[p] = make_float2(0.f, 0.f);
+      A[p] = make_float2(0.f, 0.f);
+    }
+    for (int st = 0; st < nst; st += 2) {
+      const bool two = st + 1 < nst;
+      uint4 z[2 * kRowsPerThread], cv[2 * kRowsPerThread];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && !two) break;
+        if (!dead && !wait(&full[s], ph, abort_flag)) dead = true;
+        const uint8_t* sz = stages + s * kStageBytes;
+#pragma unroll
+        for (int q = 0; q < kRowsPerThread; ++q) {
+          const int r = rg + RG * q;  // row within the stage
+          const int off = ((e * UR + r) * SC + sc0) * static_cast<int>(sizeof(InT));
+          z[h * kRowsPerThread + q] = *reinterpret_cast<const uint4*>(sz + off);
+          cv[h * kRowsPerThread + q] = *reinterpret_cast<const uint4*>(sz + kHalf + off);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      // rows of this thread in the two stages: st*UR + rg + RG*q, (st+1)*UR + rg + RG*q
+      const int v0 = st * UR + rg;
+      if (dead || !live || v0 >= a.m) continue;  // v0 is the smallest row of the chunk
+      auto row_of = [&](int u) { return v0 + (u / kRowsPerThread) * UR + RG * (u % kRowsPerThread); };
+      auto valid = [&](int u) { return (u < kRowsPerThread || two) && row_of(u) < a.m; };
+
+      // pass 1: an upper bound of the chunk's largest logit per channel (see the register-
+      // staged window kernel: max z * log2 e + max b when the bias spread is small, else the
+      // exact per-row maximum)
+      float2 cm[NP];
+      if (fast) {
+        uint4 zm = z[0];
+#pragma unroll
+        for (int u = 1; u < 2 * kRowsPerThread; ++u)
+          if (valid(u)) zm = vec_max<InT>(zm, z[u]);
+        const float4* bx = reinterpret_cast<const float4*>(bmx) + tx;
+#pragma unroll
+        for (int q = 0; q < NP / 2; ++q) {
+          const float4 bq = bx[q * kCG];
+          cm[2 * q] = f2_fma(vec_pair<InT>(zm, 2 * q), kL2e2, make_float2(bq.x, bq.y));
+          cm[2 * q + 1] = f2_fma(vec_pair<InT>(zm, 2 * q + 1), kL2e2, make_float2(bq.z, bq.w));
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
+#pragma unroll
+        for (int u = 0; u < 2 * kRowsPerThread; ++u) {
+          if (valid(u)) {
+            const float4* bp = reinterpret_cast<const float4*>(sb + row_of(u) * SC) + tx;
+#pragma unroll
+            for (int q = 0; q < NP / 2; ++q) {
+              const float4 bq = bp[q * kCG];
+              cm[2 * q] = f2_max(cm[2 * q], f2_fma(vec_pair<InT>(z[u], 2 * q), kL2e2,
+                                                   make_float2(bq.x, bq.y)));
+              cm[2 * q + 1] = f2_max(cm[2 * q + 1], f2_fma(vec_pair<InT>(z[u], 2 * q + 1), kL2e2,
+                                                           make_float2(bq.z, bq.w)));
+            }
+          }
+        }
+      }
+      // rescale the running state once per chunk
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 is valid
+        const float2 sc = make_float2(ex2_ftz(M[p].x - nm.x), ex2_ftz(M[p].y - nm.y));
+        S[p] = f2_mul(S[p], sc);
+        A[p] = f2_mul(A[p], sc);
+        M[p] = nm;
+      }
+      // pass 2: one exp2 per element
+#pragma unroll
+      for (int u = 0; u < 2 * kRowsPerThread; ++u) {
+        if (valid(u)) {
+          const float4* bp = reinterpret_cast<const float4*>(sb + row_of(u) * SC) + tx;
+#pragma unroll
+          for (int q = 0; q < NP / 2; ++q) {
+            const float4 bq = bp[q * kCG];
+            const float2 b2[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int pp = 2 * q + h;
+              const float2 l = f2_fma(vec_pair<InT>(z[u], pp), kL2e2, f2_sub(b2[h], M[pp]));
+              const float2 w = f2_ex2(l);
+              S[pp] = f2_add(S[pp], w);
+              A[pp] = f2_fma(w, vec_pair<InT>(cv[u], pp), A[pp]);
+            }
+          }
+        }
+      }
+    }
+
+    if constexpr (RG == 1) {
+      if (live && !dead) {
+        float res[CPT];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+          res[2 * p] = __fdividef(A[p].x, S[p].x);
+          res[2 * p + 1] = __fdividef(A[p].y, S[p].y);
+        }
+        store_out<OutT, CPT>(out + (k.b * a.ne + i) * a.c + ch0, res);
+      }
+    } else {
+      // row-group partials -> shared memory; one thread per (entry, channel vector) merges
+#pragma unroll
+      for (int q = 0; q < NP / 2; ++q) {
+        reinterpret_cast<float4*>(pm + ty * SC + sc0)[q] =
+            make_float4(M[2 * q].x, M[2 * q].y, M[2 * q + 1].x, M[2 * q + 1].y);
+        reinterpret_cast<float4*>(ps + ty * SC + sc0)[q] =
+            make_float4(S[2 * q].x, S[2 * q].y, S[2 * q + 1].x, S[2 * q + 1].y);
+        reinterpret_cast<float4*>(pa + ty * SC + sc0)[q] =
+            make_float4(A[2 * q].x, A[2 * q].y, A[2 * q + 1].x, A[2 * q + 1].y);
+      }
+      bar_named(2, kConsumers);
+      // one (entry, channel) per thread and item: conflict-free, every consumer busy
+      for (int item = tid; item < E * SC; item += kConsumers) {
+        const int e2 = item / SC, sc = item - (item / SC) * SC;
+        const int64_t i2 = k.g * E + e2;
+        const int64_t c2 = k.x * SC + sc;
+        if (i2 < a.ne && c2 < a.c && !dead) {
+          float gm = -INFINITY;
+#pragma unroll 4
+          for (int r = 0; r < RG; ++r) gm = fmaxf(gm, pm[(e2 * RG + r) * SC + sc]);
+          float sum = 0.f, acc = 0.f;
+#pragma unroll 4
+          for (int r = 0; r < RG; ++r) {
+            const int o = (e2 * RG + r) * SC + sc;
+            const float f = ex2_ftz(pm[o] - gm);  // 0 for row groups without rows
+            sum = fmaf(ps[o], f, sum);
+            acc = fmaf(pa[o], f, acc);
+          }
+          store_scalar<OutT>(out + (k.b * a.ne + i2) * a.c + c2, __fdividef(acc, sum));
+        }
+      }
+      bar_named(2, kConsumers);
+    }
+  }
+}
+
+// 4-D tensor map of a [batch, n, c] stream viewed as [batch][ne][m][c] (entries of m rows;
+// the n mod m tail rows are never addressed), box [1][E][UR][SC], no swizzle, zero fill.
+bool make_stream_map(CUtensorMap* map, const void* base, bool bf16, int64_t batch, int64_t n,
+                     int64_t ne, int64_t c, int m, int SC, int UR, int E) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const uint64_t es = bf16 ? 2 : 4;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c), static_cast<cuuint64_t>(m),
+                              static_cast<cuuint64_t>(ne), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(c) * es,
+                                 static_cast<cuuint64_t>(m) * c * es,
+                                 static_cast<cuuint64_t>(n) * c * es};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(SC), static_cast<cuuint32_t>(UR),
+                             static_cast<cuuint32_t>(E), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D tensor map of the fp32 bias [m, c] with a [m][SC] box (a slab's rows, natural order).
+bool make_bias_map(CUtensorMap* map, const float* B, int64_t c, int m, int SC) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc || (reinterpret_cast<uintptr_t>(B) & 15u)) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c), static_cast<cuuint64_t>(m)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(c) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(SC), static_cast<cuuint32_t>(m)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(B), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename InT, typename OutT, int RG>
+kvc_status launch_rg(const StreamProblem& p, cudaStream_t st, const DeviceInfo& di) {
+  constexpr int SC = slab<InT>();
+  constexpr int E = kTY / RG;
+  constexpr int UR = kRowsPerThread * RG;
+  const size_t smem = smem_bytes<InT>(p.m, RG);
+  if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
+  CUtensorMap mz, mc;
+  const bool bf = sizeof(InT) == 2;
+  if (!make_stream_map(&mz, p.Z0, bf, p.batch, p.n, p.ne, p.c, p.m, SC, UR, E) ||
+      !make_stream_map(&mc, p.C0, bf, p.batch, p.n, p.ne, p.c, p.m, SC, UR, E))
+    return KVC_ERR_UNSUPPORTED;
+  CUtensorMap mb;
+  const bool bias_tma = p.m <= 256 && make_bias_map(&mb, p.B0, p.c, p.m, SC);
+  if (!bias_tma) mb = mz;  // unused
+  auto kern = window_tma_kernel<InT, OutT, RG>;
+  if (resident_blocks(kern, kThreads, smem) < 1) return KVC_ERR_UNSUPPORTED;
+  Args a{p.B0, p.out, p.batch, p.ne, p.c, p.m, ceil_div(p.ne, E), 0, bias_tma ? 1 : 0};
+  a.tasks = ceil_div(p.c, SC) * p.batch * a.groups;
+  const int64_t grid = a.tasks < di.sms ? a.tasks : di.sms;
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mz, mc, mb, a);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+// Share of the SMs' task rounds that do work when `tasks` tasks are split into contiguous
+// ranges over `sms` CTAs.
+double balance(int64_t tasks, int sms) {
+  const int64_t rounds = ceil_div(tasks, sms);
+  return static_cast<double>(tasks) / (static_cast<double>(rounds) * sms);
+}
+
+template <typename InT, typename OutT>
+kvc_status launch_typed(const StreamProblem& p, cudaStream_t st) {
+  constexpr int SC = slab<InT>();
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (di.sms == 0) return KVC_ERR_CUDA;
+  // The fewest row groups whose task count keeps the SMs at least 90% busy (else the
+  // best balance); one row group needs no merge.
+  const int64_t per_group = ceil_div(p.c, SC) * p.batch;
+  int best = 16;
+  double best_bal = -1.0;
+  for (int rg = 1; rg <= 16; rg *= 2) {
+    const double bal = balance(per_group * ceil_div(p.ne, kTY / rg), di.sms);
+    if (bal >= 0.9) {
+      best = rg;
+      break;
+    }
+    if (bal > best_bal + 1e-9) {
+      best_bal = bal;
+      best = rg;
+    }
+  }
+  switch (best) {
+    case 1: return launch_rg<InT, OutT, 1>(p, st, di);
+    case 2: return launch_rg<InT, OutT, 2>(p, st, di);
+    case 4: return launch_rg<InT, OutT, 4>(p, st, di);
+    case 8: return launch_rg<InT, OutT, 8>(p, st, di);
+    default: return launch_rg<InT, OutT, 16>(p, st, di);
+  }
+}
+
+}  // namespace wtma
+
+kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st) {
+  if (p.two_segments || p.listed || p.cache || p.m < wtma::kMinRows || p.ne <= 0 ||
+      p.ne > INT32_MAX || p.batch > INT32_MAX || p.c > INT32_MAX)
+    return KVC_ERR_UNSUPPORTED;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(p.C0) | reinterpret_cast<uintptr_t>(p.Z0);
+  if (al & 15u) return KVC_ERR_UNSUPPORTED;
+  if (p.in_bf16)
+    return p.out_bf16 ? wtma::launch_typed<__nv_bfloat16, __nv_bfloat16>(p, st)
+                      : wtma::launch_typed<__nv_bfloat16, float>(p, st);
+  return p.out_bf16 ? wtma::launch_typed<float, __nv_bfloat16>(p, st)
+                    : wtma::launch_typed<float, float>(p, st);
+}
+
+unsigned int read_and_clear_window_error(bool* failed) {
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_window_error, sizeof(v)) != cudaSuccess) {
+    *failed = true;
+    return 0;
+  }
+  if (v != 0 && cudaMemcpyToSymbol(g_window_error, &zero, sizeof(zero)) != cudaSuccess)
+    *failed = true;
+  return v;
+}
+
+}  // namespace kvc

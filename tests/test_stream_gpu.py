@@ -97,6 +97,27 @@ HCA_CASES = [
     (1, 100 * 300 + 7, 136, 100),
 ]
 
+# Window counts that make the TMA-fed window kernel pick each of its row-group splits on a
+# 148-SM part (c = 512 bf16: 4 channel slabs; 148 tasks at 1, 2, 4, 8, 16 row groups per
+# entry), plus a tail of n mod m rows.
+TMA_RG_CASES = [
+    (1, 32 * 592 + 5, 512, 32),
+    (1, 32 * 296, 512, 32),
+    (1, 64 * 148 + 63, 512, 64),
+    (1, 128 * 74, 512, 128),
+    (1, 128 * 37 + 1, 512, 128),
+]
+
+
+@pytest.mark.parametrize("in_dt,out_dt", [("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32")])
+@pytest.mark.parametrize("batch,n,c,m", TMA_RG_CASES)
+def test_hca_row_group_splits(batch, n, c, m, in_dt, out_dt):
+    d = synth.stream_inputs("hca", batch, n, c, m, in_dt, seed=11 + n + m)
+    out = _run_hca(d, m, in_dt, out_dt)
+    ref = O.hca_compress(d["C"], d["Z"], d["B"], m)
+    assert kvc.device_status() == kvc.KVC_OK
+    check_close(out, ref, out_dt, f"hca {batch}x{n}x{c} m={m}")
+
 
 @pytest.mark.parametrize("in_dt,out_dt", [("f32", "f32"), ("bf16", "bf16"), ("bf16", "f32"),
                                           ("f32", "bf16")])
