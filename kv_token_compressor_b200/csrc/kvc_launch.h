@@ -96,7 +96,11 @@ unsigned int read_and_clear_indexer_error(bool* failed);
 // KVC_ERR_UNSUPPORTED when the problem or the device does not fit it (the caller then uses
 // the register-staged kernels).
 kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st);
-// Reads and clears its error word (no synchronisation): bit 0 a bounded wait gave up.
+// The TMA-fed CSA kernel (m = 4 with overlap, dense streams); KVC_ERR_UNSUPPORTED when the
+// problem or the device does not fit it.
+kvc_status launch_csa_tma(const StreamProblem& p, cudaStream_t st);
+// Reads and clears the TMA-fed kernels' error word (no synchronisation): bit 0 a bounded
+// wait gave up.
 unsigned int read_and_clear_window_error(bool* failed);
 
 // Device error words: bounded waits that gave up (fused kernels) and listed entries out

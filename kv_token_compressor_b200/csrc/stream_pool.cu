@@ -810,6 +810,12 @@ kvc_status launch_window(const StreamProblem& p, cudaStream_t st) {
 template <typename InT, typename OutT, bool LISTED, bool CACHE>
 kvc_status dispatch_stream(const StreamProblem& p, cudaStream_t st) {
   if (p.two_segments) {
+    if constexpr (!LISTED && !CACHE) {
+      if (p.m == 4) {
+        const kvc_status r = launch_csa_tma(p, st);
+        if (r != KVC_ERR_UNSUPPORTED) return r;
+      }
+    }
     switch (p.m) {
       case 1: return launch_csa_small<InT, OutT, 1, true, LISTED, CACHE>(p, st);
       case 2: return launch_csa_small<InT, OutT, 2, true, LISTED, CACHE>(p, st);

@@ -570,6 +570,241 @@ kvc_status launch_typed(const StreamProblem& p, cudaStream_t st) {
   }
 }
 
+
+// ---------------------------------------------------------------------------------
+// CSA, m = 4, two overlapping streams ("序列压缩注意力", eqs. attn-seqcomp-csa-softmax,
+// attn-seqcomp-csa-pool, attn-seqcomp-overlap-bound; "Ch 04 · CSA" §3): entry i pools the
+// a-block, rows [4i, 4i + 4) of Z^a / C^a, and the b-block, rows [4i - 4, 4i) of Z^b / C^b,
+// under one softmax over the 8 rows; entry 0 has no b-block (logit -inf, vector 0).
+//
+// A stage holds kCsaE entries: the [1][8][4][SC] boxes of Z^a and C^a at entry coordinate
+// g * 8 and of Z^b and C^b at g * 8 - 1 (the b-block of entry i is the a-row block of
+// entry i - 1 in the b streams; for the first group the coordinate is -1 and the copy
+// fills zeros, which entry 0 never reads).  Consumer thread rows pair up: ty = 2 e + h
+// takes entry e's a-block (h = 0) or b-block (h = 1), lanes l and l ^ 16 of one warp, and
+// the pair combines its maxima, sums and weighted sums with two shuffles per value.
+// Each window is short, so a warp's work per stage is one serial chain (loads, logits,
+// maximum, shuffle, exp2, sums, shuffle, divide); two independent groups of eight consumer
+// warps take alternate stages (each with its own copy of the bias) so that the SM always
+// has another chain to issue from.
+// ---------------------------------------------------------------------------------
+constexpr int kCsaE = 8;                                // entries per stage
+constexpr int kCsaStages = 6;                           // 6 x 32 KB, even: groups alternate
+constexpr int kCsaBox = kCsaE * 4 * 256;                // one stream's box: 8 KB
+constexpr int kCsaStageBytes = 4 * kCsaBox;             // Za, Ca, Zb, Cb
+constexpr int kCsaGroups = 2;
+constexpr int kCsaConsumers = kCsaGroups * kConsumers;  // 512
+constexpr int kCsaThreads = kCsaConsumers + 32;         // + one producer warp
+
+struct CsaArgs {
+  const float* Ba;  // [4, c]
+  const float* Bb;  // [4, c]
+  void* out;        // [batch, ne, c]
+  int64_t batch, ne, c;
+  int64_t groups;   // entry groups of kCsaE per sequence
+  int64_t tasks;    // slabs * batch * groups
+};
+
+template <typename InT>
+size_t csa_smem_bytes() {
+  constexpr int SC = slab<InT>();
+  return 1024 + static_cast<size_t>(kCsaStages) * kCsaStageBytes +
+         kCsaGroups * 8 * SC * sizeof(float) + 2 * kCsaStages * sizeof(uint64_t) + 16;
+}
+
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(kCsaThreads, 1)
+    csa_tma_kernel(const __grid_constant__ CUtensorMap mapZa,
+                   const __grid_constant__ CUtensorMap mapCa,
+                   const __grid_constant__ CUtensorMap mapZb,
+                   const __grid_constant__ CUtensorMap mapCb, const CsaArgs a) {
+  constexpr int CPT = VecInfo<InT>::kChannels;
+  constexpr int SC = slab<InT>();
+  constexpr int NP = CPT / 2;
+  static_assert(kCsaE * 4 * SC * sizeof(InT) == kCsaBox, "box geometry");
+  const float2 kL2e2 = make_float2(kLog2e, kLog2e);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = base;
+  float* sb_all = reinterpret_cast<float*>(base + kCsaStages * kCsaStageBytes);  // [2][8][SC]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb_all + kCsaGroups * 8 * SC);
+  uint64_t* empty = full + kCsaStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kCsaStages);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kCsaStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers / 32);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  const int64_t lo = static_cast<int64_t>(blockIdx.x) * a.tasks / gridDim.x;
+  const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * a.tasks / gridDim.x;
+  const Args ta{nullptr, nullptr, a.batch, a.ne, a.c, 4, a.groups, a.tasks, 0};  // task cursor
+
+  if (warp == kCsaConsumers / 32) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, used = 0, last_par = 0;
+      Task k(ta, lo);
+      for (int64_t t = lo; t < hi; ++t, k.next(ta)) {
+        if (!wait(&empty[s], ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], kCsaStageBytes);
+        const uint32_t dst = smem_u32(stages + s * kCsaStageBytes);
+        const int x = static_cast<int>(k.x * SC), z = static_cast<int>(k.g * kCsaE);
+        const int w = static_cast<int>(k.b);
+        tma_load_4d(dst, &mapZa, &full[s], x, 0, z, w);
+        tma_load_4d(dst + kCsaBox, &mapCa, &full[s], x, 0, z, w);
+        tma_load_4d(dst + 2 * kCsaBox, &mapZb, &full[s], x, 0, z - 1, w);
+        tma_load_4d(dst + 3 * kCsaBox, &mapCb, &full[s], x, 0, z - 1, w);
+        used |= 1u << s;
+        last_par = (last_par & ~(1u << s)) | (ph << s);
+        if (++s == kCsaStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      for (int q = 0; q < kCsaStages; ++q)
+        if (used & (1u << q)) wait(&full[q], (last_par >> q) & 1u, abort_flag, false);
+    }
+    return;
+  }
+
+  // ------------------------------------------------- consumers (warps 0..15, two groups)
+  const int grp = tid / kConsumers;  // takes the group's alternate tasks and stages
+  const int ct = tid - grp * kConsumers;
+  const int tx = ct % kCG, ty = ct / kCG;
+  const int e = ty >> 1, h = ty & 1;  // entry within the stage; a-block (0) or b-block (1)
+  const int sc0 = tx * CPT;
+  float* sb = sb_all + grp * 8 * SC;  // this group's bias rows
+  int s = grp;
+  uint32_t ph = 0;
+  bool dead = false;
+  int64_t cur_x = -1;
+  OutT* out = static_cast<OutT*>(a.out);
+
+  Task k(ta, lo);
+  if (grp == 1) k.next(ta);
+  for (int64_t t = lo + grp; t < hi; t += kCsaGroups, k.next(ta), k.next(ta)) {
+    if (k.x != cur_x) {  // the same in every thread of the group
+      if (cur_x >= 0) bar_named(1 + grp, kConsumers);  // nobody still reads the old bias
+      stage_bias(sb, a.Ba, a.Bb, 4, 8, SC, k.x * SC, a.c, ct, kConsumers,
+                 [](int sc) { return slab_bias_pos<CPT, kCG>(sc); });
+      bar_named(1 + grp, kConsumers);
+      cur_x = k.x;
+    }
+    const int64_t i = k.g * kCsaE + e;
+    const int64_t ch0 = k.x * SC + sc0;
+    const bool live = i < a.ne && ch0 < a.c;
+    const bool none = h == 1 && i == 0;  // entry 0 has no b-block
+
+    uint4 z[4], cv[4];
+    if (!dead && !wait(&full[s], ph, abort_flag)) dead = true;
+    {
+      const uint8_t* sz = stages + s * kCsaStageBytes + h * 2 * kCsaBox;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int off = ((e * 4 + r) * SC + sc0) * static_cast<int>(sizeof(InT));
+        z[r] = *reinterpret_cast<const uint4*>(sz + off);
+        cv[r] = *reinterpret_cast<const uint4*>(sz + kCsaBox + off);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    s += kCsaGroups;
+    if (s >= kCsaStages) {
+      s -= kCsaStages;
+      ph ^= 1u;
+    }
+
+    // logits of this thread's four rows (bias rows h*4 .. h*4+3), their maximum, then the
+    // pair's maximum
+    float2 l[4][NP], mx[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) mx[p] = make_float2(-INFINITY, -INFINITY);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4* bp = reinterpret_cast<const float4*>(sb + (h * 4 + r) * SC) + tx;
+#pragma unroll
+      for (int q = 0; q < NP / 2; ++q) {
+        const float4 bq = bp[q * kCG];
+        l[r][2 * q] = f2_fma(vec_pair<InT>(z[r], 2 * q), kL2e2, make_float2(bq.x, bq.y));
+        l[r][2 * q + 1] = f2_fma(vec_pair<InT>(z[r], 2 * q + 1), kL2e2, make_float2(bq.z, bq.w));
+        mx[2 * q] = f2_max(mx[2 * q], l[r][2 * q]);
+        mx[2 * q + 1] = f2_max(mx[2 * q + 1], l[r][2 * q + 1]);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      if (none) mx[p] = make_float2(-INFINITY, -INFINITY);
+      mx[p].x = fmaxf(mx[p].x, __shfl_xor_sync(0xffffffffu, mx[p].x, 16));
+      mx[p].y = fmaxf(mx[p].y, __shfl_xor_sync(0xffffffffu, mx[p].y, 16));
+    }
+    float res[CPT];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const float2 negm = make_float2(-mx[p].x, -mx[p].y);
+      float2 sum = make_float2(0.f, 0.f), acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float2 w = f2_ex2(f2_add(l[r][p], negm));
+        sum = f2_add(sum, w);
+        acc = f2_fma(w, vec_pair<InT>(cv[r], p), acc);
+      }
+      if (none) {
+        sum = make_float2(0.f, 0.f);
+        acc = make_float2(0.f, 0.f);
+      }
+      sum.x += __shfl_xor_sync(0xffffffffu, sum.x, 16);
+      sum.y += __shfl_xor_sync(0xffffffffu, sum.y, 16);
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+      res[2 * p] = __fdividef(acc.x, sum.x);
+      res[2 * p + 1] = __fdividef(acc.y, sum.y);
+    }
+    if (h == 0 && live && !dead) store_out<OutT, CPT>(out + (k.b * a.ne + i) * a.c + ch0, res);
+  }
+}
+
+template <typename InT, typename OutT>
+kvc_status launch_csa_typed(const StreamProblem& p, cudaStream_t st) {
+  constexpr int SC = slab<InT>();
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  const DeviceInfo di = device_info(dev);
+  if (di.sms == 0) return KVC_ERR_CUDA;
+  CsaArgs a{p.B0, p.B1, p.out, p.batch, p.ne, p.c, ceil_div(p.ne, kCsaE), 0};
+  a.tasks = ceil_div(p.c, SC) * p.batch * a.groups;
+  // Measured against the register-staged kernel (L2 flushed, B200): faster up to ~16 tasks
+  // per SM (c = 512 bf16: n = 1024 10.2 vs 16.4 us, n = 16384 24.6 vs 28.7 us; c = 128,
+  // n = 32768: 16.4 vs 18.5 us), then equal or slower (n = 2^18: 206 vs 197 us), where the
+  // loads-in-registers kernel already streams at ~0.97 of HBM.
+  if (a.tasks > 16 * static_cast<int64_t>(di.sms)) return KVC_ERR_UNSUPPORTED;
+  const size_t smem = csa_smem_bytes<InT>();
+  if (smem > di.smem_optin) return KVC_ERR_UNSUPPORTED;
+  const bool bf = sizeof(InT) == 2;
+  CUtensorMap m0, m1, m2, m3;
+  if (!make_stream_map(&m0, p.Z0, bf, p.batch, p.n, p.ne, p.c, 4, SC, 4, kCsaE) ||
+      !make_stream_map(&m1, p.C0, bf, p.batch, p.n, p.ne, p.c, 4, SC, 4, kCsaE) ||
+      !make_stream_map(&m2, p.Z1, bf, p.batch, p.n, p.ne, p.c, 4, SC, 4, kCsaE) ||
+      !make_stream_map(&m3, p.C1, bf, p.batch, p.n, p.ne, p.c, 4, SC, 4, kCsaE))
+    return KVC_ERR_UNSUPPORTED;
+  auto kern = csa_tma_kernel<InT, OutT>;
+  if (resident_blocks(kern, kCsaThreads, smem) < 1) return KVC_ERR_UNSUPPORTED;
+  const int64_t grid = a.tasks < di.sms ? a.tasks : di.sms;
+  kern<<<static_cast<unsigned>(grid), kCsaThreads, smem, st>>>(m0, m1, m2, m3, a);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
 }  // namespace wtma
 
 kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st) {
@@ -583,6 +818,20 @@ kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st) {
                       : wtma::launch_typed<__nv_bfloat16, float>(p, st);
   return p.out_bf16 ? wtma::launch_typed<float, __nv_bfloat16>(p, st)
                     : wtma::launch_typed<float, float>(p, st);
+}
+
+kvc_status launch_csa_tma(const StreamProblem& p, cudaStream_t st) {
+  if (!p.two_segments || p.m != 4 || p.listed || p.cache || p.ne <= 0 || p.ne > INT32_MAX ||
+      p.batch > INT32_MAX || p.c > INT32_MAX)
+    return KVC_ERR_UNSUPPORTED;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(p.C0) | reinterpret_cast<uintptr_t>(p.Z0) |
+                       reinterpret_cast<uintptr_t>(p.C1) | reinterpret_cast<uintptr_t>(p.Z1);
+  if (al & 15u) return KVC_ERR_UNSUPPORTED;
+  if (p.in_bf16)
+    return p.out_bf16 ? wtma::launch_csa_typed<__nv_bfloat16, __nv_bfloat16>(p, st)
+                      : wtma::launch_csa_typed<__nv_bfloat16, float>(p, st);
+  return p.out_bf16 ? wtma::launch_csa_typed<float, __nv_bfloat16>(p, st)
+                    : wtma::launch_csa_typed<float, float>(p, st);
 }
 
 unsigned int read_and_clear_window_error(bool* failed) {

@@ -1,6 +1,7 @@
 """GPU parity of the entry-list calls (csa_compress_entries / hca_compress_entries):
-ragged prefill, decode-style lists, agreement with the dense calls (CSA bit for bit), and
-out-of-range entries that the kernel skips and reports."""
+ragged prefill, decode-style lists, agreement with the dense calls (to bf16 rounding: the
+dense calls may take other kernels with another summation order), and out-of-range entries
+that the kernel skips and reports."""
 
 from __future__ import annotations
 
@@ -79,7 +80,10 @@ def test_lists_equal_dense_calls():
     out = kvc.csa_compress_entries(flat["Ca"], flat["Cb"], flat["Za"], flat["Zb"], t["Ba"], t["Bb"],
                                    *_list(starts, lens, ents), m=4)
     torch.cuda.synchronize()
-    assert torch.equal(out.reshape(batch, ne, c), dense)
+    # the dense call runs the TMA-fed kernel, which adds the a- and b-block sums of a window
+    # in another order than the listed kernel: equal to bf16 rounding, not bit for bit
+    diff = (out.reshape(batch, ne, c).float() - dense.float()).abs()
+    assert torch.all(diff <= 2.0 ** -7 * dense.float().abs() + 1e-6).item()
     # HCA
     h = synth.stream_inputs("hca", batch, 128 * 9 + 5, c, 128, "bf16", seed=4)
     th = {k: dev(v, "bf16") if v.ndim == 3 else dev(v, "f32") for k, v in h.items()}

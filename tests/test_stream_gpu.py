@@ -109,6 +109,26 @@ TMA_RG_CASES = [
 ]
 
 
+# CSA m = 4 problems of up to ~16 tasks (8 entries x one channel slab) per SM take the
+# TMA-fed CSA kernel: several tasks per CTA, CTAs whose task range crosses a channel slab,
+# entry 0 of every sequence, groups cut short by the entry count.
+TMA_CSA_CASES = [
+    (1, 4 * 4096 + 3, 512),
+    (2, 4 * 1000 + 2, 256),
+    (4, 4 * 9, 64),
+]
+
+
+@pytest.mark.parametrize("in_dt,out_dt", [("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32")])
+@pytest.mark.parametrize("batch,n,c", TMA_CSA_CASES)
+def test_csa_tma_tasks(batch, n, c, in_dt, out_dt):
+    d = synth.stream_inputs("csa", batch, n, c, 4, in_dt, seed=5 + n + c)
+    out = _run_csa(d, 4, True, in_dt, out_dt)
+    ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], 4, True)
+    assert kvc.device_status() == kvc.KVC_OK
+    check_close(out, ref, out_dt, f"csa {batch}x{n}x{c}")
+
+
 @pytest.mark.parametrize("in_dt,out_dt", [("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32")])
 @pytest.mark.parametrize("batch,n,c,m", TMA_RG_CASES)
 def test_hca_row_group_splits(batch, n, c, m, in_dt, out_dt):
