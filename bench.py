@@ -536,7 +536,8 @@ def _workload(name, dev):
             nbytes = (2 * ne * m + 2 * (ne - 1) * m) * c * es + 2 * m * c * 4 + ne * c * es
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // m,
                     bound="hbm", units=float(nbytes), flush=nbytes < 4 * (126 << 20),
-                    kernel=("csa_small_m_kernel" if mode == "csa" else
+                    kernel=("csa_tma_kernel (TMA-fed, small problems)" if name == "csa_f32_n1024"
+                            else "csa_small_m_kernel" if mode == "csa" else
                             "window_tma_kernel (TMA-fed, 8 row groups)"),
                     traffic_key="hca_compress_bf16_n65536" if mode == "hca" else None,
                     config={"workload": f"{mode.upper()} streams: batch 1, n={n}, c={c}, m={m}, "
