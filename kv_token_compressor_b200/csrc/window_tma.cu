@@ -1,6 +1,8 @@
-// Single-segment softmax pool over long windows (HCA, m' = 128) fed by TMA (sm_100a).
+// Softmax pools fed by TMA from a shared-memory ring (sm_100a): the single-segment window
+// kernel for long windows (HCA, m' = 128) below, and the two-stream CSA kernel (m = 4) for
+// small problems further down.
 //
-// What it computes ("序列压缩注意力", eq. attn-seqcomp-hca; "Ch 05 · HCA" §2): for every
+// What the window kernel computes ("序列压缩注意力", eq. attn-seqcomp-hca; "Ch 05 · HCA" §2): for every
 // entry i and channel ch, the softmax over the window's m rows of Z[i*m + v, ch] + B[v, ch]
 // and the weighted sum of C[i*m + v, ch], exactly as the register-staged window kernel.
 //
@@ -18,6 +20,12 @@
 // group's E entries, so every consumer thread takes four rows per stage whatever RG is,
 // and rescales its running state once per two stages (eight rows).  Tasks are ordered slab
 // first, so a CTA's contiguous range of tasks re-stages the bias rarely.
+//
+// Measured limits.  At full clock the consumers just keep up with HBM (the producer waits
+// for free stages about 3/4 of the time); under the power cap they set the pace.  A copy
+// engine box row of 256 bytes takes ~6.5 ns, so per-SM TMA throughput with these boxes is
+// itself near the SM's share of HBM, and boxes much smaller than 8 KB run far slower (an
+// entry-list variant with 1 KB boxes reached ~21 GB/s per SM and was not kept).
 #include <cuda.h>
 
 #include "kvc_common.cuh"
