@@ -271,6 +271,15 @@ KVC_API int64_t kvc_topk_max_candidates(void);
  * if the synchronisation failed, else KVC_OK. */
 KVC_API kvc_status kvc_device_status(kvc_stream stream);
 
+/* Failure-detection self-test, no fault involved: launches one CTA whose first warp waits
+ * on a shared-memory barrier that nothing completes, gives up after the kernels' wait limit
+ * (2 s), raises the CTA's abort flag and the device error word; a second warp waiting on the
+ * same barrier leaves as soon as it sees the flag.  out: device int32[2], written with
+ * out[0] = 1 (the first wait gave up) and out[1] = 1 (the second left on the flag).
+ * Afterwards kvc_device_status() reports KVC_ERR_TIMEOUT once and the context stays usable.
+ * Errors: KVC_ERR_NULL, KVC_ERR_ALIGN, KVC_ERR_POINTER, KVC_ERR_CUDA (launch). */
+KVC_API kvc_status kvc_selftest_bounded_wait(int32_t* out, kvc_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

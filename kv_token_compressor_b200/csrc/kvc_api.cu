@@ -649,4 +649,12 @@ kvc_status kvc_device_status(kvc_stream stream) {
   return kvc::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));
 }
 
+kvc_status kvc_selftest_bounded_wait(int32_t* out, kvc_stream stream) {
+  if (!out) return KVC_ERR_NULL;
+  if (!aligned(out, 4)) return KVC_ERR_ALIGN;
+  const kvc_status s = check_device_ptr(out);
+  if (s != KVC_OK) return s;
+  return kvc::launch_wait_selftest(out, reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

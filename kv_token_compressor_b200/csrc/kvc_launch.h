@@ -99,6 +99,8 @@ kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st);
 // The TMA-fed CSA kernel (m = 4 with overlap, dense streams); KVC_ERR_UNSUPPORTED when the
 // problem or the device does not fit it.
 kvc_status launch_csa_tma(const StreamProblem& p, cudaStream_t st);
+// The bounded-wait self-test kernel (kvc_selftest_bounded_wait).
+kvc_status launch_wait_selftest(int32_t* out, cudaStream_t st);
 // Reads and clears the TMA-fed kernels' error word (no synchronisation): bit 0 a bounded
 // wait gave up.
 unsigned int read_and_clear_window_error(bool* failed);

@@ -813,6 +813,36 @@ kvc_status launch_csa_typed(const StreamProblem& p, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
+
+// ---------------------------------------------------------------------------------
+// Self-test of the bounded waits (failure detection without a GPU fault): warp 0 waits on
+// an mbarrier that nothing completes until the limit, raises the CTA's abort flag and the
+// error bit; warp 1 waits on the same barrier honouring the abort flag and must leave
+// once it is raised.  out[0] = 1 if warp 0 gave up, out[1] = 1 if warp 1 left on the flag.
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(64, 1) wait_selftest_kernel(int32_t* out) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_word;
+  volatile int* abort_flag = &abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // one arrival would complete phase 0; none comes
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    out[0] = wait(&bar, 0, abort_flag, false) ? 0 : 1;
+  } else if (threadIdx.x == 32) {
+    // start a quarter of the limit later, so that it is warp 0's wait that runs out first
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < kWaitLimitNs / 4) {
+    }
+    const uint64_t t1 = global_timer_ns();
+    const bool done = wait(&bar, 0, abort_flag, true);
+    out[1] = (!done && global_timer_ns() - t1 < kWaitLimitNs) ? 1 : 0;  // left on the flag
+  }
+}
+
 }  // namespace wtma
 
 kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st) {
@@ -840,6 +870,11 @@ kvc_status launch_csa_tma(const StreamProblem& p, cudaStream_t st) {
                       : wtma::launch_csa_typed<__nv_bfloat16, float>(p, st);
   return p.out_bf16 ? wtma::launch_csa_typed<float, __nv_bfloat16>(p, st)
                     : wtma::launch_csa_typed<float, float>(p, st);
+}
+
+kvc_status launch_wait_selftest(int32_t* out, cudaStream_t st) {
+  wtma::wait_selftest_kernel<<<1, 64, 0, st>>>(out);
+  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
 }
 
 unsigned int read_and_clear_window_error(bool* failed) {

@@ -44,6 +44,7 @@ SIGNATURES = {
     "hca_compress_fused_proj": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32, _p,
                                                ctypes.c_int, _p]),
     "kvc_device_status": (ctypes.c_int, [_p]),
+    "kvc_selftest_bounded_wait": (ctypes.c_int, [_p, _p]),
     "csa_compress_scalar_logits": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64,
                                                   _i64, _i32, _i32, _p, ctypes.c_int, _p]),
     "hca_compress_scalar_logits": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i32,
@@ -396,3 +397,12 @@ def topk_max_candidates() -> int:
 def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the kernels' device error status."""
     return int(lib().kvc_device_status(_stream(stream)))
+
+
+def selftest_bounded_wait(stream=None):
+    """Run the bounded-wait self-test kernel (about 2 s); returns the device int32[2] flags
+    (first wait gave up, second waiter left on the abort flag)."""
+    torch = _torch()
+    out = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    _check(lib().kvc_selftest_bounded_wait(_ptr(out), _stream(stream)), "kvc_selftest_bounded_wait")
+    return out
