@@ -109,6 +109,22 @@ TMA_RG_CASES = [
 ]
 
 
+@pytest.mark.parametrize("in_dt", ["bf16", "f32"])
+def test_hca_bias_not_16_byte_aligned(in_dt):
+    """A bias that is 4- but not 16-byte aligned cannot be copied by the tensor engine: the
+    TMA-fed window kernel then stages it with plain loads (same results)."""
+    d = synth.stream_inputs("hca", 2, 128 * 300 + 9, 256, 128, in_dt, seed=31)
+    Bbuf = torch.zeros(128 * 256 + 1, dtype=torch.float32, device="cuda")
+    B = Bbuf[1:].view(128, 256)
+    B.copy_(torch.from_numpy(d["B"]).cuda())
+    assert B.data_ptr() % 16 == 4
+    out = kvc.hca_compress(dev(d["C"], in_dt), dev(d["Z"], in_dt), B, m=128,
+                           out_dtype=tdtype(in_dt))
+    torch.cuda.synchronize()
+    assert kvc.device_status() == kvc.KVC_OK
+    check_close(out, O.hca_compress(d["C"], d["Z"], d["B"], 128), in_dt, "hca unaligned bias")
+
+
 # CSA m = 4 problems of up to ~16 tasks (8 entries x one channel slab) per SM take the
 # TMA-fed CSA kernel: several tasks per CTA, CTAs whose task range crosses a channel slab,
 # entry 0 of every sequence, groups cut short by the entry count.
