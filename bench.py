@@ -509,6 +509,7 @@ def _workload(name, dev):
         nbytes = seqs * (4 * m * c * 2 + c * 2 + 24) + 2 * m * c * 4
         return dict(inputs=t, launch=launch, outputs=[out], tokens=seqs * m, entries=seqs,
                     bound="hbm", units=float(nbytes), flush=True, kernel="csa_small_m_kernel (listed)",
+                    traffic_key="csa_compress_entries_decode_4096",
                     resident=("Ca", "Cb", "Za", "Zb", "Ba", "Bb"),
                     config={"workload": f"decode step: {seqs} sequences (lengths U[8, 1024)) each "
                                         f"emitting its newest CSA entry, c={c}, m=4, bf16",
@@ -539,7 +540,9 @@ def _workload(name, dev):
                     kernel=("csa_tma_kernel (TMA-fed, small problems)" if name == "csa_f32_n1024"
                             else "csa_small_m_kernel" if mode == "csa" else
                             "window_tma_kernel (TMA-fed, 8 row groups)"),
-                    traffic_key="hca_compress_bf16_n65536" if mode == "hca" else None,
+                    traffic_key={"hca_n65536": "hca_compress_bf16_n65536",
+                                 "csa_f32_n1024": "csa_compress_f32_n1024",
+                                 "indexer_keys": "csa_compress_bf16_c128_n1048576"}.get(name),
                     config={"workload": f"{mode.upper()} streams: batch 1, n={n}, c={c}, m={m}, "
                                         f"{dt} in/out", "n": n, "c": c, "m": m})
     raise SystemExit(f"unknown workload {name}")
@@ -691,6 +694,27 @@ def run_profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             flush.zero_()
             kvc.hca_compress(t["C"], t["Z"], t["B"], m=M_HCA)
+    elif kind == "csa_n1024":  # the n = 1024 fp32 CSA workload itself (TMA-fed small-problem kernel)
+        t = synth.stream_inputs_torch("csa", 1, 1024, C, M_CSA, "f32", seed=0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        for _ in range(launches):
+            flush.zero_()
+            kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=M_CSA)
+    elif kind == "indexer_keys":  # CSA at c = 128 (indexer keys), n = 2^18 (268 MB of streams)
+        t = synth.stream_inputs_torch("csa", 1, 1 << 18, 128, M_CSA, "bf16", seed=0)
+        for _ in range(launches):
+            kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=M_CSA)
+    elif kind == "decode":  # a decode list: 4096 sequences of lengths U[8, 64), newest entry each
+        g = torch.Generator(device="cuda")
+        g.manual_seed(0)
+        lens = torch.randint(8, 64, (4096,), generator=g, device="cuda") // M_CSA * M_CSA
+        starts = torch.cumsum(lens, 0) - lens
+        t = synth.stream_inputs_torch("csa", 1, int(lens.sum().item()), C, M_CSA, "bf16", seed=0)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        for _ in range(launches):
+            flush.zero_()
+            kvc.csa_compress_entries(t["Ca"][0], t["Cb"][0], t["Za"][0], t["Zb"][0], t["Ba"], t["Bb"],
+                                     starts, lens, lens // M_CSA - 1, m=M_CSA)
     elif kind == "indexer":  # 4 queries x 131072 keys (K 128 MB), top-1024
         T, S = 4, 1 << 17
         t = synth.indexer_inputs_torch(T, 64, T * S, seed=0)
@@ -733,7 +757,8 @@ def main():
                              "decode_entries", "cache_long", "indexer_decode"],
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "
                          "time one kernel on its own workload")
-    ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "indexer", "csa_fused", "hca_fused"],
+    ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "csa_n1024", "indexer_keys",
+                                               "decode", "indexer", "csa_fused", "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
     if args.profile_case:
