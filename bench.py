@@ -197,6 +197,15 @@ def cpu_baseline(budget_s=12.0):
                       f"single-threaded elementwise), {dt:.1f} s"}
 
 
+def default_config(world: int) -> dict:
+    """The default step's workload description, shared by both arms."""
+    return {"workload": "long-context streams: batch 1, n=2^20, c=512, bf16 in/out; "
+                        "CSA m=4 overlap + HCA m'=128 on the same streams",
+            "batch": 1, "n": N_TOK, "c": C, "m": M_CSA, "m_hca": M_HCA,
+            "l2": "inputs 4.3 GB > 126 MB L2, no flush",
+            "parallelism": f"weak: {world} independent replicas"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -218,10 +227,10 @@ def run_reference(args):
         "entries_per_s": steps * ne / t, "n_gpus": args.gpus, "steps": steps, "warmup": warm,
         "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "long-context streams n=2^20 c=512 bf16: CSA m=4 overlap + HCA m'=128",
-                   "sample_tokens_per_step": tokens},
+        "config": default_config(args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {tokens} tokens per step"},
+                         "sample": f"first {tokens} of the {N_TOK} tokens per step (CSA m=4 + "
+                                   f"HCA m'=128, fp64 numpy, single-threaded elementwise)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -337,11 +346,7 @@ def run_ours(args):
             "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "long-context streams: batch 1, n=2^20, c=512, bf16 in/out; "
-                                   "CSA m=4 overlap + HCA m'=128 on the same streams",
-                       "batch": 1, "n": N_TOK, "c": C, "m": M_CSA, "m_hca": M_HCA,
-                       "l2": "inputs 4.3 GB > 126 MB L2, no flush",
-                       "parallelism": f"weak: {world} independent replicas"},
+            "config": default_config(world),
             "roofline": {"bound": "hbm", "kernel": "csa_compress (csa_small_m_kernel<bf16,bf16,4>)",
                          "achieved": csa_gbs, "peak": peak, "unit": "GB/s",
                          "frac": csa_gbs / peak, "peak_kind": peak_kind, "traffic": traffic,

@@ -1,0 +1,56 @@
+"""The bench's JSON line keeps its contract: the keys the driver reads, consistent units, and
+the same metric / config on both arms.  The reference arm (the fp64 oracle on the host) runs
+here on the CPU; the GPU arm is checked on the small n = 1024 workload."""
+
+from __future__ import annotations
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+             "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "e2e"}
+
+
+def _run(*args, timeout=600):
+    out = subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True,
+                         text=True, timeout=timeout)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    line = _run("--impl", "reference", "--steps", "1", "--warmup", "0")
+    assert BASE_KEYS <= set(line)
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["n_gpus"] == 1 and line["steps"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    sys.path.insert(0, ROOT)
+    import bench
+    assert line["metric"] == bench.METRIC
+    assert line["config"] == bench.default_config(1)
+
+
+@pytest.mark.gpu
+def test_gpu_arm_line_small_workload():
+    line = _run("--workload", "csa_f32_n1024", "--steps", "5", "--warmup", "3", "--no-cpu-baseline")
+    assert BASE_KEYS <= set(line)
+    assert {"roofline", "gpu_launches", "clocks"} <= set(line)
+    r = line["roofline"]
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] > 0
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert line["gpu_launches"] == 5
+    e = line["e2e"]
+    assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0 and e["value"] > 0
+    assert e["value"] < line["value"]  # host copies inside its timed region
+    assert line["warmup"] >= 3
