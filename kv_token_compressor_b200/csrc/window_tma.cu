@@ -116,17 +116,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
 // per CTA, not on every task boundary).
 struct Task {
   int64_t x, b, g;
-  __device__ Task(const Args& a, int64_t t) {
-    const int64_t per_slab = a.batch * a.groups;
+  int64_t batch, groups;
+  __device__ Task(int64_t batch_, int64_t groups_, int64_t t) : batch(batch_), groups(groups_) {
+    const int64_t per_slab = batch * groups;
     x = t / per_slab;
     const int64_t r = t - x * per_slab;
-    b = r / a.groups;
-    g = r - b * a.groups;
+    b = r / groups;
+    g = r - b * groups;
   }
-  __device__ __forceinline__ void next(const Args& a) {
-    if (++g == a.groups) {
+  __device__ __forceinline__ void next() {
+    if (++g == groups) {
       g = 0;
-      if (++b == a.batch) {
+      if (++b == batch) {
         b = 0;
         ++x;
       }
@@ -207,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t nbias = 0;               // bias loads issued
       int64_t px = -1;
       bool ok = true;
-      Task k(a, lo);
-      for (int64_t t = lo; t < hi && ok; ++t, k.next(a)) {
+      Task k(a.batch, a.groups, lo);
+      for (int64_t t = lo; t < hi && ok; ++t, k.next()) {
         if (a.bias_tma && k.x != px) {
           // the slab's bias rows, once the consumers are done with the previous slab's
           if (nbias > 0 && !wait(bias_free, (nbias - 1) & 1u, abort_flag)) break;
@@ -256,8 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t nb = 0;  // bias loads consumed
   OutT* out = static_cast<OutT*>(a.out);
 
-  Task k(a, lo);
-  for (int64_t t = lo; t < hi; ++t, k.next(a)) {
+  Task k(a.batch, a.groups, lo);
+  for (int64_t t = lo; t < hi; ++t, k.next()) {
     if (k.x != cur_x) {  // the same in every consumer thread
       bool narrow = true;
       if (a.bias_tma) {
@@ -656,15 +657,14 @@ __global__ void __launch_bounds__(kCsaThreads, 1)
 
   const int64_t lo = static_cast<int64_t>(blockIdx.x) * a.tasks / gridDim.x;
   const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * a.tasks / gridDim.x;
-  const Args ta{nullptr, nullptr, a.batch, a.ne, a.c, 4, a.groups, a.tasks, 0};  // task cursor
 
   if (warp == kCsaConsumers / 32) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0, used = 0, last_par = 0;
-      Task k(ta, lo);
-      for (int64_t t = lo; t < hi; ++t, k.next(ta)) {
+      Task k(a.batch, a.groups, lo);
+      for (int64_t t = lo; t < hi; ++t, k.next()) {
         if (!wait(&empty[s], ph ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(&full[s], kCsaStageBytes);
         const uint32_t dst = smem_u32(stages + s * kCsaStageBytes);
@@ -700,9 +700,9 @@ __global__ void __launch_bounds__(kCsaThreads, 1)
   int64_t cur_x = -1;
   OutT* out = static_cast<OutT*>(a.out);
 
-  Task k(ta, lo);
-  if (grp == 1) k.next(ta);
-  for (int64_t t = lo + grp; t < hi; t += kCsaGroups, k.next(ta), k.next(ta)) {
+  Task k(a.batch, a.groups, lo);
+  if (grp == 1) k.next();
+  for (int64_t t = lo + grp; t < hi; t += kCsaGroups, k.next(), k.next()) {
     if (k.x != cur_x) {  // the same in every thread of the group
       if (cur_x >= 0) bar_named(1 + grp, kConsumers);  // nobody still reads the old bias
       stage_bias(sb, a.Ba, a.Bb, 4, 8, SC, k.x * SC, a.c, ct, kConsumers,
