@@ -34,6 +34,8 @@
 #include "stream_common.cuh"
 #include "tc_ptx.cuh"
 
+#include <type_traits>
+
 namespace kvc {
 
 // Bit 0: a bounded wait of the TMA-fed window kernel gave up (outputs undefined).
@@ -367,28 +369,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       // rows of this thread in the two stages: st*UR + rg + RG*q, (st+1)*UR + rg + RG*q
       const int v0 = st * UR + rg;
       if (dead || !live || v0 >= a.m) continue;  // v0 is the smallest row of the chunk
-      auto row_of = [&](int u) { return v0 + (u / kRowsPerThread) * UR + RG * (u % kRowsPerThread); };
-      auto valid = [&](int u) { return (u < kRowsPerThread || two) && row_of(u) < a.m; };
+      auto row_of = [&](int u) {
+        return v0 + (u / kRowsPerThread) * UR + RG * (u % kRowsPerThread);
+      };
+      // FULL: every row of the chunk exists (the common case), so no row needs a check; the
+      // checks cost about 7% of the consumers' instructions, which set this kernel's pace
+      // under the power cap (1000-step runs: 0.351 -> 0.336 ms at n = 2^20)
+      auto chunk = [&](auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
+        auto valid = [&](int u) {
+          return FULL || ((u < kRowsPerThread || two) && row_of(u) < a.m);
+        };
 
-      // pass 1: an upper bound of the chunk's largest logit per channel (see the register-
-      // staged window kernel: max z * log2 e + max b when the bias spread is small, else the
-      // exact per-row maximum)
-      float2 cm[NP];
-      if (fast) {
-        uint4 zm = z[0];
+        // pass 1: an upper bound of the chunk's largest logit per channel (see the register-
+        // staged window kernel: max z * log2 e + max b when the bias spread is small, else the
+        // exact per-row maximum)
+        float2 cm[NP];
+        if (fast) {
+          uint4 zm = z[0];
 #pragma unroll
-        for (int u = 1; u < 2 * kRowsPerThread; ++u)
-          if (valid(u)) zm = vec_max<InT>(zm, z[u]);
-        const float4* bx = reinterpret_cast<const float4*>(bmx) + tx;
+          for (int u = 1; u < 2 * kRowsPerThread; ++u)
+            if (valid(u)) zm = vec_max<InT>(zm, z[u]);
+          const float4* bx = reinterpret_cast<const float4*>(bmx) + tx;
 #pragma unroll
-        for (int q = 0; q < NP / 2; ++q) {
-          const float4 bq = bx[q * kCG];
-          cm[2 * q] = f2_fma(vec_pair<InT>(zm, 2 * q), kL2e2, make_float2(bq.x, bq.y));
-          cm[2 * q + 1] = f2_fma(vec_pair<InT>(zm, 2 * q + 1), kL2e2, make_float2(bq.z, bq.w));
+          for (int q = 0; q < NP / 2; ++q) {
+            const float4 bq = bx[q * kCG];
+            cm[2 * q] = f2_fma(vec_pair<InT>(zm, 2 * q), kL2e2, make_float2(bq.x, bq.y));
+            cm[2 * q + 1] = f2_fma(vec_pair<InT>(zm, 2 * q + 1), kL2e2, make_float2(bq.z, bq.w));
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < NP; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
+#pragma unroll
+          for (int u = 0; u < 2 * kRowsPerThread; ++u) {
+            if (valid(u)) {
+              const float4* bp = reinterpret_cast<const float4*>(sb + row_of(u) * SC) + tx;
+#pragma unroll
+              for (int q = 0; q < NP / 2; ++q) {
+                const float4 bq = bp[q * kCG];
+                cm[2 * q] = f2_max(cm[2 * q], f2_fma(vec_pair<InT>(z[u], 2 * q), kL2e2,
+                                                     make_float2(bq.x, bq.y)));
+                cm[2 * q + 1] = f2_max(cm[2 * q + 1], f2_fma(vec_pair<InT>(z[u], 2 * q + 1), kL2e2,
+                                                             make_float2(bq.z, bq.w)));
+              }
+            }
+          }
         }
-      } else {
+        // rescale the running state once per chunk
 #pragma unroll
-        for (int p = 0; p < NP; ++p) cm[p] = make_float2(-INFINITY, -INFINITY);
+        for (int p = 0; p < NP; ++p) {
+          const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 is valid
+          const float2 sc = make_float2(ex2_ftz(M[p].x - nm.x), ex2_ftz(M[p].y - nm.y));
+          S[p] = f2_mul(S[p], sc);
+          A[p] = f2_mul(A[p], sc);
+          M[p] = nm;
+        }
+        // pass 2: one exp2 per element
 #pragma unroll
         for (int u = 0; u < 2 * kRowsPerThread; ++u) {
           if (valid(u)) {
@@ -396,43 +432,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < NP / 2; ++q) {
               const float4 bq = bp[q * kCG];
-              cm[2 * q] = f2_max(cm[2 * q], f2_fma(vec_pair<InT>(z[u], 2 * q), kL2e2,
-                                                   make_float2(bq.x, bq.y)));
-              cm[2 * q + 1] = f2_max(cm[2 * q + 1], f2_fma(vec_pair<InT>(z[u], 2 * q + 1), kL2e2,
-                                                           make_float2(bq.z, bq.w)));
+              const float2 b2[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int pp = 2 * q + h;
+                const float2 l = f2_fma(vec_pair<InT>(z[u], pp), kL2e2, f2_sub(b2[h], M[pp]));
+                const float2 w = f2_ex2(l);
+                S[pp] = f2_add(S[pp], w);
+                A[pp] = f2_fma(w, vec_pair<InT>(cv[u], pp), A[pp]);
+              }
             }
           }
         }
-      }
-      // rescale the running state once per chunk
-#pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 is valid
-        const float2 sc = make_float2(ex2_ftz(M[p].x - nm.x), ex2_ftz(M[p].y - nm.y));
-        S[p] = f2_mul(S[p], sc);
-        A[p] = f2_mul(A[p], sc);
-        M[p] = nm;
-      }
-      // pass 2: one exp2 per element
-#pragma unroll
-      for (int u = 0; u < 2 * kRowsPerThread; ++u) {
-        if (valid(u)) {
-          const float4* bp = reinterpret_cast<const float4*>(sb + row_of(u) * SC) + tx;
-#pragma unroll
-          for (int q = 0; q < NP / 2; ++q) {
-            const float4 bq = bp[q * kCG];
-            const float2 b2[2] = {make_float2(bq.x, bq.y), make_float2(bq.z, bq.w)};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int pp = 2 * q + h;
-              const float2 l = f2_fma(vec_pair<InT>(z[u], pp), kL2e2, f2_sub(b2[h], M[pp]));
-              const float2 w = f2_ex2(l);
-              S[pp] = f2_add(S[pp], w);
-              A[pp] = f2_fma(w, vec_pair<InT>(cv[u], pp), A[pp]);
-            }
-          }
-        }
-      }
+      };
+      if (two && row_of(2 * kRowsPerThread - 1) < a.m) chunk(std::true_type{});
+      else chunk(std::false_type{});
     }
 
     if constexpr (RG == 1) {
