@@ -55,6 +55,7 @@ constexpr int kHalf = kTY * kRowsPerThread * 256;  // one stream's stage: 64 row
 constexpr int kStageBytes = 2 * kHalf;             // Z then C
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
 constexpr int kMinRows = 32;                       // shorter windows use the other kernels
+constexpr float kHeadroom = 16.f;                  // log2 units a chunk may exceed the reference
 
 struct Args {
   const float* B;  // [m, c]
@@ -415,14 +416,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // rescale the running state once per chunk
+        // M is the reference subtracted from the logits.  It moves (and the running sums
+        // are rescaled) only when a chunk's bound exceeds it by more than kHeadroom log2
+        // units: the weights then stay <= 2^kHeadroom, far from overflow, and a window's
+        // largest weight stays a normal number (the reference never exceeds the window's
+        // largest logit by more than the bias spread).  The first chunk always sets it
+        // (M = -inf), and most later chunks skip the rescale.
+        bool move = false;
 #pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 is valid
-          const float2 sc = make_float2(ex2_ftz(M[p].x - nm.x), ex2_ftz(M[p].y - nm.y));
-          S[p] = f2_mul(S[p], sc);
-          A[p] = f2_mul(A[p], sc);
-          M[p] = nm;
+        for (int p = 0; p < NP; ++p)
+          move |= cm[p].x > M[p].x + kHeadroom || cm[p].y > M[p].y + kHeadroom;
+        if (move) {
+#pragma unroll
+          for (int p = 0; p < NP; ++p) {
+            const float2 nm = f2_max(M[p], cm[p]);  // finite: row v0 is valid
+            const float2 sc = make_float2(ex2_ftz(M[p].x - nm.x), ex2_ftz(M[p].y - nm.y));
+            S[p] = f2_mul(S[p], sc);
+            A[p] = f2_mul(A[p], sc);
+            M[p] = nm;
+          }
         }
         // pass 2: one exp2 per element
 #pragma unroll
