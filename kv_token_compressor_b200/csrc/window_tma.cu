@@ -18,11 +18,14 @@
 // entry's rows are dealt round-robin to RG threads, whose partial (max, sum, acc) merge in
 // shared memory at the end of the window.  A stage holds UR = 4 RG rows of each of the
 // group's E entries, so every consumer thread takes four rows per stage whatever RG is,
-// and rescales its running state once per two stages (eight rows).  Tasks are ordered slab
-// first, so a CTA's contiguous range of tasks re-stages the bias rarely.
+// bounds its logits once per two stages (an 8-row chunk), and moves its softmax reference
+// (rescaling the running sums) only when a chunk's bound exceeds it by more than 16 log2
+// units.  Tasks are ordered slab first, so a CTA's contiguous range of tasks re-stages the
+// bias rarely.
 //
 // Measured limits.  At full clock the consumers just keep up with HBM (the producer waits
-// for free stages about 3/4 of the time); under the power cap they set the pace.  A copy
+// for free stages about 3/4 of the time); under the power cap they set the pace, hence the
+// lazy reference and a check-free path for full chunks.  A copy
 // engine box row of 256 bytes takes ~6.5 ns, so per-SM TMA throughput with these boxes is
 // itself near the SM's share of HBM, and boxes much smaller than 8 KB run far slower (an
 // entry-list variant with 1 KB boxes reached ~21 GB/s per SM and was not kept).
