@@ -450,6 +450,7 @@ def _workload(name, dev):
         return dict(inputs=t, launch=launch, outputs=[idx, val], tokens=T * S * 4, entries=T * S,
                     bound="hbm", units=score_bytes, flush=False, resident=("K",),
                     kernel="indexer_score_kernel (tcgen05, keys on M, heads on N)",
+                    traffic_key="indexer_scores_decode_8x262144",
                     parts=[dict(name="indexer_score_kernel", launch=score, units=score_bytes,
                                 bound="hbm"),
                            dict(name="indexer_topk_kernel", launch=select, units=topk_bytes,
@@ -470,7 +471,7 @@ def _workload(name, dev):
         rows = ne * m + (ne - 1) * m  # a-rows of every entry + b-rows of entries 1..
         nbytes = rows * c * 2 + rows * 2 + 2 * m * 4 + ne * c * 2  # values, logits, biases, out
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=ne, bound="hbm",
-                    units=float(nbytes), flush=False, kernel="scalar_pool_kernel",
+                    units=float(nbytes), flush=False, kernel="scalar_small_m_kernel",
                     config={"workload": f"scalar-logit CSA: batch 1, n={n}, c={c}, m=4 overlap, "
                                         "bf16 streams and logits", "n": n, "c": c, "m": m})
     if name == "cache_long":
@@ -490,7 +491,7 @@ def _workload(name, dev):
         nbytes = (2 * ne * m + 2 * (ne - 1) * m) * c * 2 + 2 * m * c * 4 + ne * ((c - r) + 2 * r)
         return dict(inputs=t, launch=launch, outputs=[nope, rope], tokens=n, entries=ne,
                     bound="hbm", units=float(nbytes), flush=False,
-                    kernel="csa_small_m_kernel (cache layout)",
+                    kernel="csa_small_m_kernel (cache layout)", traffic_key="csa_cache_bf16_n1048576",
                     config={"workload": f"CSA n={n}, c={c}, m=4, bf16 streams, entries written "
                                         f"as E4M3 [c-{r}] + RoPE'd bf16 [{r}]", "n": n, "c": c,
                             "m": m, "r": r})
@@ -720,6 +721,17 @@ def run_profile_case(kind: str, launches: int = 3):
             flush.zero_()
             kvc.csa_compress_entries(t["Ca"][0], t["Cb"][0], t["Za"][0], t["Zb"][0], t["Ba"], t["Bb"],
                                      starts, lens, lens // M_CSA - 1, m=M_CSA)
+    elif kind == "scalar":  # scalar-logit CSA, n = 2^18 (the scalar workload / 4)
+        t = synth.scalar_inputs_torch("csa", 1, 1 << 18, C, M_CSA, "bf16", seed=0)
+        for _ in range(launches):
+            kvc.csa_compress_scalar_logits(t["Ca"], t["Cb"], t["za"], t["zb"], t["ba"], t["bb"], m=M_CSA)
+    elif kind == "cache":  # CSA into the cache layout, n = 2^18 (the cache workload / 4)
+        n, r = 1 << 18, 64
+        t = synth.stream_inputs_torch("csa", 1, n, C, M_CSA, "bf16", seed=0, z_row_offset=Z_OFF)
+        inv = (10000.0 ** (-torch.arange(r // 2, device="cuda", dtype=torch.float64) * 2 / r)).float()
+        for _ in range(launches):
+            kvc.csa_compress_cache(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], r, inv, 4.0,
+                                   1.5, 1.0, m=M_CSA)
     elif kind == "indexer":  # 4 queries x 131072 keys (K 128 MB), top-1024
         T, S = 4, 1 << 17
         t = synth.indexer_inputs_torch(T, 64, T * S, seed=0)
@@ -763,7 +775,8 @@ def main():
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "
                          "time one kernel on its own workload")
     ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "csa_n1024", "indexer_keys",
-                                               "decode", "indexer", "csa_fused", "hca_fused"],
+                                               "decode", "scalar", "cache", "indexer", "csa_fused",
+                                               "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
     if args.profile_case:
