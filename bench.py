@@ -472,6 +472,7 @@ def _workload(name, dev):
         nbytes = rows * c * 2 + rows * 2 + 2 * m * 4 + ne * c * 2  # values, logits, biases, out
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=ne, bound="hbm",
                     units=float(nbytes), flush=False, kernel="scalar_small_m_kernel",
+                    traffic_key="csa_scalar_bf16_n1048576",
                     config={"workload": f"scalar-logit CSA: batch 1, n={n}, c={c}, m=4 overlap, "
                                         "bf16 streams and logits", "n": n, "c": c, "m": m})
     if name == "cache_long":
