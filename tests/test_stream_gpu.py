@@ -166,6 +166,30 @@ def test_hca_shapes(batch, n, c, m, in_dt, out_dt):
     check_close(out, ref, out_dt, f"hca {batch}x{n}x{c} m={m}")
 
 
+@pytest.mark.parametrize("profile", ["ramp", "late_jump", "falling", "ramp_below_headroom"])
+def test_hca_reference_moves(profile):
+    """The TMA-fed window kernel moves its softmax reference only when a chunk's logit bound
+    exceeds it by more than its headroom: logits that climb across a window (by ~2 log2
+    units a row, or just under the headroom per 8-row chunk), one very large late row, and
+    logits that fall (later chunks far below the reference) all pool like the fp64 oracle."""
+    m, c = 128, 256
+    h = synth.stream_inputs("hca", 2, m * 40 + 3, c, m, "f32", seed=41)
+    rows = np.arange(h["Z"].shape[1]) % m
+    ln2 = np.log(2.0)
+    if profile == "ramp":
+        shift = 2.0 * rows * ln2                   # +2 log2 units per row
+    elif profile == "late_jump":
+        shift = np.where(rows == m - 1, 100.0, 0.0)  # one row ~144 log2 units up
+    elif profile == "falling":
+        shift = -1.5 * rows                        # later chunks far below the first
+    else:
+        shift = 15.5 * ln2 * (rows // 8) / 1.0     # each chunk just under 16 log2 units up
+    h["Z"] = (h["Z"] + shift[None, :, None]).astype(np.float32)
+    out = _run_hca(h, m, "f32", "f32")
+    assert kvc.device_status() == kvc.KVC_OK
+    check_close(out, O.hca_compress(h["C"], h["Z"], h["B"], m), "f32", f"hca reference {profile}")
+
+
 def test_wide_logit_range():
     """Row offsets of +-30 on the logits: the max subtraction must keep exp2 finite."""
     d = synth.stream_inputs("csa", 2, 4 * 64, 64, 4, "f32", seed=3, z_row_offset=30.0)
