@@ -409,6 +409,7 @@ def _workload(name, dev):
                     bound="tensor", units=2.0 * n * d * 4 * c, flush=False,
                     kernel=("fused_pair_kernel<CSA> (CTA pairs, M=256)" if c % 128 == 0
                             else "fused_pool_kernel<CSA>"),
+                    traffic_key="fused_csa_n32768_d7168" if (n, d, c) == (32768, 7168, 512) else None,
                     config={"workload": f"CSA fused projection + pool: H [{n}, {d}] bf16, 4 W "
                                         f"[{d}, {c}] bf16, m=4 overlap, bf16 out", "n": n,
                             "d": d, "c": c, "m": 4})
