@@ -54,3 +54,27 @@ def test_gpu_arm_line_small_workload():
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0 and e["value"] > 0
     assert e["value"] < line["value"]  # host copies inside its timed region
     assert line["warmup"] >= 3
+
+
+def test_algorithmic_bytes_match_the_window_definition():
+    """The roofline's numerator counts every stream element the windows read exactly once:
+    enumerate the windows of a small problem by brute force and compare, then check the
+    default step's figures."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for batch, n, c in ((1, 4 * 37, 64), (3, 4 * 37 + 2, 128), (2, 128 * 5 + 9, 512)):
+        ne, nh = n // 4, n // 128
+        read = set()
+        for b in range(batch):
+            for i in range(ne):  # CSA: a-block of entry i in Z^a, C^a; b-block in Z^b, C^b
+                for k in range(4):
+                    read |= {("Za", b, 4 * i + k), ("Ca", b, 4 * i + k)}
+                    if i > 0:
+                        read |= {("Zb", b, 4 * (i - 1) + k), ("Cb", b, 4 * (i - 1) + k)}
+        csa = len(read) * c * 2 + 2 * 4 * c * 4 + batch * ne * c * 2
+        hread = {(s, b, r) for b in range(batch) for i in range(nh) for r in range(128 * i, 128 * i + 128)
+                 for s in ("Z", "C")}
+        hca = len(hread) * c * 2 + 128 * c * 4 + batch * nh * c * 2
+        assert bench.algorithmic_bytes(batch, n, c) == (csa, hca)
+    assert bench.algorithmic_bytes() == (4_563_410_944, 2_148_270_080)
