@@ -77,4 +77,4 @@ def test_algorithmic_bytes_match_the_window_definition():
                  for s in ("Z", "C")}
         hca = len(hread) * c * 2 + 128 * c * 4 + batch * nh * c * 2
         assert bench.algorithmic_bytes(batch, n, c) == (csa, hca)
-    assert bench.algorithmic_bytes() == (4_563_410_944, 2_148_270_080)
+    assert bench.algorithmic_bytes() == (4_563_410_944, 2_156_134_400)
