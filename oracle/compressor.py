@@ -22,7 +22,7 @@ numpy (no blocking, fusion or reordering beyond what the equations state):
   "Ch 05 · HCA", §2 compression formulas): S = Softmax_row(Z + B) over the m' rows of
   segment i, C^Comp_i = sum S_j (.) C_j, no overlap, single stream.
 
-Readings taken where the pages are silent or disagree (each is listed in the design doc):
+Readings taken where the pages are silent or disagree:
 Z and B are per channel (n x c and m x c), the softmax is joint over the 2m rows, the
 entry count is floor(n/m) with the trailing n mod m tokens not compressed, sequences of
 a batch are independent, the fused path keeps the streams unrounded (float64 here).

@@ -17,7 +17,7 @@ selected-set equation; §5 for k):
 * Selection: the entries whose scores are among the k largest of the query's candidates
   (k = 1024 on the Pro model, 512 on Flash).
 
-Readings where the page is silent (each is listed in the design doc):
+Readings where the page is silent:
 * Candidates: query t scores the n_visible[t] keys K[key_start[t] : key_start[t] +
   n_visible[t]] of its own sequence (a decode step sees all of its sequence's entries; a
   prefill query only the entries whose blocks are complete -- the caller decides).
