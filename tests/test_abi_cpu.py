@@ -324,3 +324,80 @@ def test_indexer_topk_rejects_before_launch(L, kw, status):
 def test_indexer_topk_limits(L):
     assert L.kvc_topk_max_candidates() == 8 * 40960
     assert ix_topk(L, T=0, sc=None, idx=None) == kvc.KVC_OK
+
+
+def csa_list(L, Ca=A, Cb=A, Za=A, Zb=A, in_dt=kvc.KVC_BF16, Ba=A, Bb=A, rows=4096, c=512, m=4,
+             overlap=1, start=A, slen=A, entry=A, num=64, out=A, out_dt=kvc.KVC_BF16):
+    return L.csa_compress_entries(Ca, Cb, Za, Zb, in_dt, Ba, Bb, rows, c, m, overlap, start, slen,
+                                  entry, num, out, out_dt, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dt=9), kvc.KVC_ERR_DTYPE),
+    (dict(out_dt=3), kvc.KVC_ERR_DTYPE),
+    (dict(overlap=2), kvc.KVC_ERR_SHAPE),
+    (dict(rows=-1), kvc.KVC_ERR_SHAPE),
+    (dict(m=0), kvc.KVC_ERR_SHAPE),
+    (dict(num=-1), kvc.KVC_ERR_SHAPE),
+    (dict(c=12), kvc.KVC_ERR_SHAPE),
+    (dict(rows=1 << 62), kvc.KVC_ERR_SHAPE),        # rows * c * 4 bytes overflows
+    (dict(num=1 << 62), kvc.KVC_ERR_SHAPE),         # num * c overflows
+    (dict(start=None), kvc.KVC_ERR_NULL),
+    (dict(slen=None), kvc.KVC_ERR_NULL),
+    (dict(entry=None), kvc.KVC_ERR_NULL),
+    (dict(Ca=None), kvc.KVC_ERR_NULL),
+    (dict(Bb=None), kvc.KVC_ERR_NULL),
+    (dict(out=None), kvc.KVC_ERR_NULL),
+    (dict(start=A + 4), kvc.KVC_ERR_ALIGN),         # the lists are int64
+    (dict(entry=A + 4), kvc.KVC_ERR_ALIGN),
+    (dict(Za=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(Cb=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(Ba=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(m=161), kvc.KVC_ERR_UNSUPPORTED),         # 2 m = 322 window rows
+])
+def test_csa_entries_rejects_before_launch(L, kw, status):
+    assert csa_list(L, **kw) == status
+
+
+def test_csa_entries_overlap_off_and_empty(L):
+    # overlap = 0 lets the b-stream pointers be NULL (validation reaches the a-stream check)
+    assert csa_list(L, overlap=0, Cb=None, Zb=None, Bb=None, Ca=MIS) == kvc.KVC_ERR_ALIGN
+    # an empty list (or c == 0) is valid and reads no pointer, the lists' included
+    none = dict(Ca=None, Cb=None, Za=None, Zb=None, Ba=None, Bb=None, start=None, slen=None,
+                entry=None, out=None)
+    assert csa_list(L, num=0, **none) == kvc.KVC_OK
+    assert csa_list(L, c=0, **none) == kvc.KVC_OK
+
+
+def hca_list(L, C=A, Z=A, in_dt=kvc.KVC_BF16, B=A, rows=4096, c=512, m=128, start=A, slen=A,
+             entry=A, num=8, out=A, out_dt=kvc.KVC_BF16):
+    return L.hca_compress_entries(C, Z, in_dt, B, rows, c, m, start, slen, entry, num, out, out_dt,
+                                  None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(in_dt=2), kvc.KVC_ERR_DTYPE),
+    (dict(rows=-128), kvc.KVC_ERR_SHAPE),
+    (dict(c=20), kvc.KVC_ERR_SHAPE),
+    (dict(m=-1), kvc.KVC_ERR_SHAPE),
+    (dict(slen=None), kvc.KVC_ERR_NULL),
+    (dict(Z=None), kvc.KVC_ERR_NULL),
+    (dict(B=None), kvc.KVC_ERR_NULL),
+    (dict(slen=A + 4), kvc.KVC_ERR_ALIGN),
+    (dict(C=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(out=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(B=A + 1), kvc.KVC_ERR_ALIGN),
+    (dict(m=321), kvc.KVC_ERR_UNSUPPORTED),
+])
+def test_hca_entries_rejects_before_launch(L, kw, status):
+    assert hca_list(L, **kw) == status
+
+
+def test_hca_entries_empty(L):
+    assert hca_list(L, num=0, C=None, Z=None, B=None, start=None, slen=None, entry=None,
+                    out=None) == kvc.KVC_OK
+
+
+def test_selftest_rejects_before_launch(L):
+    assert L.kvc_selftest_bounded_wait(None, None) == kvc.KVC_ERR_NULL
+    assert L.kvc_selftest_bounded_wait(A + 2, None) == kvc.KVC_ERR_ALIGN
