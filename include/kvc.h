@@ -266,9 +266,13 @@ KVC_API kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* 
 /* The largest n_visible indexer_topk accepts (its candidates stay on chip). */
 KVC_API int64_t kvc_topk_max_candidates(void);
 
-/* Synchronises `stream`, then reports and clears the device-side error word that
- * kernels set when a bounded wait gives up: KVC_ERR_TIMEOUT if one did, KVC_ERR_CUDA
- * if the synchronisation failed, else KVC_OK. */
+/* Synchronises `stream`, then reports and clears the device-side error words that kernels
+ * set: KVC_ERR_CUDA if the synchronisation or a read of the words failed; else
+ * KVC_ERR_TIMEOUT if a bounded wait gave up (this takes precedence); else KVC_ERR_INDEX if
+ * an entry list or an indexer window named rows outside its sequence or the streams; else
+ * KVC_OK.  The words belong to the current device, not to a stream or a host thread: they
+ * collect what every kernel of this library set since the last call, and one call clears
+ * them for all callers. */
 KVC_API kvc_status kvc_device_status(kvc_stream stream);
 
 /* Failure-detection self-test, no fault involved: launches one CTA whose first warp waits
