@@ -8,6 +8,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -401,3 +402,30 @@ def test_hca_entries_empty(L):
 def test_selftest_rejects_before_launch(L):
     assert L.kvc_selftest_bounded_wait(None, None) == kvc.KVC_ERR_NULL
     assert L.kvc_selftest_bounded_wait(A + 2, None) == kvc.KVC_ERR_ALIGN
+
+
+def test_binding_raises_without_the_library(monkeypatch):
+    # No CPU fallback: with libkvc.so absent every call fails loudly.
+    monkeypatch.setattr(kvc, "_lib", None)
+    monkeypatch.setattr(kvc, "LIB_PATH", os.path.join(ROOT, "no-such-dir", "libkvc.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        kvc.num_entries(8, 4)
+    with pytest.raises(RuntimeError, match="missing"):
+        kvc.lib()
+
+
+def test_product_package_never_reaches_the_oracle():
+    # The oracle is test infrastructure: the package neither imports it nor names it in an
+    # import, and importing the package (and its binding) loads no module of it.
+    pkg = os.path.join(ROOT, "kv_token_compressor_b200")
+    for name in sorted(os.listdir(pkg)):
+        if name.endswith(".py"):
+            src = open(os.path.join(pkg, name)).read()
+            assert not re.search(r"^\s*(from|import)\s+oracle\b", src, re.M), name
+    code = ("import sys; import kv_token_compressor_b200, kv_token_compressor_b200.kvc, "
+            "kv_token_compressor_b200.synth, kv_token_compressor_b200.shard; "
+            "print(sorted(m for m in sys.modules if m == 'oracle' or m.startswith('oracle.')))")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True,
+                         text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "[]"
