@@ -45,17 +45,24 @@ __all__ = [
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returns fp32 holding them."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    u = x.view(np.uint32)
+    # u + 0x7FFF + lsb, then the low half cleared: in 32 bits this wraps only for bit
+    # patterns above 0xFFFF7FFF, which are all NaNs and are restored below.
+    r = (u >> 16) & np.uint32(1)
+    r += u
+    r += np.uint32(0x7FFF)
+    r &= np.uint32(0xFFFF0000)
+    out = r.view(np.float32)
     nan = np.isnan(x)
-    out = r.astype(np.uint32).view(np.float32).copy()
-    out[nan] = np.nan
+    if nan.any():
+        out[nan] = np.nan
     return out
 
 
 def _normal(rng, shape, var=1.0):
-    return (rng.standard_normal(shape, dtype=np.float32) * np.float32(np.sqrt(var))).astype(np.float32)
+    a = rng.standard_normal(shape, dtype=np.float32)
+    a *= np.float32(np.sqrt(var))
+    return a
 
 
 def stream_inputs(mode: str, batch: int, n: int, c: int, m: int, dtype: str = "f32",
@@ -75,7 +82,7 @@ def stream_inputs(mode: str, batch: int, n: int, c: int, m: int, dtype: str = "f
         for k in names:
             if k.startswith("Z"):
                 off = rng.uniform(-z_row_offset, z_row_offset, size=(batch, n, 1)).astype(np.float32)
-                out[k] = (out[k] + off).astype(np.float32)
+                out[k] += off
     if dtype == "bf16":
         for k in names:
             out[k] = round_to_bf16(out[k])
