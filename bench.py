@@ -187,14 +187,89 @@ def oracle_time(d):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(budget_s=12.0):
+def cpu_baseline(budget_s=12.0, all_cores=True):
     probe = 4096
     rate = probe / oracle_time(oracle_inputs(probe))
     tokens = int(max(probe, min(1 << 18, rate * budget_s)) // M_HCA * M_HCA)
     dt = oracle_time(oracle_inputs(tokens))
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {tokens} of the {N_TOK} tokens (CSA m=4 + HCA m'=128, fp64 numpy, "
-                      f"single-threaded elementwise), {dt:.1f} s"}
+    out = {"value": tokens / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+           "sample": f"first {tokens} of the {N_TOK} tokens (CSA m=4 + HCA m'=128, fp64 numpy, "
+                     f"single-threaded elementwise), {dt:.1f} s"}
+    if all_cores:
+        out["all_cores"] = cpu_baseline_all_cores(tokens / dt)
+    return out
+
+
+def _oracle_worker(seed, tokens, reps, barrier, results):
+    """One process of the all-cores oracle timing: its own seeded piece of the workload,
+    generated before the common start; then `reps` passes of the oracle as it stands."""
+    try:
+        d = oracle_inputs(tokens, seed=seed)
+        import oracle.compressor  # noqa: F401  (the import stays out of the timed region)
+
+        barrier.wait()
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle_time(d)
+        results.put(time.perf_counter() - t0)
+    except Exception as e:  # reported by the parent, which then gives no figure
+        barrier.abort()
+        results.put(repr(e))
+
+
+def cpu_baseline_all_cores(rate1, seconds=4.0, max_tokens=1 << 19, max_workers=64):
+    """The same oracle on every host core this process may use: one spawned process per
+    core, each on its own seeded piece of the workload's shape (inputs are generated in the
+    process, outside the timed region), released together by a barrier.  The figure is the
+    tokens all processes handled over the parent's wall-clock time from the release to the
+    last result.  `rate1` (tokens/s on one core) sizes each process to ~`seconds` of work;
+    `max_tokens` bounds the tokens held at once by all processes together (8 KB each);
+    at most `max_workers` processes."""
+    import multiprocessing
+
+    cores = len(os.sched_getaffinity(0))
+    if max_workers:
+        cores = min(cores, max_workers)
+    if cores < 2:
+        return None
+    tokens = int(max(M_HCA, min(max_tokens // cores, rate1 * seconds)) // M_HCA * M_HCA)
+    reps = max(1, round(rate1 * seconds / tokens))
+    ctx = multiprocessing.get_context("spawn")  # never fork a process that holds a GPU context
+    barrier, results = ctx.Barrier(cores + 1), ctx.Queue()
+    pin = {k: "1" for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    saved = {k: os.environ.get(k) for k in pin}
+    os.environ.update(pin)  # one thread per process: the processes are the parallelism
+    try:
+        procs = [ctx.Process(target=_oracle_worker, args=(1000 + 2 * w, tokens, reps, barrier,
+                                                          results), daemon=True)
+                 for w in range(cores)]
+        for p in procs:
+            p.start()
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    try:
+        barrier.wait(timeout=300)
+        t0 = time.perf_counter()
+        got = [results.get(timeout=300) for _ in procs]
+        wall = time.perf_counter() - t0
+    except Exception as e:
+        for p in procs:
+            p.terminate()
+        return {"error": f"all-cores timing failed: {e!r}"}
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+    if any(isinstance(g, str) for g in got):
+        return {"error": next(g for g in got if isinstance(g, str))}
+    return {"value": cores * tokens * reps / wall, "unit": "tokens/s", "cores": cores,
+            "kind": "oracle", "wall_s": wall, "slowest_process_s": max(got),
+            "sample": f"{cores} processes x {reps} passes over {tokens} tokens each (own seeded "
+                      f"piece of the workload's shape; CSA m=4 + HCA m'=128, fp64 numpy, one "
+                      f"thread per process)"}
 
 
 def default_config(world: int) -> dict:

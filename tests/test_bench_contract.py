@@ -78,3 +78,17 @@ def test_algorithmic_bytes_match_the_window_definition():
         hca = len(hread) * c * 2 + 128 * c * 4 + batch * nh * c * 2
         assert bench.algorithmic_bytes(batch, n, c) == (csa, hca)
     assert bench.algorithmic_bytes() == (4_563_410_944, 2_156_134_400)
+
+
+def test_cpu_baseline_all_cores_small():
+    # The all-cores oracle timing on two spawned processes with a tiny sample: it reports
+    # the processes it used and a positive rate, or no figure on a one-core host.
+    import bench
+
+    if len(os.sched_getaffinity(0)) < 2:
+        assert bench.cpu_baseline_all_cores(2e4, seconds=0.1, max_tokens=2048) is None
+        return
+    r = bench.cpu_baseline_all_cores(2e4, seconds=0.1, max_tokens=2048, max_workers=2)
+    assert "error" not in r, r
+    assert r["cores"] == 2 and r["kind"] == "oracle" and r["unit"] == "tokens/s"
+    assert r["value"] > 0 and r["wall_s"] >= r["slowest_process_s"] > 0
