@@ -429,3 +429,49 @@ def test_product_package_never_reaches_the_oracle():
                          text=True, timeout=300)
     assert out.returncode == 0, out.stderr
     assert out.stdout.strip() == "[]"
+
+
+def _header_prototypes():
+    """name -> (return type, [parameter types]) for every KVC_API declaration, with the
+    comments removed and the parameter names dropped."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    protos = {}
+    for ret, name, params in re.findall(r"KVC_API\s+([\w\s\*]+?)\s*\b(\w+)\s*\(([^)]*)\)\s*;", src):
+        types = []
+        for p in params.split(","):
+            p = " ".join(p.split())
+            if not p or p == "void":
+                continue
+            p = re.sub(r"\b\w+$", "", p).strip()  # drop the parameter name
+            types.append(p.replace(" *", "*"))
+        protos[name] = (" ".join(ret.split()).replace(" *", "*"), types)
+    return protos
+
+
+# The ctypes class each C type of the header must be bound with (pointers of any kind
+# travel as void*; enums are C ints).
+_CTYPE = {
+    "int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32, "double": ctypes.c_double,
+    "float": ctypes.c_float, "kvc_status": ctypes.c_int, "kvc_dtype": ctypes.c_int,
+    "kvc_stream": ctypes.c_void_p, "const char*": ctypes.c_char_p,
+}
+
+
+def _ctype_of(t):
+    if t.endswith("*") and t != "const char*":
+        return ctypes.c_void_p
+    return _CTYPE[t]
+
+
+def test_binding_signatures_match_the_header():
+    protos = _header_prototypes()
+    assert set(protos) == set(header_entry_points())
+    assert set(kvc.SIGNATURES) == set(protos)
+    for name, (ret, params) in protos.items():
+        res, args = kvc.SIGNATURES[name]
+        assert res is _ctype_of(ret), (name, ret)
+        assert len(args) == len(params), (name, len(args), len(params))
+        for i, (a, p) in enumerate(zip(args, params)):
+            assert a is _ctype_of(p), (name, i, p, a)
