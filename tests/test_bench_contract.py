@@ -92,3 +92,13 @@ def test_cpu_baseline_all_cores_small():
     assert "error" not in r, r
     assert r["cores"] == 2 and r["kind"] == "oracle" and r["unit"] == "tokens/s"
     assert r["value"] > 0 and r["wall_s"] >= r["slowest_process_s"] > 0
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    # Under torchrun rank 0 alone times the oracle and prints; the other ranks exit 0 silently.
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2",
+                          "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True,
+                         text=True, timeout=300, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip() == ""
