@@ -258,9 +258,17 @@ def cpu_baseline_all_cores(rate1, seconds=4.0, max_tokens=1 << 19, max_workers=6
         got = [results.get(timeout=300) for _ in procs]
         wall = time.perf_counter() - t0
     except Exception as e:
+        why = []
+        try:  # a worker that raised has queued its exception
+            while len(why) < len(procs):
+                g = results.get(timeout=5)
+                if isinstance(g, str):
+                    why.append(g)
+        except Exception:
+            pass
         for p in procs:
             p.terminate()
-        return {"error": f"all-cores timing failed: {e!r}"}
+        return {"error": f"all-cores timing failed: {e!r}" + (f" ({why[0]})" if why else "")}
     finally:
         for p in procs:
             p.join(timeout=60)
