@@ -147,11 +147,46 @@ def _out(out, shape, dtype, like):
     return out
 
 
+def _need(name, t, numel, dtype):
+    """The library will read `numel` elements of `dtype` from `t`, and it sees only the
+    pointer: refuse a tensor of another type or one too small to hold them.  None is passed
+    on (the library reports a missing pointer it needs)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call reads {numel}")
+
+
+def _streams(lead, others, overlap_only, overlap):
+    """The other streams of a call: the lead stream's dtype and at least its size."""
+    for name, t in others:
+        if overlap or name not in overlap_only:
+            _need(name, t, lead.numel(), lead.dtype)
+
+
+def _biases(m, width, overlap, **bs):
+    """Position biases: fp32, m x width values each (Bb / bb only with overlap)."""
+    torch = _torch()
+    for name, t in bs.items():
+        if overlap or name not in ("Bb", "bb"):
+            _need(name, t, m * width, torch.float32)
+
+
+def _rope_freqs(inv_freq, r, c):
+    """inv_freq: fp32, r / 2 values, when r is one the library accepts (else it reports r)."""
+    if 0 < r <= c and r % 8 == 0:
+        _need("inv_freq", inv_freq, r // 2, _torch().float32)
+
+
 def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, m: int = 4, overlap: bool = True, out=None,
                  out_dtype=None, stream=None):
     """CSA compressor over precomputed streams [batch, n, c] (bf16 or fp32) with fp32
     biases [m, c].  Returns [batch, n // m, c] in ``out_dtype`` (default: input dtype)."""
     batch, n, c = Ca.shape
+    _streams(Ca, (("Cb", Cb), ("Za", Za), ("Zb", Zb)), ("Cb", "Zb"), overlap)
+    _biases(m, c, overlap, Ba=Ba, Bb=Bb)
     out_dtype = Ca.dtype if out_dtype is None else out_dtype
     out = _out(out, (batch, n // m, c), out_dtype, Ca)
     st = lib().csa_compress(_ptr(Ca), _ptr(Cb) if overlap else None, _ptr(Za),
@@ -165,6 +200,8 @@ def csa_compress(Ca, Cb, Za, Zb, Ba, Bb, m: int = 4, overlap: bool = True, out=N
 def hca_compress(C, Z, B, m: int = 128, out=None, out_dtype=None, stream=None):
     """HCA compressor over precomputed streams C, Z [batch, n, c] with bias B [m, c]."""
     batch, n, c = C.shape
+    _streams(C, (("Z", Z),), (), True)
+    _biases(m, c, True, B=B)
     out_dtype = C.dtype if out_dtype is None else out_dtype
     out = _out(out, (batch, n // m, c), out_dtype, C)
     st = lib().hca_compress(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
@@ -180,6 +217,9 @@ def csa_compress_scalar_logits(Ca, Cb, za, zb, ba, bb, m: int = 4, overlap: bool
     batch, n, c = Ca.shape
     if tuple(za.shape) != (batch, n) or za.dtype != Ca.dtype:
         raise ValueError("za must be [batch, n] with the streams' dtype")
+    _streams(Ca, (("Cb", Cb),), ("Cb",), overlap)
+    _streams(za, (("zb", zb),), ("zb",), overlap)
+    _biases(m, 1, overlap, ba=ba, bb=bb)
     out_dtype = Ca.dtype if out_dtype is None else out_dtype
     out = _out(out, (batch, n // m, c), out_dtype, Ca)
     st = lib().csa_compress_scalar_logits(
@@ -195,6 +235,7 @@ def hca_compress_scalar_logits(C, z, b, m: int = 128, out=None, out_dtype=None, 
     batch, n, c = C.shape
     if tuple(z.shape) != (batch, n) or z.dtype != C.dtype:
         raise ValueError("z must be [batch, n] with C's dtype")
+    _biases(m, 1, True, b=b)
     out_dtype = C.dtype if out_dtype is None else out_dtype
     out = _out(out, (batch, n // m, c), out_dtype, C)
     st = lib().hca_compress_scalar_logits(_ptr(C), _ptr(z), _dtype_code(C.dtype), _ptr(b), batch, n,
@@ -216,6 +257,8 @@ def csa_compress_entries(Ca, Cb, Za, Zb, Ba, Bb, seq_start, seq_len, entry, m: i
     streams [total_rows, c].  Returns [num, c]; row k is entry entry[k] of its sequence."""
     total_rows, c = Ca.shape
     num = entry.shape[0]
+    _streams(Ca, (("Cb", Cb), ("Za", Za), ("Zb", Zb)), ("Cb", "Zb"), overlap)
+    _biases(m, c, overlap, Ba=Ba, Bb=Bb)
     out_dtype = Ca.dtype if out_dtype is None else out_dtype
     out = _out(out, (num, c), out_dtype, Ca)
     st = lib().csa_compress_entries(
@@ -232,6 +275,8 @@ def hca_compress_entries(C, Z, B, seq_start, seq_len, entry, m: int = 128, out=N
     """HCA entries listed by device int64 arrays over packed streams [total_rows, c]."""
     total_rows, c = C.shape
     num = entry.shape[0]
+    _streams(C, (("Z", Z),), (), True)
+    _biases(m, c, True, B=B)
     out_dtype = C.dtype if out_dtype is None else out_dtype
     out = _out(out, (num, c), out_dtype, C)
     st = lib().hca_compress_entries(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), total_rows, c,
@@ -268,6 +313,9 @@ def csa_compress_cache(Ca, Cb, Za, Zb, Ba, Bb, r, inv_freq, pos_stride=4.0, pos_
     """CSA entries in the cache layout: E4M3 bytes [batch, N_e, c - r] and RoPE'd bf16
     [batch, N_e, r].  The default position is the centre of the entry's own m-block."""
     batch, n, c = Ca.shape
+    _streams(Ca, (("Cb", Cb), ("Za", Za), ("Zb", Zb)), ("Cb", "Zb"), overlap)
+    _biases(m, c, overlap, Ba=Ba, Bb=Bb)
+    _rope_freqs(inv_freq, r, c)
     ne = n // m
     nope, rope = _cache_outs(batch * ne, c, r, Ca, out_nope, out_rope)
     st = lib().csa_compress_cache(
@@ -283,6 +331,9 @@ def hca_compress_cache(C, Z, B, r, inv_freq, pos_stride=128.0, pos_offset=63.5, 
                        m: int = 128, out_nope=None, out_rope=None, stream=None):
     """HCA entries in the cache layout (default position: the segment centre)."""
     batch, n, c = C.shape
+    _streams(C, (("Z", Z),), (), True)
+    _biases(m, c, True, B=B)
+    _rope_freqs(inv_freq, r, c)
     ne = n // m
     nope, rope = _cache_outs(batch * ne, c, r, C, out_nope, out_rope)
     st = lib().hca_compress_cache(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
@@ -298,6 +349,9 @@ def csa_compress_entries_cache(Ca, Cb, Za, Zb, Ba, Bb, seq_start, seq_len, entry
     """Listed CSA entries (decode-time cache insertion) in the cache layout."""
     total_rows, c = Ca.shape
     num = entry.shape[0]
+    _streams(Ca, (("Cb", Cb), ("Za", Za), ("Zb", Zb)), ("Cb", "Zb"), overlap)
+    _biases(m, c, overlap, Ba=Ba, Bb=Bb)
+    _rope_freqs(inv_freq, r, c)
     nope, rope = _cache_outs(num, c, r, Ca, out_nope, out_rope)
     st = lib().csa_compress_entries_cache(
         _ptr(Ca), _ptr(Cb) if overlap else None, _ptr(Za), _ptr(Zb) if overlap else None,
@@ -314,6 +368,9 @@ def hca_compress_entries_cache(C, Z, B, seq_start, seq_len, entry, r, inv_freq, 
     """Listed HCA entries in the cache layout."""
     total_rows, c = C.shape
     num = entry.shape[0]
+    _streams(C, (("Z", Z),), (), True)
+    _biases(m, c, True, B=B)
+    _rope_freqs(inv_freq, r, c)
     nope, rope = _cache_outs(num, c, r, C, out_nope, out_rope)
     st = lib().hca_compress_entries_cache(
         _ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), total_rows, c, m, _index(seq_start, num),
@@ -329,6 +386,11 @@ def csa_compress_fused_proj(H, W_kva, W_kvb, W_za, W_zb, Ba, Bb, batch: int, n: 
     torch = _torch()
     d = H.shape[1]
     c = W_kva.shape[1]
+    _need("H", H, batch * n * d, torch.bfloat16)
+    for name, w in (("W_kva", W_kva), ("W_kvb", W_kvb), ("W_za", W_za), ("W_zb", W_zb)):
+        if overlap or name not in ("W_kvb", "W_zb"):
+            _need(name, w, d * c, torch.bfloat16)
+    _biases(m, c, overlap, Ba=Ba, Bb=Bb)
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     out = _out(out, (batch, n // m, c), out_dtype, H)
     st = lib().csa_compress_fused_proj(
@@ -345,6 +407,10 @@ def hca_compress_fused_proj(H, W_kv, W_z, B, batch: int, n: int, m: int = 128, o
     torch = _torch()
     d = H.shape[1]
     c = W_kv.shape[1]
+    _need("H", H, batch * n * d, torch.bfloat16)
+    _need("W_kv", W_kv, d * c, torch.bfloat16)
+    _need("W_z", W_z, d * c, torch.bfloat16)
+    _biases(m, c, True, B=B)
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     out = _out(out, (batch, n // m, c), out_dtype, H)
     st = lib().hca_compress_fused_proj(_ptr(H), _ptr(W_kv), _ptr(W_z), _ptr(B), batch, n, d, c, m,
@@ -361,6 +427,11 @@ def lightning_indexer_scores(q, w, K, key_start, n_visible, max_visible: int, sc
     + s]) for s < n_visible[t] (the rest of each row untouched)."""
     torch = _torch()
     T, H, D = q.shape
+    _need("q", q, T * H * D, torch.bfloat16)
+    _need("w", w, T * H, torch.float32)
+    if K.dim() != 2 or K.shape[1] != D:
+        raise ValueError(f"K must be [rows, {D}]")
+    _need("K", K, K.shape[0] * D, torch.bfloat16)
     if scores is None:
         ld = max(4, -(-int(max_visible) // 4) * 4)
         scores = torch.zeros((T, ld), dtype=torch.float32, device=q.device)
@@ -380,6 +451,7 @@ def indexer_topk(scores, n_visible, k: int, max_visible: int, out_idx=None, out_
     past n_visible[t]."""
     torch = _torch()
     T, ld = scores.shape
+    _need("scores", scores, T * ld, torch.float32)
     out_idx = _out(out_idx, (T, k), torch.int32, scores)
     if want_scores:
         out_score = _out(out_score, (T, k), torch.float32, scores)

@@ -475,3 +475,80 @@ def test_binding_signatures_match_the_header():
         assert len(args) == len(params), (name, len(args), len(params))
         for i, (a, p) in enumerate(zip(args, params)):
             assert a is _ctype_of(p), (name, i, p, a)
+
+
+# ---- the Python binding refuses tensors the library would misread (checked before any
+# pointer is taken, so CPU tensors exercise it: a consistent call gets as far as the
+# "must be on a CUDA device" check)
+
+def _z(*shape, dt="f32"):
+    import torch
+
+    return torch.zeros(shape, dtype={"f32": torch.float32, "bf16": torch.bfloat16,
+                                     "f64": torch.float64, "i64": torch.int64}[dt])
+
+
+def _csa_args(**kw):
+    a = dict(Ca=_z(1, 64, 64, dt="bf16"), Cb=_z(1, 64, 64, dt="bf16"), Za=_z(1, 64, 64, dt="bf16"),
+             Zb=_z(1, 64, 64, dt="bf16"), Ba=_z(4, 64), Bb=_z(4, 64))
+    a.update(kw)
+    return a
+
+
+def _entries_args(**kw):
+    a = dict(Ca=_z(64, 64), Cb=_z(64, 64), Za=_z(64, 64), Zb=_z(64, 64), Ba=_z(4, 64), Bb=_z(4, 64),
+             seq_start=_z(2, dt="i64"), seq_len=_z(2, dt="i64"), entry=_z(2, dt="i64"))
+    a.update(kw)
+    return a
+
+
+BINDING_CASES = [
+    ("csa short Za", lambda: kvc.csa_compress(**_csa_args(Za=_z(1, 32, 64, dt="bf16"))), "Za holds"),
+    ("csa Zb dtype", lambda: kvc.csa_compress(**_csa_args(Zb=_z(1, 64, 64))), "Zb must be"),
+    ("csa Cb dtype", lambda: kvc.csa_compress(**_csa_args(Cb=_z(1, 64, 64))), "Cb must be"),
+    ("csa bias width", lambda: kvc.csa_compress(**_csa_args(Ba=_z(4, 32))), "Ba holds"),
+    ("csa bias dtype", lambda: kvc.csa_compress(**_csa_args(Bb=_z(4, 64, dt="bf16"))), "Bb must be"),
+    ("csa consistent", lambda: kvc.csa_compress(**_csa_args()), "CUDA device"),
+    ("csa overlap off", lambda: kvc.csa_compress(**_csa_args(Cb=None, Zb=None, Bb=_z(1)),
+                                                 overlap=False), "CUDA device"),
+    ("hca bias rows", lambda: kvc.hca_compress(_z(1, 256, 64), _z(1, 256, 64), _z(64, 64), m=128),
+     "B holds"),
+    ("hca Z dtype", lambda: kvc.hca_compress(_z(1, 256, 64), _z(1, 256, 64, dt="f64"),
+                                             _z(128, 64), m=128), "Z must be"),
+    ("scalar zb size", lambda: kvc.csa_compress_scalar_logits(
+        _z(1, 64, 64), _z(1, 64, 64), _z(1, 64), _z(1, 32), _z(4), _z(4)), "zb holds"),
+    ("scalar bias", lambda: kvc.hca_compress_scalar_logits(_z(1, 256, 64), _z(1, 256), _z(64),
+                                                           m=128), "b holds"),
+    ("entries Za", lambda: kvc.csa_compress_entries(**_entries_args(Za=_z(63, 64))), "Za holds"),
+    ("entries consistent", lambda: kvc.csa_compress_entries(**_entries_args()), "CUDA device"),
+    ("hca entries B", lambda: kvc.hca_compress_entries(
+        _z(256, 64), _z(256, 64), _z(128, 64, dt="f64"), _z(1, dt="i64"), _z(1, dt="i64"),
+        _z(1, dt="i64")), "B must be"),
+    ("cache inv_freq", lambda: kvc.csa_compress_cache(**_csa_args(), r=16, inv_freq=_z(4)),
+     "inv_freq holds"),
+    ("cache bad r reaches the library", lambda: kvc.csa_compress_cache(
+        **_csa_args(), r=12, inv_freq=_z(4)), "CUDA device"),
+    ("fused H dtype", lambda: kvc.hca_compress_fused_proj(
+        _z(256, 128), _z(128, 128, dt="bf16"), _z(128, 128, dt="bf16"), _z(128, 128), 1, 256),
+     "H must be"),
+    ("fused short H", lambda: kvc.hca_compress_fused_proj(
+        _z(255, 128, dt="bf16"), _z(128, 128, dt="bf16"), _z(128, 128, dt="bf16"), _z(128, 128),
+        1, 256), "H holds"),
+    ("fused W_zb", lambda: kvc.csa_compress_fused_proj(
+        _z(64, 128, dt="bf16"), *[_z(128, 128, dt="bf16")] * 3, _z(64, 128, dt="bf16"),
+        _z(4, 128), _z(4, 128), 1, 64), "W_zb holds"),
+    ("indexer K width", lambda: kvc.lightning_indexer_scores(
+        _z(2, 4, 128, dt="bf16"), _z(2, 4), _z(100, 64, dt="bf16"), _z(2, dt="i64"),
+        _z(2, dt="i64"), 100), "K must be"),
+    ("indexer w dtype", lambda: kvc.lightning_indexer_scores(
+        _z(2, 4, 128, dt="bf16"), _z(2, 4, dt="f64"), _z(100, 128, dt="bf16"), _z(2, dt="i64"),
+        _z(2, dt="i64"), 100), "w must be"),
+    ("topk scores dtype", lambda: kvc.indexer_topk(_z(2, 8, dt="f64"), _z(2, dt="i64"), 4, 8),
+     "scores must be"),
+]
+
+
+@pytest.mark.parametrize("name,call,msg", BINDING_CASES, ids=[c[0] for c in BINDING_CASES])
+def test_binding_refuses_tensors_the_library_would_misread(L, name, call, msg):
+    with pytest.raises(ValueError, match=msg):
+        call()
