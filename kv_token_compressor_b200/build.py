@@ -46,13 +46,19 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     if not force and not ptxas_verbose and _newer(LIB, deps):
         return LIB
     os.makedirs(BUILD_DIR, exist_ok=True)
-    objs = []
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
-    for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+    srcs = sources()
+    objs = [os.path.join(BUILD_DIR, os.path.basename(src) + ".o") for src in srcs]
+    cmds = [[nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj] for src, obj in zip(srcs, objs)]
+    # the translation units are independent: compile them side by side
+    from concurrent.futures import ThreadPoolExecutor
+
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for r in list(pool.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds)):
+            sys.stdout.write(r.stdout)
+            sys.stderr.write(r.stderr)
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args, r.stdout, r.stderr)
     tmp = LIB + ".tmp"
     subprocess.run([nvcc(), *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
