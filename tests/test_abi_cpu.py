@@ -552,3 +552,46 @@ BINDING_CASES = [
 def test_binding_refuses_tensors_the_library_would_misread(L, name, call, msg):
     with pytest.raises(ValueError, match=msg):
         call()
+
+
+C_CONSUMER = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "kvc.h"
+
+/* A plain C99 program against the C ABI.  Only calls that fail validation before any CUDA
+ * call are made, so it runs without a GPU. */
+int main(void) {
+  int bad = 0;
+  if (kvc_num_entries(1 << 20, 4) != 262144 || kvc_num_entries(1 << 20, 128) != 8192) bad |= 1;
+  if (kvc_num_entries(-1, 4) != -1) bad |= 2;
+  if (csa_compress(NULL, NULL, NULL, NULL, KVC_BF16, NULL, NULL, 1, 1024, 512, 4, 1, NULL,
+                   KVC_BF16, NULL) != KVC_ERR_NULL) bad |= 4;
+  if (hca_compress(NULL, NULL, KVC_BF16, NULL, 1, 1024, 512, 128, NULL, KVC_BF16, NULL)
+      != KVC_ERR_NULL) bad |= 8;
+  /* an empty problem is valid and touches nothing */
+  if (csa_compress(NULL, NULL, NULL, NULL, KVC_BF16, NULL, NULL, 0, 1024, 512, 4, 1, NULL,
+                   KVC_BF16, NULL) != KVC_OK) bad |= 16;
+  if (kvc_selftest_bounded_wait(NULL, NULL) != KVC_ERR_NULL) bad |= 32;
+  if (kvc_status_string(KVC_ERR_TIMEOUT) == NULL) bad |= 64;
+  if (kvc_topk_max_candidates() <= 0) bad |= 128;
+  printf("%s %d\n", kvc_status_string(KVC_ERR_SHAPE), bad);
+  return bad;
+}
+"""
+
+
+def test_plain_c_program_uses_the_abi(L, tmp_path):
+    # The header compiles as C99 (no C++ or CUDA types leak into it) and a C program linked
+    # against libkvc.so gets the documented statuses.
+    src = tmp_path / "consumer.c"
+    src.write_text(C_CONSUMER)
+    exe = tmp_path / "consumer"
+    lib_dir = os.path.dirname(kvc.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I",
+                         os.path.join(ROOT, "include"), str(src), "-L", lib_dir, "-lkvc",
+                         "-Wl,-rpath," + lib_dir, "-o", str(exe)], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    assert run.stdout.split()[-1] == "0"
