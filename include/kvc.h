@@ -49,7 +49,12 @@
  *                          entry was skipped and its output row left unwritten)
  *   An empty problem (batch == 0 or N_e == 0) is valid: KVC_OK, nothing is launched and
  *   no pointer is dereferenced.
- * Thread safety.  Calls may be made concurrently from several host threads.
+ * Thread safety.  Calls may be made concurrently from several host threads, with one
+ *   limit: a call sets its kernel's dynamic shared-memory limit to what it needs just
+ *   before launching, so two concurrent calls that run the same kernel with different
+ *   shared-memory needs (the same dtypes with different window lengths m) may see the
+ *   launch of one fail with KVC_ERR_CUDA; nothing is computed wrongly.  Serialise such
+ *   calls, or issue them from one thread.
  */
 #ifndef KVC_H
 #define KVC_H
