@@ -201,6 +201,56 @@ def cpu_baseline(budget_s=12.0, all_cores=True):
     return out
 
 
+def cpu_baseline_workload(name):
+    """The oracle, as it stands, on one host core for a named workload: the whole workload
+    for the two small streaming ones; for the fused ones, sampled entries (first, last and
+    evenly spaced) of a 4096-token H with the workload's d and c, since the work per entry
+    does not depend on n (the oracle projects only the rows an entry reads).  BLAS is held
+    to one thread.  None for the other workloads."""
+    from threadpoolctl import threadpool_limits
+
+    from kv_token_compressor_b200 import synth
+    from oracle import compressor as O
+
+    def timed(f):
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            f()
+            return time.perf_counter() - t0
+
+    if name in ("csa_f32_n1024", "hca_n65536"):
+        mode, n, m, dt = (("csa", 1024, M_CSA, "f32") if name == "csa_f32_n1024"
+                          else ("hca", 65536, M_HCA, "bf16"))
+        d = synth.stream_inputs(mode, 1, n, C, m, dt, seed=0)
+        if mode == "csa":
+            s = timed(lambda: O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"],
+                                             m, True))
+        else:
+            s = timed(lambda: O.hca_compress(d["C"], d["Z"], d["B"], m))
+        return {"value": n / s, "unit": "tokens/s", "entries_per_s": (n // m) / s, "cores": 1,
+                "kind": "oracle", "sampled": False,
+                "sample": f"the whole workload ({n} tokens; fp64 numpy, one thread), {s:.2f} s"}
+    if name in ("fused_csa", "fused_hca"):
+        csa = name == "fused_csa"
+        m, dm, n, k = (M_CSA, 7168, 4096, 48) if csa else (M_HCA, 4096, 4096, 8)
+        f = synth.fused_inputs("csa" if csa else "hca", 1, n, dm, C, m, seed=0)
+        ne = n // m
+        ents = sorted({(0, int(i)) for i in np.linspace(0, ne - 1, k).round()})
+        if csa:
+            s = timed(lambda: O.csa_compress_fused(f["H"], f["W_kva"], f["W_kvb"], f["W_za"],
+                                                   f["W_zb"], f["Ba"], f["Bb"], 1, n, m, True,
+                                                   entries=ents))
+        else:
+            s = timed(lambda: O.hca_compress_fused(f["H"], f["W_kv"], f["W_z"], f["B"], 1, n, m,
+                                                   entries=ents))
+        eps = len(ents) / s
+        return {"value": eps * m, "unit": "tokens/s", "entries_per_s": eps, "cores": 1,
+                "kind": "oracle", "sampled": True,
+                "sample": f"sampled: {len(ents)} entries of a {n}-token H, d={dm}, c={C}, m={m} "
+                          f"(fp64, one thread), {s:.2f} s; value = entries/s x m"}
+    return None
+
+
 def _oracle_worker(seed, tokens, reps, barrier, results):
     """One process of the all-cores oracle timing: its own seeded piece of the workload,
     generated before the common start; then `reps` passes of the oracle as it stands."""
@@ -748,6 +798,10 @@ def run_workload(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         }
         line["clocks"] = clocks
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline_workload(args.workload)
+            if cb is not None:
+                line["cpu_baseline"] = cb
         if w.get("parts"):
             line["kernels"] = {}
             for part in w["parts"]:

@@ -102,3 +102,17 @@ def test_reference_arm_other_ranks_do_no_work():
                          text=True, timeout=300, env=env)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip() == ""
+
+
+def test_workload_cpu_baselines():
+    # The oracle beside the other configs: the whole small CSA workload, and sampled entries
+    # of the fused HCA one (marked as sampled); workloads without one get none.
+    import bench
+
+    full = bench.cpu_baseline_workload("csa_f32_n1024")
+    assert full["kind"] == "oracle" and full["cores"] == 1 and full["sampled"] is False
+    assert full["value"] > 0 and abs(full["entries_per_s"] * 4 - full["value"]) < 1e-6 * full["value"]
+    samp = bench.cpu_baseline_workload("fused_hca")
+    assert samp["sampled"] is True and "sampled" in samp["sample"]
+    assert abs(samp["entries_per_s"] * 128 - samp["value"]) < 1e-6 * samp["value"]
+    assert bench.cpu_baseline_workload("decode_entries") is None
