@@ -116,3 +116,18 @@ def test_workload_cpu_baselines():
     assert samp["sampled"] is True and "sampled" in samp["sample"]
     assert abs(samp["entries_per_s"] * 128 - samp["value"]) < 1e-6 * samp["value"]
     assert bench.cpu_baseline_workload("decode_entries") is None
+
+
+def test_cpu_baseline_survives_a_failed_all_cores_run(monkeypatch):
+    # The one-core figure is reported even when the all-cores processes cannot be started.
+    import bench
+
+    def no_processes(*a, **k):
+        raise OSError("cannot start processes")
+
+    monkeypatch.setattr(bench, "cpu_baseline_all_cores", no_processes)
+    monkeypatch.setattr(bench, "oracle_inputs", lambda tokens, seed=0: None)
+    monkeypatch.setattr(bench, "oracle_time", lambda d: 0.5)
+    r = bench.cpu_baseline(budget_s=0.01)
+    assert r["value"] > 0 and r["cores"] == 1
+    assert r["all_cores"]["error"].startswith("all-cores timing failed")
