@@ -71,12 +71,12 @@ def _worker(rank, world, port, n, m, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("n", [4 * 61 + 2, 64])
-def test_two_gloo_ranks_match_single_process(n):
+@pytest.mark.parametrize("n,world", [(4 * 61 + 2, 2), (64, 2), (4 * 97 + 3, 3)])
+def test_gloo_ranks_match_single_process(n, world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, n, 4, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, n, 4, q)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
