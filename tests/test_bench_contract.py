@@ -131,3 +131,19 @@ def test_cpu_baseline_survives_a_failed_all_cores_run(monkeypatch):
     r = bench.cpu_baseline(budget_s=0.01)
     assert r["value"] > 0 and r["cores"] == 1
     assert r["all_cores"]["error"].startswith("all-cores timing failed")
+
+
+def test_profile_commands_name_existing_bench_options():
+    # Every summary under profiles/ gives the command that produced it; the bench options it
+    # names must still exist (argparse rejects an unknown choice before it reaches --help).
+    import glob
+    import re
+
+    used = set()
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*")):
+        used |= set(re.findall(r"--(profile-case|workload) ([a-z0-9_]+)", open(f).read()))
+    assert ("profile-case", "hca") in used
+    for opt, val in sorted(used):
+        out = subprocess.run([sys.executable, "bench.py", f"--{opt}", val, "--help"], cwd=ROOT,
+                             capture_output=True, text=True, timeout=120)
+        assert out.returncode == 0, (opt, val, out.stderr[-500:])
