@@ -41,3 +41,38 @@ def test_stream_inputs_are_seeded_and_bf16_valued():
         assert a[k].shape == (2, 64, 32)
         assert np.all(a[k].view(np.uint32) & 0xFFFF == 0), k  # bf16 values
     assert a["Ba"].shape == (4, 32)
+
+
+def test_torch_generators_shapes_dtypes_and_seeding():
+    # The device-side generators (used by the full-size GPU tests and the bench) run on any
+    # torch device; on the CPU their shapes, dtypes, seeding and ranges are checked here.
+    dev = "cpu"
+    a = synth.stream_inputs_torch("csa", 2, 256, 64, 4, "bf16", seed=1, z_row_offset=4.0, device=dev)
+    b = synth.stream_inputs_torch("csa", 2, 256, 64, 4, "bf16", seed=1, z_row_offset=4.0, device=dev)
+    for k in ("Ca", "Cb", "Za", "Zb"):
+        assert a[k].shape == (2, 256, 64) and a[k].dtype == torch.bfloat16
+        assert torch.equal(a[k], b[k])
+    for k in ("Ba", "Bb"):
+        assert a[k].shape == (4, 64) and a[k].dtype == torch.float32
+    # the logit rows carry one offset U(-4, 4) each: row means spread far wider than C's
+    za_means = a["Za"].float().mean(-1)
+    assert za_means.abs().max() > 2.0 and a["Ca"].float().mean(-1).abs().max() < 1.0
+    assert abs(a["Ba"].std().item() - 0.1 ** 0.5) < 0.05
+    h = synth.stream_inputs_torch("hca", 1, 512, 32, 128, "f32", seed=2, device=dev)
+    assert set(h) == {"C", "Z", "B"} and h["C"].dtype == torch.float32 and h["B"].shape == (128, 32)
+
+    f = synth.fused_inputs_torch("csa", 1, 64, 256, 128, 4, seed=3, device=dev)
+    assert f["H"].shape == (64, 256) and f["H"].dtype == torch.bfloat16
+    for k in ("W_kva", "W_kvb", "W_za", "W_zb"):
+        assert f[k].shape == (256, 128) and f[k].dtype == torch.bfloat16
+    # W ~ N(0, 1/d): unit-variance projections
+    assert abs(f["W_kva"].float().std().item() * 256 ** 0.5 - 1.0) < 0.05
+    fh = synth.fused_inputs_torch("hca", 2, 128, 128, 128, 128, seed=3, device=dev)
+    assert fh["H"].shape == (256, 128) and set(fh) == {"H", "W_kv", "W_z", "B"}
+
+    s = synth.scalar_inputs_torch("csa", 1, 64, 32, 4, "bf16", seed=4, device=dev)
+    assert s["za"].shape == (1, 64) and s["za"].dtype == torch.bfloat16 and s["ba"].shape == (4,)
+
+    ix = synth.indexer_inputs_torch(3, 8, 100, seed=5, device=dev)
+    assert ix["q"].shape == (3, 8, 128) and ix["q"].dtype == torch.bfloat16
+    assert ix["K"].shape == (100, 128) and ix["w"].shape == (3, 8) and ix["w"].dtype == torch.float32
