@@ -281,7 +281,7 @@ def cpu_baseline_all_cores(rate1, seconds=4.0, max_tokens=1 << 19, max_workers=6
     at most `max_workers` processes."""
     import multiprocessing
 
-    cores = len(os.sched_getaffinity(0))
+    host_cores = cores = len(os.sched_getaffinity(0))
     if max_workers:
         cores = min(cores, max_workers)
     if cores < 2:
@@ -334,7 +334,7 @@ def cpu_baseline_all_cores(rate1, seconds=4.0, max_tokens=1 << 19, max_workers=6
     if any(isinstance(g, str) for g in got):
         return {"error": next(g for g in got if isinstance(g, str))}
     return {"value": cores * tokens * reps / wall, "unit": "tokens/s", "cores": cores,
-            "kind": "oracle", "wall_s": wall, "slowest_process_s": max(got),
+            "host_cores": host_cores, "kind": "oracle", "wall_s": wall, "slowest_process_s": max(got),
             "sample": f"{cores} processes x {reps} passes over {tokens} tokens each (own seeded "
                       f"piece of the workload's shape; CSA m=4 + HCA m'=128, fp64 numpy, one "
                       f"thread per process)"}

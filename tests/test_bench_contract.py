@@ -91,6 +91,7 @@ def test_cpu_baseline_all_cores_small():
     r = bench.cpu_baseline_all_cores(2e4, seconds=0.1, max_tokens=2048, max_workers=2)
     assert "error" not in r, r
     assert r["cores"] == 2 and r["kind"] == "oracle" and r["unit"] == "tokens/s"
+    assert r["host_cores"] == len(os.sched_getaffinity(0))
     assert r["value"] > 0 and r["wall_s"] >= r["slowest_process_s"] > 0
 
 
