@@ -125,6 +125,81 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+class NvmlClockSampler:
+    """Clocks and clock-event reasons read through NVML by a host thread every ~2 ms, so
+    that even a timed region of a few tens of milliseconds holds several samples.  Reads
+    only; nothing is set.  `stop()` returns the same fields as :class:`ClockSampler`."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4))
+
+    def __init__(self, uuid, period_s=0.002):
+        import threading
+
+        import pynvml
+
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.period = period_s
+        self.samples = []
+        self.t0 = self.t1 = None
+        self.halt = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _reasons(self):
+        nv = self.nv
+        get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(get(self.h))
+
+    def _run(self):
+        nv = self.nv
+        while not self.halt.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.samples.append((time.time(), mhz, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def mark(self, start: bool):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def start(self):
+        self.thread.start()
+        time.sleep(0.05)
+
+    def stop(self):
+        self.halt.set()
+        self.thread.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        rows = [s for s in self.samples
+                if self.t0 is None or (self.t0 <= s[0] <= (self.t1 or s[0]) + 0.002)]
+        bits = {name: getattr(self.nv, attr, val) for name, attr, val in self.REASONS}
+        reasons = sorted({name for _, _, r in rows for name, b in bits.items() if r & b})
+        sm = [r[1] for r in rows]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows), "source": "nvml, ~2 ms period"}
+
+
+def clock_sampler(uuid):
+    """The NVML sampler when NVML answers, else nvidia-smi every 100 ms."""
+    try:
+        return NvmlClockSampler(uuid)
+    except Exception:
+        return ClockSampler(uuid)
+
+
 def dist_setup(n_gpus):
     import torch
 
@@ -418,7 +493,7 @@ def run_ours(args):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     props = torch.cuda.get_device_properties(dev)
     uuid = str(getattr(props, "uuid", ""))
-    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0"))
+    sampler = clock_sampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0"))
     sampler.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -474,6 +549,11 @@ def run_ours(args):
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
 
+    fused = None
+    if world == 1 and not args.no_fused:
+        del host, h_out_c, h_out_h
+        fused = time_fused(dev, stream)
+
     peak, peak_kind = peaks()
     csa_bytes, hca_bytes = algorithmic_bytes()
     csa_gbs = csa_bytes / (csa_ms * 1e-3) / 1e9
@@ -508,6 +588,8 @@ def run_ours(args):
             "e2e": {"value": world * N_TOK / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         }
+        if fused:
+            line["kernels"].update(fused)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)
@@ -515,6 +597,58 @@ def run_ours(args):
         import torch.distributed as dist
 
         dist.destroy_process_group()
+
+
+def time_fused(dev, stream, reps=20):
+    """The fused projection + pool kernels on their own workloads (CSA: H [32768, 7168],
+    c = 512; HCA: 4 x 131072 tokens, d = 4096, c = 512), timed after the default step's
+    timed region and reported beside it: CUDA events around each of `reps` back-to-back
+    launches on the launching stream after 3 warm-up launches; clocks sampled meanwhile.
+    FLOPs = 2 * tokens * d * (streams * c); fractions of the measured burst and sustained
+    bf16 GEMM rates."""
+    import torch
+
+    from kv_token_compressor_b200 import kvc
+
+    burst, kind = _peak("tensor")
+    sust, _ = _peak("tensor", sustained=True)
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", ""))
+    res = {}
+    for name in ("fused_csa", "fused_hca"):
+        w = _workload(name, dev)
+        for _ in range(3):
+            w["launch"](w["inputs"], stream)
+        torch.cuda.synchronize()
+        kernel = kvc.last_kernel()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        sampler = clock_sampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-")
+                                else (uuid or "0"))
+        sampler.start()
+        sampler.mark(True)
+        for a, b in evs:
+            a.record(stream)
+            w["launch"](w["inputs"], stream)
+            b.record(stream)
+        torch.cuda.synchronize()
+        sampler.mark(False)
+        clocks = sampler.stop()
+        if kvc.device_status(stream) != kvc.KVC_OK:
+            raise SystemExit(f"device error in {name}")
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        tf = w["units"] / (ms * 1e-3) / 1e12
+        res[name] = {"kernel": kernel, "workload": w["config"]["workload"], "ms": ms,
+                     "flops": w["units"], "TFLOP/s": tf, "frac": tf / burst,
+                     "frac_sustained": tf / sust, "peak": burst, "peak_sustained": sust,
+                     "peak_kind": kind, "unit": "TFLOP/s",
+                     "traffic": _traffic(w["traffic_key"]) if w.get("traffic_key") else None,
+                     "tokens_per_s": w["tokens"] / (ms * 1e-3),
+                     "entries_per_s": w["entries"] / (ms * 1e-3), "launches": reps,
+                     "clocks": clocks}
+        del w
+        torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------------------ other paths
@@ -720,7 +854,7 @@ def run_workload(args):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", ""))
-    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0"))
+    sampler = clock_sampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or "0"))
     sampler.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -920,6 +1054,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the fused-path kernels timed after the default step")
     ap.add_argument("--workload", default="long",
                     choices=["long", "fused_csa", "fused_hca", "hca_n65536", "csa_f32_n1024",
                              "indexer_keys", "fused_indexer_keys", "scalar_long",

@@ -49,12 +49,10 @@
  *                          entry was skipped and its output row left unwritten)
  *   An empty problem (batch == 0 or N_e == 0) is valid: KVC_OK, nothing is launched and
  *   no pointer is dereferenced.
- * Thread safety.  Calls may be made concurrently from several host threads, with one
- *   limit: a call sets its kernel's dynamic shared-memory limit to what it needs just
- *   before launching, so two concurrent calls that run the same kernel with different
- *   shared-memory needs (the same dtypes with different window lengths m) may see the
- *   launch of one fail with KVC_ERR_CUDA; nothing is computed wrongly.  Serialise such
- *   calls, or issue them from one thread.
+ * Thread safety.  Calls may be made concurrently from several host threads.  A kernel's
+ *   dynamic shared-memory limit is raised once to the device's maximum (under a lock)
+ *   and never lowered, so concurrent calls with different window lengths do not
+ *   interfere.  The device error words read by kvc_device_status() are per device.
  */
 #ifndef KVC_H
 #define KVC_H
@@ -214,7 +212,10 @@ KVC_API kvc_status hca_compress_entries_cache(
  * csa_compress pool): the four streams H W are formed on the tensor cores (bf16 in,
  * fp32 accumulate) and pooled on chip; they never reach device memory.
  *   H : [batch*n, d] bf16;  W_kva, W_kvb, W_za, W_zb : [d, c] bf16;  Ba, Bb : [m, c] fp32
- *   d % 64 == 0, c % 128 == 0;  out : [batch, N_e, c] out_dtype. */
+ *   d % 64 == 0, c % 128 == 0;  out : [batch, N_e, c] out_dtype.
+ *   The kernels implement the pages' CSA compressor only: m == 4 with overlap == 1.  Any
+ *   other valid m or overlap = 0 returns KVC_ERR_UNSUPPORTED (before any launch); the
+ *   streaming csa_compress covers those over precomputed streams. */
 KVC_API kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, const void* W_kvb,
                                    const void* W_za, const void* W_zb,
                                    const float* Ba, const float* Bb,
@@ -223,7 +224,8 @@ KVC_API kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, con
                                    void* out, kvc_dtype out_dtype, kvc_stream stream);
 
 /* HCA compressor fed by hidden states: C = H W_kv, Z = H W_z on the tensor cores, then
- * the hca_compress pool in the GEMM epilogue.  Shapes and rules as above. */
+ * the hca_compress pool in the GEMM epilogue.  Shapes and rules as above; the kernels
+ * implement m == 128 (the pages' m') only, any other valid m returns KVC_ERR_UNSUPPORTED. */
 KVC_API kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* W_z,
                                    const float* B, int64_t batch, int64_t n, int64_t d,
                                    int64_t c, int32_t m,
@@ -270,6 +272,13 @@ KVC_API kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* 
 
 /* The largest n_visible indexer_topk accepts (its candidates stay on chip). */
 KVC_API int64_t kvc_topk_max_candidates(void);
+
+/* Name of the kernel that the calling host thread's most recent successful call launched
+ * (e.g. "csa_small_m_kernel/c512", "window_tma_kernel", "fused_pair_kernel/csa"); "" before
+ * the first launch.  Static storage, never NULL.  The record is per host thread and is
+ * left unchanged by calls that launch nothing (errors, empty problems).  It shows which
+ * of the kernels behind one entry point the size-based dispatch picked. */
+KVC_API const char* kvc_last_kernel(void);
 
 /* Synchronises `stream`, then reports and clears the device-side error words that kernels
  * set: KVC_ERR_CUDA if the synchronisation or a read of the words failed; else

@@ -1165,11 +1165,11 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   }
   grid = a.units < sms ? a.units : sms;
   auto kern = fused_pool_kernel<CSA, BK, OutT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(C::SMEM)) != cudaSuccess)
-    return KVC_ERR_CUDA;
+  if (!raise_smem_limit(reinterpret_cast<const void*>(kern))) return KVC_ERR_CUDA;
   kern<<<static_cast<unsigned>(grid), kThreads, C::SMEM, st>>>(mh, mw[0], mw[1], mw[2], mw[3], a);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = CSA ? "fused_pool_kernel/csa" : "fused_pool_kernel/hca";
+  return KVC_OK;
 }
 
 // CTA-pair launch (fused_pair_kernel): clusters of two CTAs, as many as can be resident.
@@ -1191,9 +1191,7 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
       return KVC_ERR_CUDA;
   }
   auto kern = fused_pair_kernel<CSA, OutT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(C::SMEM)) != cudaSuccess)
-    return KVC_ERR_CUDA;
+  if (!raise_smem_limit(reinterpret_cast<const void*>(kern))) return KVC_ERR_CUDA;
   int clusters = 0;
   {
     cudaLaunchConfig_t cfg = {};
@@ -1229,7 +1227,9 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
   const int64_t ncl = a.units < clusters ? a.units : clusters;
   kern<<<static_cast<unsigned>(2 * ncl), pair::kThreads, C::SMEM, st>>>(mh, mw[0], mw[1], mw[2], mw[3],
                                                                    a);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = CSA ? "fused_pair_kernel/csa" : "fused_pair_kernel/hca";
+  return KVC_OK;
 }
 
 }  // namespace fused

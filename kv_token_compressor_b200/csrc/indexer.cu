@@ -752,12 +752,13 @@ kvc_status launch_indexer_scores(const IndexerProblem& p, cudaStream_t st) {
     return KVC_ERR_CUDA;
   ScoreArgs a{p.w, p.key_start, p.n_visible, p.scores, p.T, p.key_rows, p.max_visible, p.ld,
               tiles, units, p.H};
-  if (cudaFuncSetAttribute(indexer_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmem)) != cudaSuccess)
+  if (!raise_smem_limit(reinterpret_cast<const void*>(indexer_score_kernel)))
     return KVC_ERR_CUDA;
   const int64_t grid = units < sms ? units : sms;
   indexer_score_kernel<<<static_cast<unsigned>(grid), kThreads, kSmem, st>>>(mq, mk, a);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "indexer_score_kernel";
+  return KVC_OK;
 }
 
 int64_t topk_max_candidates() { return static_cast<int64_t>(idx::kCluster) * idx::kSlice; }
@@ -769,8 +770,7 @@ kvc_status launch_indexer_topk(const TopkProblem& p, cudaStream_t st) {
   TopkArgs a{p.scores, p.n_visible, p.out_idx, p.out_score, p.T, p.max_visible, p.ld, p.k};
   // Clusters of 8 CTAs (16-CTA clusters were measured slower on the decode step).
   auto try_launch = [&](auto kern, int cl, bool non_portable) -> kvc_status {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kTkSmem)) != cudaSuccess ||
+    if (!raise_smem_limit(reinterpret_cast<const void*>(kern)) ||
         (non_portable &&
          cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
              cudaSuccess)) {
@@ -796,6 +796,7 @@ kvc_status launch_indexer_topk(const TopkProblem& p, cudaStream_t st) {
     }
     cfg.gridDim = dim3(static_cast<unsigned>(p.T * cl), 1, 1);
     if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return KVC_ERR_CUDA;
+    last_kernel() = "indexer_topk_kernel";
     return KVC_OK;
   };
   return try_launch(indexer_topk_kernel<kCluster>, kCluster, false);

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/kvc.h"
+#include "kvc_host.h"
 #include "kvc_launch.h"
 
 namespace {
@@ -508,10 +509,10 @@ kvc_status hca_compress_entries_cache(const void* C, const void* Z, kvc_dtype in
   return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
-static kvc_status fused_common(FusedProblem* p, const void* H, const void* const* W, int nw,
-                               const float* B0, const float* B1, bool need_b1, int64_t batch,
-                               int64_t n, int64_t d, int64_t c, int32_t m, void* out,
-                               kvc_dtype out_dtype, bool* empty) {
+static kvc_status fused_common(FusedProblem* p, bool csa, int32_t overlap, const void* H,
+                               const void* const* W, int nw, const float* B0, const float* B1,
+                               bool need_b1, int64_t batch, int64_t n, int64_t d, int64_t c,
+                               int32_t m, void* out, kvc_dtype out_dtype, bool* empty) {
   *empty = false;
   if (!dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
   if (batch < 0 || n < 0 || d < 0 || c < 0 || m < 1) return KVC_ERR_SHAPE;
@@ -524,6 +525,8 @@ static kvc_status fused_common(FusedProblem* p, const void* H, const void* const
     return KVC_OK;
   }
   if (d == 0 || d % 64 != 0 || c % 128 != 0) return KVC_ERR_SHAPE;
+  // the tensor-core kernels implement the pages' two compressors only
+  if (csa ? (m != 4 || overlap != 1) : m != 128) return KVC_ERR_UNSUPPORTED;
   if (!H || !out || !B0 || (need_b1 && !B1)) return KVC_ERR_NULL;
   for (int i = 0; i < nw; ++i)
     if (!W[i]) return KVC_ERR_NULL;
@@ -561,11 +564,13 @@ kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, const void*
   kvc_status s;
   if (overlap) {
     const void* W[4] = {W_kva, W_kvb, W_za, W_zb};
-    s = fused_common(&p, H, W, 4, Ba, Bb, true, batch, n, d, c, m, out, out_dtype, &empty);
+    s = fused_common(&p, true, overlap, H, W, 4, Ba, Bb, true, batch, n, d, c, m, out, out_dtype,
+                     &empty);
     for (int i = 0; i < 4; ++i) p.W[i] = W[i];
   } else {  // a-streams only
     const void* W[2] = {W_kva, W_za};
-    s = fused_common(&p, H, W, 2, Ba, nullptr, false, batch, n, d, c, m, out, out_dtype, &empty);
+    s = fused_common(&p, true, overlap, H, W, 2, Ba, nullptr, false, batch, n, d, c, m, out,
+                     out_dtype, &empty);
     p.W[0] = W_kva;
     p.W[1] = nullptr;
     p.W[2] = W_za;
@@ -584,8 +589,8 @@ kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* 
   FusedProblem p{};
   bool empty = false;
   const void* W[2] = {W_kv, W_z};
-  kvc_status s =
-      fused_common(&p, H, W, 2, B, nullptr, false, batch, n, d, c, m, out, out_dtype, &empty);
+  kvc_status s = fused_common(&p, false, 0, H, W, 2, B, nullptr, false, batch, n, d, c, m, out,
+                              out_dtype, &empty);
   if (s != KVC_OK || empty) return s;
   p.W[0] = W_kv;
   p.W[1] = W_z;
@@ -644,6 +649,8 @@ kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* n_visibl
 }
 
 int64_t kvc_topk_max_candidates(void) { return kvc::topk_max_candidates(); }
+
+const char* kvc_last_kernel(void) { return kvc::last_kernel(); }
 
 kvc_status kvc_device_status(kvc_stream stream) {
   return kvc::read_and_clear_device_error(reinterpret_cast<cudaStream_t>(stream));

@@ -215,8 +215,11 @@ __device__ __forceinline__ void store_cache(const CacheFmt& cf, int64_t orow, in
     float rot[CPT];
 #pragma unroll
     for (int p = 0; p < CPT / 2; ++p) {
-      // angle in fp64 (the product of two fp32 values is exact), reduced by a multiple of
-      // 2 pi in fp64, then the fp32 sine and cosine of the remainder (|red| <= pi)
+      // angle in fp64, reduced by a multiple of 2 pi in fp64, then the fp32 sine and cosine
+      // of the remainder (|red| <= pi).  pos is exact for the usual integer or half-integer
+      // offsets and strides; the product with inv_freq and the reduction each add at most a
+      // few units of 2^-53 relative to |ang| (about 1e-10 rad at |ang| = 1e6), far below
+      // the fp32 rounding of the remainder (about 2e-7 rad near pi).
       const double ang = pos * static_cast<double>(cf.inv_freq[off / 2 + p]);
       const double turns = rint(ang * 0.15915494309189535);
       const float red = static_cast<float>(fma(-turns, 6.283185307179586, ang));

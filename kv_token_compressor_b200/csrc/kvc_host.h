@@ -33,15 +33,39 @@ inline DeviceInfo device_info(int dev) {
   return cache[dev];
 }
 
+// Raises kernel k's dynamic shared-memory limit on the current device to the most the
+// device allows beside the kernel's static shared memory.  Every launch path calls this
+// and never sets a lower limit, so concurrent host threads that run one kernel with
+// different shared-memory needs cannot undercut one another; the limit does not change
+// occupancy, which follows the shared memory a launch actually asks for.  The current
+// limit is read back each time (a context reset restores the 48 KB default).
+inline bool raise_smem_limit(const void* k) {
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const DeviceInfo di = device_info(dev);
+  if (di.sms == 0) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return false;
+  const int want = static_cast<int>(di.smem_optin) - static_cast<int>(fa.sharedSizeBytes);
+  if (fa.maxDynamicSharedSizeBytes >= want) return true;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, want) ==
+         cudaSuccess;
+}
+
+// Name of the kernel that the calling host thread's last successful launch through this
+// library ran (a string literal; "" before the first launch).  Read by kvc_last_kernel().
+inline const char*& last_kernel() {
+  static thread_local const char* name = "";
+  return name;
+}
+
 // Resident CTAs per SM of kernel k at this block size and dynamic shared memory (0 on
-// error); raises the kernel's dynamic shared-memory limit when needed.
+// error); raises the kernel's dynamic shared-memory limit first (raise_smem_limit).
 template <typename Kernel>
 int resident_blocks(Kernel k, int threads, size_t smem) {
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return 0;
-  }
+  if (!raise_smem_limit(reinterpret_cast<const void*>(k))) return 0;
   int blocks = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k, threads, smem) != cudaSuccess)
     return 0;

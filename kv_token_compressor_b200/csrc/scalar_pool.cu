@@ -234,7 +234,9 @@ kvc_status launch_small(const StreamProblem& p, cudaStream_t st) {
   ScalarArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
          dim3(cg, ey), 0, st>>>(args);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "scalar_small_m_kernel";
+  return KVC_OK;
 }
 
 template <typename InT, typename OutT, bool TWO_SEG>
@@ -254,7 +256,9 @@ kvc_status launch(const StreamProblem& p, cudaStream_t st) {
   if (grid > need) grid = need;
   ScalarArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
   kern<<<static_cast<unsigned>(grid), kScWarps * 32, smem, st>>>(args);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "scalar_pool_kernel";
+  return KVC_OK;
 }
 
 template <typename InT, typename OutT>

@@ -726,7 +726,11 @@ kvc_status launch_csa_small_ck(const StreamProblem& p, cudaStream_t st) {
   CsaSmallArgs args{p.C0, p.C1, p.Z0, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.out};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
          block, smem, st>>>(args, entry_list(p), cache_arg<CACHE>(p));
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = CK == 512   ? "csa_small_m_kernel/c512"
+                  : CK == 128 ? "csa_small_m_kernel/c128"
+                              : "csa_small_m_kernel";
+  return KVC_OK;
 }
 
 // The dense CSA (m = 4, overlap; plain outputs) at the channel counts of the workloads
@@ -762,7 +766,10 @@ kvc_status launch_window_rg(const StreamProblem& p, cudaStream_t st, const Devic
   WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, batch, p.n, p.c, p.ne, p.m, p.out};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
          dim3(kWinCG, kWinTY), smem, st>>>(args, entry_list(p), cache_arg<CACHE>(p));
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = RG == 1 ? "window_pool_kernel/rg1" : RG == 4 ? "window_pool_kernel/rg4"
+                                                               : "window_pool_kernel/rg16";
+  return KVC_OK;
 }
 
 // The pipelined few-window kernel (one segment, dense streams), same grid as above.
@@ -786,7 +793,10 @@ kvc_status launch_window_pipe(const StreamProblem& p, cudaStream_t st, const Dev
   WinArgs args{p.C0, p.Z0, p.C1, p.Z1, p.B0, p.B1, p.batch, p.n, p.c, p.ne, p.m, p.out};
   kern<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), static_cast<unsigned>(gz)),
          dim3(kWinCG, kWinTY), smem, st>>>(args);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = RG == 4 ? "window_pipe_kernel/rg4" : RG == 8 ? "window_pipe_kernel/rg8"
+                                                               : "window_pipe_kernel/rg16";
+  return KVC_OK;
 }
 
 // Row groups per entry: the fewest that still give every resident CTA slot a few

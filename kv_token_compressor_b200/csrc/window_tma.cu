@@ -566,7 +566,9 @@ kvc_status launch_rg(const StreamProblem& p, cudaStream_t st, const DeviceInfo& 
   a.tasks = ceil_div(p.c, SC) * p.batch * a.groups;
   const int64_t grid = a.tasks < di.sms ? a.tasks : di.sms;
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mz, mc, mb, a);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "window_tma_kernel";
+  return KVC_OK;
 }
 
 // Share of the SMs' task rounds that do work when `tasks` tasks are split into contiguous
@@ -839,7 +841,9 @@ kvc_status launch_csa_typed(const StreamProblem& p, cudaStream_t st) {
   if (resident_blocks(kern, kCsaThreads, smem) < 1) return KVC_ERR_UNSUPPORTED;
   const int64_t grid = a.tasks < di.sms ? a.tasks : di.sms;
   kern<<<static_cast<unsigned>(grid), kCsaThreads, smem, st>>>(m0, m1, m2, m3, a);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "csa_tma_kernel";
+  return KVC_OK;
 }
 
 
@@ -903,7 +907,9 @@ kvc_status launch_csa_tma(const StreamProblem& p, cudaStream_t st) {
 
 kvc_status launch_wait_selftest(int32_t* out, cudaStream_t st) {
   wtma::wait_selftest_kernel<<<1, 64, 0, st>>>(out);
-  return cudaGetLastError() == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "wait_selftest_kernel";
+  return KVC_OK;
 }
 
 unsigned int read_and_clear_window_error(bool* failed) {

@@ -66,6 +66,7 @@ SIGNATURES = {
                                                 _i64, _p]),
     "indexer_topk": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i32, _p, _p, _p]),
     "kvc_topk_max_candidates": (_i64, []),
+    "kvc_last_kernel": (ctypes.c_char_p, []),
 }
 
 _lib = None
@@ -99,6 +100,11 @@ def status_string(status: int) -> str:
 
 def num_entries(n: int, m: int) -> int:
     return int(lib().kvc_num_entries(n, m))
+
+
+def last_kernel() -> str:
+    """Name of the kernel this host thread's last successful launch ran ("" before any)."""
+    return lib().kvc_last_kernel().decode()
 
 
 def _check(status: int, where: str):

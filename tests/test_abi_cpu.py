@@ -180,6 +180,22 @@ def test_fused_hca_rejects_before_launch(L, kw, status):
     assert fused_hca(L, **kw) == status
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(m=8), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(m=2), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(overlap=0), kvc.KVC_ERR_UNSUPPORTED),
+])
+def test_fused_csa_only_the_pages_compressor(L, kw, status):
+    """The tensor-core path implements CSA with m = 4 and overlap only; other valid
+    ratios are refused before any CUDA call (fake pointers are never dereferenced)."""
+    assert fused_csa(L, **kw) == status
+
+
+@pytest.mark.parametrize("m", [64, 4, 256])
+def test_fused_hca_only_m_128(L, m):
+    assert fused_hca(L, m=m) == kvc.KVC_ERR_UNSUPPORTED
+
+
 def test_fused_empty(L):
     assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
     assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK
@@ -575,6 +591,8 @@ int main(void) {
   if (kvc_selftest_bounded_wait(NULL, NULL) != KVC_ERR_NULL) bad |= 32;
   if (kvc_status_string(KVC_ERR_TIMEOUT) == NULL) bad |= 64;
   if (kvc_topk_max_candidates() <= 0) bad |= 128;
+  /* nothing was launched: the record of the last kernel is still empty */
+  if (kvc_last_kernel() == NULL || kvc_last_kernel()[0] != '\0') bad |= 256;
   printf("%s %d\n", kvc_status_string(KVC_ERR_SHAPE), bad);
   return bad;
 }
