@@ -690,6 +690,26 @@ def _workload(name, dev):
                     config={"workload": f"CSA fused projection + pool: H [{n}, {d}] bf16, 4 W "
                                         f"[{d}, {c}] bf16, m=4 overlap, bf16 out", "n": n,
                             "d": d, "c": c, "m": 4})
+    if name == "fused_csa_cache":
+        n, d, c, r = 32768, 7168, 512, 64
+        t = synth.fused_inputs_torch("csa", 1, n, d, c, 4, seed=0, device=dev)
+        t["inv_freq"] = (10000.0 ** (-torch.arange(r // 2, device=dev, dtype=torch.float64)
+                                     * 2 / r)).float()
+        nope = torch.empty((n // 4, c - r), device=dev, dtype=torch.uint8)
+        rope = torch.empty((n // 4, r), device=dev, dtype=bf)
+
+        def launch(x, st):
+            kvc.csa_compress_fused_proj_cache(x["H"], x["W_kva"], x["W_kvb"], x["W_za"],
+                                              x["W_zb"], x["Ba"], x["Bb"], 1, n, r,
+                                              x["inv_freq"], out_nope=nope, out_rope=rope,
+                                              stream=st)
+        return dict(inputs=t, launch=launch, outputs=[nope, rope], tokens=n, entries=n // 4,
+                    bound="tensor", units=2.0 * n * d * 4 * c, flush=False,
+                    kernel="fused_pair_kernel<CSA, cache layout> (CTA pairs, M=256)",
+                    config={"workload": f"CSA fused projection + pool, cache layout: H [{n}, {d}] "
+                                        f"bf16, 4 W [{d}, {c}] bf16, m=4 overlap, E4M3 [c-{r}] "
+                                        f"+ RoPE'd bf16 [{r}]", "n": n, "d": d, "c": c, "m": 4,
+                            "r": r})
     if name == "fused_hca":
         b, n, d, c = 4, 131072, 4096, 512
         t = synth.fused_inputs_torch("hca", b, n, d, c, 128, seed=0, device=dev)
@@ -1057,7 +1077,7 @@ def main():
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused-path kernels timed after the default step")
     ap.add_argument("--workload", default="long",
-                    choices=["long", "fused_csa", "fused_hca", "hca_n65536", "csa_f32_n1024",
+                    choices=["long", "fused_csa", "fused_csa_cache", "fused_hca", "hca_n65536", "csa_f32_n1024",
                              "indexer_keys", "fused_indexer_keys", "scalar_long",
                              "decode_entries", "cache_long", "indexer_decode"],
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "

@@ -231,6 +231,25 @@ KVC_API kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, cons
                                    int64_t c, int32_t m,
                                    void* out, kvc_dtype out_dtype, kvc_stream stream);
 
+/* The fused compressors with the entries written in the cache layout (the same layout as
+ * csa_compress_cache above: [HCA] §4 (2) partial RoPE on the last r dimensions, the
+ * comparison article's BF16 RoPE part and FP8 rest) straight from the GEMM epilogue ([SC]
+ * flash-compressor section: RoPE and cache insertion are the fusions that sit next to the
+ * compressor), so neither the streams nor the plain entries reach device memory.
+ *   Arguments as csa_compress_fused_proj / hca_compress_fused_proj, with `out` and
+ *   `out_dtype` replaced by r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope,
+ *   out_rope as in csa_compress_cache (rows = batch * N_e; entry i of each sequence sits at
+ *   position pos_offset + pos_stride * i).  The same m / overlap restrictions apply. */
+KVC_API kvc_status csa_compress_fused_proj_cache(
+    const void* H, const void* W_kva, const void* W_kvb, const void* W_za, const void* W_zb,
+    const float* Ba, const float* Bb, int64_t batch, int64_t n, int64_t d, int64_t c, int32_t m,
+    int32_t overlap, int32_t r, const float* inv_freq, double pos_stride, double pos_offset,
+    float fp8_scale, void* out_nope, void* out_rope, kvc_stream stream);
+KVC_API kvc_status hca_compress_fused_proj_cache(
+    const void* H, const void* W_kv, const void* W_z, const float* B, int64_t batch, int64_t n,
+    int64_t d, int64_t c, int32_t m, int32_t r, const float* inv_freq, double pos_stride,
+    double pos_offset, float fp8_scale, void* out_nope, void* out_rope, kvc_stream stream);
+
 /* ---------------------------------------------------------------- lightning indexer
  * [CSA] §4 (Lightning Indexer) and §5: CSA attends only to the compressed entries that
  * its indexer ranks highest.  Query t's score for compressed indexer key s is

@@ -41,6 +41,7 @@
 #include "tc_ptx.cuh"
 
 #include <mutex>
+#include <type_traits>
 
 namespace kvc {
 
@@ -198,6 +199,25 @@ struct Args {
   int64_t units;        // CSA: pieces; HCA: tiles
 };
 
+// Extra kernel argument of the cache-layout instantiations (empty otherwise).
+template <bool CACHE>
+using FusedCacheArg = typename std::conditional<CACHE, CacheFmt, NoCache>::type;
+
+// Stores the result v of channel ch of entry `entry` of sequence b: as OutT into the plain
+// output, or in the cache layout (E4M3 below c - r, RoPE'd bf16 above).  Every lane of the
+// warp calls it together (the lanes hold consecutive channels; the RoPE pairs are
+// exchanged by a shuffle).
+template <bool CACHE, typename OutT>
+__device__ __forceinline__ void store_entry(const Args& a, const FusedCacheArg<CACHE>& cf, int b,
+                                            int64_t entry, int64_t ch, float v) {
+  const int64_t orow = static_cast<int64_t>(b) * a.ne + entry;
+  if constexpr (CACHE) {
+    store_cache_lane(cf, orow, ch, entry, v, true);
+  } else {
+    store_scalar<OutT>(static_cast<OutT*>(a.out) + orow * a.c + ch, v);
+  }
+}
+
 // CSA m = 4: piece p = (sequence b, channel group cg, entries [e0, e1)).  Its token rows
 // start one block before e0 (the b-rows of entry e0) unless e0 = 0.
 struct CsaPiece {
@@ -241,13 +261,14 @@ __device__ __forceinline__ HcaTile hca_tile(const Args& a, int64_t t) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <bool CSA, int BK, typename OutT>
+template <bool CSA, int BK, typename OutT, bool CACHE>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_pool_kernel(const __grid_constant__ CUtensorMap tmH,
                       const __grid_constant__ CUtensorMap tmW0,
                       const __grid_constant__ CUtensorMap tmW1,
                       const __grid_constant__ CUtensorMap tmW2,
-                      const __grid_constant__ CUtensorMap tmW3, const Args a) {
+                      const __grid_constant__ CUtensorMap tmW3, const Args a,
+                      const FusedCacheArg<CACHE> cf) {
   constexpr int NS = CSA ? 4 : 2;
   using C = Cfg<NS, BK>;
   constexpr int TN = C::TN;
@@ -410,7 +431,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;  // TMEM lane = channel within the tile
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    OutT* out = static_cast<OutT*>(a.out);
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int64_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -474,8 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   s += w;
                   acc = fmaf(w, carry_c[k], acc);
                 }
-                store_scalar<OutT>(out + (static_cast<int64_t>(pc.b) * a.ne + kb) * a.c + ch,
-                                   __fdividef(acc, s));
+                store_entry<CACHE, OutT>(a, cf, pc.b, kb, ch, __fdividef(acc, s));
               }
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
@@ -527,8 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             M = nm;
           }
-          store_scalar<OutT>(out + (static_cast<int64_t>(h.b) * a.ne + e) * a.c + ch,
-                             __fdividef(A, S));
+          store_entry<CACHE, OutT>(a, cf, h.b, e, ch, __fdividef(A, S));
         }
         tc_fence_before();
         mbar_arrive(tmem_empty);
@@ -720,13 +738,14 @@ __host__ __device__ constexpr uint32_t idesc_pair(int n) {
 
 // W maps: CSA W0 = W^{KV_a}, W1 = W^{KV_b}, W2 = W^{Z_a}, W3 = W^{Z_b} (the leader loads
 // W0/W2, the peer W1/W3); HCA W0 = W^{KV}, W1 = W^{Z} (both CTAs).
-template <bool CSA, typename OutT>
+template <bool CSA, typename OutT, bool CACHE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     fused_pair_kernel(const __grid_constant__ CUtensorMap tmH,
                       const __grid_constant__ CUtensorMap tmW0,
                       const __grid_constant__ CUtensorMap tmW1,
                       const __grid_constant__ CUtensorMap tmW2,
-                      const __grid_constant__ CUtensorMap tmW3, const Args a) {
+                      const __grid_constant__ CUtensorMap tmW3, const Args a,
+                      const FusedCacheArg<CACHE> cf) {
   using C = pair::Cfg;
   constexpr int S = C::STAGES;
   constexpr int R = pair::kGroups * pair::kSlotsPerGroup;  // exchange slots (CSA)
@@ -894,7 +913,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     const int gbar = 1 + eg;                // the group's named barrier (128 threads)
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(qw * 32) << 16);
     const uint32_t leader_tmem_empty = cluster_addr(smem_u32(tmem_empty), 0);
-    OutT* out = static_cast<OutT*>(a.out);
     uint32_t acc_phase = 0;
     uint32_t xcount = 0;  // CSA: exchange chunks of this group so far
     bool ok = true;
@@ -1002,8 +1020,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                   const float f = ex2_ftz(pl[blk] - mx);  // 0 when there are no b-rows
                   s += f;
                   acc = fmaf(pm[blk], f, acc);
-                  store_scalar<OutT>(out + (static_cast<int64_t>(pc.b) * a.ne + kb) * a.c + ch,
-                                     __fdividef(acc, s));
+                  store_entry<CACHE, OutT>(a, cf, pc.b, kb, ch, __fdividef(acc, s));
                 }
               }
             }
@@ -1076,8 +1093,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
             const float f0 = ex2_ftz(M - nm), f1 = ex2_ftz(M1 - nm);
             Ssum = fmaf(S1, f1, Ssum * f0);
             A = fmaf(A1, f1, A * f0);
-            store_scalar<OutT>(out + (static_cast<int64_t>(h.b) * a.ne + h.j * 2 + w) * a.c + ch,
-                               __fdividef(A, Ssum));
+            store_entry<CACHE, OutT>(a, cf, h.b, h.j * 2 + w, ch, __fdividef(A, Ssum));
           }
         }
         tc_fence_before();
@@ -1123,7 +1139,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool CSA, int BK, typename OutT>
+template <bool CACHE>
+FusedCacheArg<CACHE> fused_cache_arg(const FusedProblem& p) {
+  if constexpr (CACHE) {
+    return CacheFmt{static_cast<uint8_t*>(p.out_nope), static_cast<__nv_bfloat16*>(p.out_rope),
+                    p.inv_freq, p.c - p.r, p.r, p.pos_stride, p.pos_offset, p.fp8_scale};
+  } else {
+    return NoCache{};
+  }
+}
+
+template <bool CSA, int BK, typename OutT, bool CACHE>
 kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   constexpr int NS = CSA ? 4 : 2;
   using C = Cfg<NS, BK>;
@@ -1164,16 +1190,18 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
     a.units = p.batch * ((p.ne * 128 + C::TN - 1) / C::TN) * a.ncg;
   }
   grid = a.units < sms ? a.units : sms;
-  auto kern = fused_pool_kernel<CSA, BK, OutT>;
+  auto kern = fused_pool_kernel<CSA, BK, OutT, CACHE>;
   if (!raise_smem_limit(reinterpret_cast<const void*>(kern))) return KVC_ERR_CUDA;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::SMEM, st>>>(mh, mw[0], mw[1], mw[2], mw[3], a);
+  kern<<<static_cast<unsigned>(grid), kThreads, C::SMEM, st>>>(mh, mw[0], mw[1], mw[2], mw[3], a,
+                                                             fused_cache_arg<CACHE>(p));
   if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
-  last_kernel() = CSA ? "fused_pool_kernel/csa" : "fused_pool_kernel/hca";
+  last_kernel() = CSA ? (CACHE ? "fused_pool_kernel/csa/cache" : "fused_pool_kernel/csa")
+                      : (CACHE ? "fused_pool_kernel/hca/cache" : "fused_pool_kernel/hca");
   return KVC_OK;
 }
 
 // CTA-pair launch (fused_pair_kernel): clusters of two CTAs, as many as can be resident.
-template <bool CSA, typename OutT>
+template <bool CSA, typename OutT, bool CACHE>
 kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
   using C = pair::Cfg;
   int dev = 0, sms = 0;
@@ -1190,7 +1218,7 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
     if (!make_map(&mw[s], w, static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.c), C::BK, 64))
       return KVC_ERR_CUDA;
   }
-  auto kern = fused_pair_kernel<CSA, OutT>;
+  auto kern = fused_pair_kernel<CSA, OutT, CACHE>;
   if (!raise_smem_limit(reinterpret_cast<const void*>(kern))) return KVC_ERR_CUDA;
   int clusters = 0;
   {
@@ -1226,9 +1254,10 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
   }
   const int64_t ncl = a.units < clusters ? a.units : clusters;
   kern<<<static_cast<unsigned>(2 * ncl), pair::kThreads, C::SMEM, st>>>(mh, mw[0], mw[1], mw[2], mw[3],
-                                                                   a);
+                                                                   a, fused_cache_arg<CACHE>(p));
   if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
-  last_kernel() = CSA ? "fused_pair_kernel/csa" : "fused_pair_kernel/hca";
+  last_kernel() = CSA ? (CACHE ? "fused_pair_kernel/csa/cache" : "fused_pair_kernel/csa")
+                      : (CACHE ? "fused_pair_kernel/hca/cache" : "fused_pair_kernel/hca");
   return KVC_OK;
 }
 
@@ -1241,23 +1270,26 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
 constexpr int kBkCsa = 64;
 constexpr int kBkHca = 64;
 
-kvc_status launch_fused(const FusedProblem& p, cudaStream_t st) {
+template <typename OutT, bool CACHE>
+kvc_status launch_fused_typed(const FusedProblem& p, cudaStream_t st) {
   if (p.csa) {
     if (p.m != 4 || !p.overlap) return KVC_ERR_UNSUPPORTED;
-    const kvc_status r = p.out_bf16 ? fused::launch_pair<true, __nv_bfloat16>(p, st)
-                                    : fused::launch_pair<true, float>(p, st);
+    const kvc_status r = fused::launch_pair<true, OutT, CACHE>(p, st);
     if (r != KVC_ERR_UNSUPPORTED) return r;
-    return p.out_bf16 ? fused::launch_impl<true, kBkCsa, __nv_bfloat16>(p, st)
-                      : fused::launch_impl<true, kBkCsa, float>(p, st);
+    return fused::launch_impl<true, kBkCsa, OutT, CACHE>(p, st);
   }
   if (p.m != 128) return KVC_ERR_UNSUPPORTED;
   if ((p.c / fused::kCh) % 2 == 0) {  // channel groups pair up over the CTA pair
-    const kvc_status r = p.out_bf16 ? fused::launch_pair<false, __nv_bfloat16>(p, st)
-                                    : fused::launch_pair<false, float>(p, st);
+    const kvc_status r = fused::launch_pair<false, OutT, CACHE>(p, st);
     if (r != KVC_ERR_UNSUPPORTED) return r;
   }
-  return p.out_bf16 ? fused::launch_impl<false, kBkHca, __nv_bfloat16>(p, st)
-                    : fused::launch_impl<false, kBkHca, float>(p, st);
+  return fused::launch_impl<false, kBkHca, OutT, CACHE>(p, st);
+}
+
+kvc_status launch_fused(const FusedProblem& p, cudaStream_t st) {
+  if (p.cache) return launch_fused_typed<__nv_bfloat16, true>(p, st);
+  return p.out_bf16 ? launch_fused_typed<__nv_bfloat16, false>(p, st)
+                    : launch_fused_typed<float, false>(p, st);
 }
 
 kvc_status read_and_clear_device_error(cudaStream_t st) {

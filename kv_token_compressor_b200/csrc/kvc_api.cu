@@ -57,6 +57,38 @@ kvc_status check_stream_shape(int64_t batch, int64_t n, int64_t c, int32_t m, bo
   return KVC_OK;
 }
 
+// Checks and records the cache-layout arguments (after the problem's own checks).
+template <typename Problem>
+kvc_status set_cache(Problem* p, int32_t r, const float* inv_freq, double pos_stride,
+                           double pos_offset, float fp8_scale, void* out_nope, void* out_rope) {
+  if (r < 0 || r > p->c || r % 8 != 0) return KVC_ERR_SHAPE;
+  if (!(fp8_scale == fp8_scale) || !(pos_stride == pos_stride) || !(pos_offset == pos_offset))
+    return KVC_ERR_SHAPE;  // NaN arguments
+  const bool has_nope = p->c - r > 0, has_rope = r > 0;
+  if ((has_nope && !out_nope) || (has_rope && (!out_rope || !inv_freq))) return KVC_ERR_NULL;
+  if ((has_nope && !aligned(out_nope, 16)) || (has_rope && !aligned(out_rope, 16)) ||
+      (has_rope && !aligned(inv_freq, 4)))
+    return KVC_ERR_ALIGN;
+  const void* ps[3];
+  int np = 0;
+  if (has_nope) ps[np++] = out_nope;
+  if (has_rope) {
+    ps[np++] = out_rope;
+    ps[np++] = inv_freq;
+  }
+  kvc_status s = check_ptrs(ps, np);
+  if (s != KVC_OK) return s;
+  p->cache = true;
+  p->out_nope = out_nope;
+  p->out_rope = out_rope;
+  p->inv_freq = inv_freq;
+  p->r = r;
+  p->pos_stride = pos_stride;
+  p->pos_offset = pos_offset;
+  p->fp8_scale = fp8_scale;
+  return KVC_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -332,37 +364,6 @@ kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype in_dtype
   return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// Checks and records the cache-layout arguments (after the problem's own checks).
-static kvc_status set_cache(StreamProblem* p, int32_t r, const float* inv_freq, double pos_stride,
-                           double pos_offset, float fp8_scale, void* out_nope, void* out_rope) {
-  if (r < 0 || r > p->c || r % 8 != 0) return KVC_ERR_SHAPE;
-  if (!(fp8_scale == fp8_scale) || !(pos_stride == pos_stride) || !(pos_offset == pos_offset))
-    return KVC_ERR_SHAPE;  // NaN arguments
-  const bool has_nope = p->c - r > 0, has_rope = r > 0;
-  if ((has_nope && !out_nope) || (has_rope && (!out_rope || !inv_freq))) return KVC_ERR_NULL;
-  if ((has_nope && !aligned(out_nope, 16)) || (has_rope && !aligned(out_rope, 16)) ||
-      (has_rope && !aligned(inv_freq, 4)))
-    return KVC_ERR_ALIGN;
-  const void* ps[3];
-  int np = 0;
-  if (has_nope) ps[np++] = out_nope;
-  if (has_rope) {
-    ps[np++] = out_rope;
-    ps[np++] = inv_freq;
-  }
-  kvc_status s = check_ptrs(ps, np);
-  if (s != KVC_OK) return s;
-  p->cache = true;
-  p->out_nope = out_nope;
-  p->out_rope = out_rope;
-  p->inv_freq = inv_freq;
-  p->r = r;
-  p->pos_stride = pos_stride;
-  p->pos_offset = pos_offset;
-  p->fp8_scale = fp8_scale;
-  return KVC_OK;
-}
-
 kvc_status csa_compress_cache(const void* Ca, const void* Cb, const void* Za, const void* Zb,
                               kvc_dtype in_dtype, const float* Ba, const float* Bb, int64_t batch,
                               int64_t n, int64_t c, int32_t m, int32_t overlap, int32_t r,
@@ -509,12 +510,26 @@ kvc_status hca_compress_entries_cache(const void* C, const void* Z, kvc_dtype in
   return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Device-memory check of the fused calls' inputs (and of `out` when non-NULL).
+static kvc_status fused_ptrs(const void* H, const void* const* W, int nw, const float* B0,
+                             const float* B1, const void* out) {
+  const void* ps[3] = {H, B0, out};
+  kvc_status s = check_ptrs(ps, out ? 3 : 2);
+  if (s == KVC_OK) s = check_ptrs(W, nw);
+  if (s == KVC_OK && B1) s = check_device_ptr(B1);
+  return s;
+}
+
+// Common checks of the fused calls.  need_out: the plain output `out` is written (false
+// for the cache layout, whose outputs set_cache checks; the inputs' device-memory check is
+// then left to the caller, after the layout arguments have been checked).
 static kvc_status fused_common(FusedProblem* p, bool csa, int32_t overlap, const void* H,
                                const void* const* W, int nw, const float* B0, const float* B1,
                                bool need_b1, int64_t batch, int64_t n, int64_t d, int64_t c,
-                               int32_t m, void* out, kvc_dtype out_dtype, bool* empty) {
+                               int32_t m, void* out, kvc_dtype out_dtype, bool need_out,
+                               bool* empty) {
   *empty = false;
-  if (!dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  if (need_out && !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
   if (batch < 0 || n < 0 || d < 0 || c < 0 || m < 1) return KVC_ERR_SHAPE;
   int64_t t = 0;
   if (!mul_ok(batch, n, &t) || !mul_ok(t, d > c ? d : c, &t) || !mul_ok(t, 4, &t))
@@ -527,18 +542,17 @@ static kvc_status fused_common(FusedProblem* p, bool csa, int32_t overlap, const
   if (d == 0 || d % 64 != 0 || c % 128 != 0) return KVC_ERR_SHAPE;
   // the tensor-core kernels implement the pages' two compressors only
   if (csa ? (m != 4 || overlap != 1) : m != 128) return KVC_ERR_UNSUPPORTED;
-  if (!H || !out || !B0 || (need_b1 && !B1)) return KVC_ERR_NULL;
+  if (!H || (need_out && !out) || !B0 || (need_b1 && !B1)) return KVC_ERR_NULL;
   for (int i = 0; i < nw; ++i)
     if (!W[i]) return KVC_ERR_NULL;
-  if (!aligned(H, 16) || !aligned(out, 16) || !aligned(B0, 4)) return KVC_ERR_ALIGN;
+  if (!aligned(H, 16) || (need_out && !aligned(out, 16)) || !aligned(B0, 4)) return KVC_ERR_ALIGN;
   for (int i = 0; i < nw; ++i)
     if (!aligned(W[i], 16)) return KVC_ERR_ALIGN;
   if (need_b1 && !aligned(B1, 4)) return KVC_ERR_ALIGN;
-  const void* ps[3] = {H, out, B0};
-  kvc_status s = check_ptrs(ps, 3);
-  if (s == KVC_OK) s = check_ptrs(W, nw);
-  if (s == KVC_OK && need_b1) s = check_device_ptr(B1);
-  if (s != KVC_OK) return s;
+  if (need_out) {
+    const kvc_status s = fused_ptrs(H, W, nw, B0, need_b1 ? B1 : nullptr, out);
+    if (s != KVC_OK) return s;
+  }
   p->H = H;
   p->B0 = B0;
   p->B1 = need_b1 ? B1 : nullptr;
@@ -549,7 +563,7 @@ static kvc_status fused_common(FusedProblem* p, bool csa, int32_t overlap, const
   p->ne = ne;
   p->m = m;
   p->out_bf16 = out_dtype == KVC_BF16;
-  p->out = out;
+  p->out = need_out ? out : nullptr;
   return KVC_OK;
 }
 
@@ -565,12 +579,12 @@ kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, const void*
   if (overlap) {
     const void* W[4] = {W_kva, W_kvb, W_za, W_zb};
     s = fused_common(&p, true, overlap, H, W, 4, Ba, Bb, true, batch, n, d, c, m, out, out_dtype,
-                     &empty);
+                     true, &empty);
     for (int i = 0; i < 4; ++i) p.W[i] = W[i];
   } else {  // a-streams only
     const void* W[2] = {W_kva, W_za};
     s = fused_common(&p, true, overlap, H, W, 2, Ba, nullptr, false, batch, n, d, c, m, out,
-                     out_dtype, &empty);
+                     out_dtype, true, &empty);
     p.W[0] = W_kva;
     p.W[1] = nullptr;
     p.W[2] = W_za;
@@ -590,8 +604,52 @@ kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* 
   bool empty = false;
   const void* W[2] = {W_kv, W_z};
   kvc_status s = fused_common(&p, false, 0, H, W, 2, B, nullptr, false, batch, n, d, c, m, out,
-                              out_dtype, &empty);
+                              out_dtype, true, &empty);
   if (s != KVC_OK || empty) return s;
+  p.W[0] = W_kv;
+  p.W[1] = W_z;
+  p.csa = false;
+  p.overlap = false;
+  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status csa_compress_fused_proj_cache(const void* H, const void* W_kva, const void* W_kvb,
+                                         const void* W_za, const void* W_zb, const float* Ba,
+                                         const float* Bb, int64_t batch, int64_t n, int64_t d,
+                                         int64_t c, int32_t m, int32_t overlap, int32_t r,
+                                         const float* inv_freq, double pos_stride,
+                                         double pos_offset, float fp8_scale, void* out_nope,
+                                         void* out_rope, kvc_stream stream) {
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  FusedProblem p{};
+  bool empty = false;
+  const void* W[4] = {W_kva, W_kvb, W_za, W_zb};
+  kvc_status s = fused_common(&p, true, overlap, H, W, 4, Ba, Bb, true, batch, n, d, c, m,
+                              nullptr, KVC_BF16, false, &empty);
+  if (s != KVC_OK || empty) return s;
+  s = set_cache(&p, r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope);
+  if (s == KVC_OK) s = fused_ptrs(H, W, 4, Ba, Bb, nullptr);
+  if (s != KVC_OK) return s;
+  for (int i = 0; i < 4; ++i) p.W[i] = W[i];
+  p.csa = true;
+  p.overlap = true;
+  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_fused_proj_cache(const void* H, const void* W_kv, const void* W_z,
+                                         const float* B, int64_t batch, int64_t n, int64_t d,
+                                         int64_t c, int32_t m, int32_t r, const float* inv_freq,
+                                         double pos_stride, double pos_offset, float fp8_scale,
+                                         void* out_nope, void* out_rope, kvc_stream stream) {
+  FusedProblem p{};
+  bool empty = false;
+  const void* W[2] = {W_kv, W_z};
+  kvc_status s = fused_common(&p, false, 0, H, W, 2, B, nullptr, false, batch, n, d, c, m,
+                              nullptr, KVC_BF16, false, &empty);
+  if (s != KVC_OK || empty) return s;
+  s = set_cache(&p, r, inv_freq, pos_stride, pos_offset, fp8_scale, out_nope, out_rope);
+  if (s == KVC_OK) s = fused_ptrs(H, W, 2, B, nullptr, nullptr);
+  if (s != KVC_OK) return s;
   p.W[0] = W_kv;
   p.W[1] = W_z;
   p.csa = false;

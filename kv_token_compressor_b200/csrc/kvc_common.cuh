@@ -188,6 +188,44 @@ struct CacheFmt {
 };
 struct NoCache {};
 
+// Sine and cosine of the RoPE angle of pair j of entry `entry`: the angle is formed in
+// fp64 and reduced by a multiple of 2 pi in fp64, then the fp32 sine and cosine of the
+// remainder (|red| <= pi) are taken.  pos is exact for the usual integer or half-integer
+// offsets and strides; the product with inv_freq and the reduction each add at most a few
+// units of 2^-53 relative to |ang| (about 1e-10 rad at |ang| = 1e6), far below the fp32
+// rounding of the remainder (about 2e-7 rad near pi).
+__device__ __forceinline__ void rope_sincos(const CacheFmt& cf, int64_t entry, int64_t j,
+                                            float* sn, float* cs) {
+  const double pos = cf.pos_offset + cf.pos_stride * static_cast<double>(entry);
+  const double ang = pos * static_cast<double>(cf.inv_freq[j]);
+  const double turns = rint(ang * 0.15915494309189535);
+  const float red = static_cast<float>(fma(-turns, 6.283185307179586, ang));
+  sincosf(red, sn, cs);
+}
+
+// One result per lane of a full warp whose lanes hold consecutive channels (ch has the
+// lane's parity), stored in the cache layout: a channel below c - r as one E4M3 byte of
+// v * scale; a RoPE channel as bf16, rotated together with its pair partner, which is the
+// adjacent lane (exchanged by a shuffle, so every lane of the warp must make the call;
+// lanes with live == false store nothing).
+__device__ __forceinline__ void store_cache_lane(const CacheFmt& cf, int64_t orow, int64_t ch,
+                                                 int64_t entry, float v, bool live) {
+  const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
+  if (!live) return;
+  if (ch < cf.cn) {
+    cf.nope[orow * cf.cn + ch] =
+        static_cast<uint8_t>(__nv_cvt_float_to_fp8(v * cf.scale, __NV_SATFINITE, __NV_E4M3));
+  } else {
+    const int64_t off = ch - cf.cn;
+    float sn, cs;
+    rope_sincos(cf, entry, off >> 1, &sn, &cs);
+    const bool odd = (off & 1) != 0;
+    const float x = odd ? partner : v, y = odd ? v : partner;
+    const float res = odd ? fmaf(x, sn, y * cs) : fmaf(x, cs, -y * sn);
+    cf.rope[orow * cf.r + off] = __float2bfloat16_rn(res);
+  }
+}
+
 // Store the CPT results of channels [ch0, ch0 + CPT) of entry `entry` (output row orow)
 // in the cache layout.  A thread's vector lies wholly in one part (r % 8 == 0).
 template <int CPT>
@@ -211,20 +249,11 @@ __device__ __forceinline__ void store_cache(const CacheFmt& cf, int64_t orow, in
     }
   } else {
     const int64_t off = ch0 - cf.cn;  // channel offset inside the rope part (even)
-    const double pos = cf.pos_offset + cf.pos_stride * static_cast<double>(entry);
     float rot[CPT];
 #pragma unroll
     for (int p = 0; p < CPT / 2; ++p) {
-      // angle in fp64, reduced by a multiple of 2 pi in fp64, then the fp32 sine and cosine
-      // of the remainder (|red| <= pi).  pos is exact for the usual integer or half-integer
-      // offsets and strides; the product with inv_freq and the reduction each add at most a
-      // few units of 2^-53 relative to |ang| (about 1e-10 rad at |ang| = 1e6), far below
-      // the fp32 rounding of the remainder (about 2e-7 rad near pi).
-      const double ang = pos * static_cast<double>(cf.inv_freq[off / 2 + p]);
-      const double turns = rint(ang * 0.15915494309189535);
-      const float red = static_cast<float>(fma(-turns, 6.283185307179586, ang));
       float sn, cs;
-      sincosf(red, &sn, &cs);
+      rope_sincos(cf, entry, off / 2 + p, &sn, &cs);
       const float x = v[2 * p], y = v[2 * p + 1];
       rot[2 * p] = fmaf(x, cs, -y * sn);
       rot[2 * p + 1] = fmaf(x, sn, y * cs);

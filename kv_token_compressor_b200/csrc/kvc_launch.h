@@ -60,6 +60,15 @@ struct FusedProblem {
   bool overlap;  // CSA only
   bool out_bf16;
   void* out;
+  // Cache layout (the *_fused_proj_cache calls): when `cache`, the entries go to out_nope
+  // ([rows, c - r] E4M3) and out_rope ([rows, r] bf16) instead of `out`.
+  bool cache;
+  void* out_nope;
+  void* out_rope;
+  const float* inv_freq;
+  int64_t r;
+  double pos_stride, pos_offset;
+  float fp8_scale;
 };
 
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st);

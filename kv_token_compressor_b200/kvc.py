@@ -67,6 +67,11 @@ SIGNATURES = {
     "indexer_topk": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i32, _p, _p, _p]),
     "kvc_topk_max_candidates": (_i64, []),
     "kvc_last_kernel": (ctypes.c_char_p, []),
+    "csa_compress_fused_proj_cache": (ctypes.c_int, [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64,
+                                                     _i64, _i32, _i32, _i32, _p, _d, _d, _f, _p,
+                                                     _p, _p]),
+    "hca_compress_fused_proj_cache": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32,
+                                                     _i32, _p, _d, _d, _f, _p, _p, _p]),
 }
 
 _lib = None
@@ -423,6 +428,51 @@ def hca_compress_fused_proj(H, W_kv, W_z, B, batch: int, n: int, m: int = 128, o
                                        _ptr(out), _dtype_code(out_dtype), _stream(stream))
     _check(st, "hca_compress_fused_proj")
     return out
+
+
+def csa_compress_fused_proj_cache(H, W_kva, W_kvb, W_za, W_zb, Ba, Bb, batch: int, n: int, r: int,
+                                  inv_freq, pos_stride=4.0, pos_offset=1.5, fp8_scale=1.0,
+                                  m: int = 4, out_nope=None, out_rope=None, stream=None):
+    """Fused CSA (H [batch*n, d] bf16, W's [d, c] bf16) writing the cache layout: E4M3 bytes
+    [batch, N_e, c - r] and RoPE'd bf16 [batch, N_e, r]."""
+    torch = _torch()
+    d = H.shape[1]
+    c = W_kva.shape[1]
+    _need("H", H, batch * n * d, torch.bfloat16)
+    for name, w in (("W_kva", W_kva), ("W_kvb", W_kvb), ("W_za", W_za), ("W_zb", W_zb)):
+        _need(name, w, d * c, torch.bfloat16)
+    _biases(m, c, True, Ba=Ba, Bb=Bb)
+    _rope_freqs(inv_freq, r, c)
+    ne = n // m
+    nope, rope = _cache_outs(batch * ne, c, r, H, out_nope, out_rope)
+    st = lib().csa_compress_fused_proj_cache(
+        _ptr(H), _ptr(W_kva), _ptr(W_kvb), _ptr(W_za), _ptr(W_zb), _ptr(Ba), _ptr(Bb), batch, n, d,
+        c, m, 1, *_cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, nope, rope, c),
+        _stream(stream))
+    _check(st, "csa_compress_fused_proj_cache")
+    return nope.view(batch, ne, max(c - r, 0)), rope.view(batch, ne, max(min(r, c), 0))
+
+
+def hca_compress_fused_proj_cache(H, W_kv, W_z, B, batch: int, n: int, r: int, inv_freq,
+                                  pos_stride=128.0, pos_offset=63.5, fp8_scale=1.0, m: int = 128,
+                                  out_nope=None, out_rope=None, stream=None):
+    """Fused HCA writing the cache layout (default position: the segment centre)."""
+    torch = _torch()
+    d = H.shape[1]
+    c = W_kv.shape[1]
+    _need("H", H, batch * n * d, torch.bfloat16)
+    _need("W_kv", W_kv, d * c, torch.bfloat16)
+    _need("W_z", W_z, d * c, torch.bfloat16)
+    _biases(m, c, True, B=B)
+    _rope_freqs(inv_freq, r, c)
+    ne = n // m
+    nope, rope = _cache_outs(batch * ne, c, r, H, out_nope, out_rope)
+    st = lib().hca_compress_fused_proj_cache(
+        _ptr(H), _ptr(W_kv), _ptr(W_z), _ptr(B), batch, n, d, c, m,
+        *_cache_args(r, inv_freq, pos_stride, pos_offset, fp8_scale, nope, rope, c),
+        _stream(stream))
+    _check(st, "hca_compress_fused_proj_cache")
+    return nope.view(batch, ne, max(c - r, 0)), rope.view(batch, ne, max(min(r, c), 0))
 
 
 def lightning_indexer_scores(q, w, K, key_start, n_visible, max_visible: int, scores=None,

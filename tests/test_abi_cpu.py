@@ -196,6 +196,64 @@ def test_fused_hca_only_m_128(L, m):
     assert fused_hca(L, m=m) == kvc.KVC_ERR_UNSUPPORTED
 
 
+def fused_csa_cache(L, **kw):
+    a = dict(H=A, Wa=A, Wb=A, Za=A, Zb=A, Ba=A, Bb=A, batch=1, n=4096, d=7168, c=512, m=4,
+             overlap=1, r=64, inv=A, stride=4.0, offset=1.5, scale=1.0, nope=A, rope=A)
+    a.update(kw)
+    return L.csa_compress_fused_proj_cache(a["H"], a["Wa"], a["Wb"], a["Za"], a["Zb"], a["Ba"],
+                                           a["Bb"], a["batch"], a["n"], a["d"], a["c"], a["m"],
+                                           a["overlap"], a["r"], a["inv"], a["stride"],
+                                           a["offset"], a["scale"], a["nope"], a["rope"], None)
+
+
+def fused_hca_cache(L, **kw):
+    a = dict(H=A, Wk=A, Wz=A, B=A, batch=1, n=4096, d=4096, c=512, m=128, r=64, inv=A,
+             stride=128.0, offset=63.5, scale=1.0, nope=A, rope=A)
+    a.update(kw)
+    return L.hca_compress_fused_proj_cache(a["H"], a["Wk"], a["Wz"], a["B"], a["batch"], a["n"],
+                                           a["d"], a["c"], a["m"], a["r"], a["inv"], a["stride"],
+                                           a["offset"], a["scale"], a["nope"], a["rope"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(r=12), kvc.KVC_ERR_SHAPE),
+    (dict(r=520), kvc.KVC_ERR_SHAPE),
+    (dict(r=-8), kvc.KVC_ERR_SHAPE),
+    (dict(scale=float("nan")), kvc.KVC_ERR_SHAPE),
+    (dict(inv=None), kvc.KVC_ERR_NULL),
+    (dict(nope=None), kvc.KVC_ERR_NULL),
+    (dict(rope=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(inv=A + 2), kvc.KVC_ERR_ALIGN),
+    (dict(m=8), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(overlap=0), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(d=100), kvc.KVC_ERR_SHAPE),
+    (dict(H=None), kvc.KVC_ERR_NULL),
+])
+def test_fused_csa_cache_rejects_before_launch(L, kw, status):
+    assert fused_csa_cache(L, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(r=4), kvc.KVC_ERR_SHAPE),
+    (dict(rope=None), kvc.KVC_ERR_NULL),
+    (dict(nope=MIS), kvc.KVC_ERR_ALIGN),
+    (dict(m=64), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(Wz=None), kvc.KVC_ERR_NULL),
+])
+def test_fused_hca_cache_rejects_before_launch(L, kw, status):
+    assert fused_hca_cache(L, **kw) == status
+
+
+def test_fused_cache_optional_parts_and_empty(L):
+    # an empty problem touches nothing; r = 0 needs no RoPE output or frequencies, r = c
+    # no E4M3 output (checked up to the device-memory check, which fails without a GPU)
+    assert fused_csa_cache(L, n=3, H=None, nope=None, rope=None) == kvc.KVC_OK
+    assert fused_hca_cache(L, batch=0, H=None, nope=None, rope=None) == kvc.KVC_OK
+    for kw in (dict(r=0, rope=None, inv=None), dict(r=512, nope=None)):
+        assert fused_csa_cache(L, **kw) not in (kvc.KVC_ERR_NULL, kvc.KVC_ERR_SHAPE,
+                                                kvc.KVC_ERR_ALIGN)
+
+
 def test_fused_empty(L):
     assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
     assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK
