@@ -188,6 +188,8 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
 
 // ------------------------------------------------------------------ work schedules
 
+constexpr int kMaxClusters = 96;  // CSA CTA-pair schedule table (B200: 74 pairs)
+
 struct Args {
   const float* B0;  // CSA: B^a [m, c]; HCA: B [m, c]
   const float* B1;  // CSA: B^b [m, c]
@@ -195,8 +197,13 @@ struct Args {
   int64_t batch, n, c, ne;
   int ncg;          // channel groups of 128
   int nk;           // K steps of 64
-  int pieces_per_unit;  // CSA: entry ranges per (sequence, channel group)
-  int64_t units;        // CSA: pieces; HCA: tiles
+  int pieces_per_unit;  // single-CTA CSA: entry ranges per (sequence, channel group)
+  int64_t units;        // single-CTA CSA: pieces; HCA: tiles; CTA-pair CSA: busy clusters
+  // CTA-pair CSA: tiles per cluster, and where each cluster's first piece starts (flat
+  // (sequence, channel group) index and entry)
+  int64_t tile_budget;
+  int32_t start_g[kMaxClusters];
+  int32_t start_e[kMaxClusters];
 };
 
 // Extra kernel argument of the cache-layout instantiations (empty otherwise).
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmW0,
                       const __grid_constant__ CUtensorMap tmW1,
                       const __grid_constant__ CUtensorMap tmW2,
-                      const __grid_constant__ CUtensorMap tmW3, const Args a,
+                      const __grid_constant__ CUtensorMap tmW3, const __grid_constant__ Args a,
                       const FusedCacheArg<CACHE> cf) {
   constexpr int NS = CSA ? 4 : 2;
   using C = Cfg<NS, BK>;
@@ -592,13 +599,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 //
 // Epilogue.  TMEM is full during it (the MMAs of the next tile wait), so its latency is
 // what costs: 16 warps in 4 groups, group g taking tokens [64 g, 64 g + 64) of the tile
-// (4 warps = the 4 TMEM lane quarters).  CSA tiles advance by 63 blocks (252 rows), so the
-// first block of a tile repeats the last block of the one before and only serves as the
-// b-block of the next entry: no softmax state crosses tiles.  Each CSA group has its own
-// 2-slot ring; a slot holds, per channel, the partials of the 4 blocks preceding the
-// chunk's 4 entries (the first one the peer group carries from its previous chunk, or
-// loads once per tile), so the groups never wait on one another.  An HCA window is split
-// over two groups whose (max, sum, acc) states merge through shared memory.
+// (4 warps = the 4 TMEM lane quarters).  CSA tiles advance by 64 blocks (256 rows); the
+// b-partial of a tile's first entry is the last block of the tile before, which the
+// peer's group 3 hands to its group 0 through shared memory (one 1 KB slot guarded by two
+// barriers), so no block is projected twice.  Each CSA group has its own 2-slot ring; a
+// slot holds, per channel, the partials of the 4 blocks preceding the chunk's 4 entries
+// (the first one the peer group carries from its previous chunk, loads once per tile, or
+// takes from the carry), so within a tile the groups never wait on one another.  An HCA
+// window is split over two groups whose (max, sum, acc) states merge through shared
+// memory.
 // ==================================================================================
 namespace pair {
 
@@ -617,7 +626,10 @@ struct Cfg {
   static constexpr int STAGES = 4;
   // CSA exchange slots; HCA uses the same space for its half-window states
   static constexpr int XBUF = kGroups * kSlotsPerGroup * static_cast<int>(kSlotBytes);  // 32 KB
-  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE + XBUF + 512;
+  // CSA: the b-partial (L, mean) per channel carried from the last block of a tile to the
+  // first entry of the next (peer CTA, epilogue group 3 to group 0)
+  static constexpr int CARRY = 128 * 2 * 4;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE + XBUF + CARRY + 512;
   static_assert(STAGE % 1024 == 0 && A_BYTES % 1024 == 0, "1024-byte swizzle atoms");
   static_assert(SMEM <= 232448, "shared memory per CTA");
   static_assert(2 * 2 * 128 * 3 * 4 <= XBUF, "HCA half-window states fit the exchange space");
@@ -653,30 +665,68 @@ struct Unit {
   int ntiles;
 };
 
-// CSA: unit u = (sequence, channel group, entry range).  The a.units pieces are spread
-// over the G = batch x channel-group sequences as evenly as integers allow (group g owns
-// pieces [g U / G, (g + 1) U / G)), so every resident pair gets one piece of about equal
-// size.  A piece covers blocks [first_block, e1); tile t covers its blocks
-// [63 t, 63 t + 64), the last tile shortened to the remaining rows (multiple of 16).
-__device__ __forceinline__ Unit csa_unit(const Args& a, int64_t u) {
-  Unit q;
-  const int64_t G = a.batch * a.ncg, U = a.units;
-  const int64_t g = ((u + 1) * G + U - 1) / U - 1;
-  const int64_t start = g * U / G;
-  const int64_t P = (g + 1) * U / G - start, r = u - start;
-  q.b = static_cast<int>(g / a.ncg);
-  q.cg = static_cast<int>(g - static_cast<int64_t>(q.b) * a.ncg);
-  q.e0 = (r * a.ne) / P;
-  q.e1 = ((r + 1) * a.ne) / P;
-  q.first_block = q.e0 > 0 ? q.e0 - 1 : 0;
-  const int64_t nblocks = q.e1 - q.first_block;
-  q.rows = 4 * nblocks;
-  q.stride = 252;
-  q.ntiles = q.e1 > q.e0 ? (nblocks <= 64 ? 1 : 1 + static_cast<int>((nblocks - 64 + 62) / 63)) : 0;
-  q.row0 = static_cast<int64_t>(q.b) * a.n + 4 * q.first_block;
-  q.j = 0;
-  return q;
+// CSA schedule.  The entries of the G = batch x channel-group sequences, taken group by
+// group, are cut into pieces (sequence, channel group, entries [e0, e1)); every cluster
+// takes consecutive pieces worth at most `tile_budget` tiles, where a tile holds 64 blocks
+// of 4 rows (256 tokens).  A piece that starts inside its sequence (e0 > 0) starts one
+// block early, at the b-block of entry e0 (the halo), so its tiles cover blocks
+// [e0 - 1 + 64 t, e0 - 1 + 64 t + 64); within a piece the b-partial of a tile's first
+// entry is carried over from the tile before, so no block is projected twice.  A piece
+// ends at its sequence's end or when the budget runs out, on a full tile; only the last
+// tile of a sequence can be short.  The host picks the smallest budget with which the
+// clusters cover every entry (the cost of a tile hardly depends on its length: each one
+// streams all of W), so the busiest cluster has as few tiles as possible.
+struct CsaWalk {
+  int64_t g, e;  // the next piece starts at entry e of flat group g
+  int64_t left;  // tiles left in the cluster's budget
+};
+
+__host__ __device__ inline bool csa_next(int64_t G, int64_t ne, int ncg, int64_t n, CsaWalk* w,
+                                         Unit* q) {
+  if (w->left <= 0 || w->g >= G) return false;
+  const int64_t h = w->e > 0 ? 1 : 0;
+  const int64_t tiles_to_end = (ne - w->e + h + 63) / 64;
+  const bool to_end = tiles_to_end <= w->left;
+  const int64_t nt = to_end ? tiles_to_end : w->left;
+  const int64_t e1 = to_end ? ne : w->e + 64 * nt - h;
+  q->b = static_cast<int>(w->g / ncg);
+  q->cg = static_cast<int>(w->g - static_cast<int64_t>(q->b) * ncg);
+  q->e0 = w->e;
+  q->e1 = e1;
+  q->first_block = w->e - h;
+  q->rows = 4 * (e1 - q->first_block);
+  q->stride = 256;
+  q->ntiles = static_cast<int>(nt);
+  q->row0 = static_cast<int64_t>(q->b) * n + 4 * q->first_block;
+  q->j = 0;
+  w->left -= nt;
+  if (to_end) {
+    ++w->g;
+    w->e = 0;
+  } else {
+    w->e = e1;
+  }
+  return true;
 }
+
+// The units a cluster works through: CSA pieces from its schedule entry, HCA tiles
+// u = cid, cid + ncl, ...
+struct Sched {
+  int64_t u, step, units;
+  CsaWalk w;
+};
+template <bool CSA>
+__device__ __forceinline__ Sched sched_begin(const Args& a, int64_t cid, int64_t ncl) {
+  Sched s{cid, ncl, a.units, CsaWalk{0, 0, 0}};
+  if constexpr (CSA) {
+    if (cid < a.units && cid < kMaxClusters)
+      s.w = CsaWalk{a.start_g[cid], a.start_e[cid], a.tile_budget};
+  }
+  return s;
+}
+template <bool CSA>
+__device__ __forceinline__ bool sched_next(const Args& a, Sched* s, uint32_t rank, Unit* q);
+
 // HCA: unit u = (sequence, 256-token tile, channel-group pair), pair fastest; the leader
 // takes group 2p, the peer 2p + 1.  A tile holding one window is 128 tokens.
 __device__ __forceinline__ Unit hca_unit(const Args& a, int64_t u, uint32_t rank) {
@@ -696,6 +746,18 @@ __device__ __forceinline__ Unit hca_unit(const Args& a, int64_t u, uint32_t rank
   h.e0 = h.e1 = h.first_block = 0;
   return h;
 }
+template <bool CSA>
+__device__ __forceinline__ bool sched_next(const Args& a, Sched* s, uint32_t rank, Unit* q) {
+  if constexpr (CSA) {
+    return csa_next(a.batch * a.ncg, a.ne, a.ncg, a.n, &s->w, q);
+  } else {
+    if (s->u >= s->units) return false;
+    *q = hca_unit(a, s->u, rank);
+    s->u += s->step;
+    return true;
+  }
+}
+
 // Tokens of tile t (MMA N): 256, or the rest of the unit rounded up to 16.
 __device__ __forceinline__ int tile_tokens(const Unit& q, int t) {
   const int64_t left = q.rows - static_cast<int64_t>(t) * q.stride;
@@ -744,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                       const __grid_constant__ CUtensorMap tmW0,
                       const __grid_constant__ CUtensorMap tmW1,
                       const __grid_constant__ CUtensorMap tmW2,
-                      const __grid_constant__ CUtensorMap tmW3, const Args a,
+                      const __grid_constant__ CUtensorMap tmW3, const __grid_constant__ Args a,
                       const FusedCacheArg<CACHE> cf) {
   using C = pair::Cfg;
   constexpr int S = C::STAGES;
@@ -756,7 +818,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   // [R][128][8] CSA partials: the peer stages a slot here, then copies it to the same
   // place in the leader.  HCA: [2 windows][128][3] half-window states.
   float* xbuf = reinterpret_cast<float*>(smem + S * C::STAGE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE + C::XBUF);
+  float2* carry = reinterpret_cast<float2*>(smem + S * C::STAGE + C::XBUF);  // [128] (CSA)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE + C::XBUF + C::CARRY);
   uint64_t* full = bars;                   // [S] leader: both CTAs' bytes of a stage
   uint64_t* empty = bars + S;              // [S] each CTA: the leader's MMAs freed the stage
   uint64_t* tmem_full = bars + 2 * S;      // each CTA: accumulators of a tile complete
@@ -764,8 +827,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   uint64_t* final_bar = tmem_full + 2;     // each CTA: every MMA of the leader finished
   uint64_t* xfull = tmem_full + 3;         // [R] leader: a slot arrived (1 + its bytes)
   uint64_t* xempty = xfull + R;            // [R] peer: the leader has read a slot (1)
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(xempty + R);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(xempty + R + 1);
+  uint64_t* carry_full = xempty + R;       // peer (CSA): group 3 wrote the carry (1)
+  uint64_t* carry_empty = carry_full + 1;  // peer (CSA): group 0 has read it (1)
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(carry_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(carry_empty + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -786,6 +851,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       mbar_init(&xfull[r], 1);
       mbar_init(&xempty[r], 1);
     }
+    mbar_init(carry_full, 1);
+    mbar_init(carry_empty, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -813,8 +880,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       int pending_parity[S];
       for (int s = 0; s < S; ++s) pending_parity[s] = -1;
       bool ok = true;
-      for (int64_t u = cid; u < units && ok; u += ncl) {
-        const pair::Unit q = CSA ? pair::csa_unit(a, u) : pair::hca_unit(a, u, rank);
+      pair::Sched sc = pair::sched_begin<CSA>(a, cid, ncl);
+      pair::Unit q;
+      while (ok && pair::sched_next<CSA>(a, &sc, rank, &q)) {
         for (int t = 0; t < q.ntiles && ok; ++t) {
           const int nt = pair::tile_tokens(q, t);
           const int y = static_cast<int>(q.row0 + static_cast<int64_t>(t) * q.stride +
@@ -858,8 +926,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
         uint32_t phase = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
-        for (int64_t u = cid; u < units && ok; u += ncl) {
-          const pair::Unit q = CSA ? pair::csa_unit(a, u) : pair::hca_unit(a, u, 0);
+        pair::Sched sc = pair::sched_begin<CSA>(a, cid, ncl);
+        pair::Unit q;
+        while (ok && pair::sched_next<CSA>(a, &sc, 0, &q)) {
           for (int t = 0; t < q.ntiles && ok; ++t) {
             const uint32_t idesc = pair::idesc_pair(pair::tile_tokens(q, t));
             if (!pair::wait_pair(tmem_empty, acc_phase ^ 1u, abort_flag, peer_abort)) {
@@ -915,10 +984,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
     const uint32_t leader_tmem_empty = cluster_addr(smem_u32(tmem_empty), 0);
     uint32_t acc_phase = 0;
     uint32_t xcount = 0;  // CSA: exchange chunks of this group so far
+    uint32_t ccount = 0;  // CSA peer: carries this group has written (group 3) or read (group 0)
     bool ok = true;
-    for (int64_t u = cid; u < units && ok; u += ncl) {
+    pair::Sched sc = pair::sched_begin<CSA>(a, cid, ncl);
+    pair::Unit unit;
+    while (ok && pair::sched_next<CSA>(a, &sc, rank, &unit)) {
       if constexpr (CSA) {
-        const pair::Unit pc = pair::csa_unit(a, u);
+        const pair::Unit& pc = unit;
         const int64_t ch = static_cast<int64_t>(pc.cg) * kCh + row;
         const float* Bsrc = rank == 0 ? a.B0 : a.B1;  // B^a (leader) or B^b (peer)
         float b2[4];
@@ -933,10 +1005,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const int64_t kb_tile = pc.first_block + static_cast<int64_t>(t) * 63;
+          const int64_t kb_tile = pc.first_block + static_cast<int64_t>(t) * 64;
           if (rank == 1) {
             // partial of the block before the group's first chunk: block 16 eg - 1 of the
-            // tile (none for group 0: its block 0 is a repeat or the sequence's entry 0)
+            // tile; for group 0 the last block of the tile before (carried over from group
+            // 3), or none in a piece's first tile (its block 0 is the halo, which is no
+            // entry, or the sequence's entry 0, which has no b-rows)
             float pL = -INFINITY, pmean = 0.f;
             if (eg > 0 && c_lo < nch) {
               float cv[16], zv[16];
@@ -944,6 +1018,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
               tmem_ld16(lane_addr + 256 + (c_lo - 1) * 16, zv);
               tmem_wait_ld();
               pair::block_partial(zv + 12, cv + 12, b2, &pL, &pmean);
+            } else if (eg == 0 && t > 0) {
+              if (!bar_and(gbar, 128, pair::wait_pair(carry_full, ccount & 1u, abort_flag,
+                                                      peer_abort))) {
+                ok = false;
+                break;
+              }
+              const float2 cr = carry[row];
+              pL = cr.x;
+              pmean = cr.y;
+              bar_named(gbar, 128);  // every thread of the group has read the carry
+              if (elected) mbar_arrive(carry_empty);
+              ++ccount;
             }
 #pragma unroll 1
             for (int c = c_lo; c < c_hi; ++c, ++xcount) {
@@ -977,6 +1063,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
               pL = L[3];
               pmean = mean[3];
             }
+            // the last group hands the partial of the tile's last block to group 0, whose
+            // next tile starts with that block's entry
+            if (ok && eg == pair::kGroups - 1 && t + 1 < pc.ntiles) {
+              if (!bar_and(gbar, 128, pair::wait_pair(carry_empty, (ccount & 1u) ^ 1u, abort_flag,
+                                                      peer_abort))) {
+                ok = false;
+                break;
+              }
+              carry[row] = make_float2(pL, pmean);
+              bar_named(gbar, 128);  // every thread of the group has written
+              if (elected) mbar_arrive(carry_full);
+              ++ccount;
+            }
           } else {
 #pragma unroll 1
             for (int c = c_lo; c < c_hi; ++c, ++xcount) {
@@ -1002,8 +1101,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                 const int lb = 4 * c + blk;  // block within the tile
                 const int64_t kb = kb_tile + lb;
                 // entry kb: a-rows of block kb here, b-rows of block kb - 1 as (L, mean);
-                // block 0 of a later tile repeats the last block of the one before
-                if (kb >= pc.e0 && kb < pc.e1 && (t == 0 || lb > 0)) {
+                // a piece's halo block (e0 - 1) is no entry
+                if (kb >= pc.e0 && kb < pc.e1) {
                   float l[4], mx = pl[blk];
 #pragma unroll
                   for (int k = 0; k < 4; ++k) {
@@ -1038,7 +1137,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
           acc_phase ^= 1u;
         }
       } else {
-        const pair::Unit h = pair::hca_unit(a, u, rank);
+        const pair::Unit& h = unit;
         const int64_t ch = static_cast<int64_t>(h.cg) * kCh + row;
         const int wins = static_cast<int>(h.rows / 128);
         const int w = eg >> 1, half = eg & 1;  // window of the tile, rows [64 half, +64) of it
@@ -1200,6 +1299,49 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   return KVC_OK;
 }
 
+// CSA CTA-pair schedule (see csa_next): the smallest tile budget with which `clusters`
+// clusters cover every entry, and each cluster's starting point; returns the number of
+// clusters that get work.
+int64_t plan_csa(Args* a, int64_t clusters) {
+  const int64_t G = a->batch * a->ncg;
+  auto covers = [&](int64_t T) {
+    pair::CsaWalk w{0, 0, 0};
+    pair::Unit q;
+    for (int64_t k = 0; k < clusters && w.g < G; ++k) {
+      w.left = T;
+      while (pair::csa_next(G, a->ne, a->ncg, a->n, &w, &q)) {
+      }
+    }
+    return w.g >= G;
+  };
+  // every piece wastes less than one tile at its sequence's end: the budget lies between
+  // the average and the average plus the sequences per cluster, plus one
+  int64_t lo = (G * ((a->ne + 63) / 64) + clusters - 1) / clusters;
+  if (lo < 1) lo = 1;
+  int64_t hi = lo + (G + clusters - 1) / clusters + 1;
+  while (!covers(hi)) hi *= 2;
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if (covers(mid)) {
+      hi = mid;
+    } else {
+      lo = mid + 1;
+    }
+  }
+  a->tile_budget = lo;
+  pair::CsaWalk w{0, 0, 0};
+  pair::Unit q;
+  int64_t busy = 0;
+  for (; busy < clusters && w.g < G; ++busy) {
+    a->start_g[busy] = static_cast<int32_t>(w.g);
+    a->start_e[busy] = static_cast<int32_t>(w.e);
+    w.left = lo;
+    while (pair::csa_next(G, a->ne, a->ncg, a->n, &w, &q)) {
+    }
+  }
+  return busy;
+}
+
 // CTA-pair launch (fused_pair_kernel): clusters of two CTAs, as many as can be resident.
 template <bool CSA, typename OutT, bool CACHE>
 kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
@@ -1244,11 +1386,8 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
   a.nk = static_cast<int>(p.d / C::BK);
   a.pieces_per_unit = 1;
   if constexpr (CSA) {
-    const int64_t groups = p.batch * a.ncg;  // (sequence, channel group) pairs
-    int64_t U = clusters;                    // one piece per resident pair ...
-    if (U < groups) U = groups;              // ... but at least one per group
-    if (U > groups * p.ne) U = groups * p.ne;  // and at least one entry per piece
-    a.units = U;
+    if (clusters > kMaxClusters) clusters = kMaxClusters;
+    a.units = plan_csa(&a, clusters);
   } else {
     a.units = p.batch * ((p.ne + 1) / 2) * (a.ncg / 2);
   }
