@@ -296,7 +296,7 @@ def cpu_baseline_workload(name):
             f()
             return time.perf_counter() - t0
 
-    if name in ("csa_f32_n1024", "hca_n65536"):
+    if name in ("csa_f32_n1024", "hca_n65536", "hca_n65536_prepared"):
         mode, n, m, dt = (("csa", 1024, M_CSA, "f32") if name == "csa_f32_n1024"
                           else ("hca", 65536, M_HCA, "bf16"))
         d = synth.stream_inputs(mode, 1, n, C, m, dt, seed=0)
@@ -819,8 +819,8 @@ def _workload(name, dev):
                     config={"workload": f"decode step: {seqs} sequences (lengths U[8, 1024)) each "
                                         f"emitting its newest CSA entry, c={c}, m=4, bf16",
                             "sequences": seqs, "c": c, "m": m})
-    if name in ("hca_n65536", "csa_f32_n1024", "indexer_keys"):
-        if name == "hca_n65536":
+    if name in ("hca_n65536", "hca_n65536_prepared", "csa_f32_n1024", "indexer_keys"):
+        if name in ("hca_n65536", "hca_n65536_prepared"):
             mode, n, c, m, dt = "hca", 65536, 512, 128, "bf16"
         elif name == "csa_f32_n1024":
             mode, n, c, m, dt = "csa", 1024, 512, 4, "f32"
@@ -830,7 +830,14 @@ def _workload(name, dev):
         tdt = bf if dt == "bf16" else torch.float32
         out = torch.empty((1, n // m, c), device=dev, dtype=tdt)
         es = 2 if dt == "bf16" else 4
-        if mode == "hca":
+        if name == "hca_n65536_prepared":
+            # the bias is a weight: prepared once, outside the timed region
+            t["ws"] = kvc.hca_prepare_bias(t["B"], tdt)
+
+            def launch(x, st):
+                kvc.hca_compress_prepared(x["C"], x["Z"], x["ws"], m=m, out=out, stream=st)
+            nbytes = 2 * n * c * es + m * c * 4 + (n // m) * c * es
+        elif mode == "hca":
             def launch(x, st):
                 kvc.hca_compress(x["C"], x["Z"], x["B"], m=m, out=out, stream=st)
             nbytes = 2 * n * c * es + m * c * 4 + (n // m) * c * es
@@ -843,13 +850,17 @@ def _workload(name, dev):
         return dict(inputs=t, launch=launch, outputs=[out], tokens=n, entries=n // m,
                     bound="hbm", units=float(nbytes), flush=nbytes < 4 * (126 << 20),
                     kernel=("csa_tma_kernel (TMA-fed, small problems)" if name == "csa_f32_n1024"
+                            else "window_tma_kernel (prepared bias, 8 row groups)"
+                            if name == "hca_n65536_prepared"
                             else "csa_small_m_kernel" if mode == "csa" else
                             "window_tma_kernel (TMA-fed, 8 row groups)"),
                     traffic_key={"hca_n65536": "hca_compress_bf16_n65536",
                                  "csa_f32_n1024": "csa_compress_f32_n1024",
                                  "indexer_keys": "csa_compress_bf16_c128_n1048576"}.get(name),
                     config={"workload": f"{mode.upper()} streams: batch 1, n={n}, c={c}, m={m}, "
-                                        f"{dt} in/out", "n": n, "c": c, "m": m})
+                                        f"{dt} in/out"
+                                        + (", bias prepared once" if name.endswith("prepared")
+                                           else ""), "n": n, "c": c, "m": m})
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -1077,7 +1088,8 @@ def main():
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused-path kernels timed after the default step")
     ap.add_argument("--workload", default="long",
-                    choices=["long", "fused_csa", "fused_csa_cache", "fused_hca", "hca_n65536", "csa_f32_n1024",
+                    choices=["long", "fused_csa", "fused_csa_cache", "fused_hca", "hca_n65536",
+                             "hca_n65536_prepared", "csa_f32_n1024",
                              "indexer_keys", "fused_indexer_keys", "scalar_long",
                              "decode_entries", "cache_long", "indexer_decode"],
                     help="long (default): CSA + HCA over the 2^20-token streams; the others "

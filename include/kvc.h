@@ -47,6 +47,9 @@
  *     KVC_ERR_INDEX        reported by kvc_device_status(): an entry list read from device
  *                          memory named a window outside its sequence or the streams (that
  *                          entry was skipped and its output row left unwritten)
+ *     KVC_ERR_WORKSPACE    reported by kvc_device_status(): hca_compress_prepared was given
+ *                          a workspace that hca_prepare_bias did not fill for the same c, m
+ *                          and stream dtype (nothing was computed)
  *   An empty problem (batch == 0 or N_e == 0) is valid: KVC_OK, nothing is launched and
  *   no pointer is dereferenced.
  * Thread safety.  Calls may be made concurrently from several host threads.  A kernel's
@@ -79,7 +82,8 @@ typedef enum kvc_status {
   KVC_ERR_CUDA = 6,
   KVC_ERR_TIMEOUT = 7,
   KVC_ERR_POINTER = 8,
-  KVC_ERR_INDEX = 9
+  KVC_ERR_INDEX = 9,
+  KVC_ERR_WORKSPACE = 10
 } kvc_status;
 
 typedef enum kvc_dtype { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
@@ -118,6 +122,30 @@ KVC_API kvc_status csa_compress(const void* Ca, const void* Cb, const void* Za, 
 KVC_API kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
                         int64_t batch, int64_t n, int64_t c, int32_t m,
                         void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* Prepared position bias for the HCA compressor.  The bias B [m, c] is a learned weight,
+ * the same in every call, while every call of hca_compress stages it afresh in each CTA
+ * (scaled by log2 e, reordered for the consumers, per-channel maxima and spread for the
+ * softmax reference); on short sequences that staging is a sizeable part of the call.
+ * hca_prepare_bias does it once into a caller-owned device workspace, which
+ * hca_compress_prepared then copies into shared memory as it stands.  The result is bit
+ * for bit that of hca_compress with the same B.
+ *   hca_bias_workspace_bytes: the workspace size for (c, m, in_dtype) (the stream dtype the
+ *     workspace will serve); -1 for invalid arguments.
+ *   hca_prepare_bias: B [m, c] fp32 device (4-byte aligned) -> workspace (device, 256-byte
+ *     aligned, at least hca_bias_workspace_bytes); c % 8 == 0, 1 <= m <= 320.  Asynchronous
+ *     on `stream`; the workspace holds no pointer to B, which may change afterwards.
+ *   hca_compress_prepared: as hca_compress with B replaced by a workspace that
+ *     hca_prepare_bias filled for the same c, m and in_dtype (checked on the device: a
+ *     mismatch computes nothing and kvc_device_status() reports KVC_ERR_WORKSPACE).  The
+ *     workspace is only read; calls may share it. */
+KVC_API int64_t hca_bias_workspace_bytes(int64_t c, int32_t m, kvc_dtype in_dtype);
+KVC_API kvc_status hca_prepare_bias(const float* B, int64_t c, int32_t m, kvc_dtype in_dtype,
+                                    void* workspace, int64_t workspace_bytes, kvc_stream stream);
+KVC_API kvc_status hca_compress_prepared(const void* C, const void* Z, kvc_dtype in_dtype,
+                                         const void* workspace, int64_t workspace_bytes,
+                                         int64_t batch, int64_t n, int64_t c, int32_t m,
+                                         void* out, kvc_dtype out_dtype, kvc_stream stream);
 
 /* Scalar-logit CSA compressor ([CSA] §3 symbol table: one score per token and stream,
  * an m-dimensional position bias, and a scalar weight S_j on the whole vector C_j).
@@ -301,7 +329,8 @@ KVC_API const char* kvc_last_kernel(void);
 
 /* Synchronises `stream`, then reports and clears the device-side error words that kernels
  * set: KVC_ERR_CUDA if the synchronisation or a read of the words failed; else
- * KVC_ERR_TIMEOUT if a bounded wait gave up (this takes precedence); else KVC_ERR_INDEX if
+ * KVC_ERR_TIMEOUT if a bounded wait gave up (this takes precedence); else
+ * KVC_ERR_WORKSPACE if a prepared-bias workspace did not match its call; else KVC_ERR_INDEX if
  * an entry list or an indexer window named rows outside its sequence or the streams; else
  * KVC_OK.  The words belong to the current device, not to a stream or a host thread: they
  * collect what every kernel of this library set since the last call, and one call clears

@@ -1444,6 +1444,7 @@ kvc_status read_and_clear_device_error(cudaStream_t st) {
   const unsigned int wx = read_and_clear_window_error(&failed);
   if (failed) return KVC_ERR_CUDA;
   if (v || (ix & 1u) || (wx & 1u)) return KVC_ERR_TIMEOUT;
+  if (wx & 2u) return KVC_ERR_WORKSPACE;
   return (index_error || (ix & 2u)) ? KVC_ERR_INDEX : KVC_OK;
 }
 

@@ -110,6 +110,8 @@ const char* kvc_status_string(kvc_status s) {
     case KVC_ERR_TIMEOUT: return "KVC_ERR_TIMEOUT: a bounded wait in a kernel gave up";
     case KVC_ERR_POINTER: return "KVC_ERR_POINTER: not device memory of the current device";
     case KVC_ERR_INDEX: return "KVC_ERR_INDEX: a listed entry was out of range and skipped";
+    case KVC_ERR_WORKSPACE:
+      return "KVC_ERR_WORKSPACE: the prepared-bias workspace was not made for this call";
   }
   return "KVC_ERR_UNKNOWN";
 }
@@ -178,6 +180,68 @@ kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const 
   p.C0 = C;
   p.Z0 = Z;
   p.B0 = B;
+  p.batch = batch;
+  p.n = n;
+  p.c = c;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = false;
+  p.small_window_kernel = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int64_t hca_bias_workspace_bytes(int64_t c, int32_t m, kvc_dtype in_dtype) {
+  if (c < 1 || m < 1 || !dtype_ok(in_dtype)) return -1;
+  int64_t t = 0;
+  if (!mul_ok(c, m + 1, &t) || !mul_ok(t, 8, &t)) return -1;
+  return kvc::prep_layout(c, m, in_dtype == KVC_BF16).bytes;
+}
+
+kvc_status hca_prepare_bias(const float* B, int64_t c, int32_t m, kvc_dtype in_dtype,
+                            void* workspace, int64_t workspace_bytes, kvc_stream stream) {
+  if (!dtype_ok(in_dtype)) return KVC_ERR_DTYPE;
+  if (c < 1 || m < 1 || c % 8 != 0) return KVC_ERR_SHAPE;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  const int64_t need = hca_bias_workspace_bytes(c, m, in_dtype);
+  if (need < 0 || workspace_bytes < need) return KVC_ERR_SHAPE;
+  if (!B || !workspace) return KVC_ERR_NULL;
+  if (!aligned(B, 4) || !aligned(workspace, 256)) return KVC_ERR_ALIGN;
+  const void* ps[2] = {B, workspace};
+  const kvc_status s = check_ptrs(ps, 2);
+  if (s != KVC_OK) return s;
+  return kvc::launch_prepare_bias(B, c, m, in_dtype == KVC_BF16, workspace,
+                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_prepared(const void* C, const void* Z, kvc_dtype in_dtype,
+                                 const void* workspace, int64_t workspace_bytes, int64_t batch,
+                                 int64_t n, int64_t c, int32_t m, void* out, kvc_dtype out_dtype,
+                                 kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  const int64_t need = hca_bias_workspace_bytes(c, m, in_dtype);
+  if (need < 0 || workspace_bytes < need) return KVC_ERR_SHAPE;
+  if (!C || !Z || !workspace || !out) return KVC_ERR_NULL;
+  if (!aligned(C, 16) || !aligned(Z, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+    return KVC_ERR_ALIGN;
+  {
+    const void* ps[4] = {C, Z, workspace, out};
+    s = check_ptrs(ps, 4);
+    if (s != KVC_OK) return s;
+  }
+  const kvc::PrepLayout l = kvc::prep_layout(c, m, in_dtype == KVC_BF16);
+  StreamProblem p{};
+  p.C0 = C;
+  p.Z0 = Z;
+  p.B0 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) + l.raw_off);
+  p.prep_ws = workspace;
   p.batch = batch;
   p.n = n;
   p.c = c;

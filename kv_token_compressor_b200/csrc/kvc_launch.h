@@ -41,7 +41,41 @@ struct StreamProblem {
   int64_t r;
   double pos_stride, pos_offset;
   float fp8_scale;
+  // Prepared bias (hca_compress_prepared): the workspace of hca_prepare_bias; B0 then points
+  // at its raw copy of the bias.
+  const void* prep_ws;
 };
+
+// Workspace of hca_prepare_bias, in this order: a 256-byte header, the raw bias [m, c] fp32
+// (for the kernels that read plain rows), and for every channel slab of the TMA-fed window
+// kernel (128 channels for bf16 streams, 64 for fp32) the block that kernel copies into its
+// shared memory as it stands: the m rows scaled by log2 e in its consumers' float4 order
+// (channels past c hold 0), the per-position maximum over the rows, and 4 floats whose
+// first is 1 when every channel's spread max - min is within the fast-bound limit, else 0.
+struct PrepHeader {
+  uint32_t magic, version;
+  int32_t m, in_bf16;
+  int64_t c, slabs, slab_floats;  // slab block: (m + 1) * SC + 4 floats
+  int64_t raw_off, prep_off;      // byte offsets from the workspace start
+};
+constexpr uint32_t kPrepMagic = 0x5052564Bu;
+constexpr int64_t kPrepHeaderBytes = 256;
+struct PrepLayout {
+  int64_t sc, slabs, slab_floats, raw_off, prep_off, bytes;
+};
+inline PrepLayout prep_layout(int64_t c, int m, bool in_bf16) {
+  PrepLayout l;
+  l.sc = in_bf16 ? 128 : 64;
+  l.slabs = (c + l.sc - 1) / l.sc;
+  l.slab_floats = (static_cast<int64_t>(m) + 1) * l.sc + 4;
+  l.raw_off = kPrepHeaderBytes;
+  l.prep_off = l.raw_off + ((static_cast<int64_t>(m) * c * 4 + 255) / 256) * 256;
+  l.bytes = l.prep_off + l.slabs * l.slab_floats * 4;
+  return l;
+}
+// Fills a workspace (hca_prepare_bias); the caller has checked sizes and pointers.
+kvc_status launch_prepare_bias(const float* B, int64_t c, int m, bool in_bf16, void* ws,
+                               cudaStream_t st);
 
 kvc_status launch_stream_pool(const StreamProblem& p, cudaStream_t st);
 // Scalar-logit form: Z0 / Z1 point at [batch, n] logits, B0 / B1 at [m] biases.

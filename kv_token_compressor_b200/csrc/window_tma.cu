@@ -42,6 +42,7 @@
 namespace kvc {
 
 // Bit 0: a bounded wait of the TMA-fed window kernel gave up (outputs undefined).
+// Bit 1: a prepared-bias workspace did not belong to the call (nothing was computed).
 __device__ unsigned int g_window_error = 0;
 
 namespace wtma {
@@ -67,13 +68,22 @@ struct Args {
   int m;
   int64_t groups;  // entry groups per sequence
   int64_t tasks;   // slabs * batch * groups
-  int bias_tma;    // the bias rows arrive through mapB (else plain loads)
+  int bias_mode;   // how a slab's bias rows arrive: kBiasLoads, kBiasMap or kBiasPrepared
+  // kBiasPrepared: the workspace of hca_prepare_bias (its header, and the slabs' rows ready
+  // for shared memory, prep_stride floats apart)
+  const PrepHeader* hdr;
+  const float* prep;
+  int64_t prep_stride;
 };
 
 template <typename InT>
 constexpr int slab() {
   return kCG * VecInfo<InT>::kChannels;
 }
+
+constexpr int kBiasLoads = 0;     // plain loads (bias not 16-byte aligned, or too many rows)
+constexpr int kBiasMap = 1;       // one 2-D tensor copy of the slab's rows, then scaled here
+constexpr int kBiasPrepared = 2;  // one bulk copy of the rows hca_prepare_bias made ready
 
 // Dynamic shared memory: stages, bias rows, per-channel bias maxima, spread partials,
 // row-group partials (RG > 1), barriers (stage full / empty, bias full / free) and the
@@ -115,6 +125,17 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// One contiguous global -> shared copy of `bytes` (16-byte aligned addresses, a multiple of
+// 16 bytes), counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -184,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
   uint32_t* kmax = reinterpret_cast<uint32_t*>(red);  // [SC] bias maxima as order keys
   uint32_t* kmin = kmax + SC;                          // [SC] minima
-  if (tid < SC) {
+  if (tid < SC && a.bias_mode != kBiasPrepared) {  // (prepared: copies land on these words)
     kmax[tid] = 0u;
     kmin[tid] = 0xFFFFFFFFu;
   }
@@ -196,10 +217,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bias_full, 1);
     mbar_init(bias_free, kConsumers / 32);
     *abort_flag = 0;
+    if (a.bias_mode == kBiasPrepared) {
+      // the workspace must have been prepared for this bias shape and stream type
+      const PrepHeader h = *a.hdr;
+      if (h.magic != kPrepMagic || h.m != a.m || h.c != a.c ||
+          h.in_bf16 != (sizeof(InT) == 2 ? 1 : 0) || h.slab_floats != a.prep_stride) {
+        *abort_flag = 1;
+        atomicOr(&g_window_error, 2u);
+      }
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncthreads();
+  if (a.bias_mode == kBiasPrepared && *abort_flag) return;  // nothing issued yet
 
   const int64_t lo = static_cast<int64_t>(blockIdx.x) * a.tasks / gridDim.x;
   const int64_t hi = static_cast<int64_t>(blockIdx.x + 1) * a.tasks / gridDim.x;
@@ -216,11 +247,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       Task k(a.batch, a.groups, lo);
       for (int64_t t = lo; t < hi && ok; ++t, k.next()) {
-        if (a.bias_tma && k.x != px) {
+        if (a.bias_mode != kBiasLoads && k.x != px) {
           // the slab's bias rows, once the consumers are done with the previous slab's
           if (nbias > 0 && !wait(bias_free, (nbias - 1) & 1u, abort_flag)) break;
-          mbar_arrive_expect_tx(bias_full, static_cast<uint32_t>(a.m) * SC * 4);
-          tma_load_2d(smem_u32(sb), &mapB, bias_full, static_cast<int>(k.x * SC), 0);
+          if (a.bias_mode == kBiasMap) {
+            mbar_arrive_expect_tx(bias_full, static_cast<uint32_t>(a.m) * SC * 4);
+            tma_load_2d(smem_u32(sb), &mapB, bias_full, static_cast<int>(k.x * SC), 0);
+          } else {  // rows, maxima and spread flag, ready as they are
+            const uint32_t bytes = static_cast<uint32_t>(a.prep_stride) * 4;
+            mbar_arrive_expect_tx(bias_full, bytes);
+            bulk_load(smem_u32(sb), a.prep + k.x * a.prep_stride, bytes, bias_full);
+          }
           ++nbias;
           px = k.x;
         }
@@ -267,7 +304,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int64_t t = lo; t < hi; ++t, k.next()) {
     if (k.x != cur_x) {  // the same in every consumer thread
       bool narrow = true;
-      if (a.bias_tma) {
+      if (a.bias_mode == kBiasPrepared) {
+        if (cur_x >= 0) {  // this warp is done with the old slab's bias
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bias_free);
+        }
+        if (!dead && !wait(bias_full, nb & 1u, abort_flag)) dead = true;
+        ++nb;
+        narrow = red[0] != 0.f;  // the slab's spread flag follows its maxima
+      } else if (a.bias_mode == kBiasMap) {
         if (cur_x >= 0) {  // this warp is done with the old slab's bias
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
@@ -558,16 +604,26 @@ kvc_status launch_rg(const StreamProblem& p, cudaStream_t st, const DeviceInfo& 
       !make_stream_map(&mc, p.C0, bf, p.batch, p.n, p.ne, p.c, p.m, SC, UR, E))
     return KVC_ERR_UNSUPPORTED;
   CUtensorMap mb;
-  const bool bias_tma = p.m <= 256 && make_bias_map(&mb, p.B0, p.c, p.m, SC);
+  const bool prepared = p.prep_ws != nullptr;
+  const bool bias_tma = !prepared && p.m <= 256 && make_bias_map(&mb, p.B0, p.c, p.m, SC);
   if (!bias_tma) mb = mz;  // unused
   auto kern = window_tma_kernel<InT, OutT, RG>;
   if (resident_blocks(kern, kThreads, smem) < 1) return KVC_ERR_UNSUPPORTED;
-  Args a{p.B0, p.out, p.batch, p.ne, p.c, p.m, ceil_div(p.ne, E), 0, bias_tma ? 1 : 0};
+  Args a{p.B0, p.out, p.batch, p.ne, p.c, p.m, ceil_div(p.ne, E), 0,
+         prepared ? kBiasPrepared : bias_tma ? kBiasMap : kBiasLoads, nullptr, nullptr, 0};
+  if (prepared) {
+    const PrepLayout l = prep_layout(p.c, p.m, bf);
+    static_assert(SC == 128 || SC == 64, "prepared slab widths");
+    if (l.sc != SC) return KVC_ERR_UNSUPPORTED;
+    a.hdr = static_cast<const PrepHeader*>(p.prep_ws);
+    a.prep = reinterpret_cast<const float*>(static_cast<const uint8_t*>(p.prep_ws) + l.prep_off);
+    a.prep_stride = l.slab_floats;
+  }
   a.tasks = ceil_div(p.c, SC) * p.batch * a.groups;
   const int64_t grid = a.tasks < di.sms ? a.tasks : di.sms;
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(mz, mc, mb, a);
   if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
-  last_kernel() = "window_tma_kernel";
+  last_kernel() = prepared ? "window_tma_kernel/prepared" : "window_tma_kernel";
   return KVC_OK;
 }
 
@@ -876,7 +932,73 @@ __global__ void __launch_bounds__(64, 1) wait_selftest_kernel(int32_t* out) {
   }
 }
 
+// hca_prepare_bias: block x writes the block of channel slab x (the rows scaled by log2 e
+// at their positions in the consumers' order, with 0 past c; the per-position maxima; the
+// spread flag) and slab x's columns of the raw copy; block 0 writes the header.  The values
+// are the ones the kernel above would stage itself (the same fp32 products), so a prepared
+// call gives bit for bit the result of an unprepared one.
+template <int SC, int CPT>
+__global__ void __launch_bounds__(256) prepare_bias_kernel(const float* __restrict__ B, int64_t c,
+                                                           int m, int in_bf16, uint8_t* ws,
+                                                           PrepLayout l) {
+  const int64_t x = blockIdx.x;
+  float* raw = reinterpret_cast<float*>(ws + l.raw_off);
+  float* blk = reinterpret_cast<float*>(ws + l.prep_off) + x * l.slab_floats;
+  float* bmx = blk + static_cast<int64_t>(m) * SC;
+  bool narrow = true;
+  for (int p = threadIdx.x; p < SC; p += blockDim.x) {
+    const int64_t ch = x * SC + p;
+    const int pos = slab_bias_pos<CPT, kCG>(p);
+    float mx = -INFINITY, mn = INFINITY;
+    for (int k = 0; k < m; ++k) {
+      float v = 0.f;
+      if (ch < c) {
+        v = B[static_cast<int64_t>(k) * c + ch];
+        raw[static_cast<int64_t>(k) * c + ch] = v;
+      }
+      const float sv = v * kLog2e;
+      blk[k * SC + pos] = sv;
+      mx = fmaxf(mx, sv);
+      mn = fminf(mn, sv);
+    }
+    bmx[pos] = mx;
+    narrow = narrow && (mx - mn <= kMaxBiasSpread);  // false for infinite or NaN spreads
+  }
+  narrow = __syncthreads_and(narrow) != 0;
+  if (threadIdx.x < 4) bmx[SC + threadIdx.x] = (threadIdx.x == 0 && narrow) ? 1.f : 0.f;
+  if (x == 0 && threadIdx.x == 0) {
+    PrepHeader h;
+    h.magic = kPrepMagic;
+    h.version = 1;
+    h.m = m;
+    h.in_bf16 = in_bf16;
+    h.c = c;
+    h.slabs = l.slabs;
+    h.slab_floats = l.slab_floats;
+    h.raw_off = l.raw_off;
+    h.prep_off = l.prep_off;
+    *reinterpret_cast<PrepHeader*>(ws) = h;
+  }
+}
+
 }  // namespace wtma
+
+kvc_status launch_prepare_bias(const float* B, int64_t c, int m, bool in_bf16, void* ws,
+                               cudaStream_t st) {
+  const PrepLayout l = prep_layout(c, m, in_bf16);
+  static_assert(wtma::slab<__nv_bfloat16>() == 128 && wtma::slab<float>() == 64,
+                "prep_layout's slab widths are the window kernel's");
+  if (in_bf16) {
+    wtma::prepare_bias_kernel<128, 8><<<static_cast<unsigned>(l.slabs), 256, 0, st>>>(
+        B, c, m, 1, static_cast<uint8_t*>(ws), l);
+  } else {
+    wtma::prepare_bias_kernel<64, 4><<<static_cast<unsigned>(l.slabs), 256, 0, st>>>(
+        B, c, m, 0, static_cast<uint8_t*>(ws), l);
+  }
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = "prepare_bias_kernel";
+  return KVC_OK;
+}
 
 kvc_status launch_window_tma(const StreamProblem& p, cudaStream_t st) {
   if (p.two_segments || p.listed || p.cache || p.m < wtma::kMinRows || p.ne <= 0 ||

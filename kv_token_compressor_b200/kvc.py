@@ -25,6 +25,7 @@ KVC_ERR_CUDA = 6
 KVC_ERR_TIMEOUT = 7
 KVC_ERR_POINTER = 8
 KVC_ERR_INDEX = 9
+KVC_ERR_WORKSPACE = 10
 # kvc_dtype
 KVC_F32 = 0
 KVC_BF16 = 1
@@ -67,6 +68,10 @@ SIGNATURES = {
     "indexer_topk": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i32, _p, _p, _p]),
     "kvc_topk_max_candidates": (_i64, []),
     "kvc_last_kernel": (ctypes.c_char_p, []),
+    "hca_bias_workspace_bytes": (_i64, [_i64, _i32, ctypes.c_int]),
+    "hca_prepare_bias": (ctypes.c_int, [_p, _i64, _i32, ctypes.c_int, _p, _i64, _p]),
+    "hca_compress_prepared": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i64, _i32,
+                                             _p, ctypes.c_int, _p]),
     "csa_compress_fused_proj_cache": (ctypes.c_int, [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64,
                                                      _i64, _i32, _i32, _i32, _p, _d, _d, _f, _p,
                                                      _p, _p]),
@@ -218,6 +223,39 @@ def hca_compress(C, Z, B, m: int = 128, out=None, out_dtype=None, stream=None):
     st = lib().hca_compress(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
                             _ptr(out), _dtype_code(out_dtype), _stream(stream))
     _check(st, "hca_compress")
+    return out
+
+
+def hca_bias_workspace_bytes(c: int, m: int, in_dtype) -> int:
+    """Bytes of the prepared-bias workspace for c channels, window m, streams of in_dtype."""
+    return int(lib().hca_bias_workspace_bytes(c, m, _dtype_code(in_dtype)))
+
+
+def hca_prepare_bias(B, in_dtype, workspace=None, stream=None):
+    """Prepare the HCA bias B [m, c] (fp32, device) for hca_compress_prepared with streams of
+    in_dtype; returns the workspace (a uint8 device tensor)."""
+    torch = _torch()
+    m, c = B.shape
+    _need("B", B, m * c, torch.float32)
+    nbytes = hca_bias_workspace_bytes(c, m, in_dtype)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 0), dtype=torch.uint8, device=B.device)
+    st = lib().hca_prepare_bias(_ptr(B), c, m, _dtype_code(in_dtype), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hca_prepare_bias")
+    return workspace
+
+
+def hca_compress_prepared(C, Z, workspace, m: int = 128, out=None, out_dtype=None, stream=None):
+    """hca_compress with the bias taken from a workspace of hca_prepare_bias."""
+    batch, n, c = C.shape
+    _streams(C, (("Z", Z),), (), True)
+    out_dtype = C.dtype if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, C)
+    st = lib().hca_compress_prepared(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), batch, n, c, m,
+                                     _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "hca_compress_prepared")
     return out
 
 

@@ -254,6 +254,67 @@ def test_fused_cache_optional_parts_and_empty(L):
                                                 kvc.KVC_ERR_ALIGN)
 
 
+def test_prepared_bias_workspace_size(L):
+    # header, raw bias, and per slab (m + 1) * SC + 4 floats (SC = 128 bf16, 64 fp32)
+    raw = -(-128 * 512 * 4 // 256) * 256
+    assert L.hca_bias_workspace_bytes(512, 128, kvc.KVC_BF16) == 256 + raw + 4 * (129 * 128 + 4) * 4
+    assert L.hca_bias_workspace_bytes(512, 128, kvc.KVC_F32) == 256 + raw + 8 * (129 * 64 + 4) * 4
+    assert L.hca_bias_workspace_bytes(8, 1, kvc.KVC_BF16) == 256 + 256 + (2 * 128 + 4) * 4
+    for bad in ((0, 128, kvc.KVC_BF16), (512, 0, kvc.KVC_BF16), (512, 128, 7)):
+        assert L.hca_bias_workspace_bytes(*bad) == -1
+
+
+def prep(L, **kw):
+    need = L.hca_bias_workspace_bytes(512, 128, kvc.KVC_BF16)
+    a = dict(B=A, c=512, m=128, dt=kvc.KVC_BF16, ws=A, nbytes=need)
+    a.update(kw)
+    return L.hca_prepare_bias(a["B"], a["c"], a["m"], a["dt"], a["ws"], a["nbytes"], None)
+
+
+def hca_prep(L, **kw):
+    need = L.hca_bias_workspace_bytes(512, 128, kvc.KVC_BF16)
+    a = dict(C=A, Z=A, dt=kvc.KVC_BF16, ws=A, nbytes=need, batch=1, n=65536, c=512, m=128, out=A,
+             out_dt=kvc.KVC_BF16)
+    a.update(kw)
+    return L.hca_compress_prepared(a["C"], a["Z"], a["dt"], a["ws"], a["nbytes"], a["batch"],
+                                   a["n"], a["c"], a["m"], a["out"], a["out_dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dt=9), kvc.KVC_ERR_DTYPE),
+    (dict(c=12), kvc.KVC_ERR_SHAPE),
+    (dict(c=0), kvc.KVC_ERR_SHAPE),
+    (dict(m=0), kvc.KVC_ERR_SHAPE),
+    (dict(m=321), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(nbytes=1000), kvc.KVC_ERR_SHAPE),
+    (dict(B=None), kvc.KVC_ERR_NULL),
+    (dict(ws=None), kvc.KVC_ERR_NULL),
+    (dict(ws=A + 16), kvc.KVC_ERR_ALIGN),
+    (dict(B=A + 2), kvc.KVC_ERR_ALIGN),
+])
+def test_prepare_bias_rejects_before_launch(L, kw, status):
+    assert prep(L, **kw) == status
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(out_dt=4), kvc.KVC_ERR_DTYPE),
+    (dict(n=-1), kvc.KVC_ERR_SHAPE),
+    (dict(c=100), kvc.KVC_ERR_SHAPE),
+    (dict(nbytes=4096), kvc.KVC_ERR_SHAPE),
+    (dict(m=400), kvc.KVC_ERR_UNSUPPORTED),
+    (dict(ws=None), kvc.KVC_ERR_NULL),
+    (dict(Z=None), kvc.KVC_ERR_NULL),
+    (dict(ws=A + 64), kvc.KVC_ERR_ALIGN),
+    (dict(out=MIS), kvc.KVC_ERR_ALIGN),
+])
+def test_hca_prepared_rejects_before_launch(L, kw, status):
+    assert hca_prep(L, **kw) == status
+
+
+def test_hca_prepared_empty(L):
+    assert hca_prep(L, n=127, C=None, Z=None, ws=None, out=None) == kvc.KVC_OK
+
+
 def test_fused_empty(L):
     assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
     assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK
