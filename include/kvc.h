@@ -47,6 +47,7 @@
  *     KVC_ERR_INDEX        reported by kvc_device_status(): an entry list read from device
  *                          memory named a window outside its sequence or the streams (that
  *                          entry was skipped and its output row left unwritten)
+ *     KVC_ERR_TOO_LARGE    hca_compress_noalloc: the bias needs more than its fixed scratch
  *     KVC_ERR_WORKSPACE    reported by kvc_device_status(): hca_compress_prepared was given
  *                          a workspace that hca_prepare_bias did not fill for the same c, m
  *                          and stream dtype (nothing was computed)
@@ -83,7 +84,8 @@ typedef enum kvc_status {
   KVC_ERR_TIMEOUT = 7,
   KVC_ERR_POINTER = 8,
   KVC_ERR_INDEX = 9,
-  KVC_ERR_WORKSPACE = 10
+  KVC_ERR_WORKSPACE = 10,
+  KVC_ERR_TOO_LARGE = 11
 } kvc_status;
 
 typedef enum kvc_dtype { KVC_F32 = 0, KVC_BF16 = 1 } kvc_dtype;
@@ -146,6 +148,32 @@ KVC_API kvc_status hca_compress_prepared(const void* C, const void* Z, kvc_dtype
                                          const void* workspace, int64_t workspace_bytes,
                                          int64_t batch, int64_t n, int64_t c, int32_t m,
                                          void* out, kvc_dtype out_dtype, kvc_stream stream);
+
+/* hca_compress without any memory of the caller's beyond inputs and outputs, and without
+ * allocating any (no cudaMalloc, cudaFree or allocating library call).  This entry point
+ * has no counterpart in the pages: it serves callers that cannot allocate device memory
+ * while they run, e.g. a serving loop whose device memory is all handed out at start-up
+ * (a later cudaMalloc can fail, and can synchronise the device), or a host program with no
+ * allocator of its own to provide the workspace of hca_prepare_bias.
+ *   Arguments and result as hca_compress.  Each call prepares the bias (as hca_prepare_bias
+ *   does) into a fixed scratch array inside the library, then runs hca_compress_prepared on
+ *   it; the result is bit for bit hca_compress's.
+ *   Scratch: one 1 MiB array in device memory per device that loads the library, held until
+ *   the process exits.  A call whose workspace (hca_bias_workspace_bytes(c, m, in_dtype))
+ *   exceeds 1 MiB returns KVC_ERR_TOO_LARGE before any launch: about 8 m c bytes, e.g. c up
+ *   to 1008 at m = 128.
+ *   Set-up: the first call on a device that launches work looks up the array's device
+ *   address (cudaGetSymbolAddress, which may load the library's device code) and keeps it
+ *   for later calls on that device; make that first call before any stream capture, and
+ *   call it no more on a device after cudaDeviceReset there.
+ *   Every call shares the scratch and leaves its contents behind; each call rewrites all it
+ *   reads before reading it, so nothing needs clearing.  Calls whose work may overlap on
+ *   the GPU (other streams, other host threads) race on the scratch: issue them in order on
+ *   one stream, or synchronise between them. */
+KVC_API kvc_status hca_compress_noalloc(const void* C, const void* Z, kvc_dtype in_dtype,
+                                        const float* B, int64_t batch, int64_t n, int64_t c,
+                                        int32_t m, void* out, kvc_dtype out_dtype,
+                                        kvc_stream stream);
 
 /* Scalar-logit CSA compressor ([CSA] §3 symbol table: one score per token and stream,
  * an m-dimensional position bias, and a scalar weight S_j on the whole vector C_j).

@@ -2,6 +2,8 @@
 // Every check here runs before anything is enqueued; see include/kvc.h for the contract.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "../../include/kvc.h"
 #include "kvc_host.h"
 #include "kvc_launch.h"
@@ -91,6 +93,38 @@ kvc_status set_cache(Problem* p, int32_t r, const float* inv_freq, double pos_st
 
 }  // namespace
 
+// Scratch of hca_compress_noalloc: the prepared-bias workspace lives here instead of in
+// memory the caller allocates.  One array per device that loads the library, held until
+// the process exits; every call on a device shares it.
+constexpr int64_t kNoAllocScratchBytes = int64_t(1) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device.  In host code the array's
+// name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per device (with that device current), and kept.
+kvc_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVC_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return KVC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return KVC_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return KVC_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int64_t kvc_num_entries(int64_t n, int32_t m) {
@@ -112,6 +146,9 @@ const char* kvc_status_string(kvc_status s) {
     case KVC_ERR_INDEX: return "KVC_ERR_INDEX: a listed entry was out of range and skipped";
     case KVC_ERR_WORKSPACE:
       return "KVC_ERR_WORKSPACE: the prepared-bias workspace was not made for this call";
+    case KVC_ERR_TOO_LARGE:
+      return "KVC_ERR_TOO_LARGE: the bias needs more than the 1 MiB fixed scratch of "
+             "hca_compress_noalloc";
   }
   return "KVC_ERR_UNKNOWN";
 }
@@ -253,6 +290,53 @@ kvc_status hca_compress_prepared(const void* C, const void* Z, kvc_dtype in_dtyp
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
   return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_noalloc(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
+                                int64_t batch, int64_t n, int64_t c, int32_t m, void* out,
+                                kvc_dtype out_dtype, kvc_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(out_dtype)) return KVC_ERR_DTYPE;
+  bool empty = false;
+  int64_t ne = 0;
+  kvc_status s = check_stream_shape(batch, n, c, m, &empty, &ne);
+  if (s != KVC_OK || empty) return s;
+  if (m > kMaxWindowRows) return KVC_ERR_UNSUPPORTED;
+  const int64_t need = hca_bias_workspace_bytes(c, m, in_dtype);
+  if (need < 0) return KVC_ERR_SHAPE;
+  if (need > kNoAllocScratchBytes) return KVC_ERR_TOO_LARGE;
+  if (!C || !Z || !B || !out) return KVC_ERR_NULL;
+  if (!aligned(C, 16) || !aligned(Z, 16) || !aligned(out, 16) || !aligned(B, 4))
+    return KVC_ERR_ALIGN;
+  {
+    const void* ps[4] = {C, Z, B, out};
+    s = check_ptrs(ps, 4);
+    if (s != KVC_OK) return s;
+  }
+  void* ws = nullptr;
+  s = noalloc_scratch(&ws);
+  if (s != KVC_OK) return s;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // every byte the compressor reads from the scratch is rewritten here first: nothing in
+  // it needs to start at zero, and the previous call's contents are never read
+  s = kvc::launch_prepare_bias(B, c, m, in_dtype == KVC_BF16, ws, st);
+  if (s != KVC_OK) return s;
+  const kvc::PrepLayout l = kvc::prep_layout(c, m, in_dtype == KVC_BF16);
+  StreamProblem p{};
+  p.C0 = C;
+  p.Z0 = Z;
+  p.B0 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(ws) + l.raw_off);
+  p.prep_ws = ws;
+  p.batch = batch;
+  p.n = n;
+  p.c = c;
+  p.ne = ne;
+  p.m = m;
+  p.two_segments = false;
+  p.small_window_kernel = false;
+  p.in_bf16 = in_dtype == KVC_BF16;
+  p.out_bf16 = out_dtype == KVC_BF16;
+  p.out = out;
+  return kvc::launch_stream_pool(p, st);
 }
 
 kvc_status csa_compress_scalar_logits(const void* Ca, const void* Cb, const void* za,

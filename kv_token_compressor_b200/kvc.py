@@ -26,6 +26,7 @@ KVC_ERR_TIMEOUT = 7
 KVC_ERR_POINTER = 8
 KVC_ERR_INDEX = 9
 KVC_ERR_WORKSPACE = 10
+KVC_ERR_TOO_LARGE = 11
 # kvc_dtype
 KVC_F32 = 0
 KVC_BF16 = 1
@@ -72,6 +73,8 @@ SIGNATURES = {
     "hca_prepare_bias": (ctypes.c_int, [_p, _i64, _i32, ctypes.c_int, _p, _i64, _p]),
     "hca_compress_prepared": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i64, _i32,
                                              _p, ctypes.c_int, _p]),
+    "hca_compress_noalloc": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i32, _p,
+                                            ctypes.c_int, _p]),
     "csa_compress_fused_proj_cache": (ctypes.c_int, [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64,
                                                      _i64, _i32, _i32, _i32, _p, _d, _d, _f, _p,
                                                      _p, _p]),
@@ -256,6 +259,22 @@ def hca_compress_prepared(C, Z, workspace, m: int = 128, out=None, out_dtype=Non
                                      workspace.numel() * workspace.element_size(), batch, n, c, m,
                                      _ptr(out), _dtype_code(out_dtype), _stream(stream))
     _check(st, "hca_compress_prepared")
+    return out
+
+
+def hca_compress_noalloc(C, Z, B, m: int = 128, out=None, out_dtype=None, stream=None):
+    """hca_compress for callers that cannot allocate device memory while they run: the
+    library keeps the prepared bias in a fixed 1 MiB scratch of its own (shared by all
+    calls on a device; calls that overlap on the GPU race on it).  Pass `out` to avoid the
+    allocation this wrapper would otherwise make for the result."""
+    batch, n, c = C.shape
+    _streams(C, (("Z", Z),), (), True)
+    _biases(m, c, True, B=B)
+    out_dtype = C.dtype if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, C)
+    st = lib().hca_compress_noalloc(_ptr(C), _ptr(Z), _dtype_code(C.dtype), _ptr(B), batch, n, c, m,
+                                    _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "hca_compress_noalloc")
     return out
 
 

@@ -315,6 +315,20 @@ def test_hca_prepared_empty(L):
     assert hca_prep(L, n=127, C=None, Z=None, ws=None, out=None) == kvc.KVC_OK
 
 
+def test_noalloc_rejects_before_launch(L):
+    # sizes are checked before any CUDA call (fake pointers are never dereferenced)
+    call = lambda **kw: L.hca_compress_noalloc(
+        kw.get("C", A), A, kw.get("dt", kvc.KVC_BF16), A, 1, kw.get("n", 4096), kw.get("c", 512),
+        kw.get("m", 128), A, kvc.KVC_BF16, None)
+    assert call(c=2048) == kvc.KVC_ERR_TOO_LARGE
+    assert call(c=1024, m=128) == kvc.KVC_ERR_TOO_LARGE
+    assert call(m=400) == kvc.KVC_ERR_UNSUPPORTED
+    assert call(c=12) == kvc.KVC_ERR_SHAPE
+    assert call(dt=5) == kvc.KVC_ERR_DTYPE
+    assert call(C=None) == kvc.KVC_ERR_NULL
+    assert call(n=100, C=None) == kvc.KVC_OK  # empty: no entry, nothing touched
+
+
 def test_fused_empty(L):
     assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
     assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK
