@@ -651,6 +651,194 @@ def time_fused(dev, stream, reps=20):
     return res
 
 
+# ------------------------------------------------------------------------------ split sequence
+# --split sequence: ONE sequence of world x 2^20 tokens, each rank holding only the token
+# rows its entries read (kv_token_compressor_b200.shard.plan: contiguous entry ranges, a
+# one-block halo for the CSA b-rows; HCA windows need none).  Rows are drawn per 65536-row
+# piece from (seed, piece), so every rank, and the checker, draw the same sequence.
+
+SPLIT_SEED = 11
+
+
+def split_plan(n_total, world, rank):
+    """Rows [lo, hi) this rank holds, and its CSA and HCA shards."""
+    from kv_token_compressor_b200 import shard
+
+    pc = shard.plan(n_total, M_CSA, world, True)[rank]
+    ph = shard.plan(n_total, M_HCA, world, False)[rank]
+    return min(pc.row0, ph.row0), max(pc.row1, ph.row1), pc, ph
+
+
+def split_inputs(n_total, world, rank, c, dtype, device):
+    from kv_token_compressor_b200 import synth
+
+    lo, hi, pc, ph = split_plan(n_total, world, rank)
+    t = synth.stream_rows_torch(lo, hi, c, dtype, seed=SPLIT_SEED, z_row_offset=Z_OFF, device=device)
+    t["Ba"] = synth.bias_torch(M_CSA, c, SPLIT_SEED + 1, device=device)
+    t["Bb"] = synth.bias_torch(M_CSA, c, SPLIT_SEED + 2, device=device)
+    t["Bh"] = synth.bias_torch(M_HCA, c, SPLIT_SEED + 3, device=device)
+    return t, lo, pc, ph
+
+
+def split_compress(t, lo, pc, ph, csa_fn, hca_fn, out_c, out_h):
+    """The rank's part: CSA over its rows (halo first) into out_c [1, entries + halo, c],
+    HCA into out_h [1, entries, c].  Returns the owned entries (the halo entry dropped)."""
+    sl = {k: t[k][:, pc.row0 - lo:pc.row1 - lo] for k in ("Ca", "Cb", "Za", "Zb")}
+    if pc.entries:
+        csa_fn(sl, t["Ba"], t["Bb"], out_c)
+    if ph.entries:
+        hca_fn(t["Ca"][:, ph.row0 - lo:ph.row1 - lo], t["Za"][:, ph.row0 - lo:ph.row1 - lo],
+               t["Bh"], out_h)
+    return (out_c[:, 1:] if pc.drop_first else out_c), out_h
+
+
+def split_check(world, rank, pc, ph, owned_c, owned_h, c, dtype, device, single_csa, single_hca,
+                per_rank=16):
+    """Sampled cross-rank check: every rank sends its first, second and last owned entries
+    (the first one depends on the halo) and a few others of each compressor to rank 0 over
+    the process group; rank 0 redraws the rows each entry reads and recomputes it on its
+    own as a one-sequence problem (single_csa(rows, Ba, Bb, j) -> entry j of those rows,
+    single_hca(C, Z, B) -> their one entry, numpy float64), then compares.  The tolerance
+    allows one output rounding on each side.  Returns (entries checked, max error / max
+    |ref|, ok) on rank 0, None elsewhere."""
+    import torch
+    import torch.distributed as dist
+
+    from kv_token_compressor_b200 import synth
+
+    def pick(e0, e1, k):
+        n = e1 - e0
+        if n <= 0:
+            return []
+        rng = np.random.default_rng(1000 + rank)
+        idx = {e0, e1 - 1, min(e0 + 1, e1 - 1)} | set((e0 + rng.integers(0, n, k)).tolist())
+        return sorted(idx)[:k + 3]
+
+    rows = []
+    for mode, shard, owned in (("csa", pc, owned_c), ("hca", ph, owned_h)):
+        for e in pick(shard.e0, shard.e1, per_rank if mode == "csa" else 4):
+            v = owned[0, e - shard.e0].float().cpu()
+            rows.append(torch.cat([torch.tensor([0.0 if mode == "csa" else 1.0, float(e)]), v]))
+    width, slots = 2 + c, per_rank + 3 + 4 + 3
+    mine = torch.full((slots, width), -1.0, dtype=torch.float32)
+    for i, r in enumerate(rows):
+        mine[i] = r
+    if world > 1:
+        dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+        got = [torch.empty_like(mine, device=dev) for _ in range(world)]
+        dist.all_gather(got, mine.to(dev))
+        got = [g.cpu() for g in got]
+    else:
+        got = [mine]
+    if rank != 0:
+        return None
+    Ba = synth.bias_torch(M_CSA, c, SPLIT_SEED + 1, device=device)
+    Bb = synth.bias_torch(M_CSA, c, SPLIT_SEED + 2, device=device)
+    Bh = synth.bias_torch(M_HCA, c, SPLIT_SEED + 3, device=device)
+    worst, checked, ok = 0.0, 0, True
+    for g in got:
+        for r in g:
+            if r[1] < 0:
+                continue
+            mode, e = int(r[0]), int(r[1])
+            if mode == 0:
+                lo = M_CSA * (e - 1) if e > 0 else 0
+                x = synth.stream_rows_torch(lo, M_CSA * (e + 1), c, dtype, seed=SPLIT_SEED,
+                                            z_row_offset=Z_OFF, device=device)
+                ref = single_csa(x, Ba, Bb, 1 if e > 0 else 0)
+            else:
+                x = synth.stream_rows_torch(M_HCA * e, M_HCA * (e + 1), c, dtype, seed=SPLIT_SEED,
+                                            z_row_offset=Z_OFF, device=device)
+                ref = single_hca(x["Ca"], x["Za"], Bh)
+            err = np.abs(r[2:].double().numpy() - ref)
+            scale = max(float(np.abs(ref).max()), 1e-30)
+            if dtype == "bf16":
+                bound = 2.0 ** -7 * np.abs(ref) + 1e-5 * scale
+            else:
+                bound = 1e-5 * scale
+            ok = ok and bool(np.all(err <= bound))
+            worst = max(worst, float(err.max()) / scale)
+            checked += 1
+    return checked, worst, ok
+
+
+def run_split(args):
+    """--split sequence: one world x 2^20-token sequence, each rank compressing its own rows
+    (CSA m = 4 with the halo, HCA m' = 128); timed like the default step (CUDA events, max
+    over ranks); then the sampled cross-rank check against single-GPU recomputation."""
+    import torch
+
+    from kv_token_compressor_b200 import kvc
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    n_total = world * N_TOK
+    t, lo, pc, ph = split_inputs(n_total, world, rank, C, "bf16", dev)
+    out_c = torch.empty((1, pc.entries + int(pc.drop_first), C), device=dev, dtype=torch.bfloat16)
+    out_h = torch.empty((1, ph.entries, C), device=dev, dtype=torch.bfloat16)
+
+    def csa_fn(sl, Ba, Bb, out):
+        kvc.csa_compress(sl["Ca"], sl["Cb"], sl["Za"], sl["Zb"], Ba, Bb, m=M_CSA, out=out,
+                         stream=stream)
+
+    def hca_fn(Cs, Zs, B, out):
+        kvc.hca_compress(Cs, Zs, B, m=M_HCA, out=out, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        split_compress(t, lo, pc, ph, csa_fn, hca_fn, out_c, out_h)
+    torch.cuda.synchronize()
+    if kvc.device_status(stream) != kvc.KVC_OK:
+        raise SystemExit("device error during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        owned_c, owned_h = split_compress(t, lo, pc, ph, csa_fn, hca_fn, out_c, out_h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+    def single_csa(x, Ba, Bb, j):
+        o = kvc.csa_compress(x["Ca"], x["Cb"], x["Za"], x["Zb"], Ba, Bb, m=M_CSA,
+                             out_dtype=torch.float32)
+        return o[0, j].double().cpu().numpy()
+
+    def single_hca(Cs, Zs, B):
+        return kvc.hca_compress(Cs, Zs, B, m=M_HCA, out_dtype=torch.float32)[0, 0].double().cpu().numpy()
+
+    check = split_check(world, rank, pc, ph, owned_c, owned_h, C, "bf16", dev, single_csa,
+                        single_hca)
+    if rank == 0:
+        entries = n_total // M_CSA + n_total // M_HCA
+        line = {
+            "metric": METRIC, "value": n_total / (ms * 1e-3), "unit": "tokens/s",
+            "entries_per_s": entries / (ms * 1e-3), "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"one sequence of {world} x 2^20 tokens, c=512, bf16 in/out; "
+                                   "CSA m=4 overlap + HCA m'=128 on the same streams",
+                       "n": n_total, "c": C, "m": M_CSA, "m_hca": M_HCA,
+                       "l2": "inputs 4.3 GB per rank > 126 MB L2, no flush",
+                       "parallelism": f"sequence split over {world} ranks: contiguous entry "
+                                      "ranges, one-block CSA halo, no data-path collective"},
+            "gpu_launches": 2 * args.steps,
+            "split_check": {"entries": check[0], "max_rel_err": check[1], "ok": check[2],
+                            "against": "each sampled entry recomputed on rank 0 as a "
+                                       "one-sequence problem of its own rows"},
+        }
+        print(json.dumps(line), flush=True)
+        if not check[2]:
+            raise SystemExit("split check failed")
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------------------------------ other paths
 
 def _peak(kind, sustained=False):
@@ -1058,8 +1246,10 @@ def run_profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             kvc.lightning_indexer_scores(t["q"], t["w"], t["K"], ks, nv, S, scores=sc)
             kvc.indexer_topk(sc, nv, 1024, S)
-    elif kind == "csa_fused":
-        n, d = 4096, 7168
+    elif kind in ("csa_fused", "csa_fused_n32768"):
+        # n = 4096: one tile per pair; n = 32768: the fused CSA workload itself (0.5 GB on
+        # the device; several tiles per pair, the carried partials between them)
+        n, d = (4096 if kind == "csa_fused" else 32768), 7168
         f = synth.fused_inputs_torch("csa", 1, n, d, C, M_CSA, seed=0)
         for _ in range(launches):
             kvc.csa_compress_fused_proj(f["H"], f["W_kva"], f["W_kvb"], f["W_za"], f["W_zb"],
@@ -1085,6 +1275,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", choices=["replicas", "sequence"], default="replicas",
+                    help="replicas (default): every rank its own 2^20-token problem; sequence: "
+                         "one world x 2^20-token sequence split over the ranks (shard plan)")
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused-path kernels timed after the default step")
     ap.add_argument("--workload", default="long",
@@ -1096,7 +1289,7 @@ def main():
                          "time one kernel on its own workload")
     ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "csa_n1024", "indexer_keys",
                                                "decode", "scalar", "cache", "indexer", "csa_fused",
-                                               "hca_fused"],
+                                               "csa_fused_n32768", "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
     if args.profile_case:
@@ -1104,7 +1297,10 @@ def main():
     elif args.impl == "reference":
         run_reference(args)
     else:
-        run_ours(args) if args.workload == "long" else run_workload(args)
+        if args.split == "sequence":
+            run_split(args)
+        else:
+            run_ours(args) if args.workload == "long" else run_workload(args)
 
 
 if __name__ == "__main__":

@@ -868,7 +868,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int64_t units = a.units;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both)

@@ -34,6 +34,9 @@ __all__ = [
     "fused_inputs",
     "stream_inputs_torch",
     "fused_inputs_torch",
+    "stream_rows_torch",
+    "bias_torch",
+    "ROW_CHUNK",
     "scalar_inputs",
     "scalar_inputs_torch",
     "indexer_inputs",
@@ -130,6 +133,46 @@ def stream_inputs_torch(mode: str, batch: int, n: int, c: int, m: int, dtype: st
     for k in (("Ba", "Bb") if mode == "csa" else ("B",)):
         out[k] = torch.randn((m, c), generator=g, device=device, dtype=torch.float32) * float(np.sqrt(bias_var))
     return out
+
+
+ROW_CHUNK = 1 << 16  # rows per independently seeded piece of stream_rows_torch
+
+
+def stream_rows_torch(row0: int, row1: int, c: int, dtype: str, seed: int = 0,
+                      z_row_offset: float = 0.0, device="cuda"):
+    """Rows [row0, row1) of one long sequence's four CSA streams Ca, Cb, Za, Zb ([1, rows,
+    c], the distributions of stream_inputs_torch), drawn in pieces of ROW_CHUNK rows, each
+    from its own generator seeded by (seed, piece index): any process can draw any rows of
+    the same sequence and gets the same values (for a given device type), which lets ranks
+    that each hold a slice of one sequence, and a checker that redraws a few windows,
+    agree."""
+    import torch
+
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    names = ("Ca", "Cb", "Za", "Zb")
+    out = {k: torch.empty((1, row1 - row0, c), dtype=tdt, device=device) for k in names}
+    g = torch.Generator(device=device)
+    for piece in range(row0 // ROW_CHUNK, (max(row1, row0 + 1) - 1) // ROW_CHUNK + 1):
+        p0 = piece * ROW_CHUNK
+        g.manual_seed(seed * 1000003 + piece)
+        lo, hi = max(row0, p0), min(row1, p0 + ROW_CHUNK)
+        for k in names:
+            x = torch.randn((ROW_CHUNK, c), generator=g, device=device, dtype=torch.float32)
+            if z_row_offset and k.startswith("Z"):
+                off = torch.rand((ROW_CHUNK, 1), generator=g, device=device, dtype=torch.float32)
+                x += off * (2 * z_row_offset) - z_row_offset
+            if hi > lo:
+                out[k][0, lo - row0:hi - row0] = x[lo - p0:hi - p0].to(tdt)
+    return out
+
+
+def bias_torch(m: int, c: int, seed: int, bias_var: float = 0.1, device="cuda"):
+    """One position bias [m, c] fp32 ~ N(0, bias_var), from its own seeded generator."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn((m, c), generator=g, device=device, dtype=torch.float32) * float(np.sqrt(bias_var))
 
 
 def fused_inputs_torch(mode: str, batch: int, n: int, d: int, c: int, m: int, seed: int = 0,
