@@ -909,6 +909,7 @@ def _workload(name, dev):
         return dict(inputs=t, launch=launch, outputs=[out], tokens=b * n, entries=b * n // 128,
                     bound="tensor", units=2.0 * b * n * d * 2 * c, flush=False,
                     kernel="fused_pair_kernel<HCA> (CTA pairs, M=256)",
+                    traffic_key="fused_hca_4x131072_d4096",
                     config={"workload": f"HCA fused projection + pool: batch {b}, n={n}, H d={d} "
                                         f"bf16, W_kv, W_z [{d}, {c}], m'=128, bf16 out",
                             "batch": b, "n": n, "d": d, "c": c, "m": 128})

@@ -199,11 +199,11 @@ struct Args {
   int nk;           // K steps of 64
   int pieces_per_unit;  // single-CTA CSA: entry ranges per (sequence, channel group)
   int64_t units;        // single-CTA CSA: pieces; HCA: tiles; CTA-pair CSA: busy clusters
-  // CTA-pair CSA: tiles per cluster, and where each cluster's first piece starts (flat
-  // (sequence, channel group) index and entry)
+  // CTA-pair CSA: tiles per cluster, token ranges per sequence, and each cluster's first
+  // piece (flat piece index)
   int64_t tile_budget;
-  int32_t start_g[kMaxClusters];
-  int32_t start_e[kMaxClusters];
+  int64_t ranges;
+  int32_t start_k[kMaxClusters + 1];  // start_k[units] = the number of pieces
 };
 
 // Extra kernel argument of the cache-layout instantiations (empty otherwise).
@@ -665,49 +665,44 @@ struct Unit {
   int ntiles;
 };
 
-// CSA schedule.  The entries of the G = batch x channel-group sequences, taken group by
-// group, are cut into pieces (sequence, channel group, entries [e0, e1)); every cluster
-// takes consecutive pieces worth at most `tile_budget` tiles, where a tile holds 64 blocks
-// of 4 rows (256 tokens).  A piece that starts inside its sequence (e0 > 0) starts one
-// block early, at the b-block of entry e0 (the halo), so its tiles cover blocks
-// [e0 - 1 + 64 t, e0 - 1 + 64 t + 64); within a piece the b-partial of a tile's first
-// entry is carried over from the tile before, so no block is projected twice.  A piece
-// ends at its sequence's end or when the budget runs out, on a full tile; only the last
-// tile of a sequence can be short.  The host picks the smallest budget with which the
-// clusters cover every entry (the cost of a tile hardly depends on its length: each one
-// streams all of W), so the busiest cluster has as few tiles as possible.
-struct CsaWalk {
-  int64_t g, e;  // the next piece starts at entry e of flat group g
-  int64_t left;  // tiles left in the cluster's budget
-};
+// CSA schedule.  With a budget of T tiles per cluster (a tile holds 64 blocks of 4 rows,
+// 256 tokens), each sequence is cut into token ranges of T tiles: the first range holds
+// entries [0, 64 T), every later one 64 T - 1 entries and starts one block early, at the
+// b-block of its first entry (the halo, no entry itself).  A piece is one token range of
+// one channel group; pieces are taken in the order (sequence, range, channel group) and
+// dealt to the clusters in turn, each cluster taking consecutive pieces while they fit its
+// budget (the last range of a sequence is short, and several of its pieces share a
+// cluster).  So the clusters that hold the same token range for different channel groups
+// are neighbours that run at the same time, and the H rows they all read come from DRAM
+// about once.  Within a piece the b-partial of a tile's first entry is carried over from
+// the tile before, so no block is projected twice.  The host picks the smallest T for
+// which the resident clusters cover every piece (the cost of a tile hardly depends on its
+// length: each one streams all of W).
+__host__ __device__ inline int64_t csa_ranges(int64_t ne, int64_t T) {
+  return ne <= 64 * T ? 1 : 1 + (ne - 64 * T + 64 * T - 2) / (64 * T - 1);
+}
 
-__host__ __device__ inline bool csa_next(int64_t G, int64_t ne, int ncg, int64_t n, CsaWalk* w,
-                                         Unit* q) {
-  if (w->left <= 0 || w->g >= G) return false;
-  const int64_t h = w->e > 0 ? 1 : 0;
-  const int64_t tiles_to_end = (ne - w->e + h + 63) / 64;
-  const bool to_end = tiles_to_end <= w->left;
-  const int64_t nt = to_end ? tiles_to_end : w->left;
-  const int64_t e1 = to_end ? ne : w->e + 64 * nt - h;
-  q->b = static_cast<int>(w->g / ncg);
-  q->cg = static_cast<int>(w->g - static_cast<int64_t>(q->b) * ncg);
-  q->e0 = w->e;
-  q->e1 = e1;
-  q->first_block = w->e - h;
-  q->rows = 4 * (e1 - q->first_block);
+__host__ __device__ inline void csa_piece_of(int64_t k, int64_t ne, int ncg, int64_t n, int64_t T,
+                                             int64_t R, Unit* q) {
+  const int64_t per_seq = R * ncg;
+  q->b = static_cast<int>(k / per_seq);
+  const int64_t rem = k - static_cast<int64_t>(q->b) * per_seq;
+  const int64_t r = rem / ncg;
+  q->cg = static_cast<int>(rem - r * ncg);
+  q->e0 = r == 0 ? 0 : 64 * T + (r - 1) * (64 * T - 1);
+  const int64_t e1 = q->e0 + (r == 0 ? 64 * T : 64 * T - 1);
+  q->e1 = e1 < ne ? e1 : ne;
+  q->first_block = q->e0 > 0 ? q->e0 - 1 : 0;
+  q->rows = 4 * (q->e1 - q->first_block);
   q->stride = 256;
-  q->ntiles = static_cast<int>(nt);
+  q->ntiles = static_cast<int>((q->e1 - q->first_block + 63) / 64);
   q->row0 = static_cast<int64_t>(q->b) * n + 4 * q->first_block;
   q->j = 0;
-  w->left -= nt;
-  if (to_end) {
-    ++w->g;
-    w->e = 0;
-  } else {
-    w->e = e1;
-  }
-  return true;
 }
+
+struct CsaWalk {
+  int64_t k, end;  // pieces [k, end) are this cluster's
+};
 
 // The units a cluster works through: CSA pieces from its schedule entry, HCA tiles
 // u = cid, cid + ncl, ...
@@ -717,10 +712,9 @@ struct Sched {
 };
 template <bool CSA>
 __device__ __forceinline__ Sched sched_begin(const Args& a, int64_t cid, int64_t ncl) {
-  Sched s{cid, ncl, a.units, CsaWalk{0, 0, 0}};
+  Sched s{cid, ncl, a.units, CsaWalk{0, 0}};
   if constexpr (CSA) {
-    if (cid < a.units && cid < kMaxClusters)
-      s.w = CsaWalk{a.start_g[cid], a.start_e[cid], a.tile_budget};
+    if (cid < a.units && cid < kMaxClusters) s.w = CsaWalk{a.start_k[cid], a.start_k[cid + 1]};
   }
   return s;
 }
@@ -749,7 +743,9 @@ __device__ __forceinline__ Unit hca_unit(const Args& a, int64_t u, uint32_t rank
 template <bool CSA>
 __device__ __forceinline__ bool sched_next(const Args& a, Sched* s, uint32_t rank, Unit* q) {
   if constexpr (CSA) {
-    return csa_next(a.batch * a.ncg, a.ne, a.ncg, a.n, &s->w, q);
+    if (s->w.k >= s->w.end) return false;
+    csa_piece_of(s->w.k++, a.ne, a.ncg, a.n, a.tile_budget, a.ranges, q);
+    return true;
   } else {
     if (s->u >= s->units) return false;
     *q = hca_unit(a, s->u, rank);
@@ -1298,46 +1294,48 @@ kvc_status launch_impl(const FusedProblem& p, cudaStream_t st) {
   return KVC_OK;
 }
 
-// CSA CTA-pair schedule (see csa_next): the smallest tile budget with which `clusters`
-// clusters cover every entry, and each cluster's starting point; returns the number of
-// clusters that get work.
+// CSA CTA-pair schedule (see csa_piece_of): the smallest tile budget T with which
+// `clusters` clusters take every piece, each cluster's first piece, and the number of
+// clusters that get work (returned).
 int64_t plan_csa(Args* a, int64_t clusters) {
   const int64_t G = a->batch * a->ncg;
-  auto covers = [&](int64_t T) {
-    pair::CsaWalk w{0, 0, 0};
+  // deal the pieces of budget T to clusters in turn; calls take(k0, k1) per cluster
+  auto deal = [&](int64_t T, auto take) {
+    const int64_t R = pair::csa_ranges(a->ne, T), total = a->batch * R * a->ncg;
+    int64_t k = 0, used = 0;
     pair::Unit q;
-    for (int64_t k = 0; k < clusters && w.g < G; ++k) {
-      w.left = T;
-      while (pair::csa_next(G, a->ne, a->ncg, a->n, &w, &q)) {
+    while (k < total) {
+      const int64_t k0 = k;
+      int64_t left = T;
+      while (k < total) {
+        pair::csa_piece_of(k, a->ne, a->ncg, a->n, T, R, &q);
+        if (q.ntiles > left) break;
+        left -= q.ntiles;
+        ++k;
       }
+      take(used++, k0, k);
     }
-    return w.g >= G;
+    return used;
   };
-  // every piece wastes less than one tile at its sequence's end: the budget lies between
-  // the average and the average plus the sequences per cluster, plus one
+  auto fits = [&](int64_t T) { return deal(T, [](int64_t, int64_t, int64_t) {}) <= clusters; };
   int64_t lo = (G * ((a->ne + 63) / 64) + clusters - 1) / clusters;
   if (lo < 1) lo = 1;
-  int64_t hi = lo + (G + clusters - 1) / clusters + 1;
-  while (!covers(hi)) hi *= 2;
-  while (lo < hi) {
+  int64_t hi = lo;
+  while (!fits(hi)) hi *= 2;
+  while (lo < hi) {  // the fewest clusters needed does not grow with T
     const int64_t mid = lo + (hi - lo) / 2;
-    if (covers(mid)) {
+    if (fits(mid)) {
       hi = mid;
     } else {
       lo = mid + 1;
     }
   }
   a->tile_budget = lo;
-  pair::CsaWalk w{0, 0, 0};
-  pair::Unit q;
-  int64_t busy = 0;
-  for (; busy < clusters && w.g < G; ++busy) {
-    a->start_g[busy] = static_cast<int32_t>(w.g);
-    a->start_e[busy] = static_cast<int32_t>(w.e);
-    w.left = lo;
-    while (pair::csa_next(G, a->ne, a->ncg, a->n, &w, &q)) {
-    }
-  }
+  a->ranges = pair::csa_ranges(a->ne, lo);
+  const int64_t busy = deal(lo, [&](int64_t c, int64_t k0, int64_t k1) {
+    a->start_k[c] = static_cast<int32_t>(k0);
+    a->start_k[c + 1] = static_cast<int32_t>(k1);
+  });
   return busy;
 }
 
