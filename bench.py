@@ -898,6 +898,33 @@ def _workload(name, dev):
                                         f"bf16, 4 W [{d}, {c}] bf16, m=4 overlap, E4M3 [c-{r}] "
                                         f"+ RoPE'd bf16 [{r}]", "n": n, "d": d, "c": c, "m": 4,
                             "r": r})
+    if name in ("fused_csa_scalar", "fused_hca_scalar"):
+        csa = name == "fused_csa_scalar"
+        b, n, d, c, m = (1, 32768, 7168, 512, 4) if csa else (4, 131072, 4096, 512, 128)
+        t = synth.fused_scalar_inputs_torch("csa" if csa else "hca", b, n, d, c, m, seed=0,
+                                            device=dev)
+        out = torch.empty((b, n // m, c), device=dev, dtype=bf)
+
+        def launch(x, st):
+            if csa:
+                kvc.csa_compress_fused_proj_scalar(x["H"], x["W_kva"], x["W_kvb"], x["w_za"],
+                                                   x["w_zb"], x["ba"], x["bb"], b, n, out=out,
+                                                   stream=st)
+            else:
+                kvc.hca_compress_fused_proj_scalar(x["H"], x["W_kv"], x["w_z"], x["b"], b, n,
+                                                   out=out, stream=st)
+        streams = 2 if csa else 1
+        return dict(inputs=t, launch=launch, outputs=[out], tokens=b * n, entries=b * n // m,
+                    bound="tensor", units=2.0 * b * n * d * streams * c, flush=False,
+                    kernel=f"fused_scalar_kernel<{'CSA' if csa else 'HCA'}> (CTA pairs, M=256; "
+                           "scores on the CUDA cores beside the MMAs)",
+                    config={"workload": f"{'CSA' if csa else 'HCA'} fused projection + pool, "
+                                        f"scalar logits: batch {b}, n={n}, H d={d} bf16, "
+                                        f"{streams} value W [{d}, {c}] + {streams} score vectors "
+                                        f"[{d}], m={m}, bf16 out; FLOPs count the value "
+                                        f"projections (tensor cores), not the 2 x {streams} "
+                                        f"x n x d of the scores",
+                            "batch": b, "n": n, "d": d, "c": c, "m": m})
     if name == "fused_hca":
         b, n, d, c = 4, 131072, 4096, 512
         t = synth.fused_inputs_torch("hca", b, n, d, c, 128, seed=0, device=dev)
@@ -1293,7 +1320,8 @@ def main():
     ap.add_argument("--no-fused", action="store_true",
                     help="skip the fused-path kernels timed after the default step")
     ap.add_argument("--workload", default="long",
-                    choices=["long", "fused_csa", "fused_csa_cache", "fused_hca", "hca_n65536",
+                    choices=["long", "fused_csa", "fused_csa_cache", "fused_csa_scalar",
+                             "fused_hca_scalar", "fused_hca", "hca_n65536",
                              "hca_n65536_prepared", "csa_f32_n1024",
                              "indexer_keys", "fused_indexer_keys", "scalar_long",
                              "decode_entries", "cache_long", "indexer_decode"],

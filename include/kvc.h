@@ -287,6 +287,24 @@ KVC_API kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, cons
                                    int64_t c, int32_t m,
                                    void* out, kvc_dtype out_dtype, kvc_stream stream);
 
+/* The fused compressors in the scalar-logit form ([CSA] §3 symbol table: one score per
+ * token and stream, z^a = H w^{Z_a} and z^b = H w^{Z_b} with w in R^d, an m-dimensional
+ * bias, and one weight per window row shared by all channels; the streamed form is
+ * csa_compress_scalar_logits).  C^a = H W_kva and C^b = H W_kvb are formed on the tensor
+ * cores and the scores beside them; neither reaches device memory.
+ *   H : [batch*n, d] bf16;  W_kva, W_kvb : [d, c] bf16;  w_za, w_zb : [d] bf16 (16-byte
+ *   aligned);  ba, bb : [m] fp32;  out : [batch, N_e, c] out_dtype;  d % 64 == 0,
+ *   c % 128 == 0; CSA m == 4 with overlap == 1, HCA m == 128, else KVC_ERR_UNSUPPORTED.
+ *   Scores accumulate in fp32 from the bf16 products (exact in fp32). */
+KVC_API kvc_status csa_compress_fused_proj_scalar(
+    const void* H, const void* W_kva, const void* W_kvb, const void* w_za, const void* w_zb,
+    const float* ba, const float* bb, int64_t batch, int64_t n, int64_t d, int64_t c, int32_t m,
+    int32_t overlap, void* out, kvc_dtype out_dtype, kvc_stream stream);
+/* HCA: C = H W_kv [d, c], z = H w_z [d], b : [m] fp32; entry i pools segment i. */
+KVC_API kvc_status hca_compress_fused_proj_scalar(
+    const void* H, const void* W_kv, const void* w_z, const float* b, int64_t batch, int64_t n,
+    int64_t d, int64_t c, int32_t m, void* out, kvc_dtype out_dtype, kvc_stream stream);
+
 /* The fused compressors with the entries written in the cache layout (the same layout as
  * csa_compress_cache above: [HCA] §4 (2) partial RoPE on the last r dimensions, the
  * comparison article's BF16 RoPE part and FP8 rest) straight from the GEMM epilogue ([SC]

@@ -204,6 +204,9 @@ struct Args {
   int64_t tile_budget;
   int64_t ranges;
   int32_t start_k[kMaxClusters + 1];  // start_k[units] = the number of pieces
+  // scalar-logit form: the score vectors w^{Z_a}, w^{Z_b} (CSA) or w^{Z} (HCA), bf16 [d]
+  const void* wz0;
+  const void* wz1;
 };
 
 // Extra kernel argument of the cache-layout instantiations (empty otherwise).
@@ -1214,6 +1217,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
   cluster_sync_all();
 }
 
+#include "fused_scalar.cuh"
+
 // ------------------------------------------------------------------ host side
 
 // 2-D bf16 row-major [rows, cols] tensor map with a [box_rows, box_cols] box; the
@@ -1397,6 +1402,64 @@ kvc_status launch_pair(const FusedProblem& p, cudaStream_t st) {
   return KVC_OK;
 }
 
+// Scalar-logit CTA-pair launch (fused_scalar_kernel).  No single-CTA form: without a
+// resident pair it returns KVC_ERR_UNSUPPORTED.
+template <bool CSA, typename OutT>
+kvc_status launch_scalar(const FusedProblem& p, cudaStream_t st) {
+  using C = pair::Cfg;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return KVC_ERR_CUDA;
+  if (p.batch * p.n > (int64_t(1) << 31) - 1 - 256) return KVC_ERR_UNSUPPORTED;  // TMA y: int32
+  CUtensorMap mh, mw0, mw1;
+  if (!make_map(&mh, p.H, static_cast<uint64_t>(p.batch * p.n), static_cast<uint64_t>(p.d), 128,
+                C::BK) ||
+      !make_map(&mw0, p.W[0], static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.c), C::BK, 64) ||
+      !make_map(&mw1, CSA ? p.W[1] : p.W[0], static_cast<uint64_t>(p.d),
+                static_cast<uint64_t>(p.c), C::BK, 64))
+    return KVC_ERR_CUDA;
+  auto kern = fused_scalar_kernel<CSA, OutT>;
+  if (!raise_smem_limit(reinterpret_cast<const void*>(kern))) return KVC_ERR_CUDA;
+  int clusters = 0;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+    cfg.blockDim = dim3(pair::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = scal::Cfg::SMEM;
+    cfg.stream = st;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+      (void)cudaGetLastError();
+      return KVC_ERR_UNSUPPORTED;
+    }
+  }
+  Args a{};
+  a.B0 = p.B0;
+  a.B1 = p.B1;
+  a.out = p.out;
+  a.batch = p.batch;
+  a.n = p.n;
+  a.c = p.c;
+  a.ne = p.ne;
+  a.nk = static_cast<int>(p.d / C::BK);
+  a.wz0 = p.wz[0];
+  a.wz1 = p.wz[1];
+  const int ncg = static_cast<int>(p.c / kCh);
+  if constexpr (CSA) {
+    a.ncg = (ncg + 1) / 2;  // channel-group pairs: the leader takes group 2p, the peer 2p + 1
+    if (clusters > kMaxClusters) clusters = kMaxClusters;
+    a.units = plan_csa(&a, clusters);
+  } else {
+    a.ncg = (ncg + 3) / 4;  // channel quads: two groups per CTA
+    a.units = p.batch * ((p.ne + 1) / 2) * a.ncg;
+  }
+  const int64_t ncl = a.units < clusters ? a.units : clusters;
+  kern<<<static_cast<unsigned>(2 * ncl), pair::kThreads, scal::Cfg::SMEM, st>>>(mh, mw0, mw1, a);
+  if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
+  last_kernel() = CSA ? "fused_scalar_kernel/csa" : "fused_scalar_kernel/hca";
+  return KVC_OK;
+}
+
 }  // namespace fused
 
 // Stage K per mode.  64-deep stages: CSA 80 KB (two fit), HCA 64 KB (three).  32-deep
@@ -1423,6 +1486,14 @@ kvc_status launch_fused_typed(const FusedProblem& p, cudaStream_t st) {
 }
 
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st) {
+  if (p.scalar) {
+    if (p.csa ? (p.m != 4 || !p.overlap) : p.m != 128) return KVC_ERR_UNSUPPORTED;
+    if (p.csa)
+      return p.out_bf16 ? fused::launch_scalar<true, __nv_bfloat16>(p, st)
+                        : fused::launch_scalar<true, float>(p, st);
+    return p.out_bf16 ? fused::launch_scalar<false, __nv_bfloat16>(p, st)
+                      : fused::launch_scalar<false, float>(p, st);
+  }
   if (p.cache) return launch_fused_typed<__nv_bfloat16, true>(p, st);
   return p.out_bf16 ? launch_fused_typed<__nv_bfloat16, false>(p, st)
                     : launch_fused_typed<float, false>(p, st);

@@ -761,6 +761,47 @@ kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* 
   return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
+kvc_status csa_compress_fused_proj_scalar(const void* H, const void* W_kva, const void* W_kvb,
+                                          const void* w_za, const void* w_zb, const float* ba,
+                                          const float* bb, int64_t batch, int64_t n, int64_t d,
+                                          int64_t c, int32_t m, int32_t overlap, void* out,
+                                          kvc_dtype out_dtype, kvc_stream stream) {
+  if (overlap != 0 && overlap != 1) return KVC_ERR_SHAPE;
+  FusedProblem p{};
+  bool empty = false;
+  const void* W[4] = {W_kva, W_kvb, w_za, w_zb};
+  const kvc_status s = fused_common(&p, true, overlap, H, W, 4, ba, bb, true, batch, n, d, c, m,
+                                    out, out_dtype, true, &empty);
+  if (s != KVC_OK || empty) return s;
+  p.W[0] = W_kva;
+  p.W[1] = W_kvb;
+  p.wz[0] = w_za;
+  p.wz[1] = w_zb;
+  p.scalar = true;
+  p.csa = true;
+  p.overlap = true;
+  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvc_status hca_compress_fused_proj_scalar(const void* H, const void* W_kv, const void* w_z,
+                                          const float* b, int64_t batch, int64_t n, int64_t d,
+                                          int64_t c, int32_t m, void* out, kvc_dtype out_dtype,
+                                          kvc_stream stream) {
+  FusedProblem p{};
+  bool empty = false;
+  const void* W[2] = {W_kv, w_z};
+  const kvc_status s = fused_common(&p, false, 0, H, W, 2, b, nullptr, false, batch, n, d, c, m,
+                                    out, out_dtype, true, &empty);
+  if (s != KVC_OK || empty) return s;
+  p.W[0] = W_kv;
+  p.wz[0] = w_z;
+  p.wz[1] = w_z;
+  p.scalar = true;
+  p.csa = false;
+  p.overlap = false;
+  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 kvc_status csa_compress_fused_proj_cache(const void* H, const void* W_kva, const void* W_kvb,
                                          const void* W_za, const void* W_zb, const float* Ba,
                                          const float* Bb, int64_t batch, int64_t n, int64_t d,

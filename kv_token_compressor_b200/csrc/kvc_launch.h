@@ -103,6 +103,10 @@ struct FusedProblem {
   int64_t r;
   double pos_stride, pos_offset;
   float fp8_scale;
+  // Scalar-logit form (the *_fused_proj_scalar calls): W[0] (and W[1] for CSA) are the value
+  // projections, wz the score vectors [d] bf16, B0 / B1 the biases [m].
+  bool scalar;
+  const void* wz[2];
 };
 
 kvc_status launch_fused(const FusedProblem& p, cudaStream_t st);

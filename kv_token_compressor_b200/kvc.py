@@ -73,6 +73,10 @@ SIGNATURES = {
     "hca_prepare_bias": (ctypes.c_int, [_p, _i64, _i32, ctypes.c_int, _p, _i64, _p]),
     "hca_compress_prepared": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i64, _i32,
                                              _p, ctypes.c_int, _p]),
+    "csa_compress_fused_proj_scalar": (ctypes.c_int, [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64,
+                                                      _i64, _i32, _i32, _p, ctypes.c_int, _p]),
+    "hca_compress_fused_proj_scalar": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32,
+                                                      _p, ctypes.c_int, _p]),
     "hca_compress_noalloc": (ctypes.c_int, [_p, _p, ctypes.c_int, _p, _i64, _i64, _i64, _i32, _p,
                                             ctypes.c_int, _p]),
     "csa_compress_fused_proj_cache": (ctypes.c_int, [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64,
@@ -530,6 +534,47 @@ def hca_compress_fused_proj_cache(H, W_kv, W_z, B, batch: int, n: int, r: int, i
         _stream(stream))
     _check(st, "hca_compress_fused_proj_cache")
     return nope.view(batch, ne, max(c - r, 0)), rope.view(batch, ne, max(min(r, c), 0))
+
+
+def csa_compress_fused_proj_scalar(H, W_kva, W_kvb, w_za, w_zb, ba, bb, batch: int, n: int,
+                                   m: int = 4, out=None, out_dtype=None, stream=None):
+    """Fused scalar-logit CSA: H [batch*n, d] bf16, W_kva/W_kvb [d, c] bf16, score vectors
+    w_za/w_zb [d] bf16, biases ba/bb [m] fp32.  Returns [batch, n // m, c]."""
+    torch = _torch()
+    d = H.shape[1]
+    c = W_kva.shape[1]
+    _need("H", H, batch * n * d, torch.bfloat16)
+    for name, w in (("W_kva", W_kva), ("W_kvb", W_kvb)):
+        _need(name, w, d * c, torch.bfloat16)
+    for name, w in (("w_za", w_za), ("w_zb", w_zb)):
+        _need(name, w, d, torch.bfloat16)
+    _biases(m, 1, True, ba=ba, bb=bb)
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, H)
+    st = lib().csa_compress_fused_proj_scalar(
+        _ptr(H), _ptr(W_kva), _ptr(W_kvb), _ptr(w_za), _ptr(w_zb), _ptr(ba), _ptr(bb), batch, n,
+        d, c, m, 1, _ptr(out), _dtype_code(out_dtype), _stream(stream))
+    _check(st, "csa_compress_fused_proj_scalar")
+    return out
+
+
+def hca_compress_fused_proj_scalar(H, W_kv, w_z, b, batch: int, n: int, m: int = 128, out=None,
+                                   out_dtype=None, stream=None):
+    """Fused scalar-logit HCA: H [batch*n, d] bf16, W_kv [d, c] bf16, w_z [d] bf16, b [m]."""
+    torch = _torch()
+    d = H.shape[1]
+    c = W_kv.shape[1]
+    _need("H", H, batch * n * d, torch.bfloat16)
+    _need("W_kv", W_kv, d * c, torch.bfloat16)
+    _need("w_z", w_z, d, torch.bfloat16)
+    _biases(m, 1, True, b=b)
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    out = _out(out, (batch, n // m, c), out_dtype, H)
+    st = lib().hca_compress_fused_proj_scalar(_ptr(H), _ptr(W_kv), _ptr(w_z), _ptr(b), batch, n, d,
+                                              c, m, _ptr(out), _dtype_code(out_dtype),
+                                              _stream(stream))
+    _check(st, "hca_compress_fused_proj_scalar")
+    return out
 
 
 def lightning_indexer_scores(q, w, K, key_start, n_visible, max_visible: int, scores=None,

@@ -35,6 +35,8 @@ __all__ = [
     "stream_inputs_torch",
     "fused_inputs_torch",
     "stream_rows_torch",
+    "fused_scalar_inputs",
+    "fused_scalar_inputs_torch",
     "bias_torch",
     "ROW_CHUNK",
     "scalar_inputs",
@@ -108,6 +110,42 @@ def fused_inputs(mode: str, batch: int, n: int, d: int, c: int, m: int, seed: in
         out[k] = round_to_bf16(_normal(rng, (d, c), 1.0 / d))
     for k in (("Ba", "Bb") if mode == "csa" else ("B",)):
         out[k] = _normal(rng, (m, c), bias_var)
+    return out
+
+
+def fused_scalar_inputs(mode: str, batch: int, n: int, d: int, c: int, m: int, seed: int = 0,
+                        z_scale: float = 2.0, bias_var: float = 0.1):
+    """Host inputs of the fused scalar-logit form: H [batch*n, d] and the value projections
+    W [d, c] as in fused_inputs, score vectors w [d] ~ N(0, z_scale^2 / d) (scores of
+    spread z_scale, as scalar_inputs draws them), all rounded to bf16 (stored as fp32);
+    biases [m] fp32.  mode "csa": H, W_kva, W_kvb, w_za, w_zb, ba, bb; "hca": H, W_kv, w_z, b."""
+    rng = np.random.default_rng(seed)
+    out = {"H": round_to_bf16(_normal(rng, (batch * n, d)))}
+    for k in (("W_kva", "W_kvb") if mode == "csa" else ("W_kv",)):
+        out[k] = round_to_bf16(_normal(rng, (d, c), 1.0 / d))
+    for k in (("w_za", "w_zb") if mode == "csa" else ("w_z",)):
+        out[k] = round_to_bf16(_normal(rng, (d,), z_scale * z_scale / d))
+    for k in (("ba", "bb") if mode == "csa" else ("b",)):
+        out[k] = _normal(rng, (m,), bias_var)
+    return out
+
+
+def fused_scalar_inputs_torch(mode: str, batch: int, n: int, d: int, c: int, m: int,
+                              seed: int = 0, z_scale: float = 2.0, bias_var: float = 0.1,
+                              device="cuda"):
+    """Same distributions as :func:`fused_scalar_inputs`, generated on ``device``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = torch.bfloat16
+    out = {"H": torch.randn((batch * n, d), generator=g, device=device).to(bf)}
+    for k in (("W_kva", "W_kvb") if mode == "csa" else ("W_kv",)):
+        out[k] = (torch.randn((d, c), generator=g, device=device) * float(1.0 / np.sqrt(d))).to(bf)
+    for k in (("w_za", "w_zb") if mode == "csa" else ("w_z",)):
+        out[k] = (torch.randn((d,), generator=g, device=device) * float(z_scale / np.sqrt(d))).to(bf)
+    for k in (("ba", "bb") if mode == "csa" else ("b",)):
+        out[k] = torch.randn((m,), generator=g, device=device) * float(np.sqrt(bias_var))
     return out
 
 

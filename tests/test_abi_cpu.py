@@ -329,6 +329,25 @@ def test_noalloc_rejects_before_launch(L):
     assert call(n=100, C=None) == kvc.KVC_OK  # empty: no entry, nothing touched
 
 
+def test_fused_scalar_rejects_before_launch(L):
+    csa = lambda **kw: L.csa_compress_fused_proj_scalar(
+        kw.get("H", A), A, A, kw.get("wza", A), A, A, A, 1, kw.get("n", 4096), kw.get("d", 7168),
+        kw.get("c", 512), kw.get("m", 4), kw.get("ov", 1), A, kvc.KVC_BF16, None)
+    hca = lambda **kw: L.hca_compress_fused_proj_scalar(
+        A, A, kw.get("wz", A), A, 1, 4096, 4096, kw.get("c", 512), kw.get("m", 128), A,
+        kvc.KVC_BF16, None)
+    assert csa(m=8) == kvc.KVC_ERR_UNSUPPORTED
+    assert csa(ov=0) == kvc.KVC_ERR_UNSUPPORTED
+    assert csa(d=100) == kvc.KVC_ERR_SHAPE
+    assert csa(c=200) == kvc.KVC_ERR_SHAPE
+    assert csa(wza=None) == kvc.KVC_ERR_NULL
+    assert csa(wza=MIS) == kvc.KVC_ERR_ALIGN
+    assert csa(n=3, H=None, wza=None) == kvc.KVC_OK  # empty
+    assert hca(m=64) == kvc.KVC_ERR_UNSUPPORTED
+    assert hca(wz=None) == kvc.KVC_ERR_NULL
+    assert hca(wz=MIS) == kvc.KVC_ERR_ALIGN
+
+
 def test_fused_empty(L):
     assert fused_csa(L, n=2, H=None, out=None) == kvc.KVC_OK
     assert fused_hca(L, batch=0, H=None, out=None) == kvc.KVC_OK
