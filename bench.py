@@ -1293,6 +1293,12 @@ def run_profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             kvc.csa_compress_fused_proj(f["H"], f["W_kva"], f["W_kvb"], f["W_za"], f["W_zb"],
                                         f["Ba"], f["Bb"], 1, n)
+    elif kind == "csa_fused_scalar_n32768":  # the scalar-logit fused CSA workload itself
+        n, d = 32768, 7168
+        f = synth.fused_scalar_inputs_torch("csa", 1, n, d, C, M_CSA, seed=0)
+        for _ in range(launches):
+            kvc.csa_compress_fused_proj_scalar(f["H"], f["W_kva"], f["W_kvb"], f["w_za"], f["w_zb"],
+                                               f["ba"], f["bb"], 1, n)
     elif kind == "hca_fused":
         n, d = 16384, 4096
         f = synth.fused_inputs_torch("hca", 1, n, d, C, M_HCA, seed=0)
@@ -1329,7 +1335,8 @@ def main():
                          "time one kernel on its own workload")
     ap.add_argument("--profile-case", choices=["csa", "hca", "hca_n65536", "csa_n1024", "indexer_keys",
                                                "decode", "scalar", "cache", "indexer", "csa_fused",
-                                               "csa_fused_n32768", "hca_fused"],
+                                               "csa_fused_n32768", "csa_fused_scalar_n32768",
+                                               "hca_fused"],
                     help="run one kernel on a small case for ncu (no bench line)")
     args = ap.parse_args()
     if args.profile_case:

@@ -92,14 +92,15 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-// Sum of x * w over 8 bf16 pairs packed in two 16-byte vectors.
-__device__ __forceinline__ float dot8(const uint4& x, const uint4& w, float acc) {
+// acc (two fp32 lanes) += x * w over the 8 bf16 of two 16-byte vectors, pairwise (the
+// products of bf16 values are exact in fp32).
+__device__ __forceinline__ float2 dot8(const uint4& x, const uint4& w, float2 acc) {
   const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc = fmaf(__uint_as_float(xs[i] << 16), __uint_as_float(ws[i] << 16), acc);
-    acc = fmaf(__uint_as_float(xs[i] & 0xffff0000u), __uint_as_float(ws[i] & 0xffff0000u), acc);
-  }
+  for (int i = 0; i < 4; ++i)
+    acc = f2_fma(make_float2(__uint_as_float(xs[i] << 16), __uint_as_float(xs[i] & 0xffff0000u)),
+                 make_float2(__uint_as_float(ws[i] << 16), __uint_as_float(ws[i] & 0xffff0000u)),
+                 acc);
   return acc;
 }
 
@@ -301,8 +302,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       for (int t = 0; t < q.ntiles && ok; ++t, ++tcount) {
         const int nt = pair::tile_tokens(q, t);
         const uint32_t par = tcount % scal::kZBufs;  // this tile's score buffer
-        // ---- the tile's scores for this CTA's H rows, stage by stage, beside the MMAs
-        float z0 = 0.f, z1 = 0.f;
+        // ---- the tile's scores for this CTA's H rows, stage by stage, beside the MMAs; the
+        // w slices of the next stage are loaded while this one is summed
+        float2 z0 = make_float2(0.f, 0.f), z1 = make_float2(0.f, 0.f);
+        uint4 wn[4] = {};
+        {
+          const uint4* p0 = reinterpret_cast<const uint4*>(wz0 + 16 * lq);
+          const uint4* p1 = reinterpret_cast<const uint4*>(wz1 + 16 * lq);
+          wn[0] = __ldg(p0);
+          wn[1] = __ldg(p0 + 1);
+          if constexpr (CSA) {
+            wn[2] = __ldg(p1);
+            wn[3] = __ldg(p1 + 1);
+          }
+        }
         for (int kstep = 0; kstep < a.nk; ++kstep) {
           const bool got = rank == 0
                                ? pair::wait_pair(&full[stage], phase, abort_flag, peer_abort)
@@ -316,36 +329,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
           const int sw = lr & 7;
           const uint4 h0 = *reinterpret_cast<const uint4*>(hb + (((2 * lq) ^ sw) << 4));
           const uint4 h1 = *reinterpret_cast<const uint4*>(hb + (((2 * lq + 1) ^ sw) << 4));
-          const int k0 = kstep * C::BK + 16 * lq;
-          const uint4* w0p = reinterpret_cast<const uint4*>(wz0 + k0);
-          z0 = scal::dot8(h0, __ldg(w0p), z0);
-          z0 = scal::dot8(h1, __ldg(w0p + 1), z0);
-          if constexpr (CSA) {
-            const uint4* w1p = reinterpret_cast<const uint4*>(wz1 + k0);
-            z1 = scal::dot8(h0, __ldg(w1p), z1);
-            z1 = scal::dot8(h1, __ldg(w1p + 1), z1);
+          uint4 wc[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wc[i] = wn[i];
+          if (kstep + 1 < a.nk) {
+            const int k1 = (kstep + 1) * C::BK + 16 * lq;
+            const uint4* p0 = reinterpret_cast<const uint4*>(wz0 + k1);
+            wn[0] = __ldg(p0);
+            wn[1] = __ldg(p0 + 1);
+            if constexpr (CSA) {
+              const uint4* p1 = reinterpret_cast<const uint4*>(wz1 + k1);
+              wn[2] = __ldg(p1);
+              wn[3] = __ldg(p1 + 1);
+            }
           }
-          // these generic reads precede the next (async-proxy) fill of the stage
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          // the stage's bytes are in registers: release it (MMA commit + 16 reader warps)
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[stage]);
+          z0 = scal::dot8(h0, wc[0], z0);
+          z0 = scal::dot8(h1, wc[1], z0);
+          if constexpr (CSA) {
+            z1 = scal::dot8(h0, wc[2], z1);
+            z1 = scal::dot8(h1, wc[3], z1);
+          }
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        z0 += __shfl_xor_sync(0xffffffffu, z0, 1);
-        z0 += __shfl_xor_sync(0xffffffffu, z0, 2);
-        z1 += __shfl_xor_sync(0xffffffffu, z1, 1);
-        z1 += __shfl_xor_sync(0xffffffffu, z1, 2);
+        float s0 = z0.x + z0.y, s1 = z1.x + z1.y;
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
         if (lq == 0 && lr < nt / 2) {  // this CTA's tokens are [rank nt/2, (rank + 1) nt/2)
           const int pos = static_cast<int>(rank) * (nt / 2) + lr;
           float* zl = zbuf + par * 512;
-          zl[pos] = z0;
-          zl[256 + pos] = z1;
-          scal::st_cluster_f32(cluster_addr(smem_u32(zl + pos), peer), z0);
-          scal::st_cluster_f32(cluster_addr(smem_u32(zl + 256 + pos), peer), z1);
+          zl[pos] = s0;
+          zl[256 + pos] = s1;
+          scal::st_cluster_f32(cluster_addr(smem_u32(zl + pos), peer), s0);
+          scal::st_cluster_f32(cluster_addr(smem_u32(zl + 256 + pos), peer), s1);
         }
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
         __syncwarp();
