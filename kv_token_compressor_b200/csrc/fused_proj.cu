@@ -1425,7 +1425,7 @@ kvc_status launch_scalar(const FusedProblem& p, cudaStream_t st) {
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-    cfg.blockDim = dim3(pair::kThreads, 1, 1);
+    cfg.blockDim = dim3(scal::kThreads, 1, 1);
     cfg.dynamicSmemBytes = scal::Cfg::SMEM;
     cfg.stream = st;
     if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
@@ -1454,7 +1454,7 @@ kvc_status launch_scalar(const FusedProblem& p, cudaStream_t st) {
     a.units = p.batch * ((p.ne + 1) / 2) * a.ncg;
   }
   const int64_t ncl = a.units < clusters ? a.units : clusters;
-  kern<<<static_cast<unsigned>(2 * ncl), pair::kThreads, scal::Cfg::SMEM, st>>>(mh, mw0, mw1, a);
+  kern<<<static_cast<unsigned>(2 * ncl), scal::kThreads, scal::Cfg::SMEM, st>>>(mh, mw0, mw1, a);
   if (cudaGetLastError() != cudaSuccess) return KVC_ERR_CUDA;
   last_kernel() = CSA ? "fused_scalar_kernel/csa" : "fused_scalar_kernel/hca";
   return KVC_OK;

@@ -27,6 +27,10 @@
 namespace scal {
 
 constexpr int kEpiWarps = pair::kGroups * 4;        // 16
+// warp 0 TMA, warp 1 MMA, warp 2 relay (leader: tells the peer's score readers that a
+// stage landed; a release-ordered remote arrive in the MMA thread would hold its MMAs
+// back, measured 0.33 -> 0.71 ms), warps 3..18 epilogue
+constexpr int kThreads = 96 + kEpiWarps * 32;
 // scores [tile % 3][stream][token].  Three buffers: pooling tile t reads those of t and
 // t - 1, while the other CTA may already write those of t + 1 (its score readers can run
 // through a short K loop on prefetched stages); those of t + 2 wait for the MMAs of t + 2,
@@ -110,7 +114,7 @@ __device__ __forceinline__ float2 dot8(const uint4& x, const uint4& w, float2 ac
 // W0 = W1 = W^{KV}.  a.wz0 / a.wz1: w^{Z_a} / w^{Z_b} (CSA) or w^{Z} (HCA), bf16 [d];
 // a.B0 / a.B1: the position biases [m] fp32.
 template <bool CSA, typename OutT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(scal::kThreads, 1)
     fused_scalar_kernel(const __grid_constant__ CUtensorMap tmH,
                         const __grid_constant__ CUtensorMap tmW0,
                         const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ Args a) {
@@ -244,8 +248,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
                 ok = false;
                 break;
               }
-              // the peer's score readers learn here that their half of the stage landed
-              mbar_arrive_cluster(cluster_addr(smem_u32(&pfull[stage]), 1));
               tc_fence_after();
               const uint32_t st = smem_u32(smem + stage * C::STAGE);
 #pragma unroll
@@ -277,9 +279,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::kThreads, 1)
       }
       pair::wait_pair(final_bar, 0, abort_flag, peer_abort, false);
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ relay (leader)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      pair::Sched sc = pair::sched_begin<CSA>(a, cid, ncl);
+      pair::Unit q;
+      while (ok && scal::next_unit<CSA>(a, &sc, 0, &q)) {
+        for (int t = 0; t < q.ntiles && ok; ++t) {
+          for (int kstep = 0; kstep < a.nk; ++kstep) {
+            if (!pair::wait_pair(&full[stage], phase, abort_flag, peer_abort)) {
+              ok = false;
+              break;
+            }
+            // the peer's score readers learn here that their half of the stage landed
+            mbar_arrive_cluster(cluster_addr(smem_u32(&pfull[stage]), 1));
+            if (++stage == S) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..17)
-    const int ew = warp - 2;              // epilogue warp 0..15
+    // ------------------------------------------------------------ epilogue (warps 3..18)
+    const int ew = warp - 3;              // epilogue warp 0..15
     const int eg = ew >> 2;               // group: tokens [64 eg, 64 eg + 64) of a tile
     const int qw = warp & 3;              // TMEM lane quarter this warp may access
     const int row = qw * 32 + lane;       // TMEM lane = channel within an accumulator
