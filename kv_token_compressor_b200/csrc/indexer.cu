@@ -16,10 +16,12 @@
 // the MMAs and loads of the next, and the queries' q tiles sit in two shared-memory slots.
 //
 // Top-k (indexer_topk_kernel).  A cluster of 8 CTAs per query holds the query's scores on
-// chip (an eighth each, as order-preserving 32-bit keys), finds the exact k-th largest key
-// by a radix select over four 8-bit digits whose per-pass histograms are summed across the
-// cluster through distributed shared memory, gathers the selected entries into one CTA in
-// index order (ties at the threshold go to the smallest indices) and sorts them there.
+// chip (an eighth each, as order-preserving 32-bit keys) and finds the exact k-th largest
+// key by a radix select over four 8-bit digits; every CTA pushes its per-digit histogram
+// into the others' shared memory (st.async on mbarriers, no cluster-wide barrier per
+// digit).  The selected entries (ties at the threshold to the smallest indices) are pushed
+// in index order into every CTA's copy of the list, and each CTA places its share of the
+// list by counting, for each entry, the entries that sort before it: no sort.
 #include "kvc_common.cuh"
 #include "kvc_host.h"
 #include "kvc_launch.h"
@@ -368,8 +370,22 @@ constexpr int kSlice = 40960;    // scores held on chip per CTA
 constexpr int kMaxK = 2048;
 constexpr int kBins = 256;       // radix digits of 8 bits
 constexpr int kWarps = kTkThreads / 32;
-constexpr size_t kTkSmem =
-    kSlice * 4 + (kWarps + 1) * kBins * 4 + kMaxK * 8 + kTkThreads * 4 + 64 + 2 * kWarps * 4 + 128;
+constexpr int kCandCap = 64;     // candidate positions a warp keeps after the second digit
+constexpr int kRankChunks = kTkThreads / 128;  // the selected list is ranked in 8 chunks
+constexpr int kMaxShare = kMaxK / kCluster;    // list entries one CTA ranks and stores
+// Shared memory (bytes).  The histogram region holds the selected list once the four
+// digits are known; the receive region holds the rank sums.
+constexpr size_t kTkKeys = 0;                                            // u32 [kSlice]
+constexpr size_t kTkHist = kTkKeys + size_t(kSlice) * 4;                 // u32 [kWarps][kBins]
+constexpr size_t kTkRecv = kTkHist + size_t(kWarps) * kBins * 4;         // u32 [2][CL][kBins]
+constexpr size_t kTkCand = kTkRecv + 2 * size_t(kCluster) * kBins * 4;   // u16 [kWarps][cap]
+constexpr size_t kTkBars = kTkCand + size_t(kWarps) * kCandCap * 2;      // 4 mbarriers
+constexpr size_t kTkMisc = kTkBars + 4 * 8;
+// info [CL][2], wcnt [2][kWarps], wsum [8], per-pass digit and rank [4][2], abort flag
+constexpr size_t kTkSmem = kTkMisc + size_t(2 * kCluster + 2 * kWarps + 8 + 8 + 4) * 4;
+static_assert(kMaxK + 256 + kMaxShare <= kWarps * kBins, "selected list fits the histograms");
+static_assert(kMaxShare <= 2 * kCluster * kBins, "rank sums fit the receive buffers");
+static_assert(kTkSmem <= 227 * 1024, "top-k shared memory");
 
 struct TopkArgs {
   const float* scores;
@@ -389,66 +405,109 @@ __device__ __forceinline__ float key_value(uint32_t u) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long v) {
-  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t cluster_addr_of(const void* p, uint32_t rank) {
+// The same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
   uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+// A 4- or 8-byte store into a peer CTA's shared memory that counts its bytes on the mbarrier
+// `bar` of that CTA (both addresses from peer_addr).
+__device__ __forceinline__ void push_u32(uint32_t addr, uint32_t v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(addr),
+               "r"(v), "r"(bar)
+               : "memory");
 }
-
-// Exclusive prefix sum of v over the block's threads in thread order; total in *total.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* scratch,
-                                                         uint32_t* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+__device__ __forceinline__ void push_v2(uint32_t addr, uint32_t v0, uint32_t v1, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.u32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+      "r"(v0), "r"(v1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ bool try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __noinline__ bool tk_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(&g_indexer_error, 1u);
+      return false;
+    }
+  }
+}
+// Bounded wait for the pushes of the other CTAs (acquire at cluster scope).
+__device__ __forceinline__ bool tk_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (try_wait_cluster(bar, parity)) return true;
+  return tk_wait_slow(bar, parity, abort_flag);
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
   }
-  if (lane == 31) scratch[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t s = lane < kTkThreads / 32 ? scratch[lane] : 0u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < kTkThreads / 32) scratch[lane] = s;  // inclusive over warps
-  }
-  __syncthreads();
-  const uint32_t before = (warp > 0 ? scratch[warp - 1] : 0u) + x - v;
-  *total = scratch[kTkThreads / 32 - 1];
-  __syncthreads();  // scratch is reused by the next scan
-  return before;
+  return v;
 }
 
+// One cluster of CL CTAs per query row; CTA r holds candidates [r * per, r * per + cnt) as
+// order keys, warp w of it the contiguous segment [w * seg, (w + 1) * seg) of those.
+//  1. Radix select of the ksel-th largest key over four 8-bit digits, high to low.  Each
+//     warp counts its segment into its own histogram (the first digit while the scores
+//     load); 256 threads sum the CTA's warps and push the sums into every CTA of the
+//     cluster (st.async, counted on an mbarrier per buffer, two buffers alternating), so
+//     every CTA picks the same digit with no cluster-wide barrier.  After the second digit
+//     a warp that holds at most kCandCap keys at or above the 16-bit prefix keeps their
+//     positions, and the last digit and the selection read those alone.
+//  2. The copies of the threshold that are taken go to the lowest indices (CTAs, then
+//     warps, in index order, from the counts every CTA pushes); each CTA pushes its
+//     selected keys, in index order, to their place in every CTA's copy of the list, and
+//     each entry's index to the CTA that will store it.
+//  3. Every CTA ranks its share of the list: the entry at list position e goes to output
+//     place #{keys above it} + #{equal keys before it in the list}, counted in 8 chunks by
+//     1024 threads.  The list is in index order, so equal scores come out by index.
 template <int CL>
 __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                      // [kSlice]
-  uint32_t* hist = keys + kSlice;                                  // [kWarps][kBins]
-  uint32_t* chist = hist + kWarps * kBins;                         // [kBins] the CTA's sum
-  unsigned long long* cand = reinterpret_cast<unsigned long long*>(chist + kBins);  // [kMaxK]
-  uint32_t* scratch = reinterpret_cast<uint32_t*>(cand + kMaxK);          // [kTkThreads]
-  uint32_t* info = scratch + kTkThreads;                                   // [16]
-  uint32_t* wcnt = info + 16;                                              // [2][kWarps]
-  uint32_t* runs = wcnt + 2 * kWarps;                                      // [2][16]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + kTkKeys);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + kTkHist);
+  uint32_t* recv = reinterpret_cast<uint32_t*>(smem + kTkRecv);
+  uint16_t* cand = reinterpret_cast<uint16_t*>(smem + kTkCand);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTkBars);  // [0,1] digits, [2] counts, [3] list
+  uint32_t* info = reinterpret_cast<uint32_t*>(smem + kTkMisc);  // [CL][2] above / at, per CTA
+  uint32_t* wcnt = info + 2 * CL;                                 // [2][kWarps]
+  uint32_t* wsum = wcnt + 2 * kWarps;                             // [8]
+  uint32_t* slot = wsum + 8;                                      // [4][2] digit, rank left
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(slot + 8);
+  uint32_t* list_key = hist;                   // [kMaxK + 4] selected keys, in index order
+  uint32_t* list_idx = hist + kMaxK + 256;     // [kMaxShare] indices of this CTA's share
+  uint32_t* rank_acc = recv;                   // [kMaxShare]
 
   const uint32_t rank = blockIdx.x % CL;
   const int64_t t = blockIdx.x / CL;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t nv = a.n_visible[t];
   // the same decision in every CTA of the cluster: an out-of-range row is skipped whole
   if (nv < 0 || nv > a.max_visible) {
@@ -457,272 +516,293 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
   }
   const int k = a.k;
   const int ksel = static_cast<int>(nv < k ? nv : k);
-  // this CTA's candidates [lo, lo + cnt), a multiple of 4 apart
+  if (ksel == 0) {  // no candidates: padding only, no exchange
+    for (int e = static_cast<int>(rank) * kTkThreads + tid; e < k; e += CL * kTkThreads) {
+      a.out_idx[t * k + e] = -1;
+      if (a.out_score) a.out_score[t * k + e] = -INFINITY;
+    }
+    return;
+  }
+  // list positions [my0, my1) are ranked and stored here
+  const int q = (ksel + CL - 1) / CL;
+  const int my0 = min(ksel, static_cast<int>(rank) * q), my1 = min(ksel, my0 + q);
+  if (tid == 0) {
+    *abort_flag = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    mbar_arrive_expect_tx(&bars[0], CL * kBins * 4);
+    mbar_arrive_expect_tx(&bars[1], CL * kBins * 4);
+    mbar_arrive_expect_tx(&bars[2], CL * 8);
+    mbar_arrive_expect_tx(&bars[3], static_cast<uint32_t>(ksel + (my1 - my0)) * 4);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // this CTA's candidates [lo, lo + cnt), a multiple of 4 apart; warp segments of 32s
   const int64_t per = ((nv + CL - 1) / CL + 3) & ~int64_t(3);
   const int64_t lo = rank * per;
   const int cnt = static_cast<int>(lo < nv ? (nv - lo < per ? nv - lo : per) : 0);
-  const float* row = a.scores + t * a.ld;
+  const int seg = ((cnt + kWarps - 1) / kWarps + 31) & ~31;
+  const int s0 = min(cnt, warp * seg), s1 = min(cnt, s0 + seg);
+  uint32_t* whist = hist + warp * kBins;
+  uint16_t* wcand = cand + warp * kCandCap;
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  reinterpret_cast<uint4*>(whist)[lane] = zero4;
+  reinterpret_cast<uint4*>(whist)[lane + 32] = zero4;
+  __syncwarp();
+  cluster_arrive_relaxed();  // the barriers are initialised before any CTA pushes
 
-  if (ksel > 0) {
-    // four 16-byte loads in flight per thread
-    constexpr int kStep = kTkThreads * 4;
-    for (int i0 = tid * 4; i0 < cnt; i0 += 4 * kStep) {
-      float4 f[4];
+  // load the segment as order keys, counting the first digit on the way
+  const float* row = a.scores + t * a.ld + lo;
+  for (int i0 = s0 + 4 * lane; i0 < s1; i0 += 4 * 128) {
+    float4 f[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = i0 + r * kStep;
-        if (i + 3 < cnt) f[r] = *reinterpret_cast<const float4*>(row + lo + i);
-      }
+    for (int r = 0; r < 4; ++r) {
+      const int i = i0 + 128 * r;
+      if (i + 3 < s1) f[r] = __ldg(reinterpret_cast<const float4*>(row + i));
+    }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = i0 + r * kStep;
-        if (i + 3 < cnt) {
-          keys[i] = order_key(f[r].x);
-          keys[i + 1] = order_key(f[r].y);
-          keys[i + 2] = order_key(f[r].z);
-          keys[i + 3] = order_key(f[r].w);
-        } else {
-          for (int e = i; e < cnt; ++e) keys[e] = order_key(row[lo + e]);
+    for (int r = 0; r < 4; ++r) {
+      const int i = i0 + 128 * r;
+      if (i + 3 < s1) {
+        const uint4 u = make_uint4(order_key(f[r].x), order_key(f[r].y), order_key(f[r].z),
+                                   order_key(f[r].w));
+        *reinterpret_cast<uint4*>(keys + i) = u;
+        atomicAdd(&whist[u.x >> 24], 1u);
+        atomicAdd(&whist[u.y >> 24], 1u);
+        atomicAdd(&whist[u.z >> 24], 1u);
+        atomicAdd(&whist[u.w >> 24], 1u);
+      } else {
+        for (int e = i; e < s1; ++e) {
+          const uint32_t u = order_key(row[e]);
+          keys[e] = u;
+          atomicAdd(&whist[u >> 24], 1u);
         }
       }
     }
-    // radix select of the ksel-th largest key: four 8-bit digits, high to low.  Each warp
-    // counts into its own histogram (the keys of a query share few leading bits, so one
-    // shared histogram would serialise all warps on a handful of bins), the CTA sums its
-    // warps', and every CTA sums the cluster's CTA histograms through distributed shared
-    // memory.
-    const int warp = tid >> 5, lane = tid & 31;
-    uint32_t* whist = hist + warp * kBins;
-    // Warp w owns candidates [w * seg, (w + 1) * seg) in every pass below, its lanes on
-    // consecutive keys (no bank conflicts), so its histogram also gives its own counts of
-    // keys above and at the final threshold.
-    const int seg = ((cnt + kWarps - 1) / kWarps + 31) & ~31;
-    const int s0 = warp * seg;
-    const int s1 = s0 + seg < cnt ? s0 + seg : cnt;
-    uint32_t wgt = 0;  // keys of the segment above the threshold (summed over the passes)
-    uint32_t prefix = 0, mask = 0;
-    uint32_t kk = static_cast<uint32_t>(ksel);  // rank of the wanted key among the matches
+  }
+  __syncthreads();
+  cluster_wait();
+
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t prefix = 0, mask = 0;
+  uint32_t kk = static_cast<uint32_t>(ksel);  // rank of the wanted key among the matches
+  uint32_t wgt = 0, weq = 0;  // keys of the segment above / at the threshold
+  int ncand = 0;
+  bool use_cand = false;
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int b = tid; b < kWarps * kBins; b += kTkThreads) hist[b] = 0u;
-      __syncthreads();
-      // four loads in flight per thread; lanes of a warp that hit the same bin are
-      // serialised by the shared-memory atomics (measured cheaper than aggregating them
-      // with __match_any_sync first)
-      for (int i0 = s0 + lane; i0 < s1; i0 += 128) {
-        uint32_t u[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = i0 + 32 * r;
-          u[r] = i < s1 ? keys[i] : 0u;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const int b = pass & 1;
+    if (pass > 0) {
+      if (pass == 3 && use_cand) {
+        for (int c = lane; c < ncand; c += 32) {
+          const uint32_t u = keys[wcand[c]];
+          if ((u & mask) == prefix) atomicAdd(&whist[u & 0xFFu], 1u);
         }
+      } else {
+        // four loads in flight per thread; lanes of a warp that hit the same bin are
+        // serialised by the shared-memory atomics
+        const bool compact = pass == 2 && use_cand;
+        int n = 0;
+        for (int g0 = s0; g0 < s1; g0 += 128) {  // warp-uniform trip count (ballots)
+          uint32_t u[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = i0 + 32 * r;
-          if (i < s1 && (u[r] & mask) == prefix)
-            atomicAdd(&whist[(u[r] >> shift) & (kBins - 1)], 1u);
+          for (int r = 0; r < 4; ++r) {
+            const int i = g0 + 32 * r + lane;
+            u[r] = i < s1 ? keys[i] : 0u;
+          }
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int i = g0 + 32 * r + lane;
+            const bool in = i < s1;
+            if (in && (u[r] & mask) == prefix) atomicAdd(&whist[(u[r] >> shift) & 0xFFu], 1u);
+            if (compact) {  // every key at or above the 16-bit prefix, in index order
+              const bool c = in && u[r] >= prefix;
+              const uint32_t cb = __ballot_sync(0xffffffffu, c);
+              const int at = n + __popc(cb & lt);
+              if (c && at < kCandCap) wcand[at] = static_cast<uint16_t>(i);
+              n += __popc(cb);
+            }
+          }
         }
       }
       __syncthreads();
-      if (tid < kBins) {
-        uint32_t sum = 0;
+    }
+    if (tid < kBins) {
+      // the CTA's count of bin tid, pushed into every CTA's buffer b
+      uint32_t s = 0;
+#pragma unroll 8
+      for (int w = 0; w < kWarps; ++w) s += hist[w * kBins + tid];
+      const uint32_t dst = smem_u32(recv + (b * CL + rank) * kBins + tid);
+      const uint32_t bar = smem_u32(&bars[b]);
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) sum += hist[w * kBins + tid];
-        chist[tid] = sum;
-      }
-      cluster_sync();  // every CTA's histogram is complete
-      // thread tid < 256 takes bin 255 - tid over the cluster, so a thread-order scan
-      // counts the keys in higher bins
+      for (int r = 0; r < CL; ++r) push_u32(peer_addr(dst, r), s, peer_addr(bar, r));
+      tk_wait(&bars[b], (pass >> 1) & 1, abort_flag);
+      if (tid == 0 && pass < 2) mbar_arrive_expect_tx(&bars[b], CL * kBins * 4);  // pass + 2
+      // thread tid takes bin 255 - tid over the cluster, so a thread-order scan counts the
+      // keys in higher bins
       uint32_t tot = 0;
-      if (tid < kBins) {
-        uint32_t rv[CL];
+      const uint32_t* rb = recv + b * CL * kBins + (kBins - 1 - tid);
 #pragma unroll
-        for (int r = 0; r < CL; ++r)  // all remote loads in flight before any use
-          rv[r] = ld_cluster_u32(cluster_addr_of(chist + (kBins - 1 - tid), static_cast<uint32_t>(r)));
-#pragma unroll
-        for (int r = 0; r < CL; ++r) tot += rv[r];
-      }
-      uint32_t all;
-      const uint32_t above = block_exclusive_scan(tot, scratch, &all);
+      for (int r = 0; r < CL; ++r) tot += rb[r * kBins];
+      const uint32_t incl = warp_inclusive_scan(tot, lane);
+      if (lane == 31) wsum[warp] = incl;
+      asm volatile("bar.sync 1, %0;" ::"n"(kBins) : "memory");
+      uint32_t above = incl - tot;
+      for (int w = 0; w < warp; ++w) above += wsum[w];
       if (tot > 0 && above < kk && kk <= above + tot) {
-        info[0] = static_cast<uint32_t>(kBins - 1 - tid);
-        info[1] = kk - above;
+        slot[2 * pass] = static_cast<uint32_t>(kBins - 1 - tid);
+        slot[2 * pass + 1] = kk - above;
       }
-      __syncthreads();
-      const uint32_t digit = info[0];
-      {  // this warp's keys above the chosen digit (they all sort above the threshold)
-        uint32_t c = 0;
-        for (int b = static_cast<int>(digit) + 1 + lane; b < kBins; b += 32) c += whist[b];
+    }
+    __syncthreads();
+    const uint32_t digit = slot[2 * pass] & 0xFFu;
+    {  // this warp's keys above the chosen digit (they all sort above the threshold)
+      uint32_t c = 0;
+      for (int bin = static_cast<int>(digit) + 1 + lane; bin < kBins; bin += 32) c += whist[bin];
+      wgt += warp_sum(c);
+    }
+    if (pass == 1) {
+      ncand = static_cast<int>(wgt + whist[digit]);
+      use_cand = ncand <= kCandCap;
+    }
+    if (pass == 3) weq = whist[digit];
+    prefix |= digit << shift;
+    mask |= 0xFFu << shift;
+    kk = slot[2 * pass + 1];
+    if (pass < 3) {
+      __syncwarp();
+      reinterpret_cast<uint4*>(whist)[lane] = zero4;
+      reinterpret_cast<uint4*>(whist)[lane + 32] = zero4;
+      __syncwarp();
+    }
+  }
+  const uint32_t thr = prefix;  // the ksel-th largest key; kk of its copies are taken
+  if (lane == 0) {
+    wcnt[warp] = wgt;
+    wcnt[kWarps + warp] = weq;
+  }
+  __syncthreads();  // every warp is done with its histogram: it may now hold the list
+  if (warp == 0) {
+    const uint32_t g = warp_sum(wcnt[lane]), e = warp_sum(wcnt[kWarps + lane]);
+    if (lane < CL)
+      push_v2(peer_addr(smem_u32(info + 2 * rank), lane), g, e, peer_addr(smem_u32(&bars[2]), lane));
+  }
+  if (tid < 4) list_key[ksel + tid] = 0u;  // below every key: the rank loads read up to 3 past
+  for (int s = tid; s < kMaxShare; s += kTkThreads) rank_acc[s] = 0u;
+  tk_wait(&bars[2], 0, abort_flag);
+  // the copies of the threshold go to the lowest indices: CTAs, then warps, in order
+  uint32_t base = 0, take = 0, eq_before = 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-        wgt += c;
-      }
-      if (pass == 3 && lane == 0) {  // the warp's counts above and at the threshold
-        wcnt[warp] = wgt;
-        wcnt[kWarps + warp] = whist[digit];
-      }
-      prefix |= digit << shift;
-      mask |= static_cast<uint32_t>(kBins - 1) << shift;
-      kk = info[1];
-      cluster_sync();  // remote reads are done before the next pass rewrites the histograms
+  for (int r = 0; r < CL; ++r) {
+    const uint32_t g = info[2 * r], e = info[2 * r + 1];
+    const uint32_t tk = kk > eq_before ? min(kk - eq_before, e) : 0u;
+    if (r < static_cast<int>(rank)) base += g + tk;
+    if (r == static_cast<int>(rank)) take = tk;
+    eq_before += e;
+  }
+  uint32_t wpos, wtake;
+  {  // lane l stands for warp l: its first list position and its copies of the threshold
+    const uint32_t gl = wcnt[lane], el = wcnt[kWarps + lane];
+    const uint32_t eb = warp_inclusive_scan(el, lane) - el;
+    const uint32_t tkl = take > eb ? min(take - eb, el) : 0u;
+    const uint32_t pl = warp_inclusive_scan(gl + tkl, lane) - (gl + tkl);
+    wpos = __shfl_sync(0xffffffffu, pl, warp);
+    wtake = __shfl_sync(0xffffffffu, tkl, warp);
+  }
+  // push the selected entries, in index order, to list position P: the key to every CTA,
+  // the index to the CTA whose share holds P
+  uint32_t P = base + wpos, er = 0;
+  const uint32_t key_dst = smem_u32(list_key), idx_dst = smem_u32(list_idx);
+  const uint32_t list_bar = smem_u32(&bars[3]);
+  auto push_entry = [&](uint32_t pos, uint32_t u, uint32_t index) {
+    if (pos >= static_cast<uint32_t>(ksel)) return;  // only with a wait that gave up
+#pragma unroll
+    for (int r = 0; r < CL; ++r) push_u32(peer_addr(key_dst + 4 * pos, r), u, peer_addr(list_bar, r));
+    const uint32_t owner = pos / static_cast<uint32_t>(q);
+    push_u32(peer_addr(idx_dst + 4 * (pos - owner * q), owner), index, peer_addr(list_bar, owner));
+  };
+  if (use_cand) {
+    for (int c0 = 0; c0 < ncand; c0 += 32) {
+      const int c = c0 + lane;
+      const bool in = c < ncand;
+      const int i = in ? wcand[c] : 0;
+      const uint32_t u = in ? keys[i] : 0u;
+      const uint32_t eb = __ballot_sync(0xffffffffu, in && u == thr);
+      const bool sel = in && (u > thr || (u == thr && er + __popc(eb & lt) < wtake));
+      const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) push_entry(P + __popc(sb & lt), u, static_cast<uint32_t>(lo + i));
+      P += __popc(sb);
+      er += __popc(eb);
     }
-    const uint32_t thr = prefix;  // the ksel-th largest key; kk of its copies are taken
-    const uint32_t lt = (1u << lane) - 1u;
-    __syncthreads();  // every warp's counts are in wcnt
-    if (tid == 0) {
-      uint32_t g = 0, e = 0;
-      for (int w = 0; w < kWarps; ++w) {
-        g += wcnt[w];
-        e += wcnt[kWarps + w];
-      }
-      info[2] = g;
-      info[3] = e;
-    }
-    cluster_sync();
-    // the copies of the threshold go to the lowest indices: CTAs, then warps, in order
-    uint32_t base = 0, take = 0, eq_before = 0, run_base = 0;
-    for (uint32_t r = 0; r < CL; ++r) {
-      const uint32_t g = ld_cluster_u32(cluster_addr_of(info + 2, r));
-      const uint32_t e = ld_cluster_u32(cluster_addr_of(info + 3, r));
-      const uint32_t tk = kk > eq_before ? (kk - eq_before < e ? kk - eq_before : e) : 0u;
-      if (r < rank) base += g + tk;
-      if (r == rank) take = tk;
-      if (tid == 0) {  // every CTA's run of selected entries: [base, base + length)
-        runs[2 * r] = run_base;
-        runs[2 * r + 1] = g + tk;
-      }
-      run_base += g + tk;
-      eq_before += e;
-    }
-    uint32_t pos = base, wtake = 0, web = 0;
-    for (int w = 0; w <= warp; ++w) {
-      const uint32_t e = wcnt[kWarps + w];
-      const uint32_t tk = take > web ? (take - web < e ? take - web : e) : 0u;
-      if (w < warp) pos += wcnt[w] + tk;
-      else wtake = tk;
-      web += e;
-    }
-    // write the selected entries in index order into this CTA's run buffer
-    pos -= base;
-    uint32_t er = 0;  // threshold copies of this warp already passed
-    for (int i0 = s0; i0 < s1; i0 += 128) {
+  } else {
+    for (int g0 = s0; g0 < s1; g0 += 128) {
       uint32_t u[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const int i = i0 + 32 * r + lane;
+        const int i = g0 + 32 * r + lane;
         u[r] = i < s1 ? keys[i] : 0u;
       }
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const int i = i0 + 32 * r + lane;
+        const int i = g0 + 32 * r + lane;
         const bool in = i < s1;
         if (!__any_sync(0xffffffffu, in && u[r] >= thr)) continue;  // most groups
         const uint32_t eb = __ballot_sync(0xffffffffu, in && u[r] == thr);
         const bool sel = in && (u[r] > thr || (u[r] == thr && er + __popc(eb & lt) < wtake));
         const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-        if (sel) {
-          const uint32_t index = static_cast<uint32_t>(lo + i);
-          cand[pos + __popc(sb & lt)] =
-              (static_cast<unsigned long long>(u[r]) << 32) | (0xFFFFFFFFu - index);
-        }
-        pos += __popc(sb);
+        if (sel) push_entry(P + __popc(sb & lt), u[r], static_cast<uint32_t>(lo + i));
+        P += __popc(sb);
         er += __popc(eb);
       }
     }
   }
+  cluster_arrive_relaxed();  // no CTA leaves before every CTA is done with the others' memory
+  tk_wait(&bars[3], 0, abort_flag);
   __syncthreads();
-  // Each CTA sorts its own run descending (key, then smaller index first): a bitonic
-  // network over P = 2^ceil(log2 n) entries in registers, element e = r * 1024 + tid in
-  // x[r]; strides up to 16 are lane exchanges, 32..512 go through shared memory, 1024 is
-  // between a thread's two registers.  Threads past n hold 0, below every real entry, and
-  // only ever pair with each other.
-  const int nsel = ksel > 0 ? static_cast<int>(runs[2 * rank + 1]) : 0;
-  int P = 1;
-  while (P < nsel) P <<= 1;
-  const int E = P > kTkThreads ? 2 : 1;
-  unsigned long long x[2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int e = r * kTkThreads + tid;
-    x[r] = (r < E && e < nsel) ? cand[e] : 0ull;
-  }
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= kTkThreads) {  // E == 2: the thread's own two registers
-        const bool desc = (tid & size) == 0;
-        const unsigned long long hi = x[0] > x[1] ? x[0] : x[1], lo2 = x[0] > x[1] ? x[1] : x[0];
-        x[0] = desc ? hi : lo2;
-        x[1] = desc ? lo2 : hi;
+  // rank: chunk ch of the list against entries my0 + j, my0 + 128 + j
+  {
+    const int ch = tid >> 7, j = tid & 127;
+    const int L = ((ksel + kRankChunks - 1) / kRankChunks + 3) & ~3;
+    const int c0 = min(ksel, ch * L), c1 = min(ksel, c0 + L);
+    for (int e0 = my0; e0 < my1; e0 += 128) {
+      const int e = e0 + j;
+      if (e >= my1 || c0 >= c1) continue;
+      const uint32_t ke = list_key[e];
+      uint32_t n = 0;
+      if (c1 <= e) {  // the whole chunk lies before e: equal keys sort before it
+        for (int o = c0; o < c1; o += 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(list_key + o);
+          n += (v.x >= ke) + (v.y >= ke) + (v.z >= ke) + (v.w >= ke);
+        }
+      } else if (c0 > e) {  // the whole chunk lies after e (and the zero padding past it)
+        for (int o = c0; o < c1; o += 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(list_key + o);
+          n += (v.x > ke) + (v.y > ke) + (v.z > ke) + (v.w > ke);
+        }
       } else {
-        unsigned long long y[2];
-        if (stride >= 32) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r)
-            if (r < E) cand[r * kTkThreads + tid] = x[r];
-          __syncthreads();
-#pragma unroll
-          for (int r = 0; r < 2; ++r)
-            if (r < E) y[r] = cand[(r * kTkThreads + tid) ^ stride];
-          __syncthreads();
-        } else {
-          // a warp whose entries are all padding (past P) has nothing to exchange
-          if (E == 1 && (tid & ~31) >= P) continue;
-#pragma unroll
-          for (int r = 0; r < 2; ++r) y[r] = __shfl_xor_sync(0xffffffffu, x[r], stride);
-        }
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          if (r < E) {
-            const int e = r * kTkThreads + tid;
-            const bool lower = (e & stride) == 0, desc = (e & size) == 0;
-            const unsigned long long hi = x[r] > y[r] ? x[r] : y[r];
-            const unsigned long long lo2 = x[r] > y[r] ? y[r] : x[r];
-            x[r] = (desc == lower) ? hi : lo2;
-          }
+        for (int o = c0; o < c1; o += 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(list_key + o);
+          n += (o < e ? v.x >= ke : v.x > ke) + (o + 1 < e ? v.y >= ke : v.y > ke) +
+               (o + 2 < e ? v.z >= ke : v.z > ke) + (o + 3 < e ? v.w >= ke : v.w > ke);
         }
       }
+      atomicAdd(&rank_acc[e - my0], n);
     }
   }
-  // the sorted runs go to CTA 0, in its key space (free once every CTA is past this sync)
-  cluster_sync();
-  unsigned long long* merged = reinterpret_cast<unsigned long long*>(keys);  // [ksel], CTA 0
-  if (nsel > 0) {
-    const uint32_t mbase = cluster_addr_of(merged, 0) + 8u * runs[2 * rank];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int e = r * kTkThreads + tid;
-      if (r < E && e < nsel) st_cluster_u64(mbase + 8u * e, x[r]);
+  __syncthreads();
+  if (!*abort_flag) {
+    for (int s = tid; s < my1 - my0; s += kTkThreads) {
+      const uint32_t place = rank_acc[s];
+      if (place >= static_cast<uint32_t>(ksel)) continue;  // only with a wait that gave up
+      a.out_idx[t * k + place] = static_cast<int32_t>(list_idx[s]);
+      if (a.out_score) a.out_score[t * k + place] = key_value(list_key[my0 + s]);
     }
   }
-  cluster_sync();
-  if (rank != 0) return;
-  // CTA 0: each entry's place is its position in its run plus, for every other run, the
-  // number of entries there that sort before it (binary search; the entries are distinct)
-  for (int e = tid; e < ksel; e += kTkThreads) {
-    int r0 = 0;
-    while (r0 + 1 < CL && static_cast<uint32_t>(e) >= runs[2 * (r0 + 1)]) ++r0;
-    const unsigned long long v = merged[e];
-    uint32_t place = static_cast<uint32_t>(e) - runs[2 * r0];
-    for (int r = 0; r < CL; ++r) {
-      if (r == r0) continue;
-      const unsigned long long* run = merged + runs[2 * r];
-      int lo_ = 0, hi_ = static_cast<int>(runs[2 * r + 1]);
-      while (lo_ < hi_) {
-        const int mid = (lo_ + hi_) >> 1;
-        if (run[mid] > v) lo_ = mid + 1;
-        else hi_ = mid;
-      }
-      place += static_cast<uint32_t>(lo_);
-    }
-    a.out_idx[t * k + place] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(v));
-    if (a.out_score) a.out_score[t * k + place] = key_value(static_cast<uint32_t>(v >> 32));
-  }
-  for (int e = ksel + tid; e < k; e += kTkThreads) {  // fewer candidates than k: padding
-    a.out_idx[t * k + e] = -1;
+  for (int e = ksel + static_cast<int>(rank) * kTkThreads + tid; e < k; e += CL * kTkThreads) {
+    a.out_idx[t * k + e] = -1;  // fewer candidates than k: padding
     if (a.out_score) a.out_score[t * k + e] = -INFINITY;
   }
+  cluster_wait();
 }
 
 }  // namespace idx

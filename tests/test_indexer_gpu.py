@@ -83,7 +83,7 @@ def _topk_gpu(scores, nv, k, max_visible):
 
 
 @pytest.mark.parametrize("k", [1, 7, 512, 1024, 2048])
-@pytest.mark.parametrize("kind", ["ties", "continuous"])
+@pytest.mark.parametrize("kind", ["ties", "continuous", "sorted"])
 def test_topk_exact_given_scores(k, kind):
     rng = np.random.default_rng(k + len(kind))
     nv = [0, 1, 5, 1000, 4099, 100003, 327680]
@@ -95,6 +95,8 @@ def test_topk_exact_given_scores(k, kind):
             v[rng.random(n) < 0.5] = 0.0
         else:
             v = rng.standard_normal(n).astype(np.float32)
+        if kind == "sorted":  # the largest scores crowd into the last warps of the last CTA
+            v = np.sort(v)
         S[i, :n] = v
     idx, val = _topk_gpu(torch.from_numpy(S).cuda(), nv, k, ld)
     assert kvc.device_status() == kvc.KVC_OK
