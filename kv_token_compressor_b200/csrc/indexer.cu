@@ -371,8 +371,15 @@ constexpr int kMaxK = 2048;
 constexpr int kBins = 256;       // radix digits of 8 bits
 constexpr int kWarps = kTkThreads / 32;
 constexpr int kCandCap = 64;     // candidate positions a warp keeps after the second digit
-constexpr int kRankChunks = kTkThreads / 128;  // the selected list is ranked in 8 chunks
+constexpr int kRankChunks = kTkThreads / 128;  // threads that share one entry's rank
 constexpr int kMaxShare = kMaxK / kCluster;    // list entries one CTA ranks and stores
+constexpr int kRankBins = 256;                 // bins of key - threshold for the rank
+// u32 offsets in the histogram region once it holds the list: keys [kMaxK + 4], this CTA's
+// indices [kMaxShare], then the rank's bin starts, keys by bin and list positions by bin
+constexpr int kListIdx = kMaxK + 256;
+constexpr int kListAbove = kListIdx + kMaxShare;
+constexpr int kListBKey = kListAbove + kRankBins;
+constexpr int kListBPos = kListBKey + kMaxK;
 // Shared memory (bytes).  The histogram region holds the selected list once the four
 // digits are known; the receive region holds the rank sums.
 constexpr size_t kTkKeys = 0;                                            // u32 [kSlice]
@@ -383,8 +390,9 @@ constexpr size_t kTkBars = kTkCand + size_t(kWarps) * kCandCap * 2;      // 4 mb
 constexpr size_t kTkMisc = kTkBars + 4 * 8;
 // info [CL][2], wcnt [2][kWarps], wsum [8], per-pass digit and rank [4][2], abort flag
 constexpr size_t kTkSmem = kTkMisc + size_t(2 * kCluster + 2 * kWarps + 8 + 8 + 4) * 4;
-static_assert(kMaxK + 256 + kMaxShare <= kWarps * kBins, "selected list fits the histograms");
-static_assert(kMaxShare <= 2 * kCluster * kBins, "rank sums fit the receive buffers");
+static_assert(kListBPos + kMaxK / 2 <= kWarps * kBins, "selected list fits the histograms");
+static_assert(kMaxShare + kRankBins <= 2 * kCluster * kBins, "rank sums fit the receive buffers");
+static_assert(kRankBins == 256, "the rank's bin shift and scan assume 8-bit bins");
 static_assert(kTkSmem <= 227 * 1024, "top-k shared memory");
 
 struct TopkArgs {
@@ -502,7 +510,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
   uint32_t* slot = wsum + 8;                                      // [4][2] digit, rank left
   volatile int* abort_flag = reinterpret_cast<volatile int*>(slot + 8);
   uint32_t* list_key = hist;                   // [kMaxK + 4] selected keys, in index order
-  uint32_t* list_idx = hist + kMaxK + 256;     // [kMaxShare] indices of this CTA's share
+  uint32_t* list_idx = hist + kListIdx;        // [kMaxShare] indices of this CTA's share
   uint32_t* rank_acc = recv;                   // [kMaxShare]
 
   const uint32_t rank = blockIdx.x % CL;
@@ -585,7 +593,6 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
   const uint32_t lt = (1u << lane) - 1u;
   uint32_t prefix = 0, mask = 0;
   uint32_t kk = static_cast<uint32_t>(ksel);  // rank of the wanted key among the matches
-  uint32_t wgt = 0, weq = 0;  // keys of the segment above / at the threshold
   int ncand = 0;
   bool use_cand = false;
 #pragma unroll 1
@@ -598,10 +605,9 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
           const uint32_t u = keys[wcand[c]];
           if ((u & mask) == prefix) atomicAdd(&whist[u & 0xFFu], 1u);
         }
-      } else {
-        // four loads in flight per thread; lanes of a warp that hit the same bin are
-        // serialised by the shared-memory atomics
-        const bool compact = pass == 2 && use_cand;
+      } else if (pass == 2) {
+        // count, and keep every key at or above the 16-bit prefix, in index order, while
+        // they fit
         int n = 0;
         for (int g0 = s0; g0 < s1; g0 += 128) {  // warp-uniform trip count (ballots)
           uint32_t u[4];
@@ -613,16 +619,33 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int i = g0 + 32 * r + lane;
-            const bool in = i < s1;
-            if (in && (u[r] & mask) == prefix) atomicAdd(&whist[(u[r] >> shift) & 0xFFu], 1u);
-            if (compact) {  // every key at or above the 16-bit prefix, in index order
-              const bool c = in && u[r] >= prefix;
-              const uint32_t cb = __ballot_sync(0xffffffffu, c);
+            const bool c = i < s1 && u[r] >= prefix;
+            const uint32_t cb = __ballot_sync(0xffffffffu, c);
+            if (c) {
               const int at = n + __popc(cb & lt);
-              if (c && at < kCandCap) wcand[at] = static_cast<uint16_t>(i);
-              n += __popc(cb);
+              if (at < kCandCap) wcand[at] = static_cast<uint16_t>(i);
+              if ((u[r] & mask) == prefix) atomicAdd(&whist[(u[r] >> shift) & 0xFFu], 1u);
             }
+            n += __popc(cb);
           }
+        }
+        ncand = n;
+        use_cand = n <= kCandCap;
+      } else {
+        // 16-byte loads (segments start on multiples of 32 keys), two in flight per thread;
+        // lanes of a warp that hit the same bin are serialised by the shared-memory atomics
+        auto count4 = [&](uint4 v, int i) {
+          if (i < s1 && (v.x & mask) == prefix) atomicAdd(&whist[(v.x >> shift) & 0xFFu], 1u);
+          if (i + 1 < s1 && (v.y & mask) == prefix) atomicAdd(&whist[(v.y >> shift) & 0xFFu], 1u);
+          if (i + 2 < s1 && (v.z & mask) == prefix) atomicAdd(&whist[(v.z >> shift) & 0xFFu], 1u);
+          if (i + 3 < s1 && (v.w & mask) == prefix) atomicAdd(&whist[(v.w >> shift) & 0xFFu], 1u);
+        };
+        for (int i0 = s0 + 4 * lane; i0 < s1; i0 += 256) {
+          const int i1 = i0 + 128;
+          const uint4 v0 = *reinterpret_cast<const uint4*>(keys + i0);
+          const uint4 v1 = i1 < s1 ? *reinterpret_cast<const uint4*>(keys + i1) : make_uint4(0u, 0u, 0u, 0u);
+          count4(v0, i0);
+          count4(v1, i1);
         }
       }
       __syncthreads();
@@ -647,8 +670,12 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
       const uint32_t incl = warp_inclusive_scan(tot, lane);
       if (lane == 31) wsum[warp] = incl;
       asm volatile("bar.sync 1, %0;" ::"n"(kBins) : "memory");
-      uint32_t above = incl - tot;
-      for (int w = 0; w < warp; ++w) above += wsum[w];
+      const uint4 w0 = reinterpret_cast<const uint4*>(wsum)[0];
+      const uint4 w1 = reinterpret_cast<const uint4*>(wsum)[1];
+      const uint32_t above = incl - tot + (warp > 0 ? w0.x : 0u) + (warp > 1 ? w0.y : 0u) +
+                             (warp > 2 ? w0.z : 0u) + (warp > 3 ? w0.w : 0u) +
+                             (warp > 4 ? w1.x : 0u) + (warp > 5 ? w1.y : 0u) +
+                             (warp > 6 ? w1.z : 0u);
       if (tot > 0 && above < kk && kk <= above + tot) {
         slot[2 * pass] = static_cast<uint32_t>(kBins - 1 - tid);
         slot[2 * pass + 1] = kk - above;
@@ -656,16 +683,6 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
     }
     __syncthreads();
     const uint32_t digit = slot[2 * pass] & 0xFFu;
-    {  // this warp's keys above the chosen digit (they all sort above the threshold)
-      uint32_t c = 0;
-      for (int bin = static_cast<int>(digit) + 1 + lane; bin < kBins; bin += 32) c += whist[bin];
-      wgt += warp_sum(c);
-    }
-    if (pass == 1) {
-      ncand = static_cast<int>(wgt + whist[digit]);
-      use_cand = ncand <= kCandCap;
-    }
-    if (pass == 3) weq = whist[digit];
     prefix |= digit << shift;
     mask |= 0xFFu << shift;
     kk = slot[2 * pass + 1];
@@ -677,6 +694,30 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
     }
   }
   const uint32_t thr = prefix;  // the ksel-th largest key; kk of its copies are taken
+  uint32_t wgt = 0, weq = 0;    // keys of the warp's segment above / at the threshold
+  if (use_cand) {
+    for (int c0 = 0; c0 < ncand; c0 += 32) {
+      const bool in = c0 + lane < ncand;
+      const uint32_t u = in ? keys[wcand[c0 + lane]] : 0u;
+      wgt += __popc(__ballot_sync(0xffffffffu, in && u > thr));
+      weq += __popc(__ballot_sync(0xffffffffu, in && u == thr));
+    }
+  } else {
+    for (int g0 = s0; g0 < s1; g0 += 128) {
+      uint32_t u[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = g0 + 32 * r + lane;
+        u[r] = i < s1 ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const bool in = g0 + 32 * r + lane < s1;
+        wgt += __popc(__ballot_sync(0xffffffffu, in && u[r] > thr));
+        weq += __popc(__ballot_sync(0xffffffffu, in && u[r] == thr));
+      }
+    }
+  }
   if (lane == 0) {
     wcnt[warp] = wgt;
     wcnt[kWarps + warp] = weq;
@@ -690,18 +731,16 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
   if (tid < 4) list_key[ksel + tid] = 0u;  // below every key: the rank loads read up to 3 past
   for (int s = tid; s < kMaxShare; s += kTkThreads) rank_acc[s] = 0u;
   tk_wait(&bars[2], 0, abort_flag);
-  // the copies of the threshold go to the lowest indices: CTAs, then warps, in order
-  uint32_t base = 0, take = 0, eq_before = 0;
-#pragma unroll
-  for (int r = 0; r < CL; ++r) {
-    const uint32_t g = info[2 * r], e = info[2 * r + 1];
-    const uint32_t tk = kk > eq_before ? min(kk - eq_before, e) : 0u;
-    if (r < static_cast<int>(rank)) base += g + tk;
-    if (r == static_cast<int>(rank)) take = tk;
-    eq_before += e;
-  }
-  uint32_t wpos, wtake;
-  {  // lane l stands for warp l: its first list position and its copies of the threshold
+  // the copies of the threshold go to the lowest indices: CTAs, then warps, in order.
+  // Lane r < CL stands for CTA r, then lane w for warp w of this CTA.
+  uint32_t base, take, wpos, wtake;
+  {
+    const uint32_t gr = lane < CL ? info[2 * lane] : 0u, er_ = lane < CL ? info[2 * lane + 1] : 0u;
+    const uint32_t ebr = warp_inclusive_scan(er_, lane) - er_;
+    const uint32_t tkr = kk > ebr ? min(kk - ebr, er_) : 0u;
+    const uint32_t pr = warp_inclusive_scan(gr + tkr, lane) - (gr + tkr);
+    base = __shfl_sync(0xffffffffu, pr, rank);
+    take = __shfl_sync(0xffffffffu, tkr, rank);
     const uint32_t gl = wcnt[lane], el = wcnt[kWarps + lane];
     const uint32_t eb = warp_inclusive_scan(el, lane) - el;
     const uint32_t tkl = take > eb ? min(take - eb, el) : 0u;
@@ -759,32 +798,73 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
   cluster_arrive_relaxed();  // no CTA leaves before every CTA is done with the others' memory
   tk_wait(&bars[3], 0, abort_flag);
   __syncthreads();
-  // rank: chunk ch of the list against entries my0 + j, my0 + 128 + j
+  // rank.  Every list key is >= thr: bin b holds the keys with (key - thr) >> sh == b, sh
+  // the smallest shift that puts the largest key in bin 255.  The list is laid out by bin,
+  // highest first, and the entry at list position e goes to output place (keys in higher
+  // bins) + (keys of its own bin that sort before it: larger, or equal and earlier in the
+  // list, which is index order).  8 threads share each entry's bin.
   {
-    const int ch = tid >> 7, j = tid & 127;
-    const int L = ((ksel + kRankChunks - 1) / kRankChunks + 3) & ~3;
-    const int c0 = min(ksel, ch * L), c1 = min(ksel, c0 + L);
+    uint32_t* bcnt = recv + kMaxShare;                                   // [kRankBins]
+    uint32_t* above = hist + kListAbove;                                 // [kRankBins]
+    uint32_t* bkey = hist + kListBKey;                                   // [kMaxK]
+    uint16_t* bpos = reinterpret_cast<uint16_t*>(hist + kListBPos);      // [kMaxK]
+    uint32_t mx = 0;
+    for (int o = tid; o < ksel; o += kTkThreads) mx = max(mx, list_key[o]);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) wcnt[warp] = mx;
+    if (tid < kRankBins) bcnt[tid] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kWarps; w += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(wcnt + w);
+      mx = max(max(mx, v.x), max(v.y, max(v.z, v.w)));
+    }
+    const uint32_t maxd = mx - thr;
+    const int sh = maxd >= kRankBins ? 32 - __clz(maxd) - 8 : 0;
+    auto bin_of = [&](uint32_t key) { return min(static_cast<uint32_t>(kRankBins - 1), (key - thr) >> sh); };
+    for (int o = tid; o < ksel; o += kTkThreads) atomicAdd(&bcnt[bin_of(list_key[o])], 1u);
+    __syncthreads();
+    if (warp == 0) {  // lane l: bins 255 - 8l down to 248 - 8l; a lane-order scan counts higher bins
+      uint4* c4 = reinterpret_cast<uint4*>(bcnt);
+      uint4* a4 = reinterpret_cast<uint4*>(above);
+      const uint4 lo4 = c4[62 - 2 * lane], hi4 = c4[63 - 2 * lane];
+      const uint32_t sum = lo4.x + lo4.y + lo4.z + lo4.w + hi4.x + hi4.y + hi4.z + hi4.w;
+      uint32_t at = warp_inclusive_scan(sum, lane) - sum;
+      uint4 ahi, alo;
+      ahi.w = at; at += hi4.w;
+      ahi.z = at; at += hi4.z;
+      ahi.y = at; at += hi4.y;
+      ahi.x = at; at += hi4.x;
+      alo.w = at; at += lo4.w;
+      alo.z = at; at += lo4.z;
+      alo.y = at; at += lo4.y;
+      alo.x = at;
+      a4[63 - 2 * lane] = ahi;  // bin starts, and the bins' fill cursors
+      a4[62 - 2 * lane] = alo;
+      c4[63 - 2 * lane] = ahi;
+      c4[62 - 2 * lane] = alo;
+    }
+    __syncthreads();
+    for (int o = tid; o < ksel; o += kTkThreads) {
+      const uint32_t key = list_key[o];
+      const uint32_t at = atomicAdd(&bcnt[bin_of(key)], 1u);
+      if (at < static_cast<uint32_t>(kMaxK)) {
+        bkey[at] = key;
+        bpos[at] = static_cast<uint16_t>(o);
+      }
+    }
+    __syncthreads();
+    const int j = tid & 127, sub = tid >> 7;
     for (int e0 = my0; e0 < my1; e0 += 128) {
       const int e = e0 + j;
-      if (e >= my1 || c0 >= c1) continue;
+      if (e >= my1) continue;
       const uint32_t ke = list_key[e];
-      uint32_t n = 0;
-      if (c1 <= e) {  // the whole chunk lies before e: equal keys sort before it
-        for (int o = c0; o < c1; o += 4) {
-          const uint4 v = *reinterpret_cast<const uint4*>(list_key + o);
-          n += (v.x >= ke) + (v.y >= ke) + (v.z >= ke) + (v.w >= ke);
-        }
-      } else if (c0 > e) {  // the whole chunk lies after e (and the zero padding past it)
-        for (int o = c0; o < c1; o += 4) {
-          const uint4 v = *reinterpret_cast<const uint4*>(list_key + o);
-          n += (v.x > ke) + (v.y > ke) + (v.z > ke) + (v.w > ke);
-        }
-      } else {
-        for (int o = c0; o < c1; o += 4) {
-          const uint4 v = *reinterpret_cast<const uint4*>(list_key + o);
-          n += (o < e ? v.x >= ke : v.x > ke) + (o + 1 < e ? v.y >= ke : v.y > ke) +
-               (o + 2 < e ? v.z >= ke : v.z > ke) + (o + 3 < e ? v.w >= ke : v.w > ke);
-        }
+      const uint32_t bin = bin_of(ke);
+      const uint32_t lo_ = above[bin], hi_ = min(bcnt[bin], static_cast<uint32_t>(kMaxK));
+      uint32_t n = sub == 0 ? lo_ : 0u;
+      for (uint32_t p = lo_ + sub; p < hi_; p += kRankChunks) {
+        const uint32_t km = bkey[p];
+        n += km > ke || (km == ke && bpos[p] < e);
       }
       atomicAdd(&rank_acc[e - my0], n);
     }
