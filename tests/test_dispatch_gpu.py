@@ -149,30 +149,49 @@ def test_scalar_dispatch():
     assert_guards(buf, out.numel(), "hca scalar")
 
 
-def test_listed_dispatch():
-    """Entry lists take the register-staged kernels (one window per thread)."""
-    lens = [4 * 50 + 1, 4 * 3, 4 * 77]
-    c = 128
-    d = synth.stream_inputs("csa", 1, sum(lens), c, 4, "bf16", seed=9)
+# Entry lists (CSA, m = 4, overlap) take the register-staged kernel (one window per thread)
+# at every row width, input and output type and list length.
+CSA_LISTED = [
+    # kernel, c, in, out, sequence lengths, entry step
+    ("csa_small_m_kernel", 128, "bf16", "f32", [4 * 50 + 1, 4 * 3, 4 * 77], 3),
+    ("csa_small_m_kernel", 256, "bf16", "bf16", [4 * 20, 4 * 91 + 2, 5, 4 * 7], 1),
+    ("csa_small_m_kernel", 512, "bf16", "bf16", [4 * 33 + 3, 4 * 64, 4], 1),
+    ("csa_small_m_kernel", 64, "f32", "f32", [4 * 40, 4 * 9 + 1], 1),
+    ("csa_small_m_kernel", 128, "f32", "bf16", [4 * 17, 4 * 50 + 3], 2),
+    ("csa_small_m_kernel", 256, "f32", "f32", [4 * 70 + 1, 4 * 2], 1),
+    ("csa_small_m_kernel", 136, "bf16", "f32", [4 * 50 + 1, 4 * 3, 4 * 77], 3),
+    ("csa_small_m_kernel", 512, "bf16", "bf16", [4 * 6001 + 2], 1),  # a long list
+]
+
+
+@pytest.mark.parametrize("kernel,c,in_dt,out_dt,lens,step", CSA_LISTED,
+                         ids=[f"{k}-c{c}-{i}-{o}-{len(L)}seq" for k, c, i, o, L, _ in CSA_LISTED])
+def test_csa_listed_dispatch(kernel, c, in_dt, out_dt, lens, step):
+    d = synth.stream_inputs("csa", 1, sum(lens), c, 4, in_dt, seed=9 + c)
     starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
-    ents = [(s, e) for s, L in enumerate(lens) for e in range(0, L // 4, 3)]
-    t = {k: dev(v[0], "bf16") if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+    ents = [(s, e) for s, L in enumerate(lens) for e in range(0, L // 4, step)]
+    ents = ents[::-1]  # list order is not sequence order
+    t = {k: dev(v[0], in_dt) if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
     ss = torch.tensor([int(starts[s]) for s, _ in ents], dtype=torch.int64, device="cuda")
     sl = torch.tensor([lens[s] for s, _ in ents], dtype=torch.int64, device="cuda")
     en = torch.tensor([e for _, e in ents], dtype=torch.int64, device="cuda")
-    buf, out = guarded((len(ents), c), torch.float32)
+    buf, out = guarded((len(ents), c), tdtype(out_dt))
     kvc.csa_compress_entries(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], ss, sl, en, m=4,
-                             out=out, out_dtype=torch.float32)
-    assert kvc.last_kernel() == "csa_small_m_kernel"
+                             out=out, out_dtype=tdtype(out_dt))
+    assert kvc.last_kernel() == kernel
     assert kvc.device_status() == kvc.KVC_OK
-    ref = []
-    for s, e in ents:
-        q = slice(int(starts[s]), int(starts[s]) + lens[s])
-        ref.append(O.csa_compress(d["Ca"][:, q], d["Cb"][:, q], d["Za"][:, q], d["Zb"][:, q],
-                                  d["Ba"], d["Bb"], 4, True, entries=[(0, e)])[0])
-    check_close(out, np.array(ref), "f32", "csa listed")
+    ref = {}
+    for s, L in enumerate(lens):  # every entry of a sequence at once
+        q = slice(int(starts[s]), int(starts[s]) + L)
+        if L // 4:
+            ref[s] = O.csa_compress(d["Ca"][:, q], d["Cb"][:, q], d["Za"][:, q], d["Zb"][:, q],
+                                    d["Ba"], d["Bb"], 4, True)[0]
+    check_close(out, np.array([ref[s][e] for s, e in ents]), out_dt, f"csa listed c={c}")
     assert_guards(buf, out.numel(), "csa listed")
 
+
+def test_hca_listed_dispatch():
+    c = 128
     h = synth.stream_inputs("hca", 1, 128 * 12, c, 128, "bf16", seed=10)
     th = {k: dev(v[0], "bf16") if v.ndim == 3 else dev(v, "f32") for k, v in h.items()}
     idx = torch.arange(12, dtype=torch.int64, device="cuda")

@@ -106,6 +106,37 @@ def test_topk_exact_given_scores(k, kind):
         assert np.array_equal(val[i].astype(np.float64), ref_val), (k, kind, n)
 
 
+def test_topk_many_rows_in_waves():
+    """More rows than clusters resident at once (the launch runs in waves); each row its own
+    length and distribution."""
+    rng = np.random.default_rng(40)
+    T, ld, k = 40, 65536, 1024
+    nv = [int(x) for x in rng.integers(0, ld + 1, size=T)]
+    nv[0], nv[1] = ld, 0
+    S = np.zeros((T, ld), dtype=np.float32)
+    for i, n in enumerate(nv):
+        S[i, :n] = rng.standard_normal(n) * (1 + i % 5) + (i % 3)
+    idx, val = _topk_gpu(torch.from_numpy(S).cuda(), nv, k, ld)
+    assert kvc.device_status() == kvc.KVC_OK
+    for i, n in enumerate(nv):
+        ref_idx, ref_val = IX.topk_row(S[i, :n].astype(np.float64), k)
+        assert np.array_equal(idx[i], ref_idx), (i, n)
+        assert np.array_equal(val[i].astype(np.float64), ref_val), (i, n)
+
+
+@pytest.mark.parametrize("k", [1, 1024, 2048])
+def test_topk_all_scores_equal(k):
+    """Every score the same: the selection is the first k indices in order (every warp's
+    candidate list overflows; the rank has one bin)."""
+    nv = [327680, 4099, 2048]
+    S = np.full((len(nv), 327680), 2.5, dtype=np.float32)
+    idx, val = _topk_gpu(torch.from_numpy(S).cuda(), nv, k, 327680)
+    assert kvc.device_status() == kvc.KVC_OK
+    for i, n in enumerate(nv):
+        want = np.arange(k) if k <= n else np.concatenate([np.arange(n), -np.ones(k - n)])
+        assert np.array_equal(idx[i], want.astype(np.int32)), (k, n)
+
+
 def test_topk_signed_zero_and_negatives():
     """-0.0 and 0.0 are the same score (ties by index); negative scores order correctly."""
     v = np.array([0.0, -0.0, -1.5, 2.0, -0.0, 0.0, -3.0, 2.0, -1.5], dtype=np.float32)
