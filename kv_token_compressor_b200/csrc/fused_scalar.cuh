@@ -185,6 +185,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(scal::kThreads, 1)
       int pending_parity[S];
       for (int s = 0; s < S; ++s) pending_parity[s] = -1;
       bool ok = true;
+      const uint64_t wpol = l2_evict_last_policy();  // W stays in L2 while H streams past
       pair::Sched sc = pair::sched_begin<CSA>(a, cid, ncl);
       pair::Unit q;
       while (ok && scal::next_unit<CSA>(a, &sc, rank, &q)) {
@@ -206,11 +207,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(scal::kThreads, 1)
             uint8_t* st = smem + stage * C::STAGE;
             const int x = kstep * C::BK;
             tma_load_2d_pair(smem_u32(st + C::A_BYTES), &tmH, lbar, x, y);
-            tma_load_2d_pair(smem_u32(st + 0 * C::A_BOX), &tmW0, lbar, g0 * kCh, x);
-            tma_load_2d_pair(smem_u32(st + 1 * C::A_BOX), &tmW0, lbar, g0 * kCh + 64, x);
-            tma_load_2d_pair(smem_u32(st + 2 * C::A_BOX), CSA ? &tmW1 : &tmW0, lbar, g1 * kCh, x);
-            tma_load_2d_pair(smem_u32(st + 3 * C::A_BOX), CSA ? &tmW1 : &tmW0, lbar,
-                             g1 * kCh + 64, x);
+            tma_load_2d_pair_hint(smem_u32(st + 0 * C::A_BOX), &tmW0, lbar, g0 * kCh, x, wpol);
+            tma_load_2d_pair_hint(smem_u32(st + 1 * C::A_BOX), &tmW0, lbar, g0 * kCh + 64, x, wpol);
+            tma_load_2d_pair_hint(smem_u32(st + 2 * C::A_BOX), CSA ? &tmW1 : &tmW0, lbar, g1 * kCh,
+                                  x, wpol);
+            tma_load_2d_pair_hint(smem_u32(st + 3 * C::A_BOX), CSA ? &tmW1 : &tmW0, lbar,
+                                  g1 * kCh + 64, x, wpol);
             if (++stage == S) {
               stage = 0;
               phase ^= 1u;

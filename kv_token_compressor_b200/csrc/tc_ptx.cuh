@@ -47,6 +47,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// L2 policy that keeps the lines it loads in preference to others: for operands that every
+// CTA reads again and again (the projection weights) while other data streams past.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05 format: start >> 4 at [0,14), leading byte
 // offset >> 4 at [16,30), stride byte offset >> 4 at [32,46), version 1 at [46,48),
 // layout type at [61,64): 2 = SWIZZLE_128B, 4 = SWIZZLE_64B).
