@@ -358,7 +358,10 @@ KVC_API kvc_status lightning_indexer_scores(const void* q, const float* w, const
  *   out_score[t * k + j] (fp32, may be NULL): the matching scores, -inf past the end.
  * 1 <= k <= 2048; max_visible <= kvc_topk_max_candidates(); scores [T, ld] fp32,
  * 16-byte aligned with ld a multiple of 4; n_visible as above.  The result is exact
- * for the given scores (no NaN among them). */
+ * for the given scores (no NaN among them).  The kernel is launched as a programmatic
+ * dependent of the kernel ahead of it on the stream: it may start launching while that
+ * kernel (lightning_indexer_scores in a decode step) finishes, and reads its inputs only
+ * once that kernel has completed, so stream order holds as for any other call. */
 KVC_API kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* n_visible,
                                 int64_t T, int64_t max_visible, int32_t k, int32_t* out_idx,
                                 float* out_score, kvc_stream stream);

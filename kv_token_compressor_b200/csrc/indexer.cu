@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* final_bar = tempty + kAccBufs;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(final_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(final_bar + 2);
+  // a top-k launched next on the stream may start launching now (it reads the scores only
+  // after this grid has completed)
+  griddep_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H;
@@ -516,6 +519,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkA
   const uint32_t rank = blockIdx.x % CL;
   const int64_t t = blockIdx.x / CL;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  griddep_wait();  // launched early after the score kernel: its scores are complete from here
   const int64_t nv = a.n_visible[t];
   // the same decision in every CTA of the cluster: an out-of-range row is skipped whole
   if (nv < 0 || nv > a.max_visible) {
@@ -955,6 +959,13 @@ kvc_status launch_indexer_topk(const TopkProblem& p, cudaStream_t st) {
       return KVC_ERR_UNSUPPORTED;
     }
     cfg.gridDim = dim3(static_cast<unsigned>(p.T * cl), 1, 1);
+    // may launch while the kernel ahead of it (the scores) finishes; the kernel waits for
+    // that kernel's completion before its first read
+    cudaLaunchAttribute attr2[2] = {attr[0], {}};
+    attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr2[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr2;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return KVC_ERR_CUDA;
     last_kernel() = "indexer_topk_kernel";
     return KVC_OK;

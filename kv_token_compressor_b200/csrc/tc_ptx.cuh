@@ -47,6 +47,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic stream
+// serialisation attribute may be launched while the kernel ahead of it on the stream is
+// still running; griddep_wait() returns once that kernel has completed and its memory
+// operations are visible (at once when nothing is pending), so it comes before any read of
+// what that kernel wrote.  griddep_launch_dependents() lets such a next kernel start
+// launching early; its own wait still waits for this grid's completion.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // L2 policy that keeps the lines it loads in preference to others: for operands that every
 // CTA reads again and again (the projection weights) while other data streams past.
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
