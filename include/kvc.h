@@ -386,6 +386,17 @@ KVC_API const char* kvc_last_kernel(void);
  * them for all callers. */
 KVC_API kvc_status kvc_device_status(kvc_stream stream);
 
+/* Sync check, off by default: with `on` nonzero, every call that launches work
+ * synchronises its stream after the launch and returns what kvc_device_status() would
+ * (KVC_ERR_TIMEOUT, KVC_ERR_WORKSPACE, KVC_ERR_INDEX, ...; the device error words are read
+ * and cleared), so a kernel-side failure surfaces from the call that caused it.  A
+ * debugging mode: it serialises the host with the stream.  Process-wide; a host-side
+ * validation error is returned as before, without a synchronisation.  kvc_sync_check()
+ * returns the current setting (0 or 1).  kvc_selftest_bounded_wait keeps reporting through
+ * kvc_device_status() only. */
+KVC_API void kvc_set_sync_check(int32_t on);
+KVC_API int32_t kvc_sync_check(void);
+
 /* Failure-detection self-test, no fault involved: launches one CTA whose first warp waits
  * on a shared-memory barrier that nothing completes, gives up after the kernels' wait limit
  * (2 s), raises the CTA's abort flag and the device error word; a second warp waiting on the

@@ -2,6 +2,7 @@
 // Every check here runs before anything is enqueued; see include/kvc.h for the contract.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/kvc.h"
@@ -123,9 +124,23 @@ kvc_status noalloc_scratch(void** out) {
   return KVC_OK;
 }
 
+// kvc_set_sync_check: process-wide, off by default.
+std::atomic<int> g_sync_check{0};
+
+// The status of a call that has launched its work: with the sync check on, the stream is
+// synchronised and what the kernels reported is returned (as kvc_device_status would).
+kvc_status finish(kvc_status launched, cudaStream_t st) {
+  if (launched != KVC_OK || g_sync_check.load(std::memory_order_relaxed) == 0) return launched;
+  return kvc::read_and_clear_device_error(st);
+}
+
 }  // namespace
 
 extern "C" {
+
+void kvc_set_sync_check(int32_t on) { g_sync_check.store(on != 0 ? 1 : 0); }
+
+int32_t kvc_sync_check(void) { return g_sync_check.load(); }
 
 int64_t kvc_num_entries(int64_t n, int32_t m) {
   if (n < 0 || m < 1) return -1;
@@ -193,7 +208,8 @@ kvc_status csa_compress(const void* Ca, const void* Cb, const void* Za, const vo
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
@@ -227,7 +243,8 @@ kvc_status hca_compress(const void* C, const void* Z, kvc_dtype in_dtype, const 
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 int64_t hca_bias_workspace_bytes(int64_t c, int32_t m, kvc_dtype in_dtype) {
@@ -249,8 +266,8 @@ kvc_status hca_prepare_bias(const float* B, int64_t c, int32_t m, kvc_dtype in_d
   const void* ps[2] = {B, workspace};
   const kvc_status s = check_ptrs(ps, 2);
   if (s != KVC_OK) return s;
-  return kvc::launch_prepare_bias(B, c, m, in_dtype == KVC_BF16, workspace,
-                                  reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_prepare_bias(B, c, m, in_dtype == KVC_BF16, workspace, st), st);
 }
 
 kvc_status hca_compress_prepared(const void* C, const void* Z, kvc_dtype in_dtype,
@@ -289,7 +306,8 @@ kvc_status hca_compress_prepared(const void* C, const void* Z, kvc_dtype in_dtyp
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status hca_compress_noalloc(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
@@ -336,7 +354,7 @@ kvc_status hca_compress_noalloc(const void* C, const void* Z, kvc_dtype in_dtype
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_stream_pool(p, st);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status csa_compress_scalar_logits(const void* Ca, const void* Cb, const void* za,
@@ -378,7 +396,8 @@ kvc_status csa_compress_scalar_logits(const void* Ca, const void* Cb, const void
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_scalar_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_scalar_pool(p, st), st);
 }
 
 kvc_status hca_compress_scalar_logits(const void* C, const void* z, kvc_dtype in_dtype,
@@ -413,7 +432,8 @@ kvc_status hca_compress_scalar_logits(const void* C, const void* z, kvc_dtype in
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_scalar_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_scalar_pool(p, st), st);
 }
 
 // Common checks of the entry-list calls; fills the list fields of p.
@@ -480,7 +500,8 @@ kvc_status csa_compress_entries(const void* Ca, const void* Cb, const void* Za, 
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
@@ -509,7 +530,8 @@ kvc_status hca_compress_entries(const void* C, const void* Z, kvc_dtype in_dtype
   p.in_bf16 = in_dtype == KVC_BF16;
   p.out_bf16 = out_dtype == KVC_BF16;
   p.out = out;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status csa_compress_cache(const void* Ca, const void* Cb, const void* Za, const void* Zb,
@@ -551,7 +573,8 @@ kvc_status csa_compress_cache(const void* Ca, const void* Cb, const void* Za, co
   p.two_segments = overlap != 0;
   p.small_window_kernel = true;
   p.in_bf16 = in_dtype == KVC_BF16;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status hca_compress_cache(const void* C, const void* Z, kvc_dtype in_dtype, const float* B,
@@ -585,7 +608,8 @@ kvc_status hca_compress_cache(const void* C, const void* Z, kvc_dtype in_dtype, 
   p.two_segments = false;
   p.small_window_kernel = false;
   p.in_bf16 = in_dtype == KVC_BF16;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status csa_compress_entries_cache(const void* Ca, const void* Cb, const void* Za,
@@ -624,7 +648,8 @@ kvc_status csa_compress_entries_cache(const void* Ca, const void* Cb, const void
   p.two_segments = overlap != 0;
   p.small_window_kernel = true;
   p.in_bf16 = in_dtype == KVC_BF16;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 kvc_status hca_compress_entries_cache(const void* C, const void* Z, kvc_dtype in_dtype,
@@ -655,7 +680,8 @@ kvc_status hca_compress_entries_cache(const void* C, const void* Z, kvc_dtype in
   p.two_segments = false;
   p.small_window_kernel = false;
   p.in_bf16 = in_dtype == KVC_BF16;
-  return kvc::launch_stream_pool(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_stream_pool(p, st), st);
 }
 
 // Device-memory check of the fused calls' inputs (and of `out` when non-NULL).
@@ -741,7 +767,8 @@ kvc_status csa_compress_fused_proj(const void* H, const void* W_kva, const void*
   if (s != KVC_OK || empty) return s;
   p.csa = true;
   p.overlap = overlap != 0;
-  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_fused(p, st), st);
 }
 
 kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* W_z,
@@ -758,7 +785,8 @@ kvc_status hca_compress_fused_proj(const void* H, const void* W_kv, const void* 
   p.W[1] = W_z;
   p.csa = false;
   p.overlap = false;
-  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_fused(p, st), st);
 }
 
 kvc_status csa_compress_fused_proj_scalar(const void* H, const void* W_kva, const void* W_kvb,
@@ -780,7 +808,8 @@ kvc_status csa_compress_fused_proj_scalar(const void* H, const void* W_kva, cons
   p.scalar = true;
   p.csa = true;
   p.overlap = true;
-  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_fused(p, st), st);
 }
 
 kvc_status hca_compress_fused_proj_scalar(const void* H, const void* W_kv, const void* w_z,
@@ -799,7 +828,8 @@ kvc_status hca_compress_fused_proj_scalar(const void* H, const void* W_kv, const
   p.scalar = true;
   p.csa = false;
   p.overlap = false;
-  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_fused(p, st), st);
 }
 
 kvc_status csa_compress_fused_proj_cache(const void* H, const void* W_kva, const void* W_kvb,
@@ -822,7 +852,8 @@ kvc_status csa_compress_fused_proj_cache(const void* H, const void* W_kva, const
   for (int i = 0; i < 4; ++i) p.W[i] = W[i];
   p.csa = true;
   p.overlap = true;
-  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_fused(p, st), st);
 }
 
 kvc_status hca_compress_fused_proj_cache(const void* H, const void* W_kv, const void* W_z,
@@ -843,7 +874,8 @@ kvc_status hca_compress_fused_proj_cache(const void* H, const void* W_kv, const 
   p.W[1] = W_z;
   p.csa = false;
   p.overlap = false;
-  return kvc::launch_fused(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_fused(p, st), st);
 }
 
 kvc_status lightning_indexer_scores(const void* q, const float* w, const void* K,
@@ -869,7 +901,8 @@ kvc_status lightning_indexer_scores(const void* q, const float* w, const void* K
   kvc_status s = check_ptrs(ps, 6);
   if (s != KVC_OK) return s;
   kvc::IndexerProblem p{q, w, K, key_start, n_visible, T, key_rows, max_visible, ld, H, scores};
-  return kvc::launch_indexer_scores(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_indexer_scores(p, st), st);
 }
 
 kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* n_visible, int64_t T,
@@ -892,7 +925,8 @@ kvc_status indexer_topk(const float* scores, int64_t ld, const int64_t* n_visibl
   if (s == KVC_OK && out_score) s = check_device_ptr(out_score);
   if (s != KVC_OK) return s;
   kvc::TopkProblem p{scores, n_visible, T, max_visible, ld, k, out_idx, out_score};
-  return kvc::launch_indexer_topk(p, reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(kvc::launch_indexer_topk(p, st), st);
 }
 
 int64_t kvc_topk_max_candidates(void) { return kvc::topk_max_candidates(); }

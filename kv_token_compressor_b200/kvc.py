@@ -46,6 +46,8 @@ SIGNATURES = {
     "hca_compress_fused_proj": (ctypes.c_int, [_p, _p, _p, _p, _i64, _i64, _i64, _i64, _i32, _p,
                                                ctypes.c_int, _p]),
     "kvc_device_status": (ctypes.c_int, [_p]),
+    "kvc_set_sync_check": (None, [_i32]),
+    "kvc_sync_check": (_i32, []),
     "kvc_selftest_bounded_wait": (ctypes.c_int, [_p, _p]),
     "csa_compress_scalar_logits": (ctypes.c_int, [_p, _p, _p, _p, ctypes.c_int, _p, _p, _i64, _i64,
                                                   _i64, _i32, _i32, _p, ctypes.c_int, _p]),
@@ -627,6 +629,17 @@ def topk_max_candidates() -> int:
 def device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the kernels' device error status."""
     return int(lib().kvc_device_status(_stream(stream)))
+
+
+def set_sync_check(on: bool) -> None:
+    """Turn the library's sync check on or off: with it on, every call synchronises its
+    stream and raises KvcError for what the kernels reported (a bounded wait that gave up,
+    a listed entry out of range, ...) instead of leaving it to device_status()."""
+    lib().kvc_set_sync_check(1 if on else 0)
+
+
+def sync_check() -> bool:
+    return bool(lib().kvc_sync_check())
 
 
 def selftest_bounded_wait(stream=None):

@@ -623,7 +623,7 @@ def _header_prototypes():
 _CTYPE = {
     "int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32, "double": ctypes.c_double,
     "float": ctypes.c_float, "kvc_status": ctypes.c_int, "kvc_dtype": ctypes.c_int,
-    "kvc_stream": ctypes.c_void_p, "const char*": ctypes.c_char_p,
+    "kvc_stream": ctypes.c_void_p, "const char*": ctypes.c_char_p, "void": None,
 }
 
 
@@ -765,3 +765,16 @@ def test_plain_c_program_uses_the_abi(L, tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
     assert run.stdout.split()[-1] == "0"
+
+
+def test_sync_check_setting_round_trips():
+    """kvc_set_sync_check / kvc_sync_check: off by default, any nonzero is on."""
+    L = kvc.lib()
+    assert L.kvc_sync_check() == 0
+    try:
+        L.kvc_set_sync_check(7)
+        assert L.kvc_sync_check() == 1 and kvc.sync_check()
+        kvc.set_sync_check(False)
+        assert L.kvc_sync_check() == 0 and not kvc.sync_check()
+    finally:
+        L.kvc_set_sync_check(0)

@@ -134,6 +134,29 @@ def test_out_of_range_entries_are_skipped_and_reported():
     assert kvc.device_status() == kvc.KVC_ERR_INDEX
 
 
+def test_sync_check_reports_from_the_call():
+    """With the sync check on, the call that named an out-of-range entry raises
+    KVC_ERR_INDEX itself (and clears the word); a valid call passes."""
+    m, c = 4, 64
+    lens = [40, 12]
+    d, starts = _pack(lens, c, m, "f32", seed=11)
+    t = {k: dev(v[0], "f32") if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+    args = (t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"])
+    kvc.set_sync_check(True)
+    try:
+        with pytest.raises(kvc.KvcError) as e:
+            kvc.csa_compress_entries(*args, *_list(starts, lens, [(0, 3), (1, 5)]), m=4)
+        assert e.value.status == kvc.KVC_ERR_INDEX
+        assert kvc.device_status() == kvc.KVC_OK
+        ents = [(0, 3), (1, 2)]
+        out = kvc.csa_compress_entries(*args, *_list(starts, lens, ents), m=4,
+                                       out_dtype=torch.float32)
+        check_close(out, _csa_ref(d, starts, lens, ents, m), "f32", "sync-checked call")
+    finally:
+        kvc.set_sync_check(False)
+    assert not kvc.sync_check()
+
+
 def test_empty_list():
     x = torch.zeros((16, 64), device="cuda")
     b = torch.zeros((4, 64), device="cuda")
