@@ -489,16 +489,19 @@ __device__ __forceinline__ uint32_t warp_inclusive_scan(uint32_t v, int lane) {
 //     warp counts its segment into its own histogram (the first digit while the scores
 //     load); 256 threads sum the CTA's warps and push the sums into every CTA of the
 //     cluster (st.async, counted on an mbarrier per buffer, two buffers alternating), so
-//     every CTA picks the same digit with no cluster-wide barrier.  After the second digit
-//     a warp that holds at most kCandCap keys at or above the 16-bit prefix keeps their
-//     positions, and the last digit and the selection read those alone.
+//     every CTA picks the same digit with no cluster-wide barrier.  While it counts the
+//     third digit, a warp keeps the positions of its keys at or above the 16-bit prefix
+//     if they fit in kCandCap; the last digit, the warp's counts above and at the
+//     threshold and the selection then read those alone (else they scan the segment).
 //  2. The copies of the threshold that are taken go to the lowest indices (CTAs, then
 //     warps, in index order, from the counts every CTA pushes); each CTA pushes its
 //     selected keys, in index order, to their place in every CTA's copy of the list, and
 //     each entry's index to the CTA that will store it.
 //  3. Every CTA ranks its share of the list: the entry at list position e goes to output
-//     place #{keys above it} + #{equal keys before it in the list}, counted in 8 chunks by
-//     1024 threads.  The list is in index order, so equal scores come out by index.
+//     place #{keys above it} + #{equal keys before it in the list}: the list is binned by
+//     key minus threshold, the keys in higher bins are counted by one warp's scan, those of
+//     its own bin one by one.  The list is in index order, so equal scores come out by
+//     index.
 template <int CL>
 __global__ void __launch_bounds__(kTkThreads, 1) indexer_topk_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
