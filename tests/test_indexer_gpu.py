@@ -137,6 +137,38 @@ def test_topk_all_scores_equal(k):
         assert np.array_equal(idx[i], want.astype(np.int32)), (k, n)
 
 
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_topk_randomized_rows(seed):
+    """Seeded random batches: per row a length in [0, 327680], a distribution (continuous,
+    few values with many zeros, ascending runs, constant blocks with noise) and one k per
+    launch in [1, 2048]; every row bit for bit against the oracle's selection."""
+    rng = np.random.default_rng(1000 + seed)
+    T, ld = 16, 327680
+    k = int(rng.integers(1, 2049))
+    nv = [int(x) for x in rng.integers(0, ld + 1, size=T)]
+    nv[int(rng.integers(T))] = ld
+    S = np.full((T, ld), np.nan, dtype=np.float32)
+    for i, n in enumerate(nv):
+        kind = i % 4
+        if kind == 0:
+            v = rng.standard_normal(n) * rng.uniform(0.01, 100)
+        elif kind == 1:
+            v = rng.integers(-3, 4, size=n).astype(np.float64)
+            v[rng.random(n) < 0.6] = 0.0
+        elif kind == 2:
+            v = np.cumsum(rng.random(n)) * rng.choice([-1, 1])
+        else:
+            v = np.repeat(rng.standard_normal(max(1, n // 1000 + 1)), 1000)[:n]
+            v = v + (rng.random(n) < 0.01) * rng.standard_normal(n)
+        S[i, :n] = v.astype(np.float32)
+    idx, val = _topk_gpu(torch.from_numpy(S).cuda(), nv, k, ld)
+    assert kvc.device_status() == kvc.KVC_OK
+    for i, n in enumerate(nv):
+        ref_idx, ref_val = IX.topk_row(S[i, :n].astype(np.float64), k)
+        assert np.array_equal(idx[i], ref_idx), (seed, i, n, k)
+        assert np.array_equal(val[i].astype(np.float64), ref_val), (seed, i, n, k)
+
+
 def test_topk_signed_zero_and_negatives():
     """-0.0 and 0.0 are the same score (ties by index); negative scores order correctly."""
     v = np.array([0.0, -0.0, -1.5, 2.0, -0.0, 0.0, -3.0, 2.0, -1.5], dtype=np.float32)
