@@ -188,6 +188,28 @@ def test_topk_row_past_max_visible_is_reported():
     assert idx[1].tolist() == [0, 1, 2, -1]
 
 
+def test_scores_then_topk_on_a_user_stream():
+    """The top-k launches as a programmatic dependent of the kernel ahead of it: on a
+    stream of the caller's, back to back with the score kernel and with new inputs each
+    time, it must select from the scores just written (compared bit for bit with the
+    oracle's selection over those scores)."""
+    T, H, S, k = 3, 64, 1 << 16, 512
+    s = torch.cuda.Stream()
+    ks, nv = [i * S for i in range(T)], [S, S - 7, 40000]
+    out = torch.empty((T, S), dtype=torch.float32, device="cuda")
+    with torch.cuda.stream(s):
+        for it in range(4):
+            t = synth.indexer_inputs_torch(T, H, T * S, seed=50 + it)
+            kvc.lightning_indexer_scores(t["q"], t["w"], t["K"], _i64(ks), _i64(nv), S, scores=out)
+            idx, _ = kvc.indexer_topk(out, _i64(nv), k, S)
+            s.synchronize()
+            got, gidx = out.cpu().numpy(), idx.cpu().numpy()
+            for i in range(T):
+                ref_idx, _ = IX.topk_row(got[i, :nv[i]].astype(np.float64), k)
+                assert np.array_equal(gidx[i], ref_idx), (it, i)
+    assert kvc.device_status(s) == kvc.KVC_OK
+
+
 def test_decode_step_end_to_end():
     """A decode step: 4 sequences of 2^20 tokens (262144 compressed keys each), one query
     of 64 heads per sequence, k = 1024.  Full score rows against the fp64 oracle, the top-k
