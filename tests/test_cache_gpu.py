@@ -102,6 +102,39 @@ def test_listed_cache_insertion():
     check_close(rope, ref_rope, "bf16", "listed rope")
 
 
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_hca_listed_cache_insertion(dt):
+    """HCA decode: each sequence's newest complete 128-row entry, in a shuffled list, goes
+    into the cache layout at its own position in its sequence."""
+    m, c, r = 128, 256, 64
+    rng = np.random.default_rng(11)
+    lens = [int(x) for x in rng.integers(m, 12 * m, size=9)]
+    d = synth.stream_inputs("hca", 1, sum(lens), c, m, dt, seed=12)
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    ents = [(s, L // m - 1) for s, L in enumerate(lens)]
+    rng.shuffle(ents)
+    t = {k: dev(v[0], dt) if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+    idx = lambda xs: torch.tensor([int(x) for x in xs], dtype=torch.int64, device="cuda")
+    inv = _inv_freq(r)
+    stride, offset = 128.0, 63.5
+    nope, rope = kvc.hca_compress_entries_cache(
+        t["C"], t["Z"], t["B"], idx([starts[s] for s, _ in ents]), idx([lens[s] for s, _ in ents]),
+        idx([e for _, e in ents]), r, torch.from_numpy(inv).cuda(), pos_stride=stride,
+        pos_offset=offset, fp8_scale=1.5)
+    torch.cuda.synchronize()
+    assert kvc.device_status() == kvc.KVC_OK
+    refs, poss = [], []
+    for s, e in ents:
+        sl = slice(starts[s], starts[s] + lens[s])
+        refs.append(O.hca_compress(d["C"][:, sl], d["Z"][:, sl], d["B"], m)[0, e])
+        poss.append(offset + stride * e)
+    ent = np.array(refs)
+    ref_nope = O.round_e4m3(ent[:, :c - r] * 1.5)
+    ref_rope = O.rope_pairs(ent[:, c - r:], np.array(poss), inv.astype(np.float64))
+    _check_fp8(_fp8_values(nope), ref_nope, "hca listed nope")
+    check_close(rope, ref_rope, "bf16", "hca listed rope")
+
+
 def test_cache_rejects_bad_layout():
     x = torch.zeros((1, 64, 128), device="cuda", dtype=torch.bfloat16)
     b = torch.zeros((4, 128), device="cuda")
