@@ -225,6 +225,47 @@ def test_bias_spread_paths(mode, batch, n, c, m, spread):
     check_close(out, ref, "f32", f"{mode} m={m} bias spread {spread}")
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_random_shapes_across_dispatch(seed):
+    """Seeded random problems across the dispatch boundaries: CSA with m in {1, 2, 4, 8, 13}
+    (with and without overlap) and HCA with m in {8, 16, 32, 64, 128, 150}; c any multiple
+    of 8 up to 1024, ragged n, 1-3 sequences, every input/output dtype pair.  Each output
+    lies between canary bands that must come back untouched."""
+    rng = np.random.default_rng(500 + seed)
+    for _ in range(4):
+        batch = int(rng.integers(1, 4))
+        c = 8 * int(rng.integers(1, 129))
+        in_dt, out_dt = rng.choice(["bf16", "f32"]), rng.choice(["bf16", "f32"])
+        if rng.random() < 0.5:
+            m = int(rng.choice([1, 2, 4, 8, 13]))
+            overlap = bool(rng.random() < 0.7)
+            n = int(rng.integers(m, min(6000, 2_000_000 // c)))
+            d = synth.stream_inputs("csa", batch, n, c, m, in_dt, seed=seed * 17 + m)
+            t = {k: dev(v, in_dt) if k in ("Ca", "Cb", "Za", "Zb") else dev(v, "f32")
+                 for k, v in d.items()}
+            ne = n // m
+            buf = torch.full((batch * ne * c + 128,), -777.0, device="cuda", dtype=tdtype(out_dt))
+            out = buf[64:64 + batch * ne * c].view(batch, ne, c)
+            kvc.csa_compress(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], m=m,
+                             overlap=overlap, out=out, out_dtype=tdtype(out_dt))
+            ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], m, overlap)
+            what = f"csa b={batch} n={n} c={c} m={m} ov={overlap} {in_dt}->{out_dt} ({kvc.last_kernel()})"
+        else:
+            m = int(rng.choice([8, 16, 32, 64, 128, 150]))
+            n = int(rng.integers(m, min(40 * m, 4_000_000 // c)))
+            d = synth.stream_inputs("hca", batch, n, c, m, in_dt, seed=seed * 19 + m)
+            ne = n // m
+            buf = torch.full((batch * ne * c + 128,), -777.0, device="cuda", dtype=tdtype(out_dt))
+            out = buf[64:64 + batch * ne * c].view(batch, ne, c)
+            kvc.hca_compress(dev(d["C"], in_dt), dev(d["Z"], in_dt), dev(d["B"], "f32"), m=m, out=out,
+                             out_dtype=tdtype(out_dt))
+            ref = O.hca_compress(d["C"], d["Z"], d["B"], m)
+            what = f"hca b={batch} n={n} c={c} m={m} {in_dt}->{out_dt} ({kvc.last_kernel()})"
+        assert kvc.device_status() == kvc.KVC_OK, what
+        check_close(out, ref, out_dt, what)
+        assert bool(torch.all(buf[:64] == -777.0)) and bool(torch.all(buf[64 + batch * ne * c:] == -777.0)), what
+
+
 def test_boundary_and_mean_on_gpu():
     """Closed forms on the kernel itself: entry 0 ignores the b-streams; constant logits
     with zero bias give the mean of the window (1/8 and 1/4 weights are exact)."""
