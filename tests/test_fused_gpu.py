@@ -73,6 +73,40 @@ def test_hca_fused_small(batch, n, d, c, out_dt):
     check_close(out, ref, out_dt, f"hca fused {batch}x{n} d={d} c={c}")
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_fused_random_shapes(seed):
+    """Seeded random fused problems: d a multiple of 64 up to 640, c a multiple of 128 up to
+    768, ragged n (CSA m = 4 with overlap, HCA m' = 128), 1-3 sequences, both output types;
+    each output between canary bands that must come back untouched."""
+    rng = np.random.default_rng(900 + seed)
+    for mode in ("csa", "hca"):
+        batch = int(rng.integers(1, 4))
+        d = 64 * int(rng.integers(1, 11))
+        c = 128 * int(rng.integers(1, 7))
+        m = 4 if mode == "csa" else 128
+        n = int(rng.integers(m, 3000 if mode == "csa" else 6000))
+        out_dt = rng.choice(["bf16", "f32"])
+        h = synth.fused_inputs(mode, batch, n, d, c, m, seed=seed * 31 + d + c)
+        t = _dev(h)
+        ne = n // m
+        buf = torch.full((batch * ne * c + 128,), -555.0, device="cuda", dtype=tdtype(out_dt))
+        out = buf[64:64 + batch * ne * c].view(batch, ne, c)
+        if mode == "csa":
+            kvc.csa_compress_fused_proj(t["H"], t["W_kva"], t["W_kvb"], t["W_za"], t["W_zb"],
+                                        t["Ba"], t["Bb"], batch, n, m=4, out=out,
+                                        out_dtype=tdtype(out_dt))
+            ref = O.csa_compress_fused(h["H"], h["W_kva"], h["W_kvb"], h["W_za"], h["W_zb"],
+                                       h["Ba"], h["Bb"], batch, n, 4, True)
+        else:
+            kvc.hca_compress_fused_proj(t["H"], t["W_kv"], t["W_z"], t["B"], batch, n, m=128,
+                                        out=out, out_dtype=tdtype(out_dt))
+            ref = O.hca_compress_fused(h["H"], h["W_kv"], h["W_z"], h["B"], batch, n, 128)
+        what = f"{mode} fused b={batch} n={n} d={d} c={c} {out_dt} ({kvc.last_kernel()})"
+        assert kvc.device_status() == kvc.KVC_OK, what
+        check_close(out, ref, out_dt, what)
+        assert bool(torch.all(buf[:64] == -555.0)) and bool(torch.all(buf[64 + batch * ne * c:] == -555.0)), what
+
+
 def test_fused_matches_streaming_on_identity():
     """d = c and W = scaled identities: the fused streams are exactly (scaled) H, so the
     fused path must agree with the streaming kernel fed those streams."""
