@@ -134,6 +134,45 @@ def test_out_of_range_entries_are_skipped_and_reported():
     assert kvc.device_status() == kvc.KVC_ERR_INDEX
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_random_lists(seed):
+    """Seeded random entry lists over ragged packed sequences: CSA with m in {2, 4, 8}
+    (with and without overlap) and HCA with m in {16, 64, 128}; random entries of every
+    sequence, entry 0 included, in a shuffled order; every input/output dtype pair."""
+    rng = np.random.default_rng(700 + seed)
+    for mode in ("csa", "hca"):
+        m = int(rng.choice([2, 4, 8] if mode == "csa" else [16, 64, 128]))
+        c = 8 * int(rng.integers(1, 97))
+        in_dt, out_dt = rng.choice(["bf16", "f32"]), rng.choice(["bf16", "f32"])
+        lens = [int(x) for x in rng.integers(m, 30 * m, size=int(rng.integers(1, 9)))]
+        d, starts = _pack(lens, c, m, in_dt, seed=seed * 13 + m, mode=mode)
+        ents = [(s, int(e)) for s, L in enumerate(lens)
+                for e in rng.choice(L // m, size=min(L // m, 5), replace=False)]
+        ents.append((0, 0))
+        rng.shuffle(ents)
+        lst = _list(starts, lens, ents)
+        if mode == "csa":
+            overlap = bool(rng.random() < 0.7)
+            t = {k: dev(v[0], in_dt) if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+            out = kvc.csa_compress_entries(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], *lst,
+                                           m=m, overlap=overlap, out_dtype=tdtype(out_dt))
+            ref = []
+            for s_, e in ents:
+                sl = slice(starts[s_], starts[s_] + lens[s_])
+                ref.append(O.csa_compress(d["Ca"][:, sl], d["Cb"][:, sl], d["Za"][:, sl], d["Zb"][:, sl],
+                                          d["Ba"], d["Bb"], m, overlap, entries=[(0, e)])[0])
+        else:
+            t = {k: dev(v[0], in_dt) if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+            out = kvc.hca_compress_entries(t["C"], t["Z"], t["B"], *lst, m=m, out_dtype=tdtype(out_dt))
+            ref = []
+            for s_, e in ents:
+                sl = slice(starts[s_], starts[s_] + lens[s_])
+                ref.append(O.hca_compress(d["C"][:, sl], d["Z"][:, sl], d["B"], m)[0, e])
+        what = f"{mode} lists m={m} c={c} {in_dt}->{out_dt} ({kvc.last_kernel()})"
+        assert kvc.device_status() == kvc.KVC_OK, what
+        check_close(out, np.array(ref), out_dt, what)
+
+
 def test_sync_check_reports_from_the_call():
     """With the sync check on, the call that named an out-of-range entry raises
     KVC_ERR_INDEX itself (and clears the word); a valid call passes."""
