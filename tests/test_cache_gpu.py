@@ -135,6 +135,39 @@ def test_hca_listed_cache_insertion(dt):
     check_close(rope, ref_rope, "bf16", "hca listed rope")
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_cache_random_layouts(seed):
+    """Seeded random cache layouts: c a multiple of 8, r a multiple of 8 in [0, c] (the
+    layout's rule), position offset and stride, FP8 scale; CSA (m = 4) and HCA (m = 64 or
+    128), bf16 or fp32 streams."""
+    rng = np.random.default_rng(40 + seed)
+    for mode in ("csa", "hca"):
+        c = 8 * int(rng.integers(2, 97))
+        r = 8 * int(rng.integers(0, c // 8 + 1))
+        dt = rng.choice(["bf16", "f32"])
+        m = 4 if mode == "csa" else int(rng.choice([64, 128]))
+        batch, n = int(rng.integers(1, 3)), int(rng.integers(m, 30 * m))
+        stride, offset = float(rng.choice([1.0, 4.0, 128.0])), float(rng.uniform(0, 5000))
+        scale = float(rng.choice([0.5, 1.0, 8.0]))
+        inv = _inv_freq(max(r, 2))
+        d = synth.stream_inputs(mode, batch, n, c, m, dt, seed=seed * 5 + c)
+        t = {k: dev(v, dt) if v.ndim == 3 else dev(v, "f32") for k, v in d.items()}
+        invt = torch.from_numpy(inv).cuda()
+        if mode == "csa":
+            nope, rope = kvc.csa_compress_cache(t["Ca"], t["Cb"], t["Za"], t["Zb"], t["Ba"], t["Bb"], r,
+                                                invt, pos_stride=stride, pos_offset=offset,
+                                                fp8_scale=scale, m=m)
+            ref = O.csa_compress(d["Ca"], d["Cb"], d["Za"], d["Zb"], d["Ba"], d["Bb"], m, True)
+        else:
+            nope, rope = kvc.hca_compress_cache(t["C"], t["Z"], t["B"], r, invt, pos_stride=stride,
+                                                pos_offset=offset, fp8_scale=scale, m=m)
+            ref = O.hca_compress(d["C"], d["Z"], d["B"], m)
+        torch.cuda.synchronize()
+        what = f"{mode} cache c={c} r={r} m={m} {dt} ({kvc.last_kernel()})"
+        assert kvc.device_status() == kvc.KVC_OK, what
+        _compare(nope, rope, ref, r, inv[:r // 2], stride, offset, scale, what)
+
+
 def test_cache_rejects_bad_layout():
     x = torch.zeros((1, 64, 128), device="cuda", dtype=torch.bfloat16)
     b = torch.zeros((4, 128), device="cuda")

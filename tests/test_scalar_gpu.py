@@ -94,3 +94,37 @@ def test_scalar_long_sampled():
                                           True, entries=[(0, j)])[0])
         got.append(host64(out[0, i]))
     check_close(torch.from_numpy(np.array(got)), np.array(refs), "bf16", "csa scalar n=2^20")
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_scalar_random_shapes(seed):
+    """Seeded random scalar-logit problems: CSA with m in {1, 2, 4, 8, 12} (with and
+    without overlap) and HCA with m in {8, 32, 128, 200}; c any multiple of 8 up to 1024,
+    ragged n, 1-3 sequences, every input/output dtype pair; outputs between canary bands."""
+    rng = np.random.default_rng(300 + seed)
+    for mode in ("csa", "hca"):
+        batch = int(rng.integers(1, 4))
+        c = 8 * int(rng.integers(1, 129))
+        in_dt, out_dt = rng.choice(["bf16", "f32"]), rng.choice(["bf16", "f32"])
+        m = int(rng.choice([1, 2, 4, 8, 12] if mode == "csa" else [8, 32, 128, 200]))
+        n = int(rng.integers(m, min(40 * m + 5, 2_000_000 // c)))
+        d = synth.scalar_inputs(mode, batch, n, c, m, in_dt, seed=seed * 7 + m)
+        ne = n // m
+        buf = torch.full((batch * ne * c + 128,), -333.0, device="cuda", dtype=tdtype(out_dt))
+        out = buf[64:64 + batch * ne * c].view(batch, ne, c)
+        if mode == "csa":
+            overlap = bool(rng.random() < 0.7)
+            t = {k: dev(v, in_dt) if k in ("Ca", "Cb", "za", "zb") else dev(v, "f32") for k, v in d.items()}
+            kvc.csa_compress_scalar_logits(t["Ca"], t["Cb"], t["za"], t["zb"], t["ba"], t["bb"], m=m,
+                                           overlap=overlap, out=out, out_dtype=tdtype(out_dt))
+            ref = O.csa_compress_scalar(d["Ca"], d["Cb"] if overlap else None, d["za"],
+                                        d["zb"] if overlap else None, d["ba"],
+                                        d["bb"] if overlap else None, m, overlap)
+        else:
+            kvc.hca_compress_scalar_logits(dev(d["C"], in_dt), dev(d["z"], in_dt), dev(d["b"], "f32"),
+                                           m=m, out=out, out_dtype=tdtype(out_dt))
+            ref = O.hca_compress_scalar(d["C"], d["z"], d["b"], m)
+        what = f"{mode} scalar b={batch} n={n} c={c} m={m} {in_dt}->{out_dt} ({kvc.last_kernel()})"
+        assert kvc.device_status() == kvc.KVC_OK, what
+        check_close(out, ref, out_dt, what)
+        assert bool(torch.all(buf[:64] == -333.0)) and bool(torch.all(buf[64 + batch * ne * c:] == -333.0)), what
